@@ -1,0 +1,174 @@
+/*
+ * mla.h -- C ABI for weight-absorbed Multi-Head Latent Attention (MLA) decode on NVIDIA B200
+ * (sm_100a).  One new query token per sequence attends, across n_heads heads, to a paged
+ * per-layer cache that stores 576 numbers per token: the 512-wide latent c_KV plus the
+ * 64-wide decoupled RoPE key k_R.
+ *
+ * Sources (web pages on MLA, cited by title and section):
+ *   [LP] linuxpro.com.br, "Como a DeepSeek reescreveu o Transformer (MLA)":
+ *        "Classic attention and the cost of the KV cache" (softmax(QK^T/sqrt(d_k) + M)V, the
+ *        new token computes one query row and reads the whole cache), "MLA: compress the pair,
+ *        not the heads" (c^KV 512 + k^R 64 cached; W^UK and W^UV absorbed by associativity).
+ *   [TN] technova-ai.online, "DeepSeek AI efficiency architecture benchmarks", section
+ *        "Architectural Innovations: Multi-Head Latent Attention (MLA)": c_KV = W_DKV h_t,
+ *        K_t = W_UK c_KV, V_t = W_UV c_KV.
+ *   [IA] ia.com.br, "Como a MLA da DeepSeek cortou 93% da memoria ...", section
+ *        "Um resumo no lugar de 128 copias": RoPE kept out of the compression as 64 numbers.
+ *
+ * Conventions shared by every call
+ *   - All pointers except `dims` are DEVICE pointers owned by the caller; the library never
+ *     allocates or frees memory and keeps no state between calls other than one device status
+ *     word per GPU (see mla_get_status).
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *   - Weights are row-major [out_features, in_features] (column-vector form, [TN]):
+ *       w_dkv [d_c, D], w_kr [d_rope, D], w_q [H*(d_nope+d_rope), D] (per head d_nope rows then
+ *       d_rope rows), w_uk [H*d_nope, d_c], w_uv [H*d_v, d_c], w_o [D, H*d_v].
+ *   - Element type: dims.dtype = MLA_BF16 -> h, weights, cache, q_cat, o_heads, out are bf16;
+ *     MLA_FP32 -> all of them fp32.  o_lat and lse are fp32 in both cases.
+ *   - Cache pool: [num_pages, page_size, d_c + d_rope] rows of one layer; row = [c_KV | k_R].
+ *     page_table [batch, max_pages] int32 (row-major) maps a sequence's page index to a pool
+ *     page; only entries [0, ceil(len/page_size)) of a row are read.  Cache slots past a
+ *     sequence's length must hold finite values; they never influence a result.
+ *   - RoPE: interleaved pairs (x[2i], x[2i+1]) rotated by pos * rope_theta^(-2i/d_rope); the
+ *     same rotation is applied to k_R (shared by all heads) and to every head's query part.
+ *   - Return value: MLA_OK (0) or a negative MLA_ERR_* detected on the host before any launch
+ *     (nothing was enqueued).  Errors found on the device while a kernel runs (bad page id,
+ *     over-long sequence, timed-out wait) are OR-ed into the status word; kernels never trap.
+ *   - A workspace (device, >= 256-byte aligned, size from mla_workspace_size) is scratch
+ *     shared by the four compute calls; calls that share one workspace must be ordered (same
+ *     stream or synchronised).
+ */
+#ifndef MLA_B200_H_
+#define MLA_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* mla_stream_t; /* same type as cudaStream_t */
+
+enum { MLA_BF16 = 0, MLA_FP32 = 1 };
+
+/* Shapes.  Supported: d_c = 512, d_rope = 64, d_nope = 128, d_v = 128, page_size = 64,
+ * n_heads in {16, 32, ..., 128}, d_model a positive multiple of 64, batch >= 1.
+ * rope_theta > 0 (10000 for DeepSeek-V2/V3). */
+typedef struct mla_dims {
+  int32_t batch;     /* B: sequences, one new token each */
+  int32_t n_heads;   /* H */
+  int32_t d_c;       /* latent width of c_KV */
+  int32_t d_rope;    /* width of the decoupled RoPE key k_R and of each head's q_rope */
+  int32_t d_nope;    /* per-head non-rotary query/key width */
+  int32_t d_v;       /* per-head value width */
+  int32_t d_model;   /* D: hidden size of h_t */
+  int32_t page_size; /* tokens per cache page */
+  int32_t dtype;     /* MLA_BF16 or MLA_FP32 */
+  float rope_theta;  /* RoPE base */
+} mla_dims;
+
+/* Host-detected errors (returned). */
+#define MLA_OK 0
+#define MLA_ERR_NULL_ARG (-1)    /* a required pointer is NULL */
+#define MLA_ERR_DIMS (-2)        /* unsupported shape or dtype */
+#define MLA_ERR_ALIGN (-3)       /* a pointer is not 16-byte aligned (workspace: 256) */
+#define MLA_ERR_WORKSPACE (-4)   /* workspace missing or smaller than mla_workspace_size */
+#define MLA_ERR_ARG (-5)         /* other bad argument (negative count, bad option) */
+#define MLA_ERR_CUDA (-6)        /* a CUDA runtime call failed (launch, attribute, device) */
+#define MLA_ERR_DEVICE (-7)      /* current device is not sm_100 */
+
+/* Device-detected conditions (bits of the status word, see mla_get_status). */
+#define MLA_STATUS_BAD_PAGE 0x1u     /* a page id outside [0, num_pages) was skipped */
+#define MLA_STATUS_BAD_LENGTH 0x2u   /* a sequence length outside [0, max_pages*page_size] */
+#define MLA_STATUS_TIMEOUT 0x4u      /* a bounded wait inside a kernel gave up */
+#define MLA_STATUS_BAD_POSITION 0x8u /* an append position outside the sequence's pages */
+
+/* Scratch bytes needed by every compute call for these dims when the decode call is split
+ * into at most `num_splits` parts (0 = the library's automatic choice).  Never fails. */
+size_t mla_workspace_size(const mla_dims* dims, int32_t num_splits);
+
+/* Bytes one cached token occupies in one layer's pool: (d_c + d_rope) * element size.
+ * For DeepSeek-V3 shapes in bf16 this is 1152; times 61 layers, 70,272 bytes per token
+ * ([LP] "MLA: compress the pair, not the heads"). Returns 0 for unsupported dims. */
+int64_t mla_cache_row_bytes(const mla_dims* dims);
+
+/*
+ * mla_cache_append -- the new token's cache row ([TN]; [LP] "MLA: compress the pair ..."):
+ *   c_KV = W_DKV h_t,   k_R = RoPE(W_KR h_t, positions[b]),
+ * rounded to the cache dtype (round-to-nearest-even) and written to slot
+ * positions[b] % page_size of pool page page_table[b][positions[b] / page_size].
+ *   h        [B, D]
+ *   w_dkv, w_kr: the two projections; if BOTH are NULL, h is taken as ready rows
+ *            [B, d_c + d_rope] (already rotated) and only the paged scatter runs.
+ *   positions [B] int32, 0-based index of the new token (= rows already cached).
+ * Only the addressed slot of each sequence is written; all other pool bytes are untouched.
+ */
+int mla_cache_append(const mla_dims* dims, const void* h, const void* w_dkv, const void* w_kr,
+                     const int32_t* positions, const int32_t* page_table, int32_t max_pages,
+                     void* cache_pool, int32_t num_pages, void* workspace,
+                     size_t workspace_bytes, mla_stream_t stream);
+
+/*
+ * mla_absorb_q -- absorbed query ([LP] "MLA: compress the pair ...", associativity
+ * Q (c W_UK)^T = (Q W_UK^T) c^T):
+ *   q = W_Q h_t;  per head q_nope = q[h*192 : h*192+128],  q_rope = RoPE(q[h*192+128 : +64]);
+ *   q_lat_h = W_UK_h^T q_nope_h (512);   q_cat[b][h] = [q_lat_h | q_rope_h]   (576).
+ *   q_cat    [B, H, d_c + d_rope] (dims.dtype)
+ *   q_lo     nullable; bf16 only: [B, H, d_c + d_rope] receives the rounding remainder
+ *            q - bf16(q) of every element, so that q_cat + q_lo carries ~16 significant bits.
+ *            Pass it on to mla_decode_attn when score logits are large (|logit| >> 10).
+ * q_nope is kept at ~16 bits (bf16 hi + lo) through the W_UK product; accumulation is fp32.
+ */
+int mla_absorb_q(const mla_dims* dims, const void* h, const void* w_q, const void* w_uk,
+                 const int32_t* positions, void* q_cat, void* q_lo, void* workspace,
+                 size_t workspace_bytes, mla_stream_t stream);
+
+/*
+ * mla_decode_attn -- attention of each sequence's new query over its whole cache
+ * ([LP] "Classic attention ...": softmax(Q K^T / sqrt(d_k) + M) V, causal mask M admits every
+ * cached row since the query is the newest token), in latent space:
+ *   s_j = scale * (q_lat . c_j + q_rope . k_R,j),  j < seq_lens[b];   p = softmax(s);
+ *   o_lat[b][h] = sum_j p_j c_j (d_c wide),   lse[b][h] = log sum_j exp(s_j).
+ *   q_cat    [B, H, d_c + d_rope] (dims.dtype); q_lo nullable (bf16, see mla_absorb_q).
+ *   seq_lens [B] int32 (rows to attend, including the token just appended); 0 is allowed
+ *            and yields o_lat = 0, lse = -inf.
+ *   softmax_scale: 0 selects 1/sqrt(d_nope + d_rope).
+ *   num_splits: number of parts the concatenated page list of all sequences is divided into
+ *            (split-KV); 0 = automatic (about one part per pair of SMs).  Must not exceed the
+ *            value used for mla_workspace_size.
+ *   o_lat    [B, H, d_c] fp32;  lse [B, H] fp32, nullable.
+ */
+int mla_decode_attn(const mla_dims* dims, const void* q_cat, const void* q_lo,
+                    const void* cache_pool, int32_t num_pages, const int32_t* page_table,
+                    int32_t max_pages, const int32_t* seq_lens, float softmax_scale,
+                    int32_t num_splits, void* workspace, size_t workspace_bytes, float* o_lat,
+                    float* lse, mla_stream_t stream);
+
+/*
+ * mla_out_proj -- value up-projection and output projection ([TN] V = W_UV c_KV, moved after
+ * the weighted sum by associativity; [LP] W_O):
+ *   o_heads[b][h] = W_UV_h o_lat[b][h]  (d_v wide),   out[b] = W_O concat_h o_heads[b][h].
+ *   o_lat    [B, H, d_c] fp32 (from mla_decode_attn).
+ *   o_heads  [B, H, d_v] (dims.dtype), nullable if only `out` is wanted.
+ *   w_o, out nullable together (then only o_heads is produced).
+ */
+int mla_out_proj(const mla_dims* dims, const float* o_lat, const void* w_uv, const void* w_o,
+                 void* o_heads, void* out, void* workspace, size_t workspace_bytes,
+                 mla_stream_t stream);
+
+/* Synchronises `stream`, returns the device status word of the current device (a bitwise OR
+ * of MLA_STATUS_* raised since the last call, 0 if none) and clears it.  Returns a negative
+ * MLA_ERR_CUDA if the synchronisation itself failed. */
+int mla_get_status(mla_stream_t stream);
+
+/* Static description of a return code or status bit set. */
+const char* mla_error_string(int code);
+
+/* Library build string (for logs). */
+const char* mla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MLA_B200_H_ */

@@ -1,0 +1,215 @@
+"""Python binding of the MLA decode C ABI (``libmla_b200.so``, declared in ``include/mla.h``).
+
+Argument marshalling only: every function takes torch tensors already on the GPU, checks dtype,
+shape and contiguity, and passes raw device pointers plus the current CUDA stream to the
+library.  Every step of the computation runs in the library's kernels; there is no fallback.
+Functions keep the C names: ``mla_cache_append``, ``mla_absorb_q``, ``mla_decode_attn``,
+``mla_out_proj``, plus ``mla_workspace_size``, ``mla_cache_row_bytes``, ``mla_get_status``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmla_b200.so")
+
+MLA_BF16 = 0
+MLA_FP32 = 1
+
+STATUS_BAD_PAGE = 0x1
+STATUS_BAD_LENGTH = 0x2
+STATUS_TIMEOUT = 0x4
+STATUS_BAD_POSITION = 0x8
+
+ERRORS = {
+    -1: "MLA_ERR_NULL_ARG", -2: "MLA_ERR_DIMS", -3: "MLA_ERR_ALIGN", -4: "MLA_ERR_WORKSPACE",
+    -5: "MLA_ERR_ARG", -6: "MLA_ERR_CUDA", -7: "MLA_ERR_DEVICE",
+}
+
+
+class MlaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {ERRORS.get(code, code)} ({_error_string(code)})")
+
+
+class mla_dims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("n_heads", ctypes.c_int32), ("d_c", ctypes.c_int32),
+                ("d_rope", ctypes.c_int32), ("d_nope", ctypes.c_int32), ("d_v", ctypes.c_int32),
+                ("d_model", ctypes.c_int32), ("page_size", ctypes.c_int32),
+                ("dtype", ctypes.c_int32), ("rope_theta", ctypes.c_float)]
+
+
+def dims(batch: int, n_heads: int = 128, d_model: int = 7168, dtype=torch.bfloat16,
+         rope_theta: float = 10000.0) -> mla_dims:
+    return mla_dims(batch, n_heads, 512, 64, 128, 128, d_model, 64,
+                    MLA_BF16 if dtype == torch.bfloat16 else MLA_FP32, rope_theta)
+
+
+_lib = None
+_P = ctypes.c_void_p
+_I = ctypes.c_int32
+_SZ = ctypes.c_size_t
+_SIGS = {
+    "mla_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(mla_dims), _I]),
+    "mla_cache_row_bytes": (ctypes.c_int64, [ctypes.POINTER(mla_dims)]),
+    "mla_cache_append": (ctypes.c_int, [ctypes.POINTER(mla_dims), _P, _P, _P, _P, _P, _I, _P, _I,
+                                        _P, _SZ, _P]),
+    "mla_absorb_q": (ctypes.c_int, [ctypes.POINTER(mla_dims), _P, _P, _P, _P, _P, _P, _P, _SZ,
+                                    _P]),
+    "mla_decode_attn": (ctypes.c_int, [ctypes.POINTER(mla_dims), _P, _P, _P, _I, _P, _I, _P,
+                                       ctypes.c_float, _I, _P, _SZ, _P, _P, _P]),
+    "mla_out_proj": (ctypes.c_int, [ctypes.POINTER(mla_dims), _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "mla_get_status": (ctypes.c_int, [_P]),
+    "mla_error_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "mla_version": (ctypes.c_char_p, []),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """Load the CUDA library; fails loudly when it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m mla_latent_kv_37_b200.build`")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def _error_string(code: int) -> str:
+    try:
+        return lib().mla_error_string(code).decode()
+    except Exception:  # pragma: no cover
+        return "?"
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(rc: int, where: str):
+    if rc != 0:
+        raise MlaError(rc, where)
+
+
+def _need(t, name, dtype=None, shape=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _elem(d: mla_dims):
+    return torch.bfloat16 if d.dtype == MLA_BF16 else torch.float32
+
+
+def mla_workspace_size(d: mla_dims, num_splits: int = 0) -> int:
+    return int(lib().mla_workspace_size(ctypes.byref(d), num_splits))
+
+
+def mla_cache_row_bytes(d: mla_dims) -> int:
+    return int(lib().mla_cache_row_bytes(ctypes.byref(d)))
+
+
+def workspace(d: mla_dims, num_splits: int = 0, device="cuda") -> torch.Tensor:
+    n = mla_workspace_size(d, num_splits)
+    if n == 0:
+        raise MlaError(-2, "mla_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def mla_cache_append(d: mla_dims, h, w_dkv, w_kr, positions, page_table, cache_pool, ws=None,
+                     stream=None):
+    e = _elem(d)
+    row = d.d_c + d.d_rope
+    _need(h, "h", e, (d.batch, row) if w_dkv is None else (d.batch, d.d_model))
+    _need(w_dkv, "w_dkv", e, (d.d_c, d.d_model))
+    _need(w_kr, "w_kr", e, (d.d_rope, d.d_model))
+    _need(positions, "positions", torch.int32, (d.batch,))
+    _need(page_table, "page_table", torch.int32)
+    _need(cache_pool, "cache_pool", e)
+    _need(ws, "workspace", torch.uint8)
+    rc = lib().mla_cache_append(ctypes.byref(d), _ptr(h), _ptr(w_dkv), _ptr(w_kr), _ptr(positions),
+                                _ptr(page_table), page_table.shape[1], _ptr(cache_pool),
+                                cache_pool.shape[0], _ptr(ws), 0 if ws is None else ws.numel(),
+                                _stream(stream))
+    _check(rc, "mla_cache_append")
+
+
+def mla_absorb_q(d: mla_dims, h, w_q, w_uk, positions, q_cat, ws, q_lo=None, stream=None):
+    e = _elem(d)
+    H = d.n_heads
+    _need(h, "h", e, (d.batch, d.d_model))
+    _need(w_q, "w_q", e, (H * (d.d_nope + d.d_rope), d.d_model))
+    _need(w_uk, "w_uk", e, (H * d.d_nope, d.d_c))
+    _need(positions, "positions", torch.int32, (d.batch,))
+    _need(q_cat, "q_cat", e, (d.batch, H, d.d_c + d.d_rope))
+    _need(q_lo, "q_lo", torch.bfloat16, (d.batch, H, d.d_c + d.d_rope))
+    _need(ws, "workspace", torch.uint8)
+    rc = lib().mla_absorb_q(ctypes.byref(d), _ptr(h), _ptr(w_q), _ptr(w_uk), _ptr(positions),
+                            _ptr(q_cat), _ptr(q_lo), _ptr(ws), ws.numel(), _stream(stream))
+    _check(rc, "mla_absorb_q")
+
+
+def mla_decode_attn(d: mla_dims, q_cat, cache_pool, page_table, seq_lens, o_lat, ws, lse=None,
+                    q_lo=None, softmax_scale: float = 0.0, num_splits: int = 0, stream=None):
+    e = _elem(d)
+    H = d.n_heads
+    _need(q_cat, "q_cat", e, (d.batch, H, d.d_c + d.d_rope))
+    _need(cache_pool, "cache_pool", e)
+    _need(page_table, "page_table", torch.int32)
+    _need(seq_lens, "seq_lens", torch.int32, (d.batch,))
+    _need(o_lat, "o_lat", torch.float32, (d.batch, H, d.d_c))
+    _need(lse, "lse", torch.float32, (d.batch, H))
+    _need(q_lo, "q_lo", torch.bfloat16)
+    _need(ws, "workspace", torch.uint8)
+    rc = lib().mla_decode_attn(ctypes.byref(d), _ptr(q_cat), _ptr(q_lo), _ptr(cache_pool),
+                               cache_pool.shape[0], _ptr(page_table), page_table.shape[1],
+                               _ptr(seq_lens), float(softmax_scale), int(num_splits), _ptr(ws),
+                               ws.numel(), _ptr(o_lat), _ptr(lse), _stream(stream))
+    _check(rc, "mla_decode_attn")
+
+
+def mla_out_proj(d: mla_dims, o_lat, w_uv, ws, w_o=None, o_heads=None, out=None, stream=None):
+    e = _elem(d)
+    H = d.n_heads
+    _need(o_lat, "o_lat", torch.float32, (d.batch, H, d.d_c))
+    _need(w_uv, "w_uv", e, (H * d.d_v, d.d_c))
+    _need(w_o, "w_o", e, (d.d_model, H * d.d_v))
+    _need(o_heads, "o_heads", e, (d.batch, H, d.d_v))
+    _need(out, "out", e, (d.batch, d.d_model))
+    _need(ws, "workspace", torch.uint8)
+    rc = lib().mla_out_proj(ctypes.byref(d), _ptr(o_lat), _ptr(w_uv), _ptr(w_o), _ptr(o_heads),
+                            _ptr(out), _ptr(ws), ws.numel(), _stream(stream))
+    _check(rc, "mla_out_proj")
+
+
+def mla_get_status(stream=None) -> int:
+    rc = lib().mla_get_status(_stream(stream))
+    if rc < 0:
+        raise MlaError(rc, "mla_get_status")
+    return rc
+
+
+def version() -> str:
+    return lib().mla_version().decode()

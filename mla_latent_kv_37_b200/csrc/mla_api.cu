@@ -1,0 +1,604 @@
+// C ABI of the MLA decode library (see include/mla.h for the contract of every entry point).
+// Host side: argument validation (before any CUDA call), per-device context, TMA descriptor
+// encoding, workspace layout, launch configuration.  All device work is in the included
+// kernel headers.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "attn_f32.cuh"
+#include "attn_sm100.cuh"
+#include "epilogue.cuh"
+#include "gemm_sm100.cuh"
+
+namespace mla {
+
+__device__ unsigned int g_status_word;
+
+namespace {
+
+constexpr int kDc = 512, kDr = 64, kDn = 128, kDv = 128, kRowN = 576, kPageN = 64;
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;  // 2 s per bounded wait
+constexpr int kMinPagesPerPart = 4;
+constexpr int kMaxKSplits = 32;
+constexpr uint32_t kGemmSmemBudget = 200 * 1024;
+
+// ------------------------------------------------------------------------------------------
+// validation
+// ------------------------------------------------------------------------------------------
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_dims(const mla_dims* d) {
+  if (!d) return MLA_ERR_NULL_ARG;
+  if (d->d_c != kDc || d->d_rope != kDr || d->d_nope != kDn || d->d_v != kDv ||
+      d->page_size != kPageN)
+    return MLA_ERR_DIMS;
+  if (d->n_heads < 16 || d->n_heads > 128 || d->n_heads % 16) return MLA_ERR_DIMS;
+  if (d->d_model <= 0 || d->d_model % 64) return MLA_ERR_DIMS;
+  if (d->batch < 1) return MLA_ERR_DIMS;
+  if (d->dtype != MLA_BF16 && d->dtype != MLA_FP32) return MLA_ERR_DIMS;
+  if (d->dtype == MLA_BF16 && d->batch > 128) return MLA_ERR_DIMS;  // 2B <= 256 MMA columns
+  if (!(d->rope_theta > 0.f) || !std::isfinite(d->rope_theta)) return MLA_ERR_DIMS;
+  return MLA_OK;
+}
+
+size_t elem_size(const mla_dims* d) { return d->dtype == MLA_BF16 ? 2 : 4; }
+
+// ------------------------------------------------------------------------------------------
+// per-device context
+// ------------------------------------------------------------------------------------------
+struct DevCtx {
+  bool init = false;
+  int cc_major = 0;
+  int sms = 0;
+  int max_clusters = 0;
+  unsigned int* status = nullptr;
+};
+DevCtx g_dev[64];
+std::mutex g_mu;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int device_ctx(DevCtx** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MLA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DevCtx& c = g_dev[dev];
+  if (!c.init) {
+    if (cudaDeviceGetAttribute(&c.cc_major, cudaDevAttrComputeCapabilityMajor, dev) !=
+        cudaSuccess)
+      return MLA_ERR_CUDA;
+    if (c.cc_major != 10) return MLA_ERR_DEVICE;
+    if (cudaDeviceGetAttribute(&c.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return MLA_ERR_CUDA;
+    void* sym = nullptr;
+    if (cudaGetSymbolAddress(&sym, g_status_word) != cudaSuccess) return MLA_ERR_CUDA;
+    c.status = static_cast<unsigned int*>(sym);
+    if (!g_encode) {
+      cudaDriverEntryPointQueryResult q;
+      void* fn = nullptr;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+              cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || !fn)
+        return MLA_ERR_CUDA;
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    // kernel attributes (once per device)
+    const int attn_smem = static_cast<int>(attn::kSmemBytes);
+    if (cudaFuncSetAttribute(attn::split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             attn_smem) != cudaSuccess)
+      return MLA_ERR_CUDA;
+    if (cudaFuncSetAttribute(gemm_swapab_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kGemmSmemBudget + 2048)) != cudaSuccess)
+      return MLA_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(attn::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = attn::kSmemBytes;
+    int nclusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&nclusters, attn::split_kernel, &cfg) != cudaSuccess ||
+        nclusters <= 0)
+      nclusters = c.sms / 2;
+    c.max_clusters = nclusters;
+    c.init = true;
+  }
+  *out = &c;
+  return MLA_OK;
+}
+
+int default_parts(int sms, int max_clusters) { return max_clusters > 0 ? max_clusters : sms / 2; }
+
+// ------------------------------------------------------------------------------------------
+// GEMM configuration
+// ------------------------------------------------------------------------------------------
+int n_pad_for(int rows) { return std::max(16, (rows + 15) / 16 * 16); }
+
+int choose_k_splits(int tiles, int k_blocks, int sms) {
+  int best = 1;
+  double best_eff = 0.0;
+  const int max_s = std::max(1, std::min(kMaxKSplits, k_blocks / 2));
+  for (int s = 1; s <= max_s; ++s) {
+    const int ctas = tiles * s;
+    const int waves = (ctas + sms - 1) / sms;
+    const double eff = static_cast<double>(ctas) / (static_cast<double>(waves) * sms);
+    if (eff > best_eff + 0.02) {
+      best = s;
+      best_eff = eff;
+    }
+  }
+  return best;
+}
+
+struct GemmShape {
+  int m_total, m_tiles, k, groups, n_rows;
+  int k_blocks() const { return (k + 63) / 64; }
+};
+
+// the five products of a layer (bf16 path; the fp32 path uses k_splits = 1)
+GemmShape shape_append(const mla_dims* d) { return {kRowN, 5, d->d_model, 1, d->batch}; }
+GemmShape shape_wq(const mla_dims* d) {
+  return {d->n_heads * (kDn + kDr), d->n_heads * (kDn + kDr) / 128, d->d_model, 1, d->batch};
+}
+GemmShape shape_wuk(const mla_dims* d) { return {kDc, kDc / 128, kDn, d->n_heads, 2 * d->batch}; }
+GemmShape shape_wuv(const mla_dims* d) { return {kDv, 1, kDc, d->n_heads, 2 * d->batch}; }
+GemmShape shape_wo(const mla_dims* d) {
+  return {d->d_model, (d->d_model + 127) / 128, d->n_heads * kDv, 1, 2 * d->batch};
+}
+
+size_t partial_bytes(const GemmShape& s, int sms) {
+  const int ks = choose_k_splits(s.m_tiles * s.groups, s.k_blocks(), sms);
+  return static_cast<size_t>(ks) * s.groups * s.m_total * n_pad_for(s.n_rows) * sizeof(float);
+}
+
+// ------------------------------------------------------------------------------------------
+// workspace layout
+// ------------------------------------------------------------------------------------------
+struct Workspace {
+  size_t partial, qn, o_split, oh_split, plan, part_o, part_lse, total;
+};
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+Workspace layout(const mla_dims* d, int num_parts, int sms) {
+  const size_t B = d->batch, H = d->n_heads;
+  size_t part = 0;
+  if (d->dtype == MLA_BF16) {
+    part = std::max({partial_bytes(shape_append(d), sms), partial_bytes(shape_wq(d), sms),
+                     partial_bytes(shape_wuk(d), sms), partial_bytes(shape_wuv(d), sms),
+                     partial_bytes(shape_wo(d), sms)});
+  } else {
+    part = std::max({static_cast<size_t>(kRowN) * B, H * (kDn + kDr) * B, H * kDc * B,
+                     H * kDv * B, static_cast<size_t>(d->d_model) * B}) *
+           sizeof(float);
+  }
+  Workspace w{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  w.partial = take(part);
+  w.qn = take(2 * B * H * kDn * 4);        // bf16 hi/lo planes, or fp32
+  w.o_split = take(2 * B * H * kDc * 2);   // bf16 hi/lo of o_lat
+  w.oh_split = take(2 * B * H * kDv * 4);  // bf16 hi/lo, or fp32
+  w.plan = take(attn::PlanView::words(static_cast<int>(B), num_parts) * 4);
+  w.part_o = take((B + num_parts) * H * kDc * 4);
+  w.part_lse = take((B + num_parts) * H * 4);
+  w.total = off;
+  return w;
+}
+
+int resolve_parts(int num_splits, const DevCtx* c) {
+  return num_splits > 0 ? num_splits : default_parts(c ? c->sms : 148, c ? c->max_clusters : 74);
+}
+
+// ------------------------------------------------------------------------------------------
+// TMA descriptors
+// ------------------------------------------------------------------------------------------
+int encode(CUtensorMap* m, CUtensorMapDataType dt, const void* base, int rank,
+           const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+           CUtensorMapSwizzle sw) {
+  cuuint64_t gdim[5];
+  cuuint64_t gstr[4];
+  cuuint32_t bdim[5], estr[5];
+  for (int i = 0; i < rank; ++i) {
+    gdim[i] = dims[i];
+    bdim[i] = box[i];
+    estr[i] = 1;
+  }
+  for (int i = 0; i < rank - 1; ++i) gstr[i] = strides_bytes[i];
+  const CUresult r = g_encode(m, dt, rank, const_cast<void*>(base), gdim, gstr, bdim, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_ARG;
+}
+
+// 3-D bf16 map (k contiguous, then rows_a, then rows_b), box (64, box_a, box_b), 128B swizzle.
+int map3(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
+         uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2,
+         CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B) {
+  const uint64_t dims[3] = {d0, d1, d2};
+  const uint64_t str[2] = {s1, s2};
+  const uint32_t box[3] = {b0, b1, b2};
+  return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, 3, dims, str, box, sw);
+}
+
+// 2-D bf16 map (k contiguous, rows), box (b0, b1).
+int map2(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t s1, uint32_t b0,
+         uint32_t b1, CUtensorMapSwizzle sw) {
+  const uint64_t dims[2] = {d0, d1};
+  const uint64_t str[1] = {s1};
+  const uint32_t box[2] = {b0, b1};
+  return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, 2, dims, str, box, sw);
+}
+
+// ------------------------------------------------------------------------------------------
+// launches
+// ------------------------------------------------------------------------------------------
+int last_launch() { return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
+
+int gemm_stages(int n_pad) {
+  const uint32_t sb = gemm_stage_bytes(n_pad);
+  return std::max(2, std::min(8, static_cast<int>(kGemmSmemBudget / sb)));
+}
+
+// P[ks][g][m][n] for one product on tensor cores.
+int run_gemm(const DevCtx* c, const GemmShape& s, const CUtensorMap& a0, const CUtensorMap& a1,
+             int a1_tile_start, int a_mn_major, const CUtensorMap& bmap, float* partial,
+             cudaStream_t st, int* k_splits_out) {
+  GemmParams p{};
+  p.m_total = s.m_total;
+  p.m_tiles = s.m_tiles;
+  p.a1_tile_start = a1_tile_start;
+  p.k_blocks = s.k_blocks();
+  p.k_splits = choose_k_splits(s.m_tiles * s.groups, p.k_blocks, c->sms);
+  p.n_pad = n_pad_for(s.n_rows);
+  p.a_mn_major = a_mn_major;
+  p.stages = gemm_stages(p.n_pad);
+  p.groups = s.groups;
+  p.partial = partial;
+  p.status = c->status;
+  p.wait_ns = kDefaultWaitNs;
+  const size_t smem = static_cast<size_t>(p.stages) * gemm_stage_bytes(p.n_pad) +
+                      (2 * p.stages + 1) * 8 + 16 + 1024;
+  gemm_swapab_kernel<<<dim3(s.m_tiles, p.k_splits, s.groups), kGemmThreads, smem, st>>>(
+      a0, a1, bmap, p);
+  *k_splits_out = p.k_splits;
+  return last_launch();
+}
+
+}  // namespace
+}  // namespace mla
+
+using namespace mla;
+
+// =============================================================================================
+// C ABI
+// =============================================================================================
+extern "C" {
+
+size_t mla_workspace_size(const mla_dims* dims, int32_t num_splits) {
+  if (check_dims(dims) != MLA_OK || num_splits < 0) return 0;
+  DevCtx* c = nullptr;
+  const bool have = device_ctx(&c) == MLA_OK;
+  const int sms = have ? c->sms : 148;
+  const int parts = num_splits > 0 ? num_splits : (have ? resolve_parts(0, c) : 74);
+  return layout(dims, parts, sms).total;
+}
+
+int64_t mla_cache_row_bytes(const mla_dims* dims) {
+  if (check_dims(dims) != MLA_OK) return 0;
+  return static_cast<int64_t>(dims->d_c + dims->d_rope) * static_cast<int64_t>(elem_size(dims));
+}
+
+int mla_cache_append(const mla_dims* dims, const void* h, const void* w_dkv, const void* w_kr,
+                     const int32_t* positions, const int32_t* page_table, int32_t max_pages,
+                     void* cache_pool, int32_t num_pages, void* workspace,
+                     size_t workspace_bytes, mla_stream_t stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (!h || !positions || !page_table || !cache_pool) return MLA_ERR_NULL_ARG;
+  const bool scatter_only = (w_dkv == nullptr && w_kr == nullptr);
+  if (!scatter_only && (!w_dkv || !w_kr)) return MLA_ERR_NULL_ARG;
+  if (max_pages < 1 || num_pages < 1) return MLA_ERR_ARG;
+  if (!aligned(h, 16) || !aligned(cache_pool, 16) || (w_dkv && !aligned(w_dkv, 16)) ||
+      (w_kr && !aligned(w_kr, 16)) || !aligned(positions, 4) || !aligned(page_table, 4))
+    return MLA_ERR_ALIGN;
+  if (!scatter_only && (!workspace)) return MLA_ERR_WORKSPACE;
+  if (workspace && !aligned(workspace, 256)) return MLA_ERR_ALIGN;
+  DevCtx* c = nullptr;
+  if ((rc = device_ctx(&c))) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int B = dims->batch, D = dims->d_model;
+  const dim3 eg((kRowN / 2 + 95) / 96, B);
+  if (scatter_only) {
+    if (dims->dtype == MLA_BF16)
+      append_epilogue_kernel<__nv_bfloat16><<<eg, 96, 0, st>>>(
+          nullptr, 0, 0, static_cast<const __nv_bfloat16*>(h), positions, page_table, max_pages,
+          static_cast<__nv_bfloat16*>(cache_pool), num_pages, dims->rope_theta, c->status);
+    else
+      append_epilogue_kernel<float><<<eg, 96, 0, st>>>(
+          nullptr, 0, 0, static_cast<const float*>(h), positions, page_table, max_pages,
+          static_cast<float*>(cache_pool), num_pages, dims->rope_theta, c->status);
+    return last_launch();
+  }
+  const Workspace w = layout(dims, resolve_parts(0, c), c->sms);
+  if (workspace_bytes < w.total) return MLA_ERR_WORKSPACE;
+  float* part = reinterpret_cast<float*>(static_cast<char*>(workspace) + w.partial);
+  if (dims->dtype == MLA_BF16) {
+    const GemmShape s = shape_append(dims);
+    const int n_pad = n_pad_for(s.n_rows);
+    CUtensorMap a0, a1, bm;
+    if ((rc = map3(&a0, w_dkv, D, kDc, 1, D * 2ull, D * 2ull * kDc, 64, 128, 1))) return rc;
+    if ((rc = map3(&a1, w_kr, D, kDr, 1, D * 2ull, D * 2ull * kDr, 64, 128, 1))) return rc;
+    if ((rc = map3(&bm, h, D, 1, B, D * 2ull, D * 2ull, 64, 1, n_pad))) return rc;
+    int ks = 1;
+    if ((rc = run_gemm(c, s, a0, a1, kDc / 128, 0, bm, part, st, &ks))) return rc;
+    append_epilogue_kernel<__nv_bfloat16><<<eg, 96, 0, st>>>(
+        part, ks, n_pad, nullptr, positions, page_table, max_pages,
+        static_cast<__nv_bfloat16*>(cache_pool), num_pages, dims->rope_theta, c->status);
+  } else {
+    // fp32: rows 0..511 from W_DKV, 512..575 from W_KR, written as one [576][B] partial
+    f32_gemm_k_kernel<<<dim3(kDc / 8, 1), 256, 0, st>>>(static_cast<const float*>(w_dkv), 0, D,
+                                                       static_cast<const float*>(h), D, 0, kDc, D,
+                                                       B, part);
+    f32_gemm_k_kernel<<<dim3(kDr / 8, 1), 256, 0, st>>>(static_cast<const float*>(w_kr), 0, D,
+                                                       static_cast<const float*>(h), D, 0, kDr, D,
+                                                       B, part + static_cast<size_t>(kDc) * B);
+    append_epilogue_kernel<float><<<eg, 96, 0, st>>>(
+        part, 1, B, nullptr, positions, page_table, max_pages, static_cast<float*>(cache_pool),
+        num_pages, dims->rope_theta, c->status);
+  }
+  return last_launch();
+}
+
+int mla_absorb_q(const mla_dims* dims, const void* h, const void* w_q, const void* w_uk,
+                 const int32_t* positions, void* q_cat, void* q_lo, void* workspace,
+                 size_t workspace_bytes, mla_stream_t stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (!h || !w_q || !w_uk || !positions || !q_cat) return MLA_ERR_NULL_ARG;
+  if (!workspace) return MLA_ERR_WORKSPACE;
+  if (q_lo && dims->dtype != MLA_BF16) return MLA_ERR_ARG;
+  if (!aligned(h, 16) || !aligned(w_q, 16) || !aligned(w_uk, 16) || !aligned(q_cat, 16) ||
+      (q_lo && !aligned(q_lo, 16)) || !aligned(positions, 4))
+    return MLA_ERR_ALIGN;
+  if (!aligned(workspace, 256)) return MLA_ERR_ALIGN;
+  DevCtx* c = nullptr;
+  if ((rc = device_ctx(&c))) return rc;
+  const Workspace w = layout(dims, resolve_parts(0, c), c->sms);
+  if (workspace_bytes < w.total) return MLA_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int B = dims->batch, D = dims->d_model, H = dims->n_heads;
+  char* ws = static_cast<char*>(workspace);
+  float* part = reinterpret_cast<float*>(ws + w.partial);
+  void* qn = ws + w.qn;
+  const float theta = dims->rope_theta;
+  if (dims->dtype == MLA_BF16) {
+    __nv_bfloat16* qc = static_cast<__nv_bfloat16*>(q_cat);
+    __nv_bfloat16* ql = static_cast<__nv_bfloat16*>(q_lo);
+    // q = W_Q h
+    const GemmShape s1 = shape_wq(dims);
+    const int np1 = n_pad_for(s1.n_rows);
+    CUtensorMap a, bm;
+    if ((rc = map3(&a, w_q, D, s1.m_total, 1, D * 2ull, D * 2ull * s1.m_total, 64, 128, 1)))
+      return rc;
+    if ((rc = map3(&bm, h, D, 1, B, D * 2ull, D * 2ull, 64, 1, np1))) return rc;
+    int ks = 1;
+    if ((rc = run_gemm(c, s1, a, a, 1 << 30, 0, bm, part, st, &ks))) return rc;
+    wq_epilogue_kernel<__nv_bfloat16><<<dim3(H, B), 96, 0, st>>>(part, ks, np1, B, H, positions,
+                                                                 theta, qc, ql, qn);
+    if ((rc = last_launch())) return rc;
+    // q_lat_h = W_UK_h^T [q_nope_hi | q_nope_lo]   (A MN-major: W_UK rows are the K side)
+    const GemmShape s2 = shape_wuk(dims);
+    const int np2 = n_pad_for(s2.n_rows);
+    CUtensorMap a2, b2;
+    if ((rc = map3(&a2, w_uk, kDc, kDn, H, kDc * 2ull, kDc * 2ull * kDn, 64, 64, 1))) return rc;
+    if ((rc = map3(&b2, qn, kDn, H, 2 * B, kDn * 2ull, kDn * 2ull * H, 64, 1, np2))) return rc;
+    if ((rc = run_gemm(c, s2, a2, a2, 1 << 30, 1, b2, part, st, &ks))) return rc;
+    wuk_epilogue_kernel<__nv_bfloat16, true><<<dim3(H, B), 128, 0, st>>>(part, np2, B, H, qc, ql);
+  } else {
+    float* qc = static_cast<float*>(q_cat);
+    const int M = H * (kDn + kDr);
+    f32_gemm_k_kernel<<<dim3((M + 7) / 8, 1), 256, 0, st>>>(static_cast<const float*>(w_q), 0, D,
+                                                           static_cast<const float*>(h), D, 0, M,
+                                                           D, B, part);
+    wq_epilogue_kernel<float><<<dim3(H, B), 96, 0, st>>>(part, 1, B, B, H, positions, theta, qc,
+                                                         nullptr, qn);
+    // q_lat_h[m] = sum_k W_UK[h*128 + k][m] q_nope[b][h][k]
+    f32_gemm_mn_kernel<<<dim3(kDc / 128, H), 128, 0, st>>>(
+        static_cast<const float*>(w_uk), static_cast<size_t>(kDn) * kDc, kDc,
+        static_cast<const float*>(qn), static_cast<size_t>(H) * kDn, kDn, kDc, kDn, B, part);
+    wuk_epilogue_kernel<float, false><<<dim3(H, B), 128, 0, st>>>(part, B, B, H, qc, nullptr);
+  }
+  return last_launch();
+}
+
+int mla_decode_attn(const mla_dims* dims, const void* q_cat, const void* q_lo,
+                    const void* cache_pool, int32_t num_pages, const int32_t* page_table,
+                    int32_t max_pages, const int32_t* seq_lens, float softmax_scale,
+                    int32_t num_splits, void* workspace, size_t workspace_bytes, float* o_lat,
+                    float* lse, mla_stream_t stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (!q_cat || !cache_pool || !page_table || !seq_lens || !o_lat) return MLA_ERR_NULL_ARG;
+  if (!workspace) return MLA_ERR_WORKSPACE;
+  if (num_pages < 1 || max_pages < 1 || num_splits < 0) return MLA_ERR_ARG;
+  if (q_lo) return MLA_ERR_ARG;  // extended-precision query input: not supported yet
+  if (!(softmax_scale >= 0.f) || !std::isfinite(softmax_scale)) return MLA_ERR_ARG;
+  if (!aligned(q_cat, 16) || !aligned(cache_pool, 16) || !aligned(o_lat, 16) ||
+      !aligned(page_table, 4) || !aligned(seq_lens, 4) || (lse && !aligned(lse, 4)))
+    return MLA_ERR_ALIGN;
+  if (!aligned(workspace, 256)) return MLA_ERR_ALIGN;
+  if (static_cast<int64_t>(num_pages) * kPageN > INT32_MAX) return MLA_ERR_ARG;
+  DevCtx* c = nullptr;
+  if ((rc = device_ctx(&c))) return rc;
+  const int parts = resolve_parts(num_splits, c);
+  const Workspace w = layout(dims, parts, c->sms);
+  if (workspace_bytes < w.total) return MLA_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int B = dims->batch, H = dims->n_heads;
+  char* ws = static_cast<char*>(workspace);
+  int32_t* plan = reinterpret_cast<int32_t*>(ws + w.plan);
+  float* part_o = reinterpret_cast<float*>(ws + w.part_o);
+  float* part_lse = reinterpret_cast<float*>(ws + w.part_lse);
+  const float scale =
+      softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(kDn + kDr));
+  attn::plan_kernel<<<1, attn::kPlanThreads, 0, st>>>(seq_lens, B, max_pages, parts,
+                                                      kMinPagesPerPart, plan, c->status);
+  if ((rc = last_launch())) return rc;
+  if (dims->dtype == MLA_BF16) {
+    CUtensorMap tq_lat, tq_rope, tc_lat, tc_rope;
+    const uint64_t rows = static_cast<uint64_t>(num_pages) * kPageN;
+    if ((rc = map3(&tq_lat, q_cat, kRowN, H, B, kRowN * 2ull, kRowN * 2ull * H, 64, 128, 1)))
+      return rc;
+    if ((rc = map3(&tq_rope, q_cat, kRowN, H, B, kRowN * 2ull, kRowN * 2ull * H, 32, 128, 1,
+                   CU_TENSOR_MAP_SWIZZLE_64B)))
+      return rc;
+    if ((rc = map2(&tc_lat, cache_pool, kRowN, rows, kRowN * 2ull, 64, 64,
+                   CU_TENSOR_MAP_SWIZZLE_128B)))
+      return rc;
+    if ((rc = map2(&tc_rope, cache_pool, kRowN, rows, kRowN * 2ull, 32, 64,
+                   CU_TENSOR_MAP_SWIZZLE_64B)))
+      return rc;
+    attn::Params p{};
+    p.batch = B;
+    p.n_heads = H;
+    p.max_pages = max_pages;
+    p.num_pages = num_pages;
+    p.num_parts = parts;
+    p.page_table = page_table;
+    p.seq_lens = seq_lens;
+    p.plan = plan;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.o_lat = o_lat;
+    p.lse = lse;
+    p.part_o = part_o;
+    p.part_lse = part_lse;
+    p.status = c->status;
+    p.wait_ns = kDefaultWaitNs;
+    attn::split_kernel<<<2 * parts, attn::kThreads, attn::kSmemBytes, st>>>(tq_lat, tq_rope,
+                                                                            tc_lat, tc_rope, p);
+  } else {
+    attn::f32_split_kernel<<<dim3(parts, H), 128, 0, st>>>(
+        static_cast<const float*>(q_cat), static_cast<const float*>(cache_pool), page_table,
+        max_pages, num_pages, seq_lens, plan, B, parts, H, scale, o_lat, lse, part_o, part_lse,
+        c->status);
+  }
+  if ((rc = last_launch())) return rc;
+  attn::combine_kernel<<<dim3(H, B), 128, 0, st>>>(plan, B, parts, H, part_o, part_lse, o_lat,
+                                                   lse);
+  return last_launch();
+}
+
+int mla_out_proj(const mla_dims* dims, const float* o_lat, const void* w_uv, const void* w_o,
+                 void* o_heads, void* out, void* workspace, size_t workspace_bytes,
+                 mla_stream_t stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (!o_lat || !w_uv) return MLA_ERR_NULL_ARG;
+  if ((w_o == nullptr) != (out == nullptr)) return MLA_ERR_NULL_ARG;
+  if (!o_heads && !out) return MLA_ERR_NULL_ARG;
+  if (!workspace) return MLA_ERR_WORKSPACE;
+  if (!aligned(o_lat, 16) || !aligned(w_uv, 16) || (w_o && !aligned(w_o, 16)) ||
+      (o_heads && !aligned(o_heads, 16)) || (out && !aligned(out, 16)))
+    return MLA_ERR_ALIGN;
+  if (!aligned(workspace, 256)) return MLA_ERR_ALIGN;
+  DevCtx* c = nullptr;
+  if ((rc = device_ctx(&c))) return rc;
+  const Workspace w = layout(dims, resolve_parts(0, c), c->sms);
+  if (workspace_bytes < w.total) return MLA_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int B = dims->batch, D = dims->d_model, H = dims->n_heads;
+  char* ws = static_cast<char*>(workspace);
+  float* part = reinterpret_cast<float*>(ws + w.partial);
+  void* oh_split = out ? static_cast<void*>(ws + w.oh_split) : nullptr;
+  if (dims->dtype == MLA_BF16) {
+    __nv_bfloat16* os = reinterpret_cast<__nv_bfloat16*>(ws + w.o_split);
+    const size_t n = static_cast<size_t>(B) * H * kDc;
+    split_hi_lo_kernel<<<static_cast<unsigned>(std::min<size_t>((n + 255) / 256, 4096)), 256, 0,
+                         st>>>(o_lat, n, os);
+    if ((rc = last_launch())) return rc;
+    // o_h = W_UV_h [o_lat_hi | o_lat_lo]
+    const GemmShape s1 = shape_wuv(dims);
+    const int np1 = n_pad_for(s1.n_rows);
+    CUtensorMap a, bm;
+    if ((rc = map3(&a, w_uv, kDc, kDv, H, kDc * 2ull, kDc * 2ull * kDv, 64, 128, 1))) return rc;
+    if ((rc = map3(&bm, os, kDc, H, 2 * B, kDc * 2ull, kDc * 2ull * H, 64, 1, np1))) return rc;
+    int ks = 1;
+    if ((rc = run_gemm(c, s1, a, a, 1 << 30, 0, bm, part, st, &ks))) return rc;
+    wuv_epilogue_kernel<__nv_bfloat16, true><<<dim3(H, B), kDv, 0, st>>>(
+        part, ks, np1, B, H, static_cast<__nv_bfloat16*>(o_heads), oh_split);
+    if ((rc = last_launch())) return rc;
+    if (out) {
+      const GemmShape s2 = shape_wo(dims);
+      const int np2 = n_pad_for(s2.n_rows);
+      const uint64_t K = static_cast<uint64_t>(H) * kDv;
+      CUtensorMap a2, b2;
+      if ((rc = map3(&a2, w_o, K, D, 1, K * 2, K * 2 * D, 64, 128, 1))) return rc;
+      if ((rc = map3(&b2, oh_split, K, 1, 2 * B, K * 2, K * 2, 64, 1, np2))) return rc;
+      if ((rc = run_gemm(c, s2, a2, a2, 1 << 30, 0, b2, part, st, &ks))) return rc;
+      wo_epilogue_kernel<__nv_bfloat16, true><<<dim3((D + 255) / 256, B), 256, 0, st>>>(
+          part, ks, np2, B, D, static_cast<__nv_bfloat16*>(out));
+    }
+  } else {
+    f32_gemm_k_kernel<<<dim3(kDv / 8, H), 256, 0, st>>>(
+        static_cast<const float*>(w_uv), static_cast<size_t>(kDv) * kDc, kDc, o_lat,
+        static_cast<size_t>(H) * kDc, kDc, kDv, kDc, B, part);
+    wuv_epilogue_kernel<float, false><<<dim3(H, B), kDv, 0, st>>>(
+        part, 1, B, B, H, static_cast<float*>(o_heads), oh_split);
+    if (out) {
+      const int K = H * kDv;
+      if ((rc = last_launch())) return rc;
+      f32_gemm_k_kernel<<<dim3((D + 7) / 8, 1), 256, 0, st>>>(
+          static_cast<const float*>(w_o), 0, K, static_cast<const float*>(oh_split), K, 0, D, K,
+          B, part);
+      wo_epilogue_kernel<float, false><<<dim3((D + 255) / 256, B), 256, 0, st>>>(
+          part, 1, B, B, D, static_cast<float*>(out));
+    }
+  }
+  return last_launch();
+}
+
+int mla_get_status(mla_stream_t stream) {
+  DevCtx* c = nullptr;
+  int rc = device_ctx(&c);
+  if (rc) return rc;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpy(&v, c->status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  if (cudaMemset(c->status, 0, sizeof(unsigned int)) != cudaSuccess) return MLA_ERR_CUDA;
+  return static_cast<int>(v & 0x7fffffffu);
+}
+
+const char* mla_error_string(int code) {
+  switch (code) {
+    case MLA_OK: return "ok";
+    case MLA_ERR_NULL_ARG: return "a required pointer is NULL";
+    case MLA_ERR_DIMS: return "unsupported shape or dtype";
+    case MLA_ERR_ALIGN: return "misaligned pointer";
+    case MLA_ERR_WORKSPACE: return "workspace missing or too small";
+    case MLA_ERR_ARG: return "invalid argument";
+    case MLA_ERR_CUDA: return "CUDA runtime error";
+    case MLA_ERR_DEVICE: return "device is not sm_100 (B200)";
+    default: break;
+  }
+  if (code > 0) {
+    if (code & MLA_STATUS_TIMEOUT) return "device: bounded wait timed out";
+    if (code & MLA_STATUS_BAD_PAGE) return "device: page id out of range";
+    if (code & MLA_STATUS_BAD_LENGTH) return "device: sequence length out of range";
+    if (code & MLA_STATUS_BAD_POSITION) return "device: append position out of range";
+  }
+  return "unknown code";
+}
+
+const char* mla_version(void) { return "mla_latent_kv_37_b200 0.1 (sm_100a)"; }
+
+}  // extern "C"

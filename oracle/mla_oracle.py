@@ -118,12 +118,17 @@ def query_heads(h, w_q, n_heads: int, d_nope: int, d_rope: int, pos: int,
 def gather_rows(pool, page_table_row, n_rows: int, page_size: int = PAGE) -> np.ndarray:
     """Rows 0..n_rows-1 of one sequence: row j lives in page page_table_row[j // page_size],
     slot j % page_size."""
-    pool = f64(pool)
     pt = np.asarray(page_table_row, dtype=np.int64)
-    out = np.empty((n_rows, pool.shape[-1]), dtype=np.float64)
-    for j in range(n_rows):
-        out[j] = pool[pt[j // page_size], j % page_size]
-    return out
+    n_pages = -(-n_rows // page_size)
+    if n_pages == 0:
+        return np.zeros((0, pool.shape[-1]), dtype=np.float64)
+    if hasattr(pool, "detach"):
+        import torch
+        pages = f64(pool[torch.from_numpy(pt[:n_pages])])
+    else:
+        pages = f64(np.asarray(pool)[pt[:n_pages]])
+    # pages[i][k] is row i * page_size + k
+    return pages.reshape(n_pages * page_size, -1)[:n_rows].copy()
 
 
 # ---------------------------------------------------------------------------------------------
@@ -193,6 +198,26 @@ def decode_attention(q_nope, q_rope, c_kv, k_r, w_uk, w_uv, scale: float | None 
         o_heads[i] = p @ v_h
         o_lat[i] = p @ c_kv
     return {"o_heads": o_heads, "o_lat": o_lat, "lse": lse}
+
+
+def latent_attention(q_lat, q_rope, c_kv, k_r, scale: float | None = None):
+    """Diagnostic for the attention step alone, stated in latent space: scores
+    s_j = scale * (q_lat . c_j + q_rope . k_R,j), p = softmax(s), o_lat = sum_j p_j c_j.
+    The end-to-end reference is decode_attention (no absorption); this form equals it by the
+    associativity the pages state ([LP] "MLA: compress the pair, not the heads") and is
+    pinned against it.  q_lat [H, d_c], q_rope [H, d_R]; returns o_lat [H, d_c], lse [H]."""
+    q_lat, q_rope = f64(q_lat), f64(q_rope)
+    c_kv, k_r = f64(c_kv), f64(k_r)
+    H = q_lat.shape[0]
+    if scale is None:
+        scale = 1.0 / math.sqrt(128 + q_rope.shape[1])
+    if c_kv.shape[0] == 0:
+        return np.zeros((H, c_kv.shape[1])), np.full(H, -np.inf)
+    s = (q_lat @ c_kv.T + q_rope @ k_r.T) * scale          # [H, n]
+    m = s.max(axis=1, keepdims=True)
+    e = np.exp(s - m)
+    tot = e.sum(axis=1, keepdims=True)
+    return (e / tot) @ c_kv, (m + np.log(tot))[:, 0]
 
 
 def output_projection(o_heads, w_o) -> np.ndarray:

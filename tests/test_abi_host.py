@@ -1,0 +1,119 @@
+"""C-ABI checks that need no GPU: the library builds and loads, exports every function that
+include/mla.h declares, and rejects bad arguments on the host before touching CUDA."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mla.h")
+
+
+@pytest.fixture(scope="module")
+def M():
+    from mla_latent_kv_37_b200 import build
+    build.build()
+    import mla_latent_kv_37_b200 as m
+    return m
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mla_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_four_calls():
+    names = _declared()
+    for n in ("mla_cache_append", "mla_absorb_q", "mla_decode_attn", "mla_out_proj"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(M):
+    out = subprocess.run(["nm", "-D", "--defined-only", M.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (mla_\w+)", out))
+    missing = [n for n in _declared() if n not in exported]
+    assert not missing, missing
+    lib = ctypes.CDLL(M.LIB_PATH)
+    for n in _declared():
+        assert getattr(lib, n)
+
+
+def _d(M, **kw):
+    d = M.dims(4, 128, 7168)
+    for k, v in kw.items():
+        setattr(d, k, v)
+    return d
+
+
+def test_layout_constants(M):
+    import torch
+    assert M.mla_cache_row_bytes(M.dims(1)) == 1152
+    # 61 layers of one token: the 70,272 bytes the MLA pages print
+    assert 61 * M.mla_cache_row_bytes(M.dims(1)) == 70272
+    assert M.mla_cache_row_bytes(M.dims(1, 16, 1024, dtype=torch.float32)) == 2304
+    assert M.mla_cache_row_bytes(_d(M, d_c=256)) == 0
+
+
+@pytest.mark.parametrize("field,value", [("d_c", 256), ("d_rope", 32), ("d_nope", 64),
+                                         ("d_v", 64), ("page_size", 32), ("n_heads", 24),
+                                         ("n_heads", 256), ("d_model", 100), ("batch", 0),
+                                         ("dtype", 7), ("rope_theta", 0.0), ("batch", 129)])
+def test_unsupported_dims_rejected(M, field, value):
+    d = _d(M, **{field: value})
+    assert M.mla_workspace_size(d) == 0
+    L = M.lib()
+    fake = ctypes.c_void_p(0x10000)
+    rc = L.mla_decode_attn(ctypes.byref(d), fake, None, fake, 10, fake, 4, fake, 0.0, 0, fake,
+                           1 << 30, fake, None, None)
+    assert rc == -2
+
+
+def test_null_and_alignment_errors(M):
+    d = _d(M)
+    L = M.lib()
+    f = ctypes.c_void_p(0x10000)
+    odd = ctypes.c_void_p(0x10008)  # 8-byte aligned only
+    assert L.mla_decode_attn(None, f, None, f, 10, f, 4, f, 0.0, 0, f, 1 << 30, f, None, None) == -1
+    assert L.mla_decode_attn(ctypes.byref(d), None, None, f, 10, f, 4, f, 0.0, 0, f, 1 << 30, f,
+                             None, None) == -1
+    assert L.mla_decode_attn(ctypes.byref(d), odd, None, f, 10, f, 4, f, 0.0, 0, f, 1 << 30, f,
+                             None, None) == -3
+    assert L.mla_decode_attn(ctypes.byref(d), f, None, f, 10, f, 4, f, 0.0, 0, None, 1 << 30, f,
+                             None, None) == -4
+    assert L.mla_decode_attn(ctypes.byref(d), f, None, f, 0, f, 4, f, 0.0, 0, f, 1 << 30, f, None,
+                             None) == -5
+    assert L.mla_decode_attn(ctypes.byref(d), f, None, f, 10, f, 4, f, -1.0, 0, f, 1 << 30, f,
+                             None, None) == -5
+    assert L.mla_cache_append(ctypes.byref(d), f, f, None, f, f, 4, f, 10, f, 1 << 30, None) == -1
+    assert L.mla_absorb_q(ctypes.byref(d), f, f, f, f, f, None, None, 0, None) == -4
+    assert L.mla_out_proj(ctypes.byref(d), f, f, f, None, None, f, 1 << 30, None) == -1
+    assert L.mla_out_proj(ctypes.byref(d), f, f, None, None, None, f, 1 << 30, None) == -1
+
+
+def test_valid_call_without_gpu_fails_loudly(M):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    d = _d(M)
+    f = ctypes.c_void_p(0x10000)
+    rc = M.lib().mla_decode_attn(ctypes.byref(d), f, None, f, 10, f, 4, f, 0.0, 0, f, 1 << 30, f,
+                                 None, None)
+    assert rc in (-6, -7)
+
+
+def test_workspace_size_is_positive_and_grows_with_splits(M):
+    d = _d(M)
+    a, b = M.mla_workspace_size(d, 8), M.mla_workspace_size(d, 200)
+    assert 0 < a < b
+    assert a % 256 == 0
+
+
+def test_error_strings(M):
+    L = M.lib()
+    for code in (0, -1, -2, -3, -4, -5, -6, -7, 1, 4):
+        assert L.mla_error_string(code)
+    assert b"sm_100a" in L.mla_version()

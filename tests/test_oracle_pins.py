@@ -278,6 +278,22 @@ def test_absorbed_form_equals_reconstructed_form():
                                    rtol=1e-11, atol=1e-12)
 
 
+def test_latent_attention_equals_reconstructed_form():
+    rng = np.random.default_rng(18)
+    H, n = 3, 70
+    w = _tiny_weights(rng, H, 8)
+    w.w_uk /= math.sqrt(512)
+    c, kr = rng.standard_normal((n, 512)), rng.standard_normal((n, 64))
+    qn, qr = rng.standard_normal((H, 128)), rng.standard_normal((H, 64))
+    naive = O.decode_attention(qn, qr, c, kr, w.w_uk, w.w_uv)
+    q_lat = np.stack([w.w_uk[h * 128:(h + 1) * 128].T @ qn[h] for h in range(H)])
+    o_lat, lse = O.latent_attention(q_lat, qr, c, kr)
+    np.testing.assert_allclose(o_lat, naive["o_lat"], rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(lse, naive["lse"], rtol=1e-12)
+    z, zl = O.latent_attention(q_lat, qr, np.zeros((0, 512)), np.zeros((0, 64)))
+    assert np.all(z == 0) and np.all(np.isneginf(zl))
+
+
 def test_incremental_decode_equals_full_causal_recompute():
     """The KV-cache experiment ([MD] "KV Cache"): each decode step with a cache of the earlier
     rows gives the same output as the matching row of full causal attention recomputed over
@@ -372,6 +388,7 @@ def test_gather_rows_follows_page_table_and_ignores_unused_slots():
     assert np.array_equal(O.gather_rows(pool, table, n), rows)
     pool[table[2], 22:] = -5.0  # change every slot past the length
     assert np.array_equal(O.gather_rows(pool, table, n), rows)
+    assert O.gather_rows(pool, table, 0).shape == (0, 576)
 
 
 def test_decode_step_appends_at_position_and_attends_to_itself():
