@@ -168,6 +168,19 @@ const char* mla_error_string(int code);
 /* Library build string (for logs). */
 const char* mla_version(void);
 
+/* Number of kernels this library has launched in this process (all devices, all calls). */
+uint64_t mla_launch_count(void);
+
+/* Profiling hook.  After this call, the i-th bf16 mla_decode_attn call (i < count) records
+ * begin[i] just before and end[i] just after its split-KV kernel on the call's stream, so the
+ * caller can time that kernel alone with cudaEventElapsedTime.  begin/end are host arrays of
+ * cudaEvent_t created by the caller (timing enabled), kept alive until the calls are done.
+ * count = 0 switches recording off.  Returns MLA_OK or MLA_ERR_ARG. */
+int mla_set_profile_events(void* const* begin, void* const* end, int32_t count);
+
+/* How many event pairs have been recorded since the last mla_set_profile_events. */
+int32_t mla_profile_events_used(void);
+
 #ifdef __cplusplus
 }
 #endif

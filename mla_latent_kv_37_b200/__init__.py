@@ -66,6 +66,10 @@ _SIGS = {
     "mla_get_status": (ctypes.c_int, [_P]),
     "mla_error_string": (ctypes.c_char_p, [ctypes.c_int]),
     "mla_version": (ctypes.c_char_p, []),
+    "mla_launch_count": (ctypes.c_uint64, []),
+    "mla_set_profile_events": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p),
+                                              ctypes.POINTER(ctypes.c_void_p), _I]),
+    "mla_profile_events_used": (ctypes.c_int32, []),
 }
 
 
@@ -213,3 +217,28 @@ def mla_get_status(stream=None) -> int:
 
 def version() -> str:
     return lib().mla_version().decode()
+
+
+def mla_launch_count() -> int:
+    return int(lib().mla_launch_count())
+
+
+_prof_keep = None
+
+
+def mla_set_profile_events(begin, end) -> None:
+    """begin/end: equal-length lists of torch.cuda.Event(enable_timing=True)."""
+    global _prof_keep
+    n = len(begin)
+    assert len(end) == n
+    for e in list(begin) + list(end):
+        if e.cuda_event == 0:  # events are created lazily by torch
+            e.record()
+    arr_b = (ctypes.c_void_p * max(n, 1))(*[e.cuda_event for e in begin])
+    arr_e = (ctypes.c_void_p * max(n, 1))(*[e.cuda_event for e in end])
+    _prof_keep = (arr_b, arr_e, begin, end)
+    _check(lib().mla_set_profile_events(arr_b, arr_e, n), "mla_set_profile_events")
+
+
+def mla_profile_events_used() -> int:
+    return int(lib().mla_profile_events_used())

@@ -8,6 +8,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "attn_f32.cuh"
@@ -60,6 +61,12 @@ struct DevCtx {
 };
 DevCtx g_dev[64];
 std::mutex g_mu;
+std::atomic<unsigned long long> g_launches{0};
+// profiling hook: events recorded around the split-KV kernel of successive decode calls
+cudaEvent_t* g_prof_begin = nullptr;
+cudaEvent_t* g_prof_end = nullptr;
+int g_prof_count = 0;
+int g_prof_next = 0;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 int device_ctx(DevCtx** out) {
@@ -240,7 +247,10 @@ int map2(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t s1
 // ------------------------------------------------------------------------------------------
 // launches
 // ------------------------------------------------------------------------------------------
-int last_launch() { return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
+int last_launch(int kernels = 1) {
+  g_launches.fetch_add(static_cast<unsigned long long>(kernels), std::memory_order_relaxed);
+  return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
 
 int gemm_stages(int n_pad) {
   const uint32_t sb = gemm_stage_bytes(n_pad);
@@ -347,9 +357,11 @@ int mla_cache_append(const mla_dims* dims, const void* h, const void* w_dkv, con
     f32_gemm_k_kernel<<<dim3(kDc / 8, 1), 256, 0, st>>>(static_cast<const float*>(w_dkv), 0, D,
                                                        static_cast<const float*>(h), D, 0, kDc, D,
                                                        B, part);
+    if ((rc = last_launch())) return rc;
     f32_gemm_k_kernel<<<dim3(kDr / 8, 1), 256, 0, st>>>(static_cast<const float*>(w_kr), 0, D,
                                                        static_cast<const float*>(h), D, 0, kDr, D,
                                                        B, part + static_cast<size_t>(kDc) * B);
+    if ((rc = last_launch())) return rc;
     append_epilogue_kernel<float><<<eg, 96, 0, st>>>(
         part, 1, B, nullptr, positions, page_table, max_pages, static_cast<float*>(cache_pool),
         num_pages, dims->rope_theta, c->status);
@@ -408,12 +420,15 @@ int mla_absorb_q(const mla_dims* dims, const void* h, const void* w_q, const voi
     f32_gemm_k_kernel<<<dim3((M + 7) / 8, 1), 256, 0, st>>>(static_cast<const float*>(w_q), 0, D,
                                                            static_cast<const float*>(h), D, 0, M,
                                                            D, B, part);
+    if ((rc = last_launch())) return rc;
     wq_epilogue_kernel<float><<<dim3(H, B), 96, 0, st>>>(part, 1, B, B, H, positions, theta, qc,
                                                          nullptr, qn);
+    if ((rc = last_launch())) return rc;
     // q_lat_h[m] = sum_k W_UK[h*128 + k][m] q_nope[b][h][k]
     f32_gemm_mn_kernel<<<dim3(kDc / 128, H), 128, 0, st>>>(
         static_cast<const float*>(w_uk), static_cast<size_t>(kDn) * kDc, kDc,
         static_cast<const float*>(qn), static_cast<size_t>(H) * kDn, kDn, kDc, kDn, B, part);
+    if ((rc = last_launch())) return rc;
     wuk_epilogue_kernel<float, false><<<dim3(H, B), 128, 0, st>>>(part, B, B, H, qc, nullptr);
   }
   return last_launch();
@@ -482,8 +497,15 @@ int mla_decode_attn(const mla_dims* dims, const void* q_cat, const void* q_lo,
     p.part_lse = part_lse;
     p.status = c->status;
     p.wait_ns = kDefaultWaitNs;
+    const bool prof = g_prof_next < g_prof_count;
+    if (prof && cudaEventRecord(g_prof_begin[g_prof_next], st) != cudaSuccess) return MLA_ERR_CUDA;
     attn::split_kernel<<<2 * parts, attn::kThreads, attn::kSmemBytes, st>>>(tq_lat, tq_rope,
                                                                             tc_lat, tc_rope, p);
+    if (prof) {
+      if ((rc = last_launch())) return rc;
+      if (cudaEventRecord(g_prof_end[g_prof_next++], st) != cudaSuccess) return MLA_ERR_CUDA;
+      g_launches.fetch_sub(1, std::memory_order_relaxed);  // counted again below
+    }
   } else {
     attn::f32_split_kernel<<<dim3(parts, H), 128, 0, st>>>(
         static_cast<const float*>(q_cat), static_cast<const float*>(cache_pool), page_table,
@@ -545,24 +567,28 @@ int mla_out_proj(const mla_dims* dims, const float* o_lat, const void* w_uv, con
       if ((rc = run_gemm(c, s2, a2, a2, 1 << 30, 0, b2, part, st, &ks))) return rc;
       wo_epilogue_kernel<__nv_bfloat16, true><<<dim3((D + 255) / 256, B), 256, 0, st>>>(
           part, ks, np2, B, D, static_cast<__nv_bfloat16*>(out));
+      if ((rc = last_launch())) return rc;
     }
   } else {
     f32_gemm_k_kernel<<<dim3(kDv / 8, H), 256, 0, st>>>(
         static_cast<const float*>(w_uv), static_cast<size_t>(kDv) * kDc, kDc, o_lat,
         static_cast<size_t>(H) * kDc, kDc, kDv, kDc, B, part);
+    if ((rc = last_launch())) return rc;
     wuv_epilogue_kernel<float, false><<<dim3(H, B), kDv, 0, st>>>(
         part, 1, B, B, H, static_cast<float*>(o_heads), oh_split);
+    if ((rc = last_launch())) return rc;
     if (out) {
       const int K = H * kDv;
-      if ((rc = last_launch())) return rc;
       f32_gemm_k_kernel<<<dim3((D + 7) / 8, 1), 256, 0, st>>>(
           static_cast<const float*>(w_o), 0, K, static_cast<const float*>(oh_split), K, 0, D, K,
           B, part);
+      if ((rc = last_launch())) return rc;
       wo_epilogue_kernel<float, false><<<dim3((D + 255) / 256, B), 256, 0, st>>>(
           part, 1, B, B, D, static_cast<float*>(out));
+      if ((rc = last_launch())) return rc;
     }
   }
-  return last_launch();
+  return MLA_OK;
 }
 
 int mla_get_status(mla_stream_t stream) {
@@ -600,5 +626,19 @@ const char* mla_error_string(int code) {
 }
 
 const char* mla_version(void) { return "mla_latent_kv_37_b200 0.1 (sm_100a)"; }
+
+uint64_t mla_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int mla_set_profile_events(void* const* begin, void* const* end, int32_t count) {
+  if (count < 0 || (count > 0 && (!begin || !end))) return MLA_ERR_ARG;
+  std::lock_guard<std::mutex> lock(g_mu);
+  g_prof_begin = reinterpret_cast<cudaEvent_t*>(const_cast<void**>(begin));
+  g_prof_end = reinterpret_cast<cudaEvent_t*>(const_cast<void**>(end));
+  g_prof_count = count;
+  g_prof_next = 0;
+  return MLA_OK;
+}
+
+int32_t mla_profile_events_used(void) { return g_prof_next; }
 
 }  // extern "C"
