@@ -6,19 +6,27 @@
 //     s_j = scale * <q, c_j>,  p = softmax_j(s),  o_lat = sum_j p_j c_KV,j   (512 wide),
 // every cached row j < len_b being visible to the newest token.
 //
-// Design (B200): all H = 128 heads of a sequence share every cache row, so the per-page work
+// Design (B200).  All H = 128 heads of a sequence share every cache row, so the per-page work
 // is two dense contractions, S = Q C^T ([128 x 576] x [576 x 64]) and O += P C_lat
-// ([128 x 64] x [64 x 512]).  O (128 x 512 fp32) alone fills a whole SM's tensor memory, so
-// each work unit runs on a CLUSTER OF TWO CTAs that split the 576 columns of every row:
-//   CTA r loads latent columns [256r, 256r+256) and RoPE columns [512+32r, 512+32r+32) of
-//   q_cat and of each cache page (TMA, 128B/64B swizzle), computes the partial scores of its
-//   288 columns, sends them to its peer through distributed shared memory (st.async with
-//   byte-counted mbarrier completion) and adds the peer's partial -- both CTAs then hold the
-//   same full S and run the same online softmax -- and accumulates its own 256 columns of O.
-// Per CTA the tensor memory holds O (256 cols), S double-buffered (2 x 64) and P as bf16
-// (2 x 32, the A operand of the PV product read straight from TMEM); shared memory holds the
-// Q half (72 KiB), a 3-stage page ring (3 x 36 KiB) and the 32 KiB score-exchange buffer.
-// HBM traffic is each cache byte once.
+// ([128 x 64] x [64 x 512]).  O (128 x 512 fp32) alone would fill a whole SM's tensor memory,
+// so each work unit runs on a CLUSTER OF TWO CTAs that split the 576 columns of every row:
+// CTA r owns latent columns [256r, 256r+256) and RoPE columns [512+32r, 512+32r+32).
+//   * TMEM (512 columns): O half 256 | query latent half 128 (A operand of QK) | two S
+//     buffers of 64.  P (bf16) is written over the S buffer it came from (A operand of PV).
+//     The 32 RoPE columns of the query half sit in shared memory (A operand, 64B swizzle).
+//   * Pages arrive by TMA (128B/64B swizzle) into a 4-stage ring; each byte leaves HBM once.
+//   * S_r = Q_r C_r^T is a partial score; the pair exchanges partials.  Distributed shared
+//     memory moves ~16 B/clk per SM, so a partial travels as 16-bit fixed point relative to
+//     its row's largest magnitude (error <= 2^-16 of it, ~1e-4 in the softmax logit), staged
+//     in shared memory and sent with ONE bulk copy (cp.async.bulk, completion counted in bytes
+//     on the peer's mbarrier).
+//   * Two warpgroups share the per-page softmax work: the "send" warpgroup drains S_t,
+//     quantises and stages it; the "softmax" warpgroup drains S_t again, adds the peer's
+//     decoded partial, runs the online softmax and writes P_t.  With S double-buffered, QK of
+//     page t+1 and the exchange of page t+1 run while page t is being softmaxed.
+//   * Each CTA normalises its own half of O with its own running sum (its copy of the scores
+//     differs from the peer's only by the 16-bit rounding of the received half), so the halves
+//     need no further agreement.
 //
 // The concatenated page list of all sequences is cut into `num_parts` contiguous ranges of
 // (nearly) equal length, one per cluster; a range may end inside a sequence and may span
@@ -26,34 +34,38 @@
 // split over several ranges gets normalised partials that the combine kernel merges with
 // log-sum-exp weights.
 //
-// Roles in each CTA (192 threads): warps 0-3 softmax (thread i owns head row i = TMEM lane i),
-// warp 4 TMA producer, warp 5 MMA issuer.  Online softmax keeps a per-row reference maximum
-// and rescales O only when the running maximum grows by more than 2^8.
+// Roles (384 threads): warps 0-3 softmax + epilogue (thread i owns head row i = TMEM lane i),
+// warps 4-7 send, warp 8 TMA producer, warp 9 MMA issuer, warp 10 bulk-copy sender, warp 11
+// cluster-scope signals.  The online softmax keeps a per-row reference maximum and rescales O
+// only when the running maximum grows by more than 2^8.
 #pragma once
 #include "ptx_sm100.cuh"
 
 namespace mla {
 namespace attn {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 384;
 constexpr int kPage = 64;
 constexpr int kRow = 576;
-constexpr int kStages = 3;
-constexpr uint32_t kQLatBox = 128 * 128;                  // 128 rows x 64 bf16
-constexpr uint32_t kQBytes = 4 * kQLatBox + 128 * 64;     // + rope box 128 rows x 32 bf16
+constexpr int kStages = 4;
 constexpr uint32_t kCLatBox = 64 * 128;                   // 64 rows x 64 bf16
 constexpr uint32_t kStageBytes = 4 * kCLatBox + 64 * 64;  // + rope box 64 rows x 32 bf16
-constexpr uint32_t kXBytes = 128 * 64 * 4;                // fp32 partial scores
-constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffStage = kQBytes;
-constexpr uint32_t kOffX = kOffStage + kStages * kStageBytes;
-constexpr uint32_t kOffBar = kOffX + kXBytes;
+constexpr uint32_t kXPayload = 128 * 128;                 // 128 rows x 64 x 16-bit
+constexpr uint32_t kXBytes = kXPayload + 128 * 4;         // + one fp32 step per row
+constexpr uint32_t kQRopeBytes = 128 * 64;                // 128 rows x 32 bf16
+constexpr uint32_t kOffStage = 0;
+constexpr uint32_t kOffSend = kOffStage + kStages * kStageBytes;
+constexpr uint32_t kOffRecv = kOffSend + 2 * kXBytes;
+constexpr uint32_t kOffQRope = kOffRecv + 2 * kXBytes;
+constexpr uint32_t kOffBar = kOffQRope + kQRopeBytes;
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // barriers + alignment slack
 // TMEM columns
-constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemP = 384, kTmemCols = 512;
+constexpr uint32_t kTmemO = 0, kTmemQ = 256, kTmemS = 384, kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 static_assert(kSmemBytes <= 232448, "shared memory budget");
+static_assert(kTmemS + 2 * 64 == kTmemCols, "tensor memory budget");
+static_assert(kXBytes % 16 == 0 && kOffQRope % 1024 == 0, "alignment");
 
 struct Params {
   int batch;
@@ -61,6 +73,7 @@ struct Params {
   int max_pages;
   int num_pages;
   int num_parts;  // clusters launched
+  const __nv_bfloat16* q_cat;  // [B][H][576]
   const int32_t* page_table;
   const int32_t* seq_lens;
   const int32_t* plan;
@@ -205,23 +218,6 @@ __global__ void __launch_bounds__(kPlanThreads)
   }
 }
 
-// ------------------------------------------------------------------------------------------
-// The split kernel
-// ------------------------------------------------------------------------------------------
-struct Bars {
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
-  uint64_t q_full, q_empty;
-  uint64_t s_full[2], s_free[2];
-  uint64_t p_full[2], pv_done[2];
-  uint64_t x_full, x_free;
-  uint64_t o_free;
-  uint64_t drain;
-  uint32_t tmem_base;
-  int abort_flag;
-};
-static_assert(sizeof(Bars) <= 256, "barrier block");
-
 // Iterates the segments (one per sequence touched) of a part.
 struct SegIter {
   const int32_t* pages;
@@ -245,15 +241,64 @@ struct SegIter {
   }
 };
 
-__device__ __forceinline__ uint32_t xbuf_off(int row, int chunk) {
-  return static_cast<uint32_t>(row) * 256u + static_cast<uint32_t>((chunk ^ (row & 15)) * 16);
+// Exchange buffer row layout: 8 chunks of 16 B, XOR-swizzled so that 8 consecutive rows hit
+// 8 different bank groups.
+__device__ __forceinline__ uint32_t xrow_off(int row, int chunk) {
+  return static_cast<uint32_t>(row) * 128u + static_cast<uint32_t>((chunk ^ (row & 7)) * 16);
 }
 
+// 16-bit fixed point (offset binary: u = q + 32768 for q in [-32767, 32767]) without the
+// quarter-rate int<->float conversion instructions.  Encoding: fma(x, 1/step, 1.5*2^23 + 32768)
+// rounds to nearest even and leaves u in the low 16 mantissa bits.  Decoding: the bits
+// 0x4B000000 | u are the float 2^23 + u exactly.
+constexpr float kEncBias = 12615680.0f;  // 1.5 * 2^23 + 32768
+constexpr float kDecBias = 8421376.0f;   // 2^23 + 32768
+constexpr uint32_t kDecBits = 0x4B000000u;
+
+__device__ __forceinline__ uint32_t enc_u16x2(float a, float b, float inv_step) {
+  const uint32_t ua = __float_as_uint(fmaf(a, inv_step, kEncBias));
+  const uint32_t ub = __float_as_uint(fmaf(b, inv_step, kEncBias));
+  return __byte_perm(ua, ub, 0x5410);  // low halves: a -> bits 0-15, b -> bits 16-31
+}
+__device__ __forceinline__ float dec_lo(uint32_t v) {
+  return __uint_as_float(__byte_perm(v, kDecBits, 0x7610)) - kDecBias;
+}
+__device__ __forceinline__ float dec_hi(uint32_t v) {
+  return __uint_as_float(__byte_perm(v, kDecBits, 0x7632)) - kDecBias;
+}
+
+
+// ------------------------------------------------------------------------------------------
+// The split kernel
+// ------------------------------------------------------------------------------------------
+// Every mbarrier below completes one phase per use and is waited phase by phase, never more
+// than one phase behind its current state (buffers that could run two pages ahead of their
+// waiter have one barrier per buffer), so parity waits cannot alias.
+struct Bars {
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t q_full;        // TMA: the segment's query RoPE half landed in shared memory
+  uint64_t q_empty;       // MMA: the segment's last QK finished (commit)
+  uint64_t q_ready;       // softmax WG: the segment's query latent half is in TMEM (128)
+  uint64_t s_full[2];     // MMA: S buffer i written (commit)
+  uint64_t staged[2];     // send WG: S drained, partial staged in send[i] (128)
+  uint64_t p_full[2];     // softmax WG: P written over S buffer i (128)
+  uint64_t pv_done;       // MMA: PV finished (commit, once per page)
+  uint64_t consumed[2];   // softmax WG: recv[i] read (128)
+  uint64_t x_full[2];     // the peer's partial landed in recv[i] (bulk-copy bytes)
+  uint64_t peer_done[2];  // the peer consumed our partial from its recv[i] (1 remote arrival)
+  uint64_t o_free;        // softmax WG: the epilogue drained O (128)
+  uint64_t seg_done;      // MMA: every PV of the segment finished (commit, once per segment)
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+static_assert(sizeof(Bars) <= 256, "barrier block");
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    split_kernel(const __grid_constant__ CUtensorMap tm_q_lat,
-                 const __grid_constant__ CUtensorMap tm_q_rope,
-                 const __grid_constant__ CUtensorMap tm_c_lat,
-                 const __grid_constant__ CUtensorMap tm_c_rope, const Params p) {
+    split_kernel(const __grid_constant__ CUtensorMap tm_c_lat,
+                 const __grid_constant__ CUtensorMap tm_c_rope,
+                 const __grid_constant__ CUtensorMap tm_q_rope, const Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -271,21 +316,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     mbar_init(&bars->q_full, 1);
     mbar_init(&bars->q_empty, 1);
+    mbar_init(&bars->q_ready, 128);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->s_full[i], 1);
-      mbar_init(&bars->s_free[i], 128);
+      mbar_init(&bars->staged[i], 128);
       mbar_init(&bars->p_full[i], 128);
-      mbar_init(&bars->pv_done[i], 1);
+      mbar_init(&bars->consumed[i], 128);
+      mbar_init(&bars->x_full[i], 1);
+      mbar_init(&bars->peer_done[i], 1);
     }
-    mbar_init(&bars->x_full, 1);
-    mbar_init(&bars->x_free, 128);
+    mbar_init(&bars->pv_done, 1);
     mbar_init(&bars->o_free, 128);
+    mbar_init(&bars->seg_done, 1);
     mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
     fence_mbar_init_cluster();
-    mbar_arrive_expect_tx(&bars->x_full, kXBytes);  // arm for the first tile
+    mbar_arrive_expect_tx(&bars->x_full[0], kXBytes);  // armed for pages 0 and 1
+    mbar_arrive_expect_tx(&bars->x_full[1], kXBytes);
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(&bars->tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -302,32 +351,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int g_begin = active ? plan.part_start()[part] : 0;
   const int g_end = active ? plan.part_start()[part + 1] : 0;
   const int b_begin = active ? plan.part_seq()[part] : p.batch;
-
-  uint8_t* sQ = smem + kOffQ;
   uint8_t* sStage = smem + kOffStage;
-  uint8_t* sX = smem + kOffX;
+  uint8_t* sQRope = smem + kOffQRope;
+  const uint32_t send_base = smem_u32(smem + kOffSend);
+  const uint32_t recv_base = smem_u32(smem + kOffRecv);
 
-  if (warp == 4) {
-    // =================== TMA producer ===================
+  if (warp == 8) {
+    // =================== TMA producer: page ring + query RoPE half ===================
     SegIter it{plan.seq_pages(), plan.seq_prefix(), p.batch, g_begin, g_end, b_begin};
-    int seq, p0, p1, t = 0, sg = 0, issued_stage = 0;
+    int seq, p0, p1, t = 0, sg = 0, issued = 0;
     bool ok = true;
     const uint64_t pol_stream = l2_policy_evict_first();
     if (lane == 0) {
-      tma_prefetch_desc(&tm_q_lat);
-      tma_prefetch_desc(&tm_q_rope);
       tma_prefetch_desc(&tm_c_lat);
       tma_prefetch_desc(&tm_c_rope);
+      tma_prefetch_desc(&tm_q_rope);
     }
     while (ok && it.next(seq, p0, p1)) {
       if (lane == 0) {
         if (sg > 0) ok = mbar_wait(&bars->q_empty, (sg - 1) & 1, wc);
         if (ok) {
-          mbar_arrive_expect_tx(&bars->q_full, kQBytes);
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            tma_load_3d(sQ + i * kQLatBox, &tm_q_lat, &bars->q_full, 256 * rank + 64 * i, 0, seq);
-          tma_load_3d(sQ + 4 * kQLatBox, &tm_q_rope, &bars->q_full, 512 + 32 * rank, 0, seq);
+          mbar_arrive_expect_tx(&bars->q_full, kQRopeBytes);
+          tma_load_3d(sQRope, &tm_q_rope, &bars->q_full, 512 + 32 * rank, 0, seq);
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -354,7 +399,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                  256 * rank + 64 * i, y, pol_stream);
               tma_load_2d_hint(dst + 4 * kCLatBox, &tm_c_rope, &bars->full[s], 512 + 32 * rank,
                                y, pol_stream);
-              issued_stage = t + 1;
+              issued = t + 1;
             }
           }
           ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -366,138 +411,250 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (lane == 0 && bars->abort_flag) {
       volatile int never = 0;
       WaitCtx drain{&never, p.status, p.wait_ns};
-      for (int i = max(0, issued_stage - kStages); i < issued_stage; ++i)
+      for (int i = max(0, issued - kStages); i < issued; ++i)
         mbar_wait(&bars->full[i % kStages], (i / kStages) & 1, drain);
       if (sg > 0) mbar_wait(&bars->q_full, (sg - 1) & 1, drain);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // =================== MMA issuer ===================
     if (lane == 0) {
       const uint32_t idesc_qk = idesc_bf16(128, 64, 0, 0);
       const uint32_t idesc_pv = idesc_bf16(128, 256, 0, 1);
-      const uint32_t q_base = smem_u32(sQ);
+      const uint32_t qrope = smem_u32(sQRope);
       SegIter it{plan.seq_pages(), plan.seq_prefix(), p.batch, g_begin, g_end, b_begin};
       int seq, p0, p1, t = 0, sg = 0;
       bool ok = true;
+      // S_tt = Q_r C_r^T into S buffer tt & 1: latent half A from TMEM, RoPE half A from smem
+      auto issue_qk = [&](int tt, bool last_of_seg) -> bool {
+        const int s = tt % kStages;
+        if (!mbar_wait(&bars->full[s], (tt / kStages) & 1, wc)) return false;
+        tc_fence_after();
+        const uint32_t st = smem_u32(sStage + s * kStageBytes);
+        const uint32_t d = tmem + kTmemS + (tt & 1) * 64;
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          mma_ts(d, tmem + kTmemQ + 8 * j,
+                 smem_desc(st + (j >> 2) * kCLatBox + (j & 3) * 32, 16, 1024, kSwizzle128B),
+                 idesc_qk, j > 0 ? 1u : 0u);
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+          mma_ss(d, smem_desc(qrope + j * 32, 16, 512, kSwizzle64B),
+                 smem_desc(st + 4 * kCLatBox + j * 32, 16, 512, kSwizzle64B), idesc_qk, 1u);
+        mma_commit(&bars->s_full[tt & 1]);
+        if (last_of_seg) mma_commit(&bars->q_empty);
+        return true;
+      };
+      // O += P_tt C_lat: A = P (bf16, over S buffer tt & 1), B = the page's latent half
       auto issue_pv = [&](int tt, bool first_of_seg) -> bool {
         if (first_of_seg && sg > 0 && !mbar_wait(&bars->o_free, (sg - 1) & 1, wc)) return false;
         if (!mbar_wait(&bars->p_full[tt & 1], (tt >> 1) & 1, wc)) return false;
         tc_fence_after();
         const uint32_t st = smem_u32(sStage + (tt % kStages) * kStageBytes);
-        const uint32_t a_tmem = tmem + kTmemP + (tt & 1) * 32;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t bdesc = smem_desc(st + kk * 2048, 8192, 1024, kSwizzle128B);
-          mma_ts(tmem + kTmemO, a_tmem + kk * 8, bdesc, idesc_pv,
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ts(tmem + kTmemO, tmem + kTmemS + (tt & 1) * 64 + kk * 8,
+                 smem_desc(st + kk * 2048, 8192, 1024, kSwizzle128B), idesc_pv,
                  (first_of_seg && kk == 0) ? 0u : 1u);
-        }
-        mma_commit(&bars->pv_done[tt & 1]);
+        mma_commit(&bars->pv_done);
         mma_commit(&bars->empty[tt % kStages]);
         return true;
       };
       while (ok && it.next(seq, p0, p1)) {
-        const int n_tiles = p1 - p0;
-        ok = mbar_wait(&bars->q_full, sg & 1, wc);
-        for (int i = 0; ok && i < n_tiles; ++i, ++t) {
-          const int s = t % kStages;
-          const int sb = t & 1;
-          if (!mbar_wait(&bars->full[s], (t / kStages) & 1, wc)) { ok = false; break; }
-          if (t >= 2 && !mbar_wait(&bars->s_free[sb], ((t >> 1) - 1) & 1, wc)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t st = smem_u32(sStage + s * kStageBytes);
-          const uint32_t d = tmem + kTmemS + sb * 64;
-          int n_mma = 0;
-#pragma unroll
-          for (int box = 0; box < 4; ++box)
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk, ++n_mma)
-              mma_ss(d, smem_desc(q_base + box * kQLatBox + kk * 32, 16, 1024, kSwizzle128B),
-                     smem_desc(st + box * kCLatBox + kk * 32, 16, 1024, kSwizzle128B), idesc_qk,
-                     n_mma > 0 ? 1u : 0u);
-#pragma unroll
-          for (int kk = 0; kk < 2; ++kk)
-            mma_ss(d, smem_desc(q_base + 4 * kQLatBox + kk * 32, 16, 512, kSwizzle64B),
-                   smem_desc(st + 4 * kCLatBox + kk * 32, 16, 512, kSwizzle64B), idesc_qk, 1u);
-          mma_commit(&bars->s_full[sb]);
-          if (i == n_tiles - 1) mma_commit(&bars->q_empty);
-          if (i > 0 && !issue_pv(t - 1, i == 1)) { ok = false; break; }
+        const int n = p1 - p0, t0 = t;
+        ok = mbar_wait(&bars->q_ready, sg & 1, wc) && mbar_wait(&bars->q_full, sg & 1, wc);
+        if (ok) ok = issue_qk(t0, n == 1);
+        if (ok && n > 1) ok = issue_qk(t0 + 1, n == 2);
+        for (int i = 0; ok && i < n; ++i) {
+          const int tt = t0 + i;
+          if (!(ok = issue_pv(tt, i == 0))) break;
+          if (i == n - 1) mma_commit(&bars->seg_done);
+          // PV_tt done: O is current and S buffer tt & 1 (holding P_tt) is free
+          if (!(ok = mbar_wait(&bars->pv_done, tt & 1, wc))) break;
+          if (i + 2 < n) ok = issue_qk(tt + 2, i + 3 == n);
         }
-        if (ok && !issue_pv(t - 1, n_tiles == 1)) ok = false;
+        t += n;
         ++sg;
       }
-      // no MMA may be in flight when TMEM is released
-      if (bars->abort_flag) {
+      if (bars->abort_flag) {  // no MMA may be in flight when TMEM is released
         mma_commit(&bars->drain);
         volatile int never = 0;
         WaitCtx drain{&never, p.status, p.wait_ns};
         mbar_wait(&bars->drain, 0, drain);
       }
     }
-  } else {
-    // =================== softmax / correction / epilogue (warps 0-3) ===================
-    const int row = threadIdx.x;  // head row = TMEM lane
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t x_base = smem_u32(sX);
-    const uint32_t peer_x_base = mapa_shared(smem_u32(sX), peer);
-    const uint32_t peer_xfull = mapa_shared(smem_u32(&bars->x_full), peer);
-    const uint32_t peer_xfree = mapa_shared(smem_u32(&bars->x_free), peer);
+  } else if (warp == 10 || warp == 11) {
+    // =================== exchange: bulk copies out (10), cluster-scope signals (11) ===========
+    if (lane == 0) {
+      const uint32_t peer_recv = mapa_shared(recv_base, peer);
+      const uint32_t peer_xfull[2] = {mapa_shared(smem_u32(&bars->x_full[0]), peer),
+                                      mapa_shared(smem_u32(&bars->x_full[1]), peer)};
+      const uint32_t peer_done_r[2] = {mapa_shared(smem_u32(&bars->peer_done[0]), peer),
+                                       mapa_shared(smem_u32(&bars->peer_done[1]), peer)};
+      SegIter it{plan.seq_pages(), plan.seq_prefix(), p.batch, g_begin, g_end, b_begin};
+      int seq, p0, p1, t = 0;
+      bool ok = true;
+      while (ok && it.next(seq, p0, p1)) {
+        const int n = p1 - p0;
+        for (int tt = t; ok && tt < t + n; ++tt) {
+          const int buf = tt & 1;
+          if (warp == 10) {
+            // the page's partial is staged in send[buf]: ship it
+            if (!(ok = mbar_wait(&bars->staged[buf], (tt >> 1) & 1, wc))) break;
+            bulk_copy_s2cluster(peer_recv + buf * kXBytes, send_base + buf * kXBytes, kXBytes,
+                                peer_xfull[buf]);
+          } else {
+            // every softmax row has read recv[buf]: re-arm it for page tt + 2, tell the peer
+            if (!(ok = mbar_wait(&bars->consumed[buf], (tt >> 1) & 1, wc))) break;
+            mbar_arrive_expect_tx(&bars->x_full[buf], kXBytes);
+            mbar_arrive_remote(peer_done_r[buf]);
+          }
+        }
+        t += n;
+      }
+    }
+  } else if (warp >= 4) {
+    // =================== send warpgroup (warps 4-7) ===================
+    const int row = threadIdx.x - 128;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     SegIter it{plan.seq_pages(), plan.seq_prefix(), p.batch, g_begin, g_end, b_begin};
-    int seq, p0, p1, t = 0, sg = 0;
+    int seq, p0, p1, t = 0;
     bool ok = true;
-    const float NEG_INF = -__int_as_float(0x7f800000);
     while (ok && it.next(seq, p0, p1)) {
-      const int n_tiles = p1 - p0;
+      const int n = p1 - p0;
       const int len = min(p.seq_lens[seq], p.max_pages * kPage);
-      float m_ref = NEG_INF, l_sum = 0.f;
-      for (int i = 0; ok && i < n_tiles; ++i, ++t) {
-        const int sb = t & 1;
-        if (!warp_wait(&bars->s_full[sb], (t >> 1) & 1, wc)) { ok = false; break; }
+      for (int i = 0; i < n; ++i) {
+        const int tt = t + i, buf = tt & 1;
+        if (!(ok = warp_wait(&bars->s_full[buf], (tt >> 1) & 1, wc))) break;
         tc_fence_after();
         float s[64];
         {
           uint32_t r[32];
-          tmem_ld32(tmem + kTmemS + sb * 64 + lane_off, r);
+          tmem_ld32(tmem + kTmemS + buf * 64 + lane_off, r);
           tmem_wait_ld();
 #pragma unroll
           for (int k = 0; k < 32; ++k) s[k] = __uint_as_float(r[k]);
-          tmem_ld32(tmem + kTmemS + sb * 64 + 32 + lane_off, r);
+          tmem_ld32(tmem + kTmemS + buf * 64 + 32 + lane_off, r);
           tmem_wait_ld();
 #pragma unroll
           for (int k = 0; k < 32; ++k) s[32 + k] = __uint_as_float(r[k]);
         }
         tc_fence_before();
-        mbar_arrive(&bars->s_free[sb]);
-        // ---- exchange partial scores with the peer CTA ----
-        if (t >= 1 && !warp_wait<true>(&bars->x_free, (t - 1) & 1, wc)) { ok = false; break; }
-#pragma unroll
-        for (int c = 0; c < 16; ++c)
-          st_async_v4(peer_x_base + xbuf_off(row, c), s[4 * c], s[4 * c + 1], s[4 * c + 2],
-                      s[4 * c + 3], peer_xfull);
-        if (!warp_wait<true>(&bars->x_full, t & 1, wc)) { ok = false; break; }
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          float4 v;
-          asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                       : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                       : "r"(x_base + xbuf_off(row, c)));
-          s[4 * c] += v.x;
-          s[4 * c + 1] += v.y;
-          s[4 * c + 2] += v.z;
-          s[4 * c + 3] += v.w;
-        }
-        mbar_arrive_remote(peer_xfree);
-        if (row == 0) mbar_arrive_expect_tx(&bars->x_full, kXBytes);
-        // ---- online softmax (identical in both CTAs) ----
         const int valid = min(kPage, len - (p0 + i) * kPage);
+        if (valid < kPage) {
+#pragma unroll
+          for (int k = 0; k < 64; ++k) s[k] = k < valid ? s[k] : 0.f;  // never sent
+        }
+        float mabs = 0.f;
+#pragma unroll
+        for (int k = 0; k < 64; ++k) mabs = fmaxf(mabs, fabsf(s[k]));
+        const float inv = mabs > 0.f ? 32767.f / mabs : 0.f;
+        if (tt >= 2 && !(ok = warp_wait<true>(&bars->peer_done[buf], ((tt >> 1) - 1) & 1, wc)))
+          break;
+        const uint32_t base = send_base + buf * kXBytes;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint32_t a = enc_u16x2(s[8 * c], s[8 * c + 1], inv);
+          const uint32_t b = enc_u16x2(s[8 * c + 2], s[8 * c + 3], inv);
+          const uint32_t cc = enc_u16x2(s[8 * c + 4], s[8 * c + 5], inv);
+          const uint32_t d = enc_u16x2(s[8 * c + 6], s[8 * c + 7], inv);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(base + xrow_off(row, c)),
+                       "r"(a), "r"(b), "r"(cc), "r"(d)
+                       : "memory");
+        }
+        asm volatile("st.shared.f32 [%0], %1;" ::"r"(base + kXPayload + row * 4),
+                     "f"(mabs * (1.f / 32767.f))
+                     : "memory");
+        fence_proxy_async_smem();  // generic-proxy writes -> visible to the bulk copy
+        mbar_arrive(&bars->staged[buf]);
+      }
+      t += n;
+    }
+  } else {
+    // =================== softmax warpgroup (warps 0-3) + epilogue ===================
+    const int row = threadIdx.x;  // head row = TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const float NEG_INF = -__int_as_float(0x7f800000);
+    const bool row_ok = row < p.n_heads;
+    SegIter it{plan.seq_pages(), plan.seq_prefix(), p.batch, g_begin, g_end, b_begin};
+    int seq, p0, p1, t = 0, sg = 0;
+    bool ok = true;
+    while (ok && it.next(seq, p0, p1)) {
+      const int n = p1 - p0, t0 = t;
+      const int len = min(p.seq_lens[seq], p.max_pages * kPage);
+      // ---- this CTA's latent half of the query row -> TMEM (A operand of QK) ----
+      {
+        const uint4* src = reinterpret_cast<const uint4*>(
+            p.q_cat + (static_cast<size_t>(seq) * p.n_heads + (row_ok ? row : 0)) * kRow);
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint4 v = row_ok ? __ldg(src + (256 * rank + 64 * c) / 8 + k)
+                                   : make_uint4(0u, 0u, 0u, 0u);
+            r[4 * k] = v.x;
+            r[4 * k + 1] = v.y;
+            r[4 * k + 2] = v.z;
+            r[4 * k + 3] = v.w;
+          }
+          tmem_st32(tmem + kTmemQ + 32 * c + lane_off, r);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bars->q_ready);
+      }
+      float m_ref = NEG_INF, l_sum = 0.f;
+      for (int i = 0; i < n; ++i) {
+        const int tt = t0 + i, buf = tt & 1;
+        const bool first = i == 0;
+        // ---- own exact partial ----
+        if (!(ok = warp_wait(&bars->s_full[buf], (tt >> 1) & 1, wc))) break;
+        tc_fence_after();
+        float s[64];
+        {
+          uint32_t r[32];
+          tmem_ld32(tmem + kTmemS + buf * 64 + lane_off, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) s[k] = __uint_as_float(r[k]);
+          tmem_ld32(tmem + kTmemS + buf * 64 + 32 + lane_off, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) s[32 + k] = __uint_as_float(r[k]);
+        }
+        // ---- plus the peer's decoded partial ----
+        if (!(ok = warp_wait<true>(&bars->x_full[buf], (tt >> 1) & 1, wc))) break;
+        {
+          const uint32_t base = recv_base + buf * kXBytes;
+          float dq;
+          asm volatile("ld.shared.f32 %0, [%1];" : "=f"(dq) : "r"(base + kXPayload + row * 4));
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint32_t v[4];
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
+                         : "r"(base + xrow_off(row, c)));
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              s[8 * c + 2 * k] = fmaf(dec_lo(v[k]), dq, s[8 * c + 2 * k]);
+              s[8 * c + 2 * k + 1] = fmaf(dec_hi(v[k]), dq, s[8 * c + 2 * k + 1]);
+            }
+          }
+          mbar_arrive(&bars->consumed[buf]);
+        }
+        // ---- online softmax ----
+        const int valid = min(kPage, len - (p0 + i) * kPage);
+        if (valid < kPage) {
+#pragma unroll
+          for (int k = 0; k < 64; ++k) s[k] = k < valid ? s[k] : NEG_INF;
+        }
         float mx = NEG_INF;
 #pragma unroll
-        for (int k = 0; k < 64; ++k) {
-          s[k] = (k < valid) ? s[k] * p.scale_log2 : NEG_INF;
-          mx = fmaxf(mx, s[k]);
-        }
+        for (int k = 0; k < 64; ++k) mx = fmaxf(mx, s[k]);
+        mx *= p.scale_log2;  // log2 units (scale > 0 keeps the arg max)
         float alpha = 1.f;
         bool rescale = false;
-        if (i == 0) {
+        if (first) {
           m_ref = mx;
         } else if (mx > m_ref + kRescaleThreshold) {
           alpha = ex2_approx(m_ref - mx);
@@ -508,16 +665,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         uint32_t pk[32];
 #pragma unroll
         for (int k = 0; k < 32; ++k) {
-          const float e0 = ex2_approx(s[2 * k] - m_ref);
-          const float e1 = ex2_approx(s[2 * k + 1] - m_ref);
+          const float e0 = ex2_approx(fmaf(s[2 * k], p.scale_log2, -m_ref));
+          const float e1 = ex2_approx(fmaf(s[2 * k + 1], p.scale_log2, -m_ref));
           rs += e0 + e1;
           pk[k] = pack_bf16x2(e0, e1);
         }
         l_sum = l_sum * alpha + rs;
-        if (__any_sync(0xffffffffu, rescale)) {
-          // O must hold PV of the previous tile before it is rescaled
-          const int tp = t - 1;
-          if (!warp_wait(&bars->pv_done[tp & 1], (tp >> 1) & 1, wc)) { ok = false; break; }
+        if (!first && __any_sync(0xffffffffu, rescale)) {
+          // O must hold PV of the previous page before it is rescaled
+          if (!(ok = warp_wait(&bars->pv_done, (tt - 1) & 1, wc))) break;
           tc_fence_after();
 #pragma unroll 1
           for (int c = 0; c < 256; c += 32) {
@@ -528,17 +684,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * alpha);
             tmem_st32(tmem + kTmemO + c + lane_off, r);
           }
-          tmem_wait_st();
         }
-        tmem_st32(tmem + kTmemP + sb * 32 + lane_off, pk);
+        // ---- P over the S buffer, once the send warpgroup has drained it ----
+        if (!(ok = warp_wait(&bars->staged[buf], (tt >> 1) & 1, wc))) break;
+        tc_fence_after();
+        tmem_st32(tmem + kTmemS + buf * 64 + lane_off, pk);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bars->p_full[sb]);
+        mbar_arrive(&bars->p_full[buf]);
       }
       if (!ok) break;
       // ---- segment epilogue: O / l -> global ----
-      const int tl = t - 1;
-      if (!warp_wait(&bars->pv_done[tl & 1], (tl >> 1) & 1, wc)) { ok = false; break; }
+      if (!(ok = warp_wait(&bars->seg_done, sg & 1, wc))) break;
       tc_fence_after();
       const int nparts = plan.seq_nparts()[seq];
       const float lse_nat = (m_ref + __log2f(l_sum)) * 0.69314718055994531f;
@@ -553,7 +710,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         dst = p.part_o + (static_cast<size_t>(slot) * p.n_heads + row) * 512 + 256 * rank;
         dst_lse = p.part_lse + static_cast<size_t>(slot) * p.n_heads + row;
       }
-      const bool row_ok = row < p.n_heads;
 #pragma unroll 1
       for (int c = 0; c < 256; c += 32) {
         uint32_t r[32];
@@ -563,7 +719,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           float4* d4 = reinterpret_cast<float4*>(dst + c);
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            d4[k] = make_float4(__uint_as_float(r[4 * k]) * inv_l, __uint_as_float(r[4 * k + 1]) * inv_l,
+            d4[k] = make_float4(__uint_as_float(r[4 * k]) * inv_l,
+                                __uint_as_float(r[4 * k + 1]) * inv_l,
                                 __uint_as_float(r[4 * k + 2]) * inv_l,
                                 __uint_as_float(r[4 * k + 3]) * inv_l);
         }
@@ -571,19 +728,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (row_ok && rank == 0 && dst_lse) *dst_lse = lse_nat;
       tc_fence_before();
       mbar_arrive(&bars->o_free);
+      t += n;
       ++sg;
     }
-    // the peer's last remote operations on this CTA's shared memory must have landed
-    if (t > 0) {
+    // The peer's remote arrivals for our last two partials must land before this CTA exits.
+    {
       volatile int never = 0;
       WaitCtx drain{&never, p.status, p.wait_ns};
-      mbar_wait<true>(&bars->x_free, (t - 1) & 1, ok ? wc : drain);
+      for (int u = max(0, t - 2); u < t; ++u)
+        mbar_wait<true>(&bars->peer_done[u & 1], (u >> 1) & 1, ok ? wc : drain);
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }

@@ -468,10 +468,8 @@ int mla_decode_attn(const mla_dims* dims, const void* q_cat, const void* q_lo,
                                                       kMinPagesPerPart, plan, c->status);
   if ((rc = last_launch())) return rc;
   if (dims->dtype == MLA_BF16) {
-    CUtensorMap tq_lat, tq_rope, tc_lat, tc_rope;
+    CUtensorMap tc_lat, tc_rope, tq_rope;
     const uint64_t rows = static_cast<uint64_t>(num_pages) * kPageN;
-    if ((rc = map3(&tq_lat, q_cat, kRowN, H, B, kRowN * 2ull, kRowN * 2ull * H, 64, 128, 1)))
-      return rc;
     if ((rc = map3(&tq_rope, q_cat, kRowN, H, B, kRowN * 2ull, kRowN * 2ull * H, 32, 128, 1,
                    CU_TENSOR_MAP_SWIZZLE_64B)))
       return rc;
@@ -487,6 +485,7 @@ int mla_decode_attn(const mla_dims* dims, const void* q_cat, const void* q_lo,
     p.max_pages = max_pages;
     p.num_pages = num_pages;
     p.num_parts = parts;
+    p.q_cat = static_cast<const __nv_bfloat16*>(q_cat);
     p.page_table = page_table;
     p.seq_lens = seq_lens;
     p.plan = plan;
@@ -499,8 +498,8 @@ int mla_decode_attn(const mla_dims* dims, const void* q_cat, const void* q_lo,
     p.wait_ns = kDefaultWaitNs;
     const bool prof = g_prof_next < g_prof_count;
     if (prof && cudaEventRecord(g_prof_begin[g_prof_next], st) != cudaSuccess) return MLA_ERR_CUDA;
-    attn::split_kernel<<<2 * parts, attn::kThreads, attn::kSmemBytes, st>>>(tq_lat, tq_rope,
-                                                                            tc_lat, tc_rope, p);
+    attn::split_kernel<<<2 * parts, attn::kThreads, attn::kSmemBytes, st>>>(tc_lat, tc_rope,
+                                                                            tq_rope, p);
     if (prof) {
       if ((rc = last_launch())) return rc;
       if (cudaEventRecord(g_prof_end[g_prof_next++], st) != cudaSuccess) return MLA_ERR_CUDA;

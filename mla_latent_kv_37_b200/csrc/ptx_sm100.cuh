@@ -200,6 +200,21 @@ __device__ __forceinline__ void st_async_v4(uint32_t cluster_addr, float a, floa
       : "memory");
 }
 
+// Make generic-proxy shared-memory writes visible to the async proxy (bulk copies, TMA).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Bulk copy of `bytes` from this CTA's shared memory to a peer CTA's shared memory
+// (shared::cluster address); completion is counted in bytes on the peer's mbarrier.
+__device__ __forceinline__ void bulk_copy_s2cluster(uint32_t dst_cluster, uint32_t src,
+                                                    uint32_t bytes, uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(dst_cluster), "r"(src), "r"(bytes), "r"(bar_cluster)
+      : "memory");
+}
+
 // ------------------------------------------------------------------------------------------
 // tcgen05: tensor memory and the 5th-generation tensor core
 // ------------------------------------------------------------------------------------------
