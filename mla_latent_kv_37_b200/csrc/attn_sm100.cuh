@@ -12,8 +12,9 @@
 // so each work unit runs on a CLUSTER OF TWO CTAs that split the 576 columns of every row:
 // CTA r owns latent columns [256r, 256r+256) and RoPE columns [512+32r, 512+32r+32).
 //   * TMEM (512 columns): O half 256 | query latent half 128 (A operand of QK) | two S
-//     buffers of 64.  P (bf16) is written over the S buffer it came from (A operand of PV).
-//     The 32 RoPE columns of the query half sit in shared memory (A operand, 64B swizzle).
+//     buffers of 64.  The 32 RoPE columns of the query half sit in shared memory (A operand,
+//     64B swizzle), and so does P (bf16, 128B swizzle, A operand of PV), so an S buffer is
+//     free again as soon as it has been drained and QK runs two pages ahead of the softmax.
 //   * Pages arrive by TMA (128B/64B swizzle) into a 4-stage ring; each byte leaves HBM once.
 //   * S_r = Q_r C_r^T is a partial score; the pair exchanges partials.  Distributed shared
 //     memory moves ~16 B/clk per SM, so a partial travels as 16-bit fixed point relative to
@@ -53,11 +54,13 @@ constexpr uint32_t kStageBytes = 4 * kCLatBox + 64 * 64;  // + rope box 64 rows 
 constexpr uint32_t kXPayload = 128 * 128;                 // 128 rows x 64 x 16-bit
 constexpr uint32_t kXBytes = kXPayload + 128 * 4;         // + one fp32 step per row
 constexpr uint32_t kQRopeBytes = 128 * 64;                // 128 rows x 32 bf16
+constexpr uint32_t kPBytes = 128 * 128;                   // P: 128 rows x 64 bf16
 constexpr uint32_t kOffStage = 0;
-constexpr uint32_t kOffSend = kOffStage + kStages * kStageBytes;
-constexpr uint32_t kOffRecv = kOffSend + 2 * kXBytes;
-constexpr uint32_t kOffQRope = kOffRecv + 2 * kXBytes;
-constexpr uint32_t kOffBar = kOffQRope + kQRopeBytes;
+constexpr uint32_t kOffP = kOffStage + kStages * kStageBytes;  // one P buffer
+constexpr uint32_t kOffQRope = kOffP + kPBytes;
+constexpr uint32_t kOffSend = kOffQRope + kQRopeBytes;  // two send buffers
+constexpr uint32_t kOffRecv = kOffSend + 2 * kXBytes;   // one receive buffer
+constexpr uint32_t kOffBar = kOffRecv + kXBytes;
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // barriers + alignment slack
 // TMEM columns
 constexpr uint32_t kTmemO = 0, kTmemQ = 256, kTmemS = 384, kTmemCols = 512;
@@ -65,7 +68,7 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 static_assert(kTmemS + 2 * 64 == kTmemCols, "tensor memory budget");
-static_assert(kXBytes % 16 == 0 && kOffQRope % 1024 == 0, "alignment");
+static_assert(kXBytes % 16 == 0 && kOffP % 1024 == 0 && kOffQRope % 1024 == 0, "alignment");
 
 struct Params {
   int batch;
@@ -281,12 +284,13 @@ struct Bars {
   uint64_t q_empty;       // MMA: the segment's last QK finished (commit)
   uint64_t q_ready;       // softmax WG: the segment's query latent half is in TMEM (128)
   uint64_t s_full[2];     // MMA: S buffer i written (commit)
-  uint64_t staged[2];     // send WG: S drained, partial staged in send[i] (128)
-  uint64_t p_full[2];     // softmax WG: P written over S buffer i (128)
-  uint64_t pv_done;       // MMA: PV finished (commit, once per page)
-  uint64_t consumed[2];   // softmax WG: recv[i] read (128)
-  uint64_t x_full[2];     // the peer's partial landed in recv[i] (bulk-copy bytes)
-  uint64_t peer_done[2];  // the peer consumed our partial from its recv[i] (1 remote arrival)
+  uint64_t s_free[2];     // both warpgroups drained S buffer i (256)
+  uint64_t staged[2];     // send WG: partial staged in send[i] (128)
+  uint64_t p_full;        // softmax WG: P written (128)
+  uint64_t pv_done;       // MMA: PV finished, P buffer free (commit, once per page)
+  uint64_t consumed;      // softmax WG: recv read (128)
+  uint64_t x_full;        // the peer's partial landed in recv (bulk-copy bytes)
+  uint64_t peer_done[2];  // the peer consumed our partial of a page of parity i (1 remote)
   uint64_t o_free;        // softmax WG: the epilogue drained O (128)
   uint64_t seg_done;      // MMA: every PV of the segment finished (commit, once per segment)
   uint64_t drain;
@@ -319,20 +323,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mbar_init(&bars->q_ready, 128);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->s_full[i], 1);
+      mbar_init(&bars->s_free[i], 256);
       mbar_init(&bars->staged[i], 128);
-      mbar_init(&bars->p_full[i], 128);
-      mbar_init(&bars->consumed[i], 128);
-      mbar_init(&bars->x_full[i], 1);
       mbar_init(&bars->peer_done[i], 1);
     }
+    mbar_init(&bars->p_full, 128);
     mbar_init(&bars->pv_done, 1);
+    mbar_init(&bars->consumed, 128);
+    mbar_init(&bars->x_full, 1);
     mbar_init(&bars->o_free, 128);
     mbar_init(&bars->seg_done, 1);
     mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
     fence_mbar_init_cluster();
-    mbar_arrive_expect_tx(&bars->x_full[0], kXBytes);  // armed for pages 0 and 1
-    mbar_arrive_expect_tx(&bars->x_full[1], kXBytes);
+    mbar_arrive_expect_tx(&bars->x_full, kXBytes);  // armed for page 0
   }
   if (warp == 9) {
     tmem_alloc(&bars->tmem_base, kTmemCols);
@@ -444,34 +448,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (last_of_seg) mma_commit(&bars->q_empty);
         return true;
       };
-      // O += P_tt C_lat: A = P (bf16, over S buffer tt & 1), B = the page's latent half
+      // O += P_tt C_lat: A = P (bf16, shared memory), B = the page's latent half
+      const uint32_t p_base = smem_u32(smem + kOffP);
       auto issue_pv = [&](int tt, bool first_of_seg) -> bool {
         if (first_of_seg && sg > 0 && !mbar_wait(&bars->o_free, (sg - 1) & 1, wc)) return false;
-        if (!mbar_wait(&bars->p_full[tt & 1], (tt >> 1) & 1, wc)) return false;
+        if (!mbar_wait(&bars->p_full, tt & 1, wc)) return false;
         tc_fence_after();
         const uint32_t st = smem_u32(sStage + (tt % kStages) * kStageBytes);
+        const uint32_t pa = p_base;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_ts(tmem + kTmemO, tmem + kTmemS + (tt & 1) * 64 + kk * 8,
+          mma_ss(tmem + kTmemO, smem_desc(pa + kk * 32, 16, 1024, kSwizzle128B),
                  smem_desc(st + kk * 2048, 8192, 1024, kSwizzle128B), idesc_pv,
                  (first_of_seg && kk == 0) ? 0u : 1u);
         mma_commit(&bars->pv_done);
         mma_commit(&bars->empty[tt % kStages]);
         return true;
       };
+      // S buffer of page tt (tt >= 2) is free once both warpgroups drained page tt - 2
+      auto s_ready = [&](int tt) -> bool {
+        return tt < 2 || mbar_wait(&bars->s_free[tt & 1], ((tt >> 1) - 1) & 1, wc);
+      };
       while (ok && it.next(seq, p0, p1)) {
         const int n = p1 - p0, t0 = t;
         ok = mbar_wait(&bars->q_ready, sg & 1, wc) && mbar_wait(&bars->q_full, sg & 1, wc);
-        if (ok) ok = issue_qk(t0, n == 1);
-        if (ok && n > 1) ok = issue_qk(t0 + 1, n == 2);
+        if (ok) ok = s_ready(t0) && issue_qk(t0, n == 1);
+        if (ok && n > 1) ok = s_ready(t0 + 1) && issue_qk(t0 + 1, n == 2);
+        // softmax order per page: drain S_i (s_free) ... write P_i (p_full)
         for (int i = 0; ok && i < n; ++i) {
           const int tt = t0 + i;
+          if (i + 2 < n && !(ok = s_ready(tt + 2) && issue_qk(tt + 2, i + 3 == n))) break;
           if (!(ok = issue_pv(tt, i == 0))) break;
-          if (i == n - 1) mma_commit(&bars->seg_done);
-          // PV_tt done: O is current and S buffer tt & 1 (holding P_tt) is free
-          if (!(ok = mbar_wait(&bars->pv_done, tt & 1, wc))) break;
-          if (i + 2 < n) ok = issue_qk(tt + 2, i + 3 == n);
         }
+        if (ok) mma_commit(&bars->seg_done);
         t += n;
         ++sg;
       }
@@ -486,8 +495,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // =================== exchange: bulk copies out (10), cluster-scope signals (11) ===========
     if (lane == 0) {
       const uint32_t peer_recv = mapa_shared(recv_base, peer);
-      const uint32_t peer_xfull[2] = {mapa_shared(smem_u32(&bars->x_full[0]), peer),
-                                      mapa_shared(smem_u32(&bars->x_full[1]), peer)};
+      const uint32_t peer_xfull = mapa_shared(smem_u32(&bars->x_full), peer);
       const uint32_t peer_done_r[2] = {mapa_shared(smem_u32(&bars->peer_done[0]), peer),
                                        mapa_shared(smem_u32(&bars->peer_done[1]), peer)};
       SegIter it{plan.seq_pages(), plan.seq_prefix(), p.batch, g_begin, g_end, b_begin};
@@ -498,14 +506,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int tt = t; ok && tt < t + n; ++tt) {
           const int buf = tt & 1;
           if (warp == 10) {
-            // the page's partial is staged in send[buf]: ship it
+            // the page's partial is staged in send[buf] and the peer's (single) receive buffer
+            // has been read for page tt - 1: ship it
             if (!(ok = mbar_wait(&bars->staged[buf], (tt >> 1) & 1, wc))) break;
-            bulk_copy_s2cluster(peer_recv + buf * kXBytes, send_base + buf * kXBytes, kXBytes,
-                                peer_xfull[buf]);
+            if (tt >= 1 && !(ok = mbar_wait<true>(&bars->peer_done[(tt - 1) & 1],
+                                                 ((tt - 1) >> 1) & 1, wc)))
+              break;
+            bulk_copy_s2cluster(peer_recv, send_base + buf * kXBytes, kXBytes, peer_xfull);
           } else {
-            // every softmax row has read recv[buf]: re-arm it for page tt + 2, tell the peer
-            if (!(ok = mbar_wait(&bars->consumed[buf], (tt >> 1) & 1, wc))) break;
-            mbar_arrive_expect_tx(&bars->x_full[buf], kXBytes);
+            // every softmax row has read recv: re-arm it for page tt + 1, tell the peer
+            if (!(ok = mbar_wait(&bars->consumed, tt & 1, wc))) break;
+            mbar_arrive_expect_tx(&bars->x_full, kXBytes);
             mbar_arrive_remote(peer_done_r[buf]);
           }
         }
@@ -539,6 +550,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int k = 0; k < 32; ++k) s[32 + k] = __uint_as_float(r[k]);
         }
         tc_fence_before();
+        mbar_arrive(&bars->s_free[buf]);
         const int valid = min(kPage, len - (p0 + i) * kPage);
         if (valid < kPage) {
 #pragma unroll
@@ -622,10 +634,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int k = 0; k < 32; ++k) s[32 + k] = __uint_as_float(r[k]);
         }
+        tc_fence_before();
+        mbar_arrive(&bars->s_free[buf]);
         // ---- plus the peer's decoded partial ----
-        if (!(ok = warp_wait<true>(&bars->x_full[buf], (tt >> 1) & 1, wc))) break;
+        if (!(ok = warp_wait<true>(&bars->x_full, tt & 1, wc))) break;
         {
-          const uint32_t base = recv_base + buf * kXBytes;
+          const uint32_t base = recv_base;
           float dq;
           asm volatile("ld.shared.f32 %0, [%1];" : "=f"(dq) : "r"(base + kXPayload + row * 4));
 #pragma unroll
@@ -640,7 +654,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               s[8 * c + 2 * k + 1] = fmaf(dec_hi(v[k]), dq, s[8 * c + 2 * k + 1]);
             }
           }
-          mbar_arrive(&bars->consumed[buf]);
+          mbar_arrive(&bars->consumed);
         }
         // ---- online softmax ----
         const int valid = min(kPage, len - (p0 + i) * kPage);
@@ -685,13 +699,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tmem_st32(tmem + kTmemO + c + lane_off, r);
           }
         }
-        // ---- P over the S buffer, once the send warpgroup has drained it ----
-        if (!(ok = warp_wait(&bars->staged[buf], (tt >> 1) & 1, wc))) break;
-        tc_fence_after();
-        tmem_st32(tmem + kTmemS + buf * 64 + lane_off, pk);
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&bars->p_full[buf]);
+        // ---- P -> shared memory (canonical K-major, 128B swizzle) once PV of page tt - 1
+        // has read it ----
+        if (tt >= 1 && !(ok = warp_wait(&bars->pv_done, (tt - 1) & 1, wc))) break;
+        {
+          const uint32_t pa = smem_u32(smem + kOffP);
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pa + xrow_off(row, c)),
+                         "r"(pk[4 * c]), "r"(pk[4 * c + 1]), "r"(pk[4 * c + 2]),
+                         "r"(pk[4 * c + 3])
+                         : "memory");
+        }
+        fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
+        mbar_arrive(&bars->p_full);
       }
       if (!ok) break;
       // ---- segment epilogue: O / l -> global ----
