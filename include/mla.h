@@ -157,6 +157,33 @@ int mla_out_proj(const mla_dims* dims, const float* o_lat, const void* w_uv, con
                  void* o_heads, void* out, void* workspace, size_t workspace_bytes,
                  mla_stream_t stream);
 
+/*
+ * mla_decode_attn_static_scratch -- mla_decode_attn for callers that cannot allocate device
+ * memory.  (The MLA pages have no counterpart to this: it is a deployment convenience.)
+ * A process whose memory manager already owns all of the GPU's memory, or a code path where a
+ * cudaMalloc -- which may synchronise the device or fail under memory pressure -- is not
+ * acceptable, cannot provide the workspace mla_decode_attn needs.  This entry point takes the
+ * same arguments minus the workspace and keeps the split-KV scratch (page plan and per-part
+ * partial results) in a fixed array of MLA_STATIC_SCRATCH_BYTES in the library's own device
+ * data, which every GPU that loads the library holds until the process exits.  It allocates
+ * nothing.  Results equal mla_decode_attn's for the same arguments.
+ *   - The scratch needed is about (batch + parts) * n_heads * 2 KiB (parts = num_splits, or
+ *     the automatic choice); calls needing more than MLA_STATIC_SCRATCH_BYTES return
+ *     MLA_ERR_WORKSPACE without launching anything (pass a smaller num_splits).
+ *   - The first call on each device looks the array's device address up (one-time set-up,
+ *     cached per device); make that first call before any stream capture.
+ *   - All calls on a device share the one array and leave their contents in it; nothing in it
+ *     needs to start at zero.  Calls that overlap on the GPU (different streams, or threads
+ *     without synchronisation) race on the scratch: order them on one stream.
+ */
+#define MLA_STATIC_SCRATCH_BYTES (64u * 1024u * 1024u)
+int mla_decode_attn_static_scratch(const mla_dims* dims, const void* q_cat, const void* q_lo,
+                                   const void* cache_pool, int32_t num_pages,
+                                   const int32_t* page_table, int32_t max_pages,
+                                   const int32_t* seq_lens, float softmax_scale,
+                                   int32_t num_splits, float* o_lat, float* lse,
+                                   mla_stream_t stream);
+
 /* Synchronises `stream`, returns the device status word of the current device (a bitwise OR
  * of MLA_STATUS_* raised since the last call, 0 if none) and clears it.  Returns a negative
  * MLA_ERR_CUDA if the synchronisation itself failed. */

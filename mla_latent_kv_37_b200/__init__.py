@@ -63,6 +63,9 @@ _SIGS = {
     "mla_decode_attn": (ctypes.c_int, [ctypes.POINTER(mla_dims), _P, _P, _P, _I, _P, _I, _P,
                                        ctypes.c_float, _I, _P, _SZ, _P, _P, _P]),
     "mla_out_proj": (ctypes.c_int, [ctypes.POINTER(mla_dims), _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "mla_decode_attn_static_scratch": (ctypes.c_int, [ctypes.POINTER(mla_dims), _P, _P, _P, _I,
+                                                      _P, _I, _P, ctypes.c_float, _I, _P, _P,
+                                                      _P]),
     "mla_get_status": (ctypes.c_int, [_P]),
     "mla_error_string": (ctypes.c_char_p, [ctypes.c_int]),
     "mla_version": (ctypes.c_char_p, []),
@@ -192,6 +195,28 @@ def mla_decode_attn(d: mla_dims, q_cat, cache_pool, page_table, seq_lens, o_lat,
                                _ptr(seq_lens), float(softmax_scale), int(num_splits), _ptr(ws),
                                ws.numel(), _ptr(o_lat), _ptr(lse), _stream(stream))
     _check(rc, "mla_decode_attn")
+
+
+def mla_decode_attn_static_scratch(d: mla_dims, q_cat, cache_pool, page_table, seq_lens, o_lat,
+                                   lse=None, softmax_scale: float = 0.0, num_splits: int = 0,
+                                   stream=None):
+    """mla_decode_attn without a workspace: the library's own fixed scratch array is used, for
+    callers that cannot allocate device memory (see include/mla.h)."""
+    e = _elem(d)
+    H = d.n_heads
+    _need(q_cat, "q_cat", e, (d.batch, H, d.d_c + d.d_rope))
+    _need(cache_pool, "cache_pool", e)
+    _need(page_table, "page_table", torch.int32)
+    _need(seq_lens, "seq_lens", torch.int32, (d.batch,))
+    _need(o_lat, "o_lat", torch.float32, (d.batch, H, d.d_c))
+    _need(lse, "lse", torch.float32, (d.batch, H))
+    rc = lib().mla_decode_attn_static_scratch(ctypes.byref(d), _ptr(q_cat), None,
+                                              _ptr(cache_pool), cache_pool.shape[0],
+                                              _ptr(page_table), page_table.shape[1],
+                                              _ptr(seq_lens), float(softmax_scale),
+                                              int(num_splits), _ptr(o_lat), _ptr(lse),
+                                              _stream(stream))
+    _check(rc, "mla_decode_attn_static_scratch")
 
 
 def mla_out_proj(d: mla_dims, o_lat, w_uv, ws, w_o=None, o_heads=None, out=None, stream=None):

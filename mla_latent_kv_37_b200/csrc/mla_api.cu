@@ -641,3 +641,133 @@ int mla_set_profile_events(void* const* begin, void* const* end, int32_t count) 
 int32_t mla_profile_events_used(void) { return g_prof_next; }
 
 }  // extern "C"
+
+// =============================================================================================
+// Decode attention with scratch memory owned by the library (no allocation by anyone).
+//
+// Some callers cannot allocate device memory for a workspace: a process whose memory manager
+// has already reserved all of the GPU's memory for itself, or a code path where a cudaMalloc
+// (which can synchronise the device or fail under memory pressure) is not acceptable.  For them
+// the split-KV scratch of mla_decode_attn (the page plan and the per-part partial results)
+// lives in one fixed-size array in the library's own device data.  Every GPU that loads the
+// library holds MLA_STATIC_SCRATCH_BYTES for it until the process exits.
+// =============================================================================================
+static __device__ __align__(256) unsigned char g_decode_scratch[MLA_STATIC_SCRATCH_BYTES];
+
+namespace {
+void* g_scratch_addr[64];  // device address of g_decode_scratch, per device
+std::mutex g_scratch_mu;
+
+// Host code sees `g_decode_scratch` only as a stand-in symbol: its device address is looked
+// up once per device, with that device current, and cached.
+int decode_scratch_addr(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MLA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) return MLA_ERR_CUDA;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return MLA_OK;
+}
+
+struct DecodeScratch {
+  size_t plan, part_o, part_lse, total;
+};
+
+DecodeScratch decode_scratch_layout(int B, int H, int parts) {
+  DecodeScratch d{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  d.plan = take(attn::PlanView::words(B, parts) * 4);
+  d.part_o = take(static_cast<size_t>(B + parts) * H * kDc * 4);
+  d.part_lse = take(static_cast<size_t>(B + parts) * H * 4);
+  d.total = off;
+  return d;
+}
+}  // namespace
+
+extern "C" int mla_decode_attn_static_scratch(const mla_dims* dims, const void* q_cat,
+                                              const void* q_lo, const void* cache_pool,
+                                              int32_t num_pages, const int32_t* page_table,
+                                              int32_t max_pages, const int32_t* seq_lens,
+                                              float softmax_scale, int32_t num_splits,
+                                              float* o_lat, float* lse, mla_stream_t stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (!q_cat || !cache_pool || !page_table || !seq_lens || !o_lat) return MLA_ERR_NULL_ARG;
+  if (num_pages < 1 || max_pages < 1 || num_splits < 0) return MLA_ERR_ARG;
+  if (q_lo) return MLA_ERR_ARG;
+  if (!(softmax_scale >= 0.f) || !std::isfinite(softmax_scale)) return MLA_ERR_ARG;
+  if (!aligned(q_cat, 16) || !aligned(cache_pool, 16) || !aligned(o_lat, 16) ||
+      !aligned(page_table, 4) || !aligned(seq_lens, 4) || (lse && !aligned(lse, 4)))
+    return MLA_ERR_ALIGN;
+  if (static_cast<int64_t>(num_pages) * kPageN > INT32_MAX) return MLA_ERR_ARG;
+  DevCtx* c = nullptr;
+  if ((rc = device_ctx(&c))) return rc;
+  const int B = dims->batch, H = dims->n_heads;
+  const int parts = resolve_parts(num_splits, c);
+  const DecodeScratch w = decode_scratch_layout(B, H, parts);
+  if (w.total > MLA_STATIC_SCRATCH_BYTES) return MLA_ERR_WORKSPACE;  // beyond the fixed size
+  void* scratch = nullptr;
+  if ((rc = decode_scratch_addr(&scratch))) return rc;
+  // Nothing in the scratch has to start at zero: the plan kernel writes every plan word and
+  // the split kernel writes every partial slot before the combine kernel reads it.
+  char* ws = static_cast<char*>(scratch);
+  int32_t* plan = reinterpret_cast<int32_t*>(ws + w.plan);
+  float* part_o = reinterpret_cast<float*>(ws + w.part_o);
+  float* part_lse = reinterpret_cast<float*>(ws + w.part_lse);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const float scale =
+      softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(kDn + kDr));
+  attn::plan_kernel<<<1, attn::kPlanThreads, 0, st>>>(seq_lens, B, max_pages, parts,
+                                                      kMinPagesPerPart, plan, c->status);
+  if ((rc = last_launch())) return rc;
+  if (dims->dtype == MLA_BF16) {
+    CUtensorMap tc_lat, tc_rope, tq_rope;
+    const uint64_t rows = static_cast<uint64_t>(num_pages) * kPageN;
+    if ((rc = map3(&tq_rope, q_cat, kRowN, H, B, kRowN * 2ull, kRowN * 2ull * H, 32, 128, 1,
+                   CU_TENSOR_MAP_SWIZZLE_64B)))
+      return rc;
+    if ((rc = map2(&tc_lat, cache_pool, kRowN, rows, kRowN * 2ull, 64, 64,
+                   CU_TENSOR_MAP_SWIZZLE_128B)))
+      return rc;
+    if ((rc = map2(&tc_rope, cache_pool, kRowN, rows, kRowN * 2ull, 32, 64,
+                   CU_TENSOR_MAP_SWIZZLE_64B)))
+      return rc;
+    attn::Params p{};
+    p.batch = B;
+    p.n_heads = H;
+    p.max_pages = max_pages;
+    p.num_pages = num_pages;
+    p.num_parts = parts;
+    p.q_cat = static_cast<const __nv_bfloat16*>(q_cat);
+    p.page_table = page_table;
+    p.seq_lens = seq_lens;
+    p.plan = plan;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.o_lat = o_lat;
+    p.lse = lse;
+    p.part_o = part_o;
+    p.part_lse = part_lse;
+    p.status = c->status;
+    p.wait_ns = kDefaultWaitNs;
+    attn::split_kernel<<<2 * parts, attn::kThreads, attn::kSmemBytes, st>>>(tc_lat, tc_rope,
+                                                                            tq_rope, p);
+  } else {
+    attn::f32_split_kernel<<<dim3(parts, H), 128, 0, st>>>(
+        static_cast<const float*>(q_cat), static_cast<const float*>(cache_pool), page_table,
+        max_pages, num_pages, seq_lens, plan, B, parts, H, scale, o_lat, lse, part_o, part_lse,
+        c->status);
+  }
+  if ((rc = last_launch())) return rc;
+  attn::combine_kernel<<<dim3(H, B), 128, 0, st>>>(plan, B, parts, H, part_o, part_lse, o_lat,
+                                                   lse);
+  return last_launch();
+}
