@@ -148,15 +148,15 @@ __global__ void wuk_epilogue_kernel(const float* __restrict__ part, int n_pad, i
   }
 }
 
-// o_lat fp32 [n] -> [2][n] bf16 hi/lo planes.
-__global__ void split_hi_lo_kernel(const float* __restrict__ x, size_t n,
+// o_lat fp32 [n] -> bf16 hi/lo planes: out[i] = hi, out[plane + i] = lo (plane >= n).
+__global__ void split_hi_lo_kernel(const float* __restrict__ x, size_t n, size_t plane,
                                    __nv_bfloat16* __restrict__ out) {
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {
     const float v = x[i];
     const __nv_bfloat16 hi = __float2bfloat16_rn(v);
     out[i] = hi;
-    out[n + i] = __float2bfloat16_rn(v - __bfloat162float(hi));
+    out[plane + i] = __float2bfloat16_rn(v - __bfloat162float(hi));
   }
 }
 

@@ -1,0 +1,517 @@
+// Persistent "stream-K" weight-streaming GEMM on tcgen05 with the product's epilogue fused in.
+//
+//   Y_g[m][n] = sum_k A_g[m][k] * X_g[n][k]       (A = weights, X = a few activation rows)
+//
+// Decode projections multiply large weight matrices by a handful of token vectors, so their
+// cost is the time to stream the weights from HBM once.  The work -- every (128-row tile,
+// 64-wide K block) pair of every group -- is one list of I iterations cut into P equal
+// contiguous ranges, one per CTA (P <= number of SMs), so every SM streams the same number of
+// weight bytes in one wave and its TMA -> shared memory -> tcgen05.mma pipeline never drains
+// between tiles.  A CTA's range splits into segments at tile boundaries; each segment is
+// accumulated in one of two TMEM buffers (so the epilogue of one segment overlaps the MMAs of
+// the next).
+//
+// A tile covered by one CTA is finished straight from TMEM.  A tile shared by several CTAs is
+// finished by whichever contributor arrives last: each contributor writes its partial sum to
+// slot (its CTA index - the tile's first CTA index) of the tile's partial area and counts
+// itself on the tile's counter; the one that completes the count adds the slots in slot order
+// (so the result does not depend on arrival order) and runs the epilogue.  Nobody waits for
+// another CTA.  Counters are tagged with a per-launch epoch in their upper 32 bits, so stale
+// counts from earlier launches read as zero and the workspace never needs clearing.
+//
+// Roles (192 threads): warp 0 TMA producer, warp 1 MMA issuer + TMEM owner, warps 2-5
+// epilogue (warp w reads TMEM lanes 32*(w%4) .. +31, i.e. tile rows).
+//
+// Operand layouts in shared memory (128-byte swizzle, filled by TMA):
+//   A K-major : box (64 k, 128 m)   -> [128 rows][128 B], SBO = 1024 B
+//   A MN-major: 2 boxes (64 m, 64 k) -> [64 k rows][128 B] per 64-m half, LBO = 8 KiB
+//   X         : box (64 k, 1, n_pad) -> [n_pad rows][128 B], SBO = 1024 B
+#pragma once
+#include "ptx_sm100.cuh"
+
+namespace mla {
+namespace sk {
+
+constexpr int kThreads = 192;
+constexpr uint32_t kATileBytes = 128 * 64 * 2;
+constexpr int kRopePairs = 32;  // d_rope / 2
+
+struct Params {
+  int m_total;        // rows per group
+  int m_tiles;        // 128-row tiles per group
+  int groups;         // independent products (heads) sharing the launch
+  int a1_tile_start;  // tiles (within a group) >= this read map A1, rows relative to it
+  int k_blocks;       // 64-wide K blocks per tile
+  int n_pad;          // MMA N (multiple of 16, <= 256)
+  int n_lo;           // > 0: columns [n_lo, 2 n_lo) hold the low halves of columns [0, n_lo)
+  int n_out;          // valid output columns (the batch)
+  int a_mn_major;     // 0: A K-major, 1: A MN-major
+  int stages;         // shared-memory ring depth
+  int max_slots;      // partial slots per tile
+  long long iters;    // m_tiles * groups * k_blocks
+  uint32_t epoch;     // launch tag for the tile counters (never 0)
+  float* partial;     // [tiles][max_slots][n_pad][128]
+  unsigned long long* counters;  // [tiles]
+  const int32_t* positions;      // RoPE positions [n_out] (products with RoPE rows)
+  float rope_theta;
+  unsigned int* status;
+  uint64_t wait_ns;
+};
+
+__host__ __device__ inline uint32_t stage_bytes(int n_pad) {
+  return kATileBytes + static_cast<uint32_t>(n_pad) * 128u;
+}
+
+// First iteration of CTA c's range, and the CTA whose range holds iteration i.
+__host__ __device__ inline long long range_start(long long c, long long iters, long long ctas) {
+  return c * iters / ctas;
+}
+__host__ __device__ inline int cta_of(long long i, long long iters, long long ctas) {
+  return static_cast<int>(((i + 1) * ctas - 1) / iters);
+}
+
+// Count this contributor in on the tile counter; returns the count including itself.
+__device__ __forceinline__ uint32_t count_in(unsigned long long* ctr, uint32_t epoch,
+                                             unsigned int* status) {
+  unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(ctr);
+  for (int it = 0; it < (1 << 20); ++it) {
+    const unsigned long long nv = (static_cast<uint32_t>(cur >> 32) == epoch)
+                                      ? cur + 1ull
+                                      : ((static_cast<unsigned long long>(epoch) << 32) | 1ull);
+    const unsigned long long prev = atomicCAS(ctr, cur, nv);
+    if (prev == cur) return static_cast<uint32_t>(nv);
+    cur = prev;
+  }
+  atomicOr(status, MLA_STATUS_TIMEOUT);
+  return 0;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Epilogues.  apply() is called by all 32 lanes of a warp together (lane = tile row), for 16
+// output columns c0 .. c0+15 of row r of group g; v[j] is the finished value of column c0 + j.
+// RoPE rows exchange their pair partner with the neighbouring lane (pairs are (even, odd)
+// rows, and a warp's 32 rows never straddle a RoPE boundary).
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ void rope_rotate(const float2* tab, int b, int pair, bool odd,
+                                            float v, float partner, float& out) {
+  const float2 cs = tab[b * kRopePairs + pair];
+  // (x0, x1) -> (x0 c - x1 s, x0 s + x1 c); this lane holds x1 when odd.
+  out = odd ? (partner * cs.y + v * cs.x) : (v * cs.x - partner * cs.y);
+}
+
+// Cache append: rows 0..511 = c_KV, 512..575 = k_R (rotated); scattered into the page slot.
+struct EpiAppend {
+  static constexpr bool kRope = true;
+  const int32_t* positions;
+  const int32_t* page_table;
+  int max_pages;
+  __nv_bfloat16* pool;
+  int num_pages;
+  unsigned int* status;
+  __device__ void apply(const float2* tab, int, int r, bool valid, int c0, int n_out,
+                        float (&v)[16]) const {
+    constexpr int kRow = 576, kDc = 512, kPage = 64;
+    const bool rope = r >= kDc;  // warp-uniform
+    float p[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) p[j] = __shfl_xor_sync(0xffffffffu, v[j], 1);
+    if (!valid) return;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int b = c0 + j;
+      if (b >= n_out) break;
+      const int pos = positions[b];
+      if (pos < 0 || pos >= max_pages * kPage) {
+        atomicOr(status, MLA_STATUS_BAD_POSITION);
+        continue;
+      }
+      const int page = page_table[static_cast<size_t>(b) * max_pages + pos / kPage];
+      if (page < 0 || page >= num_pages) {
+        atomicOr(status, MLA_STATUS_BAD_PAGE);
+        continue;
+      }
+      float x = v[j];
+      if (rope) rope_rotate(tab, b, (r - kDc) >> 1, r & 1, v[j], p[j], x);
+      pool[(static_cast<size_t>(page) * kPage + pos % kPage) * kRow + r] = __float2bfloat16_rn(x);
+    }
+  }
+};
+
+// q = W_Q h: per head rows 0..127 -> q_nope as bf16 hi/lo planes [2][n_lo_pad][H][128],
+// rows 128..191 -> RoPE(q_rope) into q_cat[b][h][512..575] (+ its bf16 remainder in q_lo).
+struct EpiWq {
+  static constexpr bool kRope = true;
+  int H;
+  int b_pad;  // rows per hi/lo plane
+  __nv_bfloat16* q_cat;
+  __nv_bfloat16* q_lo;
+  __nv_bfloat16* qn;
+  __device__ void apply(const float2* tab, int, int r, bool valid, int c0, int n_out,
+                        float (&v)[16]) const {
+    constexpr int kDn = 128, kDq = 192, kRow = 576, kDc = 512;
+    const int h = r / kDq, d = r - h * kDq;
+    const bool rope = d >= kDn;  // warp-uniform
+    float p[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) p[j] = __shfl_xor_sync(0xffffffffu, v[j], 1);
+    if (!valid) return;
+    const size_t plane = static_cast<size_t>(b_pad) * H * kDn;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int b = c0 + j;
+      if (b >= n_out) break;
+      if (!rope) {
+        const size_t o = (static_cast<size_t>(b) * H + h) * kDn + d;
+        const __nv_bfloat16 hi = __float2bfloat16_rn(v[j]);
+        qn[o] = hi;
+        qn[plane + o] = __float2bfloat16_rn(v[j] - __bfloat162float(hi));
+      } else {
+        float x;
+        rope_rotate(tab, b, (d - kDn) >> 1, d & 1, v[j], p[j], x);
+        const size_t o = (static_cast<size_t>(b) * H + h) * kRow + kDc + (d - kDn);
+        const __nv_bfloat16 e = __float2bfloat16_rn(x);
+        q_cat[o] = e;
+        if (q_lo) q_lo[o] = __float2bfloat16_rn(x - __bfloat162float(e));
+      }
+    }
+  }
+};
+
+// q_lat_h = W_UK_h^T q_nope_h (hi + lo already summed) -> q_cat[b][h][0..511] (+ q_lo).
+struct EpiWuk {
+  static constexpr bool kRope = false;
+  int H;
+  __nv_bfloat16* q_cat;
+  __nv_bfloat16* q_lo;
+  __device__ void apply(const float2*, int g, int r, bool valid, int c0, int n_out,
+                        float (&v)[16]) const {
+    constexpr int kRow = 576;
+    if (!valid) return;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int b = c0 + j;
+      if (b >= n_out) break;
+      const size_t o = (static_cast<size_t>(b) * H + g) * kRow + r;
+      const __nv_bfloat16 e = __float2bfloat16_rn(v[j]);
+      q_cat[o] = e;
+      if (q_lo) q_lo[o] = __float2bfloat16_rn(v[j] - __bfloat162float(e));
+    }
+  }
+};
+
+// o_h = W_UV_h o_lat_h -> o_heads[b][h][0..127] and/or bf16 hi/lo planes [2][b_pad][H*128].
+struct EpiWuv {
+  static constexpr bool kRope = false;
+  int H;
+  int b_pad;
+  __nv_bfloat16* o_heads;
+  __nv_bfloat16* oh;
+  __device__ void apply(const float2*, int g, int r, bool valid, int c0, int n_out,
+                        float (&v)[16]) const {
+    constexpr int kDv = 128;
+    if (!valid) return;
+    const size_t plane = static_cast<size_t>(b_pad) * H * kDv;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int b = c0 + j;
+      if (b >= n_out) break;
+      const size_t o = (static_cast<size_t>(b) * H + g) * kDv + r;
+      const __nv_bfloat16 hi = __float2bfloat16_rn(v[j]);
+      if (o_heads) o_heads[o] = hi;
+      if (oh) {
+        oh[o] = hi;
+        oh[plane + o] = __float2bfloat16_rn(v[j] - __bfloat162float(hi));
+      }
+    }
+  }
+};
+
+// out = W_O [o_1 .. o_H] -> out[b][0..D-1].
+struct EpiWo {
+  static constexpr bool kRope = false;
+  int D;
+  __nv_bfloat16* out;
+  __device__ void apply(const float2*, int, int r, bool valid, int c0, int n_out,
+                        float (&v)[16]) const {
+    if (!valid) return;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int b = c0 + j;
+      if (b >= n_out) break;
+      out[static_cast<size_t>(b) * D + r] = __float2bfloat16_rn(v[j]);
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------------------------
+template <class Epi>
+__global__ void __launch_bounds__(kThreads, 1)
+    streamk_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,
+                        const __grid_constant__ CUtensorMap tmA1,
+                        const __grid_constant__ CUtensorMap tmX, const Params p, const Epi epi) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sbytes = stage_bytes(p.n_pad);
+  float2* rope_tab = reinterpret_cast<float2*>(smem + p.stages * sbytes);
+  const int tab_entries = Epi::kRope ? p.n_out * kRopePairs : 0;
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(
+      smem + p.stages * sbytes + ((tab_entries * 8 + 15) & ~15));
+  uint64_t* empty_bar = full_bar + p.stages;
+  uint64_t* acc_full = empty_bar + p.stages;   // [2]
+  uint64_t* acc_empty = acc_full + 2;          // [2], 4 arrivals (one per epilogue warp)
+  uint64_t* epi_sync = acc_empty + 2;          // 4 arrivals
+  uint64_t* fin_ready = epi_sync + 1;          // 1 arrival
+  uint64_t* mma_done = fin_ready + 1;          // final drain of the MMA pipe
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* fin_flag = abort_flag + 1;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long c = blockIdx.x;
+  const long long P = gridDim.x;
+  const long long i_begin = range_start(c, p.iters, P);
+  const long long i_end = range_start(c + 1, p.iters, P);
+  const long long kb = p.k_blocks;
+  uint32_t tmem_cols = 32;
+  while (tmem_cols < 2u * static_cast<uint32_t>(p.n_pad)) tmem_cols <<= 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.stages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);
+    }
+    mbar_init(epi_sync, 4);
+    mbar_init(fin_ready, 1);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    *fin_flag = 0;
+    fence_mbar_init_cluster();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, tmem_cols);
+    tmem_relinquish();
+  }
+  if (Epi::kRope) {
+    // cos/sin of pos_b * theta^(-2i/64) for every (column b, pair i), in double precision
+    for (int e = threadIdx.x; e < tab_entries; e += kThreads) {
+      const int b = e / kRopePairs, i = e - b * kRopePairs;
+      const double inv_freq = pow(static_cast<double>(p.rope_theta), -2.0 * i / (2 * kRopePairs));
+      double sn, cs;
+      sincos(static_cast<double>(p.positions[b]) * inv_freq, &sn, &cs);
+      rope_tab[e] = make_float2(static_cast<float>(cs), static_cast<float>(sn));
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  WaitCtx wc{abort_flag, p.status, p.wait_ns};
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      tma_prefetch_desc(&tmA0);
+      tma_prefetch_desc(&tmA1);
+      tma_prefetch_desc(&tmX);
+      const uint64_t pol_w = l2_policy_evict_first();
+      const uint64_t pol_x = l2_policy_evict_last();
+      long long issued = 0;
+      for (long long i = i_begin; i < i_end; ++i, ++issued) {
+        const int s = static_cast<int>(issued % p.stages);
+        const uint32_t ph = static_cast<uint32_t>((issued / p.stages) & 1);
+        if (issued >= p.stages && !mbar_wait(&empty_bar[s], ph ^ 1, wc)) break;
+        const long long t = i / kb;
+        const int kbi = static_cast<int>(i - t * kb);
+        const int g = static_cast<int>(t / p.m_tiles);
+        const int mt = static_cast<int>(t - static_cast<long long>(g) * p.m_tiles);
+        const bool use_a1 = mt >= p.a1_tile_start;
+        const CUtensorMap* tmA = use_a1 ? &tmA1 : &tmA0;
+        const int m_row0 = (use_a1 ? mt - p.a1_tile_start : mt) * 128;
+        uint8_t* a_dst = smem + s * sbytes;
+        uint8_t* x_dst = a_dst + kATileBytes;
+        mbar_arrive_expect_tx(&full_bar[s], sbytes);
+        const int k0 = kbi * 64;
+        if (p.a_mn_major) {
+          tma_load_3d_hint(a_dst, tmA, &full_bar[s], m_row0, k0, g, pol_w);
+          tma_load_3d_hint(a_dst + 8192, tmA, &full_bar[s], m_row0 + 64, k0, g, pol_w);
+        } else {
+          tma_load_3d_hint(a_dst, tmA, &full_bar[s], k0, m_row0, g, pol_w);
+        }
+        tma_load_3d_hint(x_dst, &tmX, &full_bar[s], k0, g, 0, pol_x);
+      }
+      if (*abort_flag) {
+        // wait (bounded, ignoring the abort flag) for every copy still landing in the ring
+        volatile int never = 0;
+        WaitCtx drain{&never, p.status, p.wait_ns};
+        for (long long j = (issued > p.stages ? issued - p.stages : 0); j < issued; ++j)
+          mbar_wait(&full_bar[j % p.stages], static_cast<uint32_t>((j / p.stages) & 1), drain);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(128, p.n_pad, p.a_mn_major, 0);
+      long long it = 0;  // iteration counter (ring position)
+      int seg = 0;
+      bool ok = true;
+      for (long long i = i_begin; i < i_end && ok; ++seg) {
+        const long long t = i / kb;
+        const long long seg_end = min(i_end, (t + 1) * kb);
+        const int buf = seg & 1;
+        if (!mbar_wait(&acc_empty[buf], static_cast<uint32_t>(((seg >> 1) & 1) ^ 1), wc)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * p.n_pad);
+        for (; i < seg_end; ++i, ++it) {
+          const int s = static_cast<int>(it % p.stages);
+          if (!mbar_wait(&full_bar[s], static_cast<uint32_t>((it / p.stages) & 1), wc)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(smem + s * sbytes);
+          const uint32_t x_base = a_base + kATileBytes;
+          const bool first = (i == t * kb) || (i == i_begin);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t adesc = p.a_mn_major
+                                       ? smem_desc(a_base + kk * 2048, 8192, 1024, kSwizzle128B)
+                                       : smem_desc(a_base + kk * 32, 16, 1024, kSwizzle128B);
+            const uint64_t xdesc = smem_desc(x_base + kk * 32, 16, 1024, kSwizzle128B);
+            mma_ss(d_tmem, adesc, xdesc, idesc, (first && kk == 0) ? 0u : 1u);
+          }
+          mma_commit(&empty_bar[s]);
+        }
+        if (ok) mma_commit(&acc_full[buf]);
+      }
+      mma_commit(mma_done);  // fires once every issued MMA has completed
+    }
+  } else {
+    // ---------------- epilogue ----------------
+    const int quarter = warp & 3;
+    const int m_local = quarter * 32 + lane;
+    const int n_cols = p.n_lo > 0 ? p.n_lo : p.n_pad;  // columns that are outputs
+    int seg = 0, multi = 0;
+    for (long long i = i_begin; i < i_end; ++seg) {
+      const long long t = i / kb;
+      const long long seg_end = min(i_end, (t + 1) * kb);
+      i = seg_end;
+      const int g = static_cast<int>(t / p.m_tiles);
+      const int mt = static_cast<int>(t - static_cast<long long>(g) * p.m_tiles);
+      const int r = mt * 128 + m_local;
+      const bool valid = r < p.m_total;
+      const int c_first = cta_of(t * kb, p.iters, P);
+      const int c_last = cta_of((t + 1) * kb - 1, p.iters, P);
+      const int buf = seg & 1;
+      if (!warp_wait(&acc_full[buf], static_cast<uint32_t>((seg >> 1) & 1), wc)) break;
+      tc_fence_after();
+      const uint32_t tacc = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                            static_cast<uint32_t>(buf * p.n_pad);
+      if (c_first == c_last) {
+        // whole tile in this CTA: finish from TMEM
+        for (int c0 = 0; c0 < n_cols; c0 += 16) {
+          uint32_t a[16];
+          float v[16];
+          tmem_ld16(tacc + c0, a);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(a[j]);
+          if (p.n_lo > 0) {
+            tmem_ld16(tacc + p.n_lo + c0, a);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] += __uint_as_float(a[j]);
+          }
+          epi.apply(rope_tab, g, r, valid, c0, p.n_out, v);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        continue;
+      }
+      // shared tile: publish this CTA's partial, count in, finish if last
+      const int slot = static_cast<int>(c - c_first);
+      const int n_contrib = c_last - c_first + 1;
+      float* part_tile =
+          p.partial + static_cast<size_t>(t) * p.max_slots * p.n_pad * 128 + m_local;
+      {
+        float* dst = part_tile + static_cast<size_t>(slot) * p.n_pad * 128;
+        for (int c0 = 0; c0 < p.n_pad; c0 += 16) {
+          uint32_t a[16];
+          tmem_ld16(tacc + c0, a);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) __stcg(dst + (c0 + j) * 128, __uint_as_float(a[j]));
+        }
+      }
+      tc_fence_before();
+      __threadfence();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&acc_empty[buf]);
+        mbar_arrive(epi_sync);
+      }
+      const uint32_t ph = static_cast<uint32_t>(multi & 1);
+      ++multi;
+      if (warp == 2 && lane == 0) {
+        int fin = 0;
+        if (mbar_wait(epi_sync, ph, wc)) {
+          const uint32_t n = count_in(&p.counters[t], p.epoch, p.status);
+          fin = (n == static_cast<uint32_t>(n_contrib)) ? 1 : 0;
+          __threadfence();
+        }
+        *fin_flag = fin;
+        mbar_arrive(fin_ready);
+      }
+      if (!warp_wait(fin_ready, ph, wc)) break;
+      if (!*fin_flag) continue;
+      for (int c0 = 0; c0 < n_cols; c0 += 16) {
+        float v[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] = __ldcg(part_tile + (c0 + j) * 128);
+        for (int s = 1; s < n_contrib; ++s) {
+          const float* src = part_tile + static_cast<size_t>(s) * p.n_pad * 128;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[j] += __ldcg(src + (c0 + j) * 128);
+        }
+        if (p.n_lo > 0) {
+          float w[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) w[j] = __ldcg(part_tile + (p.n_lo + c0 + j) * 128);
+          for (int s = 1; s < n_contrib; ++s) {
+            const float* src = part_tile + static_cast<size_t>(s) * p.n_pad * 128;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) w[j] += __ldcg(src + (p.n_lo + c0 + j) * 128);
+          }
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[j] += w[j];
+        }
+        epi.apply(rope_tab, g, r, valid, c0, p.n_out, v);
+      }
+    }
+  }
+
+  // Never release TMEM while issued MMAs may still write it.
+  if (warp == 1 && lane == 0) {
+    volatile int never = 0;
+    WaitCtx drain{&never, p.status, p.wait_ns};
+    mbar_wait(mma_done, 0, drain);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, tmem_cols);
+  }
+}
+
+}  // namespace sk
+}  // namespace mla

@@ -14,7 +14,7 @@
 #include "attn_f32.cuh"
 #include "attn_sm100.cuh"
 #include "epilogue.cuh"
-#include "gemm_sm100.cuh"
+#include "gemm_streamk.cuh"
 
 namespace mla {
 
@@ -25,8 +25,9 @@ namespace {
 constexpr int kDc = 512, kDr = 64, kDn = 128, kDv = 128, kRowN = 576, kPageN = 64;
 constexpr uint64_t kDefaultWaitNs = 2000000000ull;  // 2 s per bounded wait
 constexpr int kMinPagesPerPart = 4;
-constexpr int kMaxKSplits = 32;
-constexpr uint32_t kGemmSmemBudget = 200 * 1024;
+constexpr int kSkMinIters = 8;            // fewest K blocks a stream-K CTA streams
+constexpr int kSkMaxStages = 12;
+constexpr size_t kSmemPerBlockMax = 232448;  // 227 KiB opt-in limit per CTA
 
 // ------------------------------------------------------------------------------------------
 // validation
@@ -98,8 +99,17 @@ int device_ctx(DevCtx** out) {
     if (cudaFuncSetAttribute(attn::split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              attn_smem) != cudaSuccess)
       return MLA_ERR_CUDA;
-    if (cudaFuncSetAttribute(gemm_swapab_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kGemmSmemBudget + 2048)) != cudaSuccess)
+    const int sk_smem = static_cast<int>(kSmemPerBlockMax);
+    if (cudaFuncSetAttribute(sk::streamk_gemm_kernel<sk::EpiAppend>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, sk_smem) != cudaSuccess ||
+        cudaFuncSetAttribute(sk::streamk_gemm_kernel<sk::EpiWq>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, sk_smem) != cudaSuccess ||
+        cudaFuncSetAttribute(sk::streamk_gemm_kernel<sk::EpiWuk>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, sk_smem) != cudaSuccess ||
+        cudaFuncSetAttribute(sk::streamk_gemm_kernel<sk::EpiWuv>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, sk_smem) != cudaSuccess ||
+        cudaFuncSetAttribute(sk::streamk_gemm_kernel<sk::EpiWo>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, sk_smem) != cudaSuccess)
       return MLA_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2, 1, 1);
@@ -121,61 +131,92 @@ int default_parts(int sms, int max_clusters) { return max_clusters > 0 ? max_clu
 // ------------------------------------------------------------------------------------------
 // GEMM configuration
 // ------------------------------------------------------------------------------------------
-int n_pad_for(int rows) { return std::max(16, (rows + 15) / 16 * 16); }
+int round16(int x) { return (x + 15) / 16 * 16; }
 
-int choose_k_splits(int tiles, int k_blocks, int sms) {
-  int best = 1;
-  double best_eff = 0.0;
-  const int max_s = std::max(1, std::min(kMaxKSplits, k_blocks / 2));
-  for (int s = 1; s <= max_s; ++s) {
-    const int ctas = tiles * s;
-    const int waves = (ctas + sms - 1) / sms;
-    const double eff = static_cast<double>(ctas) / (static_cast<double>(waves) * sms);
-    if (eff > best_eff + 0.02) {
-      best = s;
-      best_eff = eff;
-    }
-  }
-  return best;
-}
-
+// One weight product of a layer: rows per group, 128-row tiles per group, K, groups, and the
+// activation columns (n_pad on the MMA's N side; n_lo > 0 when columns [n_lo, 2 n_lo) carry the
+// bf16 low halves of an fp32 input).
 struct GemmShape {
-  int m_total, m_tiles, k, groups, n_rows;
+  int m_total, m_tiles, k, groups, n_pad, n_lo;
   int k_blocks() const { return (k + 63) / 64; }
 };
 
-// the five products of a layer (bf16 path; the fp32 path uses k_splits = 1)
-GemmShape shape_append(const mla_dims* d) { return {kRowN, 5, d->d_model, 1, d->batch}; }
-GemmShape shape_wq(const mla_dims* d) {
-  return {d->n_heads * (kDn + kDr), d->n_heads * (kDn + kDr) / 128, d->d_model, 1, d->batch};
+// the five products of a layer on the bf16 path
+GemmShape shape_append(const mla_dims* d) {
+  return {kRowN, 5, d->d_model, 1, round16(d->batch), 0};
 }
-GemmShape shape_wuk(const mla_dims* d) { return {kDc, kDc / 128, kDn, d->n_heads, 2 * d->batch}; }
-GemmShape shape_wuv(const mla_dims* d) { return {kDv, 1, kDc, d->n_heads, 2 * d->batch}; }
+GemmShape shape_wq(const mla_dims* d) {
+  const int m = d->n_heads * (kDn + kDr);
+  return {m, m / 128, d->d_model, 1, round16(d->batch), 0};
+}
+GemmShape shape_wuk(const mla_dims* d) {
+  return {kDc, kDc / 128, kDn, d->n_heads, 2 * round16(d->batch), round16(d->batch)};
+}
+GemmShape shape_wuv(const mla_dims* d) {
+  return {kDv, 1, kDc, d->n_heads, 2 * round16(d->batch), round16(d->batch)};
+}
 GemmShape shape_wo(const mla_dims* d) {
-  return {d->d_model, (d->d_model + 127) / 128, d->n_heads * kDv, 1, 2 * d->batch};
+  return {d->d_model, (d->d_model + 127) / 128, d->n_heads * kDv, 1, 2 * round16(d->batch),
+          round16(d->batch)};
 }
 
-size_t partial_bytes(const GemmShape& s, int sms) {
-  const int ks = choose_k_splits(s.m_tiles * s.groups, s.k_blocks(), sms);
-  return static_cast<size_t>(ks) * s.groups * s.m_total * n_pad_for(s.n_rows) * sizeof(float);
+// Stream-K launch plan: CTAs, partial slots per tile, ring depth, shared memory.
+struct SkPlan {
+  int ctas = 1, max_slots = 1, stages = 2, tiles = 0;
+  long long iters = 0;
+  size_t smem = 0, partial_bytes = 0;
+};
+
+SkPlan sk_plan(const GemmShape& s, bool rope, int n_out, int sms) {
+  SkPlan q;
+  q.tiles = s.m_tiles * s.groups;
+  const long long kb = s.k_blocks();
+  q.iters = static_cast<long long>(q.tiles) * kb;
+  long long P = std::min<long long>(sms, (q.iters + kSkMinIters - 1) / kSkMinIters);
+  P = std::max<long long>(1, std::min(P, q.iters));
+  q.ctas = static_cast<int>(P);
+  for (long long t = 0; t < q.tiles; ++t) {
+    const int cf = sk::cta_of(t * kb, q.iters, P), cl = sk::cta_of((t + 1) * kb - 1, q.iters, P);
+    q.max_slots = std::max(q.max_slots, cl - cf + 1);
+  }
+  const size_t tab = rope ? (static_cast<size_t>(n_out) * sk::kRopePairs * 8 + 15) / 16 * 16 : 0;
+  const size_t fixed = 1024 + tab + 256;  // alignment slack, RoPE table, barriers and flags
+  const size_t sb = sk::stage_bytes(s.n_pad);
+  q.stages = static_cast<int>(std::min<size_t>(kSkMaxStages, (kSmemPerBlockMax - fixed) / sb));
+  q.smem = fixed + static_cast<size_t>(q.stages) * sb;
+  q.partial_bytes = q.max_slots > 1 ? static_cast<size_t>(q.tiles) * q.max_slots * s.n_pad *
+                                          128 * sizeof(float)
+                                    : 0;
+  return q;
+}
+
+std::atomic<uint32_t> g_sk_epoch{0x5EED0000u};
+uint32_t next_epoch() {
+  uint32_t e = g_sk_epoch.fetch_add(1, std::memory_order_relaxed) + 1;
+  if (e == 0) e = g_sk_epoch.fetch_add(1, std::memory_order_relaxed) + 1;
+  return e;
 }
 
 // ------------------------------------------------------------------------------------------
 // workspace layout
 // ------------------------------------------------------------------------------------------
 struct Workspace {
-  size_t partial, qn, o_split, oh_split, plan, part_o, part_lse, total;
+  size_t partial, counters, qn, o_split, oh_split, plan, part_o, part_lse, total;
 };
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 Workspace layout(const mla_dims* d, int num_parts, int sms) {
-  const size_t B = d->batch, H = d->n_heads;
-  size_t part = 0;
+  const size_t B = d->batch, H = d->n_heads, Bp = round16(d->batch);
+  size_t part = 0, ctr = 0;
   if (d->dtype == MLA_BF16) {
-    part = std::max({partial_bytes(shape_append(d), sms), partial_bytes(shape_wq(d), sms),
-                     partial_bytes(shape_wuk(d), sms), partial_bytes(shape_wuv(d), sms),
-                     partial_bytes(shape_wo(d), sms)});
+    const GemmShape shapes[5] = {shape_append(d), shape_wq(d), shape_wuk(d), shape_wuv(d),
+                                 shape_wo(d)};
+    for (const GemmShape& s : shapes) {
+      const SkPlan q = sk_plan(s, true, d->batch, sms);
+      part = std::max(part, q.partial_bytes);
+      ctr = std::max(ctr, static_cast<size_t>(q.tiles) * 8);
+    }
   } else {
     part = std::max({static_cast<size_t>(kRowN) * B, H * (kDn + kDr) * B, H * kDc * B,
                      H * kDv * B, static_cast<size_t>(d->d_model) * B}) *
@@ -189,9 +230,10 @@ Workspace layout(const mla_dims* d, int num_parts, int sms) {
     return o;
   };
   w.partial = take(part);
-  w.qn = take(2 * B * H * kDn * 4);        // bf16 hi/lo planes, or fp32
-  w.o_split = take(2 * B * H * kDc * 2);   // bf16 hi/lo of o_lat
-  w.oh_split = take(2 * B * H * kDv * 4);  // bf16 hi/lo, or fp32
+  w.counters = take(ctr);
+  w.qn = take(std::max(2 * Bp * H * kDn * 2, B * H * kDn * 4));      // bf16 hi/lo, or fp32
+  w.o_split = take(2 * Bp * H * kDc * 2);                             // bf16 hi/lo of o_lat
+  w.oh_split = take(std::max(2 * Bp * H * kDv * 2, B * H * kDv * 4)); // bf16 hi/lo, or fp32
   w.plan = take(attn::PlanView::words(static_cast<int>(B), num_parts) * 4);
   w.part_o = take((B + num_parts) * H * kDc * 4);
   w.part_lse = take((B + num_parts) * H * 4);
@@ -252,33 +294,34 @@ int last_launch(int kernels = 1) {
   return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
-int gemm_stages(int n_pad) {
-  const uint32_t sb = gemm_stage_bytes(n_pad);
-  return std::max(2, std::min(8, static_cast<int>(kGemmSmemBudget / sb)));
-}
-
-// P[ks][g][m][n] for one product on tensor cores.
-int run_gemm(const DevCtx* c, const GemmShape& s, const CUtensorMap& a0, const CUtensorMap& a1,
-             int a1_tile_start, int a_mn_major, const CUtensorMap& bmap, float* partial,
-             cudaStream_t st, int* k_splits_out) {
-  GemmParams p{};
+// One weight product on the tensor cores, its epilogue fused (stream-K, see gemm_streamk.cuh).
+template <class Epi>
+int run_streamk(const DevCtx* c, const GemmShape& s, int n_out, const int32_t* positions,
+                float theta, const CUtensorMap& a0, const CUtensorMap& a1, int a1_tile_start,
+                int a_mn_major, const CUtensorMap& xmap, char* ws, const Workspace& w,
+                const Epi& epi, cudaStream_t st) {
+  const SkPlan q = sk_plan(s, Epi::kRope, n_out, c->sms);
+  sk::Params p{};
   p.m_total = s.m_total;
   p.m_tiles = s.m_tiles;
+  p.groups = s.groups;
   p.a1_tile_start = a1_tile_start;
   p.k_blocks = s.k_blocks();
-  p.k_splits = choose_k_splits(s.m_tiles * s.groups, p.k_blocks, c->sms);
-  p.n_pad = n_pad_for(s.n_rows);
+  p.n_pad = s.n_pad;
+  p.n_lo = s.n_lo;
+  p.n_out = n_out;
   p.a_mn_major = a_mn_major;
-  p.stages = gemm_stages(p.n_pad);
-  p.groups = s.groups;
-  p.partial = partial;
+  p.stages = q.stages;
+  p.max_slots = q.max_slots;
+  p.iters = q.iters;
+  p.epoch = next_epoch();
+  p.partial = reinterpret_cast<float*>(ws + w.partial);
+  p.counters = reinterpret_cast<unsigned long long*>(ws + w.counters);
+  p.positions = positions;
+  p.rope_theta = theta;
   p.status = c->status;
   p.wait_ns = kDefaultWaitNs;
-  const size_t smem = static_cast<size_t>(p.stages) * gemm_stage_bytes(p.n_pad) +
-                      (2 * p.stages + 1) * 8 + 16 + 1024;
-  gemm_swapab_kernel<<<dim3(s.m_tiles, p.k_splits, s.groups), kGemmThreads, smem, st>>>(
-      a0, a1, bmap, p);
-  *k_splits_out = p.k_splits;
+  sk::streamk_gemm_kernel<Epi><<<q.ctas, sk::kThreads, q.smem, st>>>(a0, a1, xmap, p, epi);
   return last_launch();
 }
 
@@ -339,19 +382,18 @@ int mla_cache_append(const mla_dims* dims, const void* h, const void* w_dkv, con
   }
   const Workspace w = layout(dims, resolve_parts(0, c), c->sms);
   if (workspace_bytes < w.total) return MLA_ERR_WORKSPACE;
-  float* part = reinterpret_cast<float*>(static_cast<char*>(workspace) + w.partial);
+  char* ws = static_cast<char*>(workspace);
+  float* part = reinterpret_cast<float*>(ws + w.partial);
   if (dims->dtype == MLA_BF16) {
     const GemmShape s = shape_append(dims);
-    const int n_pad = n_pad_for(s.n_rows);
     CUtensorMap a0, a1, bm;
     if ((rc = map3(&a0, w_dkv, D, kDc, 1, D * 2ull, D * 2ull * kDc, 64, 128, 1))) return rc;
     if ((rc = map3(&a1, w_kr, D, kDr, 1, D * 2ull, D * 2ull * kDr, 64, 128, 1))) return rc;
-    if ((rc = map3(&bm, h, D, 1, B, D * 2ull, D * 2ull, 64, 1, n_pad))) return rc;
-    int ks = 1;
-    if ((rc = run_gemm(c, s, a0, a1, kDc / 128, 0, bm, part, st, &ks))) return rc;
-    append_epilogue_kernel<__nv_bfloat16><<<eg, 96, 0, st>>>(
-        part, ks, n_pad, nullptr, positions, page_table, max_pages,
-        static_cast<__nv_bfloat16*>(cache_pool), num_pages, dims->rope_theta, c->status);
+    if ((rc = map3(&bm, h, D, 1, B, D * 2ull, D * 2ull, 64, 1, s.n_pad))) return rc;
+    sk::EpiAppend e{positions, page_table, max_pages, static_cast<__nv_bfloat16*>(cache_pool),
+                    num_pages, c->status};
+    return run_streamk(c, s, B, positions, dims->rope_theta, a0, a1, kDc / 128, 0, bm, ws, w, e,
+                       st);
   } else {
     // fp32: rows 0..511 from W_DKV, 512..575 from W_KR, written as one [576][B] partial
     f32_gemm_k_kernel<<<dim3(kDc / 8, 1), 256, 0, st>>>(static_cast<const float*>(w_dkv), 0, D,
@@ -394,26 +436,25 @@ int mla_absorb_q(const mla_dims* dims, const void* h, const void* w_q, const voi
   if (dims->dtype == MLA_BF16) {
     __nv_bfloat16* qc = static_cast<__nv_bfloat16*>(q_cat);
     __nv_bfloat16* ql = static_cast<__nv_bfloat16*>(q_lo);
-    // q = W_Q h
+    // q = W_Q h -> q_nope hi/lo planes [2][Bp][H][128] and RoPE(q_rope) into q_cat
     const GemmShape s1 = shape_wq(dims);
-    const int np1 = n_pad_for(s1.n_rows);
+    const int Bp = s1.n_pad;
     CUtensorMap a, bm;
     if ((rc = map3(&a, w_q, D, s1.m_total, 1, D * 2ull, D * 2ull * s1.m_total, 64, 128, 1)))
       return rc;
-    if ((rc = map3(&bm, h, D, 1, B, D * 2ull, D * 2ull, 64, 1, np1))) return rc;
-    int ks = 1;
-    if ((rc = run_gemm(c, s1, a, a, 1 << 30, 0, bm, part, st, &ks))) return rc;
-    wq_epilogue_kernel<__nv_bfloat16><<<dim3(H, B), 96, 0, st>>>(part, ks, np1, B, H, positions,
-                                                                 theta, qc, ql, qn);
-    if ((rc = last_launch())) return rc;
+    if ((rc = map3(&bm, h, D, 1, B, D * 2ull, D * 2ull, 64, 1, s1.n_pad))) return rc;
+    __nv_bfloat16* qnb = static_cast<__nv_bfloat16*>(qn);
+    sk::EpiWq e1{H, Bp, qc, ql, qnb};
+    if ((rc = run_streamk(c, s1, B, positions, theta, a, a, 1 << 30, 0, bm, ws, w, e1, st)))
+      return rc;
     // q_lat_h = W_UK_h^T [q_nope_hi | q_nope_lo]   (A MN-major: W_UK rows are the K side)
     const GemmShape s2 = shape_wuk(dims);
-    const int np2 = n_pad_for(s2.n_rows);
     CUtensorMap a2, b2;
     if ((rc = map3(&a2, w_uk, kDc, kDn, H, kDc * 2ull, kDc * 2ull * kDn, 64, 64, 1))) return rc;
-    if ((rc = map3(&b2, qn, kDn, H, 2 * B, kDn * 2ull, kDn * 2ull * H, 64, 1, np2))) return rc;
-    if ((rc = run_gemm(c, s2, a2, a2, 1 << 30, 1, b2, part, st, &ks))) return rc;
-    wuk_epilogue_kernel<__nv_bfloat16, true><<<dim3(H, B), 128, 0, st>>>(part, np2, B, H, qc, ql);
+    if ((rc = map3(&b2, qn, kDn, H, 2 * Bp, kDn * 2ull, kDn * 2ull * H, 64, 1, s2.n_pad)))
+      return rc;
+    sk::EpiWuk e2{H, qc, ql};
+    return run_streamk(c, s2, B, nullptr, theta, a2, a2, 1 << 30, 1, b2, ws, w, e2, st);
   } else {
     float* qc = static_cast<float*>(q_cat);
     const int M = H * (kDn + kDr);
@@ -541,32 +582,30 @@ int mla_out_proj(const mla_dims* dims, const float* o_lat, const void* w_uv, con
   void* oh_split = out ? static_cast<void*>(ws + w.oh_split) : nullptr;
   if (dims->dtype == MLA_BF16) {
     __nv_bfloat16* os = reinterpret_cast<__nv_bfloat16*>(ws + w.o_split);
+    const GemmShape s1 = shape_wuv(dims);
+    const int Bp = s1.n_lo;
     const size_t n = static_cast<size_t>(B) * H * kDc;
     split_hi_lo_kernel<<<static_cast<unsigned>(std::min<size_t>((n + 255) / 256, 4096)), 256, 0,
-                         st>>>(o_lat, n, os);
+                         st>>>(o_lat, n, static_cast<size_t>(Bp) * H * kDc, os);
     if ((rc = last_launch())) return rc;
     // o_h = W_UV_h [o_lat_hi | o_lat_lo]
-    const GemmShape s1 = shape_wuv(dims);
-    const int np1 = n_pad_for(s1.n_rows);
     CUtensorMap a, bm;
     if ((rc = map3(&a, w_uv, kDc, kDv, H, kDc * 2ull, kDc * 2ull * kDv, 64, 128, 1))) return rc;
-    if ((rc = map3(&bm, os, kDc, H, 2 * B, kDc * 2ull, kDc * 2ull * H, 64, 1, np1))) return rc;
-    int ks = 1;
-    if ((rc = run_gemm(c, s1, a, a, 1 << 30, 0, bm, part, st, &ks))) return rc;
-    wuv_epilogue_kernel<__nv_bfloat16, true><<<dim3(H, B), kDv, 0, st>>>(
-        part, ks, np1, B, H, static_cast<__nv_bfloat16*>(o_heads), oh_split);
-    if ((rc = last_launch())) return rc;
+    if ((rc = map3(&bm, os, kDc, H, 2 * Bp, kDc * 2ull, kDc * 2ull * H, 64, 1, s1.n_pad)))
+      return rc;
+    sk::EpiWuv e1{H, Bp, static_cast<__nv_bfloat16*>(o_heads),
+                  static_cast<__nv_bfloat16*>(oh_split)};
+    if ((rc = run_streamk(c, s1, B, nullptr, 0.f, a, a, 1 << 30, 0, bm, ws, w, e1, st)))
+      return rc;
     if (out) {
       const GemmShape s2 = shape_wo(dims);
-      const int np2 = n_pad_for(s2.n_rows);
       const uint64_t K = static_cast<uint64_t>(H) * kDv;
       CUtensorMap a2, b2;
       if ((rc = map3(&a2, w_o, K, D, 1, K * 2, K * 2 * D, 64, 128, 1))) return rc;
-      if ((rc = map3(&b2, oh_split, K, 1, 2 * B, K * 2, K * 2, 64, 1, np2))) return rc;
-      if ((rc = run_gemm(c, s2, a2, a2, 1 << 30, 0, b2, part, st, &ks))) return rc;
-      wo_epilogue_kernel<__nv_bfloat16, true><<<dim3((D + 255) / 256, B), 256, 0, st>>>(
-          part, ks, np2, B, D, static_cast<__nv_bfloat16*>(out));
-      if ((rc = last_launch())) return rc;
+      if ((rc = map3(&b2, oh_split, K, 1, 2 * Bp, K * 2, K * 2, 64, 1, s2.n_pad))) return rc;
+      sk::EpiWo e2{D, static_cast<__nv_bfloat16*>(out)};
+      if ((rc = run_streamk(c, s2, B, nullptr, 0.f, a2, a2, 1 << 30, 0, b2, ws, w, e2, st)))
+        return rc;
     }
   } else {
     f32_gemm_k_kernel<<<dim3(kDv / 8, H), 256, 0, st>>>(
