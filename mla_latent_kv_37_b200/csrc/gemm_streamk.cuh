@@ -42,15 +42,17 @@ struct Params {
   int groups;         // independent products (heads) sharing the launch
   int a1_tile_start;  // tiles (within a group) >= this read map A1, rows relative to it
   int k_blocks;       // 64-wide K blocks per tile
+  int kbs;            // K blocks per pipeline stage (one TMA box of A per stage)
+  int units;          // stages' worth of work per tile: ceil(k_blocks / kbs)
   int n_pad;          // MMA N (multiple of 16, <= 256)
   int n_lo;           // > 0: columns [n_lo, 2 n_lo) hold the low halves of columns [0, n_lo)
   int n_out;          // valid output columns (the batch)
   int a_mn_major;     // 0: A K-major, 1: A MN-major
   int stages;         // shared-memory ring depth
   int max_slots;      // partial slots per tile
-  long long iters;    // m_tiles * groups * k_blocks
+  long long iters;    // m_tiles * groups * units
   uint32_t epoch;     // launch tag for the tile counters (never 0)
-  float* partial;     // [tiles][max_slots][n_pad][128]
+  float* partial;     // [tiles][max_slots][n_pad / 4][128][4]
   unsigned long long* counters;  // [tiles]
   const int32_t* positions;      // RoPE positions [n_out] (products with RoPE rows)
   float rope_theta;
@@ -58,8 +60,10 @@ struct Params {
   uint64_t wait_ns;
 };
 
-__host__ __device__ inline uint32_t stage_bytes(int n_pad) {
-  return kATileBytes + static_cast<uint32_t>(n_pad) * 128u;
+// A stage holds kbs K blocks: A [kbs][128 rows][128 B] (K-major) or [2][64 kbs][128 B]
+// (MN-major), then X [kbs][n_pad][128 B].
+__host__ __device__ inline uint32_t stage_bytes(int n_pad, int kbs) {
+  return static_cast<uint32_t>(kbs) * (kATileBytes + static_cast<uint32_t>(n_pad) * 128u);
 }
 
 // First iteration of CTA c's range, and the CTA whose range holds iteration i.
@@ -243,6 +247,51 @@ struct EpiWo {
   }
 };
 
+// Sum of 16 columns of one row over slots 0 .. n-1, added in slot order.  src points at the
+// row's first float4 of the 16 columns in slot 0; four slots' loads are in flight at a time.
+__device__ __forceinline__ void sum_slots(const float4* src, size_t slot_stride, int n,
+                                          float (&v)[16]) {
+  float4 x[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) x[q] = __ldcg(src + q * 128);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    v[4 * q] = x[q].x;
+    v[4 * q + 1] = x[q].y;
+    v[4 * q + 2] = x[q].z;
+    v[4 * q + 3] = x[q].w;
+  }
+  int s = 1;
+  for (; s + 3 < n; s += 4) {
+    float4 y[4][4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) y[u][q] = __ldcg(src + (s + u) * slot_stride + q * 128);
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        v[4 * q] += y[u][q].x;
+        v[4 * q + 1] += y[u][q].y;
+        v[4 * q + 2] += y[u][q].z;
+        v[4 * q + 3] += y[u][q].w;
+      }
+  }
+  for (; s < n; ++s) {
+    float4 y[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) y[q] = __ldcg(src + s * slot_stride + q * 128);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      v[4 * q] += y[q].x;
+      v[4 * q + 1] += y[q].y;
+      v[4 * q + 2] += y[q].z;
+      v[4 * q + 3] += y[q].w;
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------------------------
 template <class Epi>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -252,7 +301,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  const uint32_t sbytes = stage_bytes(p.n_pad);
+  const uint32_t sbytes = stage_bytes(p.n_pad, p.kbs);
+  const uint32_t a_bytes = static_cast<uint32_t>(p.kbs) * kATileBytes;
   float2* rope_tab = reinterpret_cast<float2*>(smem + p.stages * sbytes);
   const int tab_entries = Epi::kRope ? p.n_out * kRopePairs : 0;
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(
@@ -273,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const long long P = gridDim.x;
   const long long i_begin = range_start(c, p.iters, P);
   const long long i_end = range_start(c + 1, p.iters, P);
-  const long long kb = p.k_blocks;
+  const long long kb = p.units;  // work units per tile
   uint32_t tmem_cols = 32;
   while (tmem_cols < 2u * static_cast<uint32_t>(p.n_pad)) tmem_cols <<= 1;
 
@@ -327,23 +377,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ph = static_cast<uint32_t>((issued / p.stages) & 1);
         if (issued >= p.stages && !mbar_wait(&empty_bar[s], ph ^ 1, wc)) break;
         const long long t = i / kb;
-        const int kbi = static_cast<int>(i - t * kb);
+        const int kb0 = static_cast<int>(i - t * kb) * p.kbs;
         const int g = static_cast<int>(t / p.m_tiles);
         const int mt = static_cast<int>(t - static_cast<long long>(g) * p.m_tiles);
         const bool use_a1 = mt >= p.a1_tile_start;
         const CUtensorMap* tmA = use_a1 ? &tmA1 : &tmA0;
         const int m_row0 = (use_a1 ? mt - p.a1_tile_start : mt) * 128;
         uint8_t* a_dst = smem + s * sbytes;
-        uint8_t* x_dst = a_dst + kATileBytes;
+        uint8_t* x_dst = a_dst + a_bytes;
         mbar_arrive_expect_tx(&full_bar[s], sbytes);
-        const int k0 = kbi * 64;
         if (p.a_mn_major) {
-          tma_load_3d_hint(a_dst, tmA, &full_bar[s], m_row0, k0, g, pol_w);
-          tma_load_3d_hint(a_dst + 8192, tmA, &full_bar[s], m_row0 + 64, k0, g, pol_w);
+          // [g][k][m] with m contiguous: box (64 m, 64 kbs k) per 64-row half of the tile
+          tma_load_3d_hint(a_dst, tmA, &full_bar[s], m_row0, kb0 * 64, g, pol_w);
+          tma_load_3d_hint(a_dst + a_bytes / 2, tmA, &full_bar[s], m_row0 + 64, kb0 * 64, g,
+                           pol_w);
         } else {
-          tma_load_3d_hint(a_dst, tmA, &full_bar[s], k0, m_row0, g, pol_w);
+          // view (64 k, rows, groups, k blocks): box (64, 128, 1, kbs)
+          tma_load_4d_hint(a_dst, tmA, &full_bar[s], 0, m_row0, g, kb0, pol_w);
         }
-        tma_load_3d_hint(x_dst, &tmX, &full_bar[s], k0, g, 0, pol_x);
+        // view (64 k, groups, n, k blocks): box (64, 1, n_pad, kbs)
+        tma_load_4d_hint(x_dst, &tmX, &full_bar[s], 0, g, 0, kb0, pol_x);
       }
       if (*abort_flag) {
         // wait (bounded, ignoring the abort flag) for every copy still landing in the ring
@@ -378,14 +431,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const uint32_t a_base = smem_u32(smem + s * sbytes);
-          const uint32_t x_base = a_base + kATileBytes;
+          const uint32_t x_base = a_base + a_bytes;
           const bool first = (i == t * kb) || (i == i_begin);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t adesc = p.a_mn_major
-                                       ? smem_desc(a_base + kk * 2048, 8192, 1024, kSwizzle128B)
-                                       : smem_desc(a_base + kk * 32, 16, 1024, kSwizzle128B);
-            const uint64_t xdesc = smem_desc(x_base + kk * 32, 16, 1024, kSwizzle128B);
+          for (int kk = 0; kk < 4 * p.kbs; ++kk) {
+            const uint32_t kq = static_cast<uint32_t>(kk >> 2), kr = static_cast<uint32_t>(kk & 3);
+            const uint64_t adesc =
+                p.a_mn_major
+                    ? smem_desc(a_base + kk * 2048, a_bytes / 2, 1024, kSwizzle128B)
+                    : smem_desc(a_base + kq * kATileBytes + kr * 32, 16, 1024, kSwizzle128B);
+            const uint64_t xdesc =
+                smem_desc(x_base + kq * static_cast<uint32_t>(p.n_pad) * 128u + kr * 32, 16, 1024,
+                          kSwizzle128B);
             mma_ss(d_tmem, adesc, xdesc, idesc, (first && kk == 0) ? 0u : 1u);
           }
           mma_commit(&empty_bar[s]);
@@ -440,16 +496,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       // shared tile: publish this CTA's partial, count in, finish if last
       const int slot = static_cast<int>(c - c_first);
       const int n_contrib = c_last - c_first + 1;
-      float* part_tile =
-          p.partial + static_cast<size_t>(t) * p.max_slots * p.n_pad * 128 + m_local;
+      // slot layout [n_pad / 4][128 rows][4 columns]: a warp moves 512 contiguous bytes
+      float4* part_tile = reinterpret_cast<float4*>(p.partial) +
+                          static_cast<size_t>(t) * p.max_slots * (p.n_pad / 4) * 128 + m_local;
+      const size_t slot_stride = static_cast<size_t>(p.n_pad / 4) * 128;  // in float4
       {
-        float* dst = part_tile + static_cast<size_t>(slot) * p.n_pad * 128;
+        float4* dst = part_tile + slot * slot_stride;
         for (int c0 = 0; c0 < p.n_pad; c0 += 16) {
           uint32_t a[16];
           tmem_ld16(tacc + c0, a);
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) __stcg(dst + (c0 + j) * 128, __uint_as_float(a[j]));
+          for (int q4 = 0; q4 < 4; ++q4)
+            __stcg(dst + (c0 / 4 + q4) * 128,
+                   make_float4(__uint_as_float(a[4 * q4]), __uint_as_float(a[4 * q4 + 1]),
+                               __uint_as_float(a[4 * q4 + 2]), __uint_as_float(a[4 * q4 + 3])));
         }
       }
       tc_fence_before();
@@ -475,22 +536,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!*fin_flag) continue;
       for (int c0 = 0; c0 < n_cols; c0 += 16) {
         float v[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] = __ldcg(part_tile + (c0 + j) * 128);
-        for (int s = 1; s < n_contrib; ++s) {
-          const float* src = part_tile + static_cast<size_t>(s) * p.n_pad * 128;
-#pragma unroll
-          for (int j = 0; j < 16; ++j) v[j] += __ldcg(src + (c0 + j) * 128);
-        }
+        sum_slots(part_tile + (c0 / 4) * 128, slot_stride, n_contrib, v);
         if (p.n_lo > 0) {
           float w[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) w[j] = __ldcg(part_tile + (p.n_lo + c0 + j) * 128);
-          for (int s = 1; s < n_contrib; ++s) {
-            const float* src = part_tile + static_cast<size_t>(s) * p.n_pad * 128;
-#pragma unroll
-            for (int j = 0; j < 16; ++j) w[j] += __ldcg(src + (p.n_lo + c0 + j) * 128);
-          }
+          sum_slots(part_tile + ((p.n_lo + c0) / 4) * 128, slot_stride, n_contrib, w);
 #pragma unroll
           for (int j = 0; j < 16; ++j) v[j] += w[j];
         }

@@ -25,8 +25,9 @@ namespace {
 constexpr int kDc = 512, kDr = 64, kDn = 128, kDv = 128, kRowN = 576, kPageN = 64;
 constexpr uint64_t kDefaultWaitNs = 2000000000ull;  // 2 s per bounded wait
 constexpr int kMinPagesPerPart = 4;
-constexpr int kSkMinIters = 8;            // fewest K blocks a stream-K CTA streams
-constexpr int kSkMaxStages = 12;
+constexpr int kSkMinUnits = 2;    // fewest stages' worth of weights a stream-K CTA streams
+constexpr int kSkMaxContrib = 4;  // aim for at most this many CTAs sharing one tile
+constexpr int kSkMaxStages = 8;
 constexpr size_t kSmemPerBlockMax = 232448;  // 227 KiB opt-in limit per CTA
 
 // ------------------------------------------------------------------------------------------
@@ -160,9 +161,9 @@ GemmShape shape_wo(const mla_dims* d) {
           round16(d->batch)};
 }
 
-// Stream-K launch plan: CTAs, partial slots per tile, ring depth, shared memory.
+// Stream-K launch plan: K blocks per stage, CTAs, partial slots per tile, ring depth, smem.
 struct SkPlan {
-  int ctas = 1, max_slots = 1, stages = 2, tiles = 0;
+  int kbs = 1, units = 1, ctas = 1, max_slots = 1, stages = 2, tiles = 0;
   long long iters = 0;
   size_t smem = 0, partial_bytes = 0;
 };
@@ -170,19 +171,26 @@ struct SkPlan {
 SkPlan sk_plan(const GemmShape& s, bool rope, int n_out, int sms) {
   SkPlan q;
   q.tiles = s.m_tiles * s.groups;
-  const long long kb = s.k_blocks();
-  q.iters = static_cast<long long>(q.tiles) * kb;
-  long long P = std::min<long long>(sms, (q.iters + kSkMinIters - 1) / kSkMinIters);
+  const size_t tab = rope ? (static_cast<size_t>(n_out) * sk::kRopePairs * 8 + 15) / 16 * 16 : 0;
+  const size_t fixed = 1024 + tab + 256;  // alignment slack, RoPE table, barriers and flags
+  const size_t budget = kSmemPerBlockMax - fixed;
+  // Large TMA boxes (several K blocks of 128 weight rows) keep HBM streaming efficient.
+  q.kbs = 4;
+  while (q.kbs > 1 && (q.kbs > s.k_blocks() || 2 * sk::stage_bytes(s.n_pad, q.kbs) > budget))
+    q.kbs /= 2;
+  q.units = (s.k_blocks() + q.kbs - 1) / q.kbs;
+  q.iters = static_cast<long long>(q.tiles) * q.units;
+  long long P = std::min<long long>(sms, (q.iters + kSkMinUnits - 1) / kSkMinUnits);
+  P = std::min<long long>(P, static_cast<long long>(q.tiles) * kSkMaxContrib);
   P = std::max<long long>(1, std::min(P, q.iters));
   q.ctas = static_cast<int>(P);
   for (long long t = 0; t < q.tiles; ++t) {
-    const int cf = sk::cta_of(t * kb, q.iters, P), cl = sk::cta_of((t + 1) * kb - 1, q.iters, P);
+    const int cf = sk::cta_of(t * q.units, q.iters, P);
+    const int cl = sk::cta_of((t + 1) * q.units - 1, q.iters, P);
     q.max_slots = std::max(q.max_slots, cl - cf + 1);
   }
-  const size_t tab = rope ? (static_cast<size_t>(n_out) * sk::kRopePairs * 8 + 15) / 16 * 16 : 0;
-  const size_t fixed = 1024 + tab + 256;  // alignment slack, RoPE table, barriers and flags
-  const size_t sb = sk::stage_bytes(s.n_pad);
-  q.stages = static_cast<int>(std::min<size_t>(kSkMaxStages, (kSmemPerBlockMax - fixed) / sb));
+  const size_t sb = sk::stage_bytes(s.n_pad, q.kbs);
+  q.stages = static_cast<int>(std::min<size_t>(kSkMaxStages, budget / sb));
   q.smem = fixed + static_cast<size_t>(q.stages) * sb;
   q.partial_bytes = q.max_slots > 1 ? static_cast<size_t>(q.tiles) * q.max_slots * s.n_pad *
                                           128 * sizeof(float)
@@ -286,6 +294,28 @@ int map2(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t s1
   return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, 2, dims, str, box, sw);
 }
 
+// Weights [groups][rows][K] (K contiguous) as a 4-D view (64 k, rows, groups, K / 64) so that
+// one box (64, 128, 1, kbs) brings kbs consecutive 128-byte pieces of 128 weight rows.
+int map_weights(CUtensorMap* m, const void* base, uint64_t rows, uint64_t groups, uint64_t K,
+                int kbs) {
+  const uint64_t dims[4] = {64, rows, groups, K / 64};
+  const uint64_t str[3] = {K * 2, rows * K * 2, 128};
+  const uint32_t box[4] = {64, 128, 1, static_cast<uint32_t>(kbs)};
+  return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, 4, dims, str, box,
+                CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// Activations X: element (k, g, n) at n * n_stride + g * g_stride + 2 k (bytes), as the view
+// (64 k, groups, n, K / 64) with box (64, 1, n_pad, kbs); rows n >= n_rows read as zero.
+int map_acts(CUtensorMap* m, const void* base, uint64_t groups, uint64_t n_rows, uint64_t K,
+             uint64_t g_stride, uint64_t n_stride, int n_pad, int kbs) {
+  const uint64_t dims[4] = {64, groups, n_rows, K / 64};
+  const uint64_t str[3] = {g_stride, n_stride, 128};
+  const uint32_t box[4] = {64, 1, static_cast<uint32_t>(n_pad), static_cast<uint32_t>(kbs)};
+  return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, 4, dims, str, box,
+                CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
 // ------------------------------------------------------------------------------------------
 // launches
 // ------------------------------------------------------------------------------------------
@@ -296,17 +326,19 @@ int last_launch(int kernels = 1) {
 
 // One weight product on the tensor cores, its epilogue fused (stream-K, see gemm_streamk.cuh).
 template <class Epi>
-int run_streamk(const DevCtx* c, const GemmShape& s, int n_out, const int32_t* positions,
-                float theta, const CUtensorMap& a0, const CUtensorMap& a1, int a1_tile_start,
-                int a_mn_major, const CUtensorMap& xmap, char* ws, const Workspace& w,
-                const Epi& epi, cudaStream_t st) {
-  const SkPlan q = sk_plan(s, Epi::kRope, n_out, c->sms);
+int run_streamk(const DevCtx* c, const GemmShape& s, const SkPlan& q, int n_out,
+                const int32_t* positions, float theta, const CUtensorMap& a0,
+                const CUtensorMap& a1, int a1_tile_start, int a_mn_major,
+                const CUtensorMap& xmap, char* ws, const Workspace& w, const Epi& epi,
+                cudaStream_t st) {
   sk::Params p{};
   p.m_total = s.m_total;
   p.m_tiles = s.m_tiles;
   p.groups = s.groups;
   p.a1_tile_start = a1_tile_start;
   p.k_blocks = s.k_blocks();
+  p.kbs = q.kbs;
+  p.units = q.units;
   p.n_pad = s.n_pad;
   p.n_lo = s.n_lo;
   p.n_out = n_out;
@@ -386,14 +418,15 @@ int mla_cache_append(const mla_dims* dims, const void* h, const void* w_dkv, con
   float* part = reinterpret_cast<float*>(ws + w.partial);
   if (dims->dtype == MLA_BF16) {
     const GemmShape s = shape_append(dims);
+    const SkPlan q = sk_plan(s, true, B, c->sms);
     CUtensorMap a0, a1, bm;
-    if ((rc = map3(&a0, w_dkv, D, kDc, 1, D * 2ull, D * 2ull * kDc, 64, 128, 1))) return rc;
-    if ((rc = map3(&a1, w_kr, D, kDr, 1, D * 2ull, D * 2ull * kDr, 64, 128, 1))) return rc;
-    if ((rc = map3(&bm, h, D, 1, B, D * 2ull, D * 2ull, 64, 1, s.n_pad))) return rc;
+    if ((rc = map_weights(&a0, w_dkv, kDc, 1, D, q.kbs))) return rc;
+    if ((rc = map_weights(&a1, w_kr, kDr, 1, D, q.kbs))) return rc;
+    if ((rc = map_acts(&bm, h, 1, B, D, D * 2ull, D * 2ull, s.n_pad, q.kbs))) return rc;
     sk::EpiAppend e{positions, page_table, max_pages, static_cast<__nv_bfloat16*>(cache_pool),
                     num_pages, c->status};
-    return run_streamk(c, s, B, positions, dims->rope_theta, a0, a1, kDc / 128, 0, bm, ws, w, e,
-                       st);
+    return run_streamk(c, s, q, B, positions, dims->rope_theta, a0, a1, kDc / 128, 0, bm, ws, w,
+                       e, st);
   } else {
     // fp32: rows 0..511 from W_DKV, 512..575 from W_KR, written as one [576][B] partial
     f32_gemm_k_kernel<<<dim3(kDc / 8, 1), 256, 0, st>>>(static_cast<const float*>(w_dkv), 0, D,
@@ -439,22 +472,24 @@ int mla_absorb_q(const mla_dims* dims, const void* h, const void* w_q, const voi
     // q = W_Q h -> q_nope hi/lo planes [2][Bp][H][128] and RoPE(q_rope) into q_cat
     const GemmShape s1 = shape_wq(dims);
     const int Bp = s1.n_pad;
+    const SkPlan q1 = sk_plan(s1, true, B, c->sms);
     CUtensorMap a, bm;
-    if ((rc = map3(&a, w_q, D, s1.m_total, 1, D * 2ull, D * 2ull * s1.m_total, 64, 128, 1)))
-      return rc;
-    if ((rc = map3(&bm, h, D, 1, B, D * 2ull, D * 2ull, 64, 1, s1.n_pad))) return rc;
+    if ((rc = map_weights(&a, w_q, s1.m_total, 1, D, q1.kbs))) return rc;
+    if ((rc = map_acts(&bm, h, 1, B, D, D * 2ull, D * 2ull, s1.n_pad, q1.kbs))) return rc;
     __nv_bfloat16* qnb = static_cast<__nv_bfloat16*>(qn);
     sk::EpiWq e1{H, Bp, qc, ql, qnb};
-    if ((rc = run_streamk(c, s1, B, positions, theta, a, a, 1 << 30, 0, bm, ws, w, e1, st)))
+    if ((rc = run_streamk(c, s1, q1, B, positions, theta, a, a, 1 << 30, 0, bm, ws, w, e1, st)))
       return rc;
     // q_lat_h = W_UK_h^T [q_nope_hi | q_nope_lo]   (A MN-major: W_UK rows are the K side)
     const GemmShape s2 = shape_wuk(dims);
+    const SkPlan q2 = sk_plan(s2, false, B, c->sms);
     CUtensorMap a2, b2;
-    if ((rc = map3(&a2, w_uk, kDc, kDn, H, kDc * 2ull, kDc * 2ull * kDn, 64, 64, 1))) return rc;
-    if ((rc = map3(&b2, qn, kDn, H, 2 * Bp, kDn * 2ull, kDn * 2ull * H, 64, 1, s2.n_pad)))
+    if ((rc = map3(&a2, w_uk, kDc, kDn, H, kDc * 2ull, kDc * 2ull * kDn, 64, 64 * q2.kbs, 1)))
+      return rc;
+    if ((rc = map_acts(&b2, qn, H, 2 * Bp, kDn, kDn * 2ull, kDn * 2ull * H, s2.n_pad, q2.kbs)))
       return rc;
     sk::EpiWuk e2{H, qc, ql};
-    return run_streamk(c, s2, B, nullptr, theta, a2, a2, 1 << 30, 1, b2, ws, w, e2, st);
+    return run_streamk(c, s2, q2, B, nullptr, theta, a2, a2, 1 << 30, 1, b2, ws, w, e2, st);
   } else {
     float* qc = static_cast<float*>(q_cat);
     const int M = H * (kDn + kDr);
@@ -589,22 +624,24 @@ int mla_out_proj(const mla_dims* dims, const float* o_lat, const void* w_uv, con
                          st>>>(o_lat, n, static_cast<size_t>(Bp) * H * kDc, os);
     if ((rc = last_launch())) return rc;
     // o_h = W_UV_h [o_lat_hi | o_lat_lo]
+    const SkPlan q1 = sk_plan(s1, false, B, c->sms);
     CUtensorMap a, bm;
-    if ((rc = map3(&a, w_uv, kDc, kDv, H, kDc * 2ull, kDc * 2ull * kDv, 64, 128, 1))) return rc;
-    if ((rc = map3(&bm, os, kDc, H, 2 * Bp, kDc * 2ull, kDc * 2ull * H, 64, 1, s1.n_pad)))
+    if ((rc = map_weights(&a, w_uv, kDv, H, kDc, q1.kbs))) return rc;
+    if ((rc = map_acts(&bm, os, H, 2 * Bp, kDc, kDc * 2ull, kDc * 2ull * H, s1.n_pad, q1.kbs)))
       return rc;
     sk::EpiWuv e1{H, Bp, static_cast<__nv_bfloat16*>(o_heads),
                   static_cast<__nv_bfloat16*>(oh_split)};
-    if ((rc = run_streamk(c, s1, B, nullptr, 0.f, a, a, 1 << 30, 0, bm, ws, w, e1, st)))
+    if ((rc = run_streamk(c, s1, q1, B, nullptr, 0.f, a, a, 1 << 30, 0, bm, ws, w, e1, st)))
       return rc;
     if (out) {
       const GemmShape s2 = shape_wo(dims);
       const uint64_t K = static_cast<uint64_t>(H) * kDv;
+      const SkPlan q2 = sk_plan(s2, false, B, c->sms);
       CUtensorMap a2, b2;
-      if ((rc = map3(&a2, w_o, K, D, 1, K * 2, K * 2 * D, 64, 128, 1))) return rc;
-      if ((rc = map3(&b2, oh_split, K, 1, 2 * Bp, K * 2, K * 2, 64, 1, s2.n_pad))) return rc;
+      if ((rc = map_weights(&a2, w_o, D, 1, K, q2.kbs))) return rc;
+      if ((rc = map_acts(&b2, oh_split, 1, 2 * Bp, K, K * 2, K * 2, s2.n_pad, q2.kbs))) return rc;
       sk::EpiWo e2{D, static_cast<__nv_bfloat16*>(out)};
-      if ((rc = run_streamk(c, s2, B, nullptr, 0.f, a2, a2, 1 << 30, 0, b2, ws, w, e2, st)))
+      if ((rc = run_streamk(c, s2, q2, B, nullptr, 0.f, a2, a2, 1 << 30, 0, b2, ws, w, e2, st)))
         return rc;
     }
   } else {
