@@ -125,6 +125,19 @@ int mla_absorb_q(const mla_dims* dims, const void* h, const void* w_q, const voi
                  size_t workspace_bytes, mla_stream_t stream);
 
 /*
+ * mla_append_absorb -- mla_cache_append followed by mla_absorb_q in one call, same arguments
+ * and same results (up to the order of fp32 additions).  Both start by multiplying the new
+ * hidden states h by a weight matrix; here W_DKV, W_KR and W_Q stream through one product, so
+ * the small cache-append projection shares the launch of the large query projection.  All
+ * pointers are required except q_lo.  The fp32 path runs the two calls in order.
+ */
+int mla_append_absorb(const mla_dims* dims, const void* h, const void* w_dkv, const void* w_kr,
+                      const void* w_q, const void* w_uk, const int32_t* positions,
+                      const int32_t* page_table, int32_t max_pages, void* cache_pool,
+                      int32_t num_pages, void* q_cat, void* q_lo, void* workspace,
+                      size_t workspace_bytes, mla_stream_t stream);
+
+/*
  * mla_decode_attn -- attention of each sequence's new query over its whole cache
  * ([LP] "Classic attention ...": softmax(Q K^T / sqrt(d_k) + M) V, causal mask M admits every
  * cached row since the query is the newest token), in latent space:

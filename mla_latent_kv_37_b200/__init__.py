@@ -60,6 +60,8 @@ _SIGS = {
                                         _P, _SZ, _P]),
     "mla_absorb_q": (ctypes.c_int, [ctypes.POINTER(mla_dims), _P, _P, _P, _P, _P, _P, _P, _SZ,
                                     _P]),
+    "mla_append_absorb": (ctypes.c_int, [ctypes.POINTER(mla_dims), _P, _P, _P, _P, _P, _P, _P,
+                                         _I, _P, _I, _P, _P, _P, _SZ, _P]),
     "mla_decode_attn": (ctypes.c_int, [ctypes.POINTER(mla_dims), _P, _P, _P, _I, _P, _I, _P,
                                        ctypes.c_float, _I, _P, _SZ, _P, _P, _P]),
     "mla_out_proj": (ctypes.c_int, [ctypes.POINTER(mla_dims), _P, _P, _P, _P, _P, _P, _SZ, _P]),
@@ -176,6 +178,29 @@ def mla_absorb_q(d: mla_dims, h, w_q, w_uk, positions, q_cat, ws, q_lo=None, str
     rc = lib().mla_absorb_q(ctypes.byref(d), _ptr(h), _ptr(w_q), _ptr(w_uk), _ptr(positions),
                             _ptr(q_cat), _ptr(q_lo), _ptr(ws), ws.numel(), _stream(stream))
     _check(rc, "mla_absorb_q")
+
+
+def mla_append_absorb(d: mla_dims, h, w_dkv, w_kr, w_q, w_uk, positions, page_table, cache_pool,
+                      q_cat, ws, q_lo=None, stream=None):
+    """mla_cache_append + mla_absorb_q in one call (one shared projection launch)."""
+    e = _elem(d)
+    H = d.n_heads
+    _need(h, "h", e, (d.batch, d.d_model))
+    _need(w_dkv, "w_dkv", e, (d.d_c, d.d_model))
+    _need(w_kr, "w_kr", e, (d.d_rope, d.d_model))
+    _need(w_q, "w_q", e, (H * (d.d_nope + d.d_rope), d.d_model))
+    _need(w_uk, "w_uk", e, (H * d.d_nope, d.d_c))
+    _need(positions, "positions", torch.int32, (d.batch,))
+    _need(page_table, "page_table", torch.int32)
+    _need(cache_pool, "cache_pool", e)
+    _need(q_cat, "q_cat", e, (d.batch, H, d.d_c + d.d_rope))
+    _need(q_lo, "q_lo", torch.bfloat16, (d.batch, H, d.d_c + d.d_rope))
+    _need(ws, "workspace", torch.uint8)
+    rc = lib().mla_append_absorb(ctypes.byref(d), _ptr(h), _ptr(w_dkv), _ptr(w_kr), _ptr(w_q),
+                                 _ptr(w_uk), _ptr(positions), _ptr(page_table),
+                                 page_table.shape[1], _ptr(cache_pool), cache_pool.shape[0],
+                                 _ptr(q_cat), _ptr(q_lo), _ptr(ws), ws.numel(), _stream(stream))
+    _check(rc, "mla_append_absorb")
 
 
 def mla_decode_attn(d: mla_dims, q_cat, cache_pool, page_table, seq_lens, o_lat, ws, lse=None,

@@ -65,6 +65,9 @@ constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // barriers + alignment s
 // TMEM columns
 constexpr uint32_t kTmemO = 0, kTmemQ = 256, kTmemS = 384, kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// Registers per thread the split kernel must be built with when it re-divides them between
+// warpgroups (setmaxnreg); 0 = no re-division.
+constexpr int kLaunchRegs = 0;
 
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 static_assert(kTmemS + 2 * 64 == kTmemCols, "tensor memory budget");
@@ -248,6 +251,27 @@ struct SegIter {
 // 8 different bank groups.
 __device__ __forceinline__ uint32_t xrow_off(int row, int chunk) {
   return static_cast<uint32_t>(row) * 128u + static_cast<uint32_t>((chunk ^ (row & 7)) * 16);
+}
+
+// Reductions over a row's 64 values as 8 independent chains (a single 64-long chain of
+// dependent instructions would dominate a page's softmax time).
+__device__ __forceinline__ float max64(const float* s) {
+  float m[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) m[j] = s[j];
+#pragma unroll
+  for (int k = 8; k < 64; ++k) m[k & 7] = fmaxf(m[k & 7], s[k]);
+  return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])),
+               fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
+}
+__device__ __forceinline__ float maxabs64(const float* s) {
+  float m[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) m[j] = fabsf(s[j]);
+#pragma unroll
+  for (int k = 8; k < 64; ++k) m[k & 7] = fmaxf(m[k & 7], fabsf(s[k]));
+  return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])),
+               fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
 }
 
 // 16-bit fixed point (offset binary: u = q + 32768 for q in [-32767, 32767]) without the
@@ -556,9 +580,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int k = 0; k < 64; ++k) s[k] = k < valid ? s[k] : 0.f;  // never sent
         }
-        float mabs = 0.f;
-#pragma unroll
-        for (int k = 0; k < 64; ++k) mabs = fmaxf(mabs, fabsf(s[k]));
+        const float mabs = maxabs64(s);
         const float inv = mabs > 0.f ? 32767.f / mabs : 0.f;
         if (tt >= 2 && !(ok = warp_wait<true>(&bars->peer_done[buf], ((tt >> 1) - 1) & 1, wc)))
           break;
@@ -662,9 +684,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int k = 0; k < 64; ++k) s[k] = k < valid ? s[k] : NEG_INF;
         }
-        float mx = NEG_INF;
-#pragma unroll
-        for (int k = 0; k < 64; ++k) mx = fmaxf(mx, s[k]);
+        float mx = max64(s);
         mx *= p.scale_log2;  // log2 units (scale > 0 keeps the arg max)
         float alpha = 1.f;
         bool rescale = false;
@@ -675,15 +695,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           m_ref = mx;
           rescale = true;
         }
-        float rs = 0.f;
+        float rsum[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         uint32_t pk[32];
 #pragma unroll
         for (int k = 0; k < 32; ++k) {
           const float e0 = ex2_approx(fmaf(s[2 * k], p.scale_log2, -m_ref));
           const float e1 = ex2_approx(fmaf(s[2 * k + 1], p.scale_log2, -m_ref));
-          rs += e0 + e1;
+          rsum[k & 7] += e0 + e1;
           pk[k] = pack_bf16x2(e0, e1);
         }
+        const float rs = ((rsum[0] + rsum[1]) + (rsum[2] + rsum[3])) +
+                         ((rsum[4] + rsum[5]) + (rsum[6] + rsum[7]));
         l_sum = l_sum * alpha + rs;
         if (!first && __any_sync(0xffffffffu, rescale)) {
           // O must hold PV of the previous page before it is rescaled

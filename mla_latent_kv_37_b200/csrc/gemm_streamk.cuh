@@ -41,6 +41,7 @@ struct Params {
   int m_tiles;        // 128-row tiles per group
   int groups;         // independent products (heads) sharing the launch
   int a1_tile_start;  // tiles (within a group) >= this read map A1, rows relative to it
+  int a2_tile_start;  // tiles >= this read map A2, rows relative to it (>= a1_tile_start)
   int k_blocks;       // 64-wide K blocks per tile
   int kbs;            // K blocks per pipeline stage (one TMA box of A per stage)
   int units;          // stages' worth of work per tile: ceil(k_blocks / kbs)
@@ -96,6 +97,31 @@ __device__ __forceinline__ uint32_t count_in(unsigned long long* ctr, uint32_t e
 // RoPE rows exchange their pair partner with the neighbouring lane (pairs are (even, odd)
 // rows, and a warp's 32 rows never straddle a RoPE boundary).
 // ---------------------------------------------------------------------------------------------
+// cos and sin of the RoPE angle pos * theta^(-2 pair / 64).  The angle (up to ~1.3e5 rad at
+// 128K positions) is formed in double precision and reduced modulo 2 pi with 2 pi split into
+// a double head and a tail (Cody and Waite's two-constant reduction); what is left,
+// |r| <= pi, goes to the float sincos.  Absolute error ~2e-7, far below the bf16 rounding
+// that follows.
+__device__ __forceinline__ float2 rope_cs(float theta, int pair, int pos) {
+  constexpr double kTwoPiHi = 6.283185307179586;       // nearest double to 2 pi
+  constexpr double kTwoPiLo = 2.4492935982947064e-16;  // 2 pi - kTwoPiHi
+  constexpr double kInvTwoPi = 0.15915494309189535;
+  const double inv_freq = pow(static_cast<double>(theta), -2.0 * pair / (2 * kRopePairs));
+  const double a = static_cast<double>(pos) * inv_freq;
+  const double k = rint(a * kInvTwoPi);
+  const double r = fma(-k, kTwoPiLo, fma(-k, kTwoPiHi, a));
+  float sn, cs;
+  sincosf(static_cast<float>(r), &sn, &cs);
+  return make_float2(cs, sn);
+}
+
+// Fill the [n][32] (cos, sin) table for the n RoPE positions (epilogue warps, once per CTA).
+__device__ __forceinline__ void rope_table(float2* tab, const int32_t* positions, int n,
+                                           float theta, int tid, int nthreads) {
+  for (int e = tid; e < n * kRopePairs; e += nthreads)
+    tab[e] = rope_cs(theta, e % kRopePairs, positions[e / kRopePairs]);
+}
+
 __device__ __forceinline__ void rope_rotate(const float2* tab, int b, int pair, bool odd,
                                             float v, float partner, float& out) {
   const float2 cs = tab[b * kRopePairs + pair];
@@ -103,6 +129,9 @@ __device__ __forceinline__ void rope_rotate(const float2* tab, int b, int pair, 
   out = odd ? (partner * cs.y + v * cs.x) : (v * cs.x - partner * cs.y);
 }
 
+// Every epilogue gets a shared-memory area of smem_bytes(n_out) bytes that its prepare()
+// fills once per CTA (epilogue warps only, before the first tile is finished), so that the
+// per-element work reads no global memory besides the partial sums.
 // Cache append: rows 0..511 = c_KV, 512..575 = k_R (rotated); scattered into the page slot.
 struct EpiAppend {
   static constexpr bool kRope = true;
@@ -112,9 +141,36 @@ struct EpiAppend {
   __nv_bfloat16* pool;
   int num_pages;
   unsigned int* status;
-  __device__ void apply(const float2* tab, int, int r, bool valid, int c0, int n_out,
+  float theta;
+  // [n][32] float2 RoPE table, then [n] int64 offsets of the destination rows (-1: invalid)
+  __host__ __device__ static size_t smem_bytes(int n) {
+    return static_cast<size_t>(n) * (kRopePairs * 8 + 8);
+  }
+  __device__ void prepare(uint8_t* sm, int n, int tid, int nthreads) const {
+    constexpr int kRow = 576, kPage = 64;
+    rope_table(reinterpret_cast<float2*>(sm), positions, n, theta, tid, nthreads);
+    long long* off = reinterpret_cast<long long*>(sm + static_cast<size_t>(n) * kRopePairs * 8);
+    for (int b = tid; b < n; b += nthreads) {
+      long long o = -1;
+      const int pos = positions[b];
+      if (pos < 0 || pos >= max_pages * kPage) {
+        atomicOr(status, MLA_STATUS_BAD_POSITION);
+      } else {
+        const int page = page_table[static_cast<size_t>(b) * max_pages + pos / kPage];
+        if (page < 0 || page >= num_pages)
+          atomicOr(status, MLA_STATUS_BAD_PAGE);
+        else
+          o = (static_cast<long long>(page) * kPage + pos % kPage) * kRow;
+      }
+      off[b] = o;
+    }
+  }
+  __device__ void apply(const uint8_t* sm, int, int r, bool valid, int c0, int n_out,
                         float (&v)[16]) const {
-    constexpr int kRow = 576, kDc = 512, kPage = 64;
+    constexpr int kDc = 512;
+    const float2* tab = reinterpret_cast<const float2*>(sm);
+    const long long* off =
+        reinterpret_cast<const long long*>(sm + static_cast<size_t>(n_out) * kRopePairs * 8);
     const bool rope = r >= kDc;  // warp-uniform
     float p[16];
 #pragma unroll
@@ -124,19 +180,11 @@ struct EpiAppend {
     for (int j = 0; j < 16; ++j) {
       const int b = c0 + j;
       if (b >= n_out) break;
-      const int pos = positions[b];
-      if (pos < 0 || pos >= max_pages * kPage) {
-        atomicOr(status, MLA_STATUS_BAD_POSITION);
-        continue;
-      }
-      const int page = page_table[static_cast<size_t>(b) * max_pages + pos / kPage];
-      if (page < 0 || page >= num_pages) {
-        atomicOr(status, MLA_STATUS_BAD_PAGE);
-        continue;
-      }
+      const long long o = off[b];
+      if (o < 0) continue;
       float x = v[j];
       if (rope) rope_rotate(tab, b, (r - kDc) >> 1, r & 1, v[j], p[j], x);
-      pool[(static_cast<size_t>(page) * kPage + pos % kPage) * kRow + r] = __float2bfloat16_rn(x);
+      pool[o + r] = __float2bfloat16_rn(x);
     }
   }
 };
@@ -150,9 +198,18 @@ struct EpiWq {
   __nv_bfloat16* q_cat;
   __nv_bfloat16* q_lo;
   __nv_bfloat16* qn;
-  __device__ void apply(const float2* tab, int, int r, bool valid, int c0, int n_out,
+  const int32_t* positions;
+  float theta;
+  __host__ __device__ static size_t smem_bytes(int n) {
+    return static_cast<size_t>(n) * kRopePairs * 8;
+  }
+  __device__ void prepare(uint8_t* sm, int n, int tid, int nthreads) const {
+    rope_table(reinterpret_cast<float2*>(sm), positions, n, theta, tid, nthreads);
+  }
+  __device__ void apply(const uint8_t* sm, int, int r, bool valid, int c0, int n_out,
                         float (&v)[16]) const {
     constexpr int kDn = 128, kDq = 192, kRow = 576, kDc = 512;
+    const float2* tab = reinterpret_cast<const float2*>(sm);
     const int h = r / kDq, d = r - h * kDq;
     const bool rope = d >= kDn;  // warp-uniform
     float p[16];
@@ -182,12 +239,35 @@ struct EpiWq {
 };
 
 // q_lat_h = W_UK_h^T q_nope_h (hi + lo already summed) -> q_cat[b][h][0..511] (+ q_lo).
+// Cache append and q = W_Q h in one launch (both multiply the same hidden states): rows
+// [0, 640) are the append tiles (W_DKV then W_KR; rows 576..639 padding), rows from 640 on are
+// W_Q's.  Both use the RoPE table that EpiAppend::prepare builds at the start of the area.
+struct EpiAppendWq {
+  static constexpr bool kRope = true;
+  static constexpr int kSplitRow = 640;
+  EpiAppend a;
+  EpiWq q;
+  __host__ __device__ static size_t smem_bytes(int n) { return EpiAppend::smem_bytes(n); }
+  __device__ void prepare(uint8_t* sm, int n, int tid, int nthreads) const {
+    a.prepare(sm, n, tid, nthreads);
+  }
+  __device__ void apply(const uint8_t* sm, int g, int r, bool valid, int c0, int n_out,
+                        float (&v)[16]) const {
+    if (r < kSplitRow)  // warp-uniform: a warp's rows lie in one tile
+      a.apply(sm, g, r, valid && r < 576, c0, n_out, v);
+    else
+      q.apply(sm, g, r - kSplitRow, valid, c0, n_out, v);
+  }
+};
+
 struct EpiWuk {
   static constexpr bool kRope = false;
   int H;
   __nv_bfloat16* q_cat;
   __nv_bfloat16* q_lo;
-  __device__ void apply(const float2*, int g, int r, bool valid, int c0, int n_out,
+  __host__ __device__ static size_t smem_bytes(int) { return 0; }
+  __device__ void prepare(uint8_t*, int, int, int) const {}
+  __device__ void apply(const uint8_t*, int g, int r, bool valid, int c0, int n_out,
                         float (&v)[16]) const {
     constexpr int kRow = 576;
     if (!valid) return;
@@ -210,7 +290,9 @@ struct EpiWuv {
   int b_pad;
   __nv_bfloat16* o_heads;
   __nv_bfloat16* oh;
-  __device__ void apply(const float2*, int g, int r, bool valid, int c0, int n_out,
+  __host__ __device__ static size_t smem_bytes(int) { return 0; }
+  __device__ void prepare(uint8_t*, int, int, int) const {}
+  __device__ void apply(const uint8_t*, int g, int r, bool valid, int c0, int n_out,
                         float (&v)[16]) const {
     constexpr int kDv = 128;
     if (!valid) return;
@@ -235,7 +317,9 @@ struct EpiWo {
   static constexpr bool kRope = false;
   int D;
   __nv_bfloat16* out;
-  __device__ void apply(const float2*, int, int r, bool valid, int c0, int n_out,
+  __host__ __device__ static size_t smem_bytes(int) { return 0; }
+  __device__ void prepare(uint8_t*, int, int, int) const {}
+  __device__ void apply(const uint8_t*, int, int r, bool valid, int c0, int n_out,
                         float (&v)[16]) const {
     if (!valid) return;
 #pragma unroll
@@ -297,16 +381,16 @@ template <class Epi>
 __global__ void __launch_bounds__(kThreads, 1)
     streamk_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,
                         const __grid_constant__ CUtensorMap tmA1,
+                        const __grid_constant__ CUtensorMap tmA2,
                         const __grid_constant__ CUtensorMap tmX, const Params p, const Epi epi) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const uint32_t sbytes = stage_bytes(p.n_pad, p.kbs);
   const uint32_t a_bytes = static_cast<uint32_t>(p.kbs) * kATileBytes;
-  float2* rope_tab = reinterpret_cast<float2*>(smem + p.stages * sbytes);
-  const int tab_entries = Epi::kRope ? p.n_out * kRopePairs : 0;
+  uint8_t* epi_smem = smem + p.stages * sbytes;
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(
-      smem + p.stages * sbytes + ((tab_entries * 8 + 15) & ~15));
+      epi_smem + ((Epi::smem_bytes(p.n_out) + 15) & ~static_cast<size_t>(15)));
   uint64_t* empty_bar = full_bar + p.stages;
   uint64_t* acc_full = empty_bar + p.stages;   // [2]
   uint64_t* acc_empty = acc_full + 2;          // [2], 4 arrivals (one per epilogue warp)
@@ -347,16 +431,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(tmem_slot, tmem_cols);
     tmem_relinquish();
   }
-  if (Epi::kRope) {
-    // cos/sin of pos_b * theta^(-2i/64) for every (column b, pair i), in double precision
-    for (int e = threadIdx.x; e < tab_entries; e += kThreads) {
-      const int b = e / kRopePairs, i = e - b * kRopePairs;
-      const double inv_freq = pow(static_cast<double>(p.rope_theta), -2.0 * i / (2 * kRopePairs));
-      double sn, cs;
-      sincos(static_cast<double>(p.positions[b]) * inv_freq, &sn, &cs);
-      rope_tab[e] = make_float2(static_cast<float>(cs), static_cast<float>(sn));
-    }
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -368,6 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tmA0);
       tma_prefetch_desc(&tmA1);
+      tma_prefetch_desc(&tmA2);
       tma_prefetch_desc(&tmX);
       const uint64_t pol_w = l2_policy_evict_first();
       const uint64_t pol_x = l2_policy_evict_last();
@@ -380,9 +455,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int kb0 = static_cast<int>(i - t * kb) * p.kbs;
         const int g = static_cast<int>(t / p.m_tiles);
         const int mt = static_cast<int>(t - static_cast<long long>(g) * p.m_tiles);
-        const bool use_a1 = mt >= p.a1_tile_start;
-        const CUtensorMap* tmA = use_a1 ? &tmA1 : &tmA0;
-        const int m_row0 = (use_a1 ? mt - p.a1_tile_start : mt) * 128;
+        const CUtensorMap* tmA = &tmA0;
+        int m_row0 = mt * 128;
+        if (mt >= p.a2_tile_start) {
+          tmA = &tmA2;
+          m_row0 = (mt - p.a2_tile_start) * 128;
+        } else if (mt >= p.a1_tile_start) {
+          tmA = &tmA1;
+          m_row0 = (mt - p.a1_tile_start) * 128;
+        }
         uint8_t* a_dst = smem + s * sbytes;
         uint8_t* x_dst = a_dst + a_bytes;
         mbar_arrive_expect_tx(&full_bar[s], sbytes);
@@ -454,6 +535,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- epilogue ----------------
     const int quarter = warp & 3;
     const int m_local = quarter * 32 + lane;
+    // per-CTA epilogue tables while the first tiles stream in (epilogue warps only)
+    epi.prepare(epi_smem, p.n_out, threadIdx.x - 64, 128);
+    asm volatile("bar.sync 1, 128;" ::: "memory");
     const int n_cols = p.n_lo > 0 ? p.n_lo : p.n_pad;  // columns that are outputs
     int seg = 0, multi = 0;
     for (long long i = i_begin; i < i_end; ++seg) {
@@ -486,7 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int j = 0; j < 16; ++j) v[j] += __uint_as_float(a[j]);
           }
-          epi.apply(rope_tab, g, r, valid, c0, p.n_out, v);
+          epi.apply(epi_smem, g, r, valid, c0, p.n_out, v);
         }
         tc_fence_before();
         __syncwarp();
@@ -543,7 +627,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 16; ++j) v[j] += w[j];
         }
-        epi.apply(rope_tab, g, r, valid, c0, p.n_out, v);
+        epi.apply(epi_smem, g, r, valid, c0, p.n_out, v);
       }
     }
   }

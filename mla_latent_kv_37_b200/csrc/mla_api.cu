@@ -27,7 +27,7 @@ constexpr uint64_t kDefaultWaitNs = 2000000000ull;  // 2 s per bounded wait
 constexpr int kMinPagesPerPart = 4;
 constexpr int kSkMinUnits = 2;    // fewest stages' worth of weights a stream-K CTA streams
 constexpr int kSkMaxContrib = 4;  // aim for at most this many CTAs sharing one tile
-constexpr int kSkMaxStages = 8;
+constexpr int kSkMaxStages = 12;
 constexpr size_t kSmemPerBlockMax = 232448;  // 227 KiB opt-in limit per CTA
 
 // ------------------------------------------------------------------------------------------
@@ -96,6 +96,12 @@ int device_ctx(DevCtx** out) {
       g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     }
     // kernel attributes (once per device)
+    // The split kernel re-divides its registers between warpgroups (setmaxnreg); that is only
+    // sound if it was built with exactly the per-thread count the division assumes.
+    cudaFuncAttributes fa{};
+    if (cudaFuncGetAttributes(&fa, attn::split_kernel) != cudaSuccess ||
+        (attn::kLaunchRegs != 0 && fa.numRegs != attn::kLaunchRegs))
+      return MLA_ERR_CUDA;
     const int attn_smem = static_cast<int>(attn::kSmemBytes);
     if (cudaFuncSetAttribute(attn::split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              attn_smem) != cudaSuccess)
@@ -110,6 +116,8 @@ int device_ctx(DevCtx** out) {
         cudaFuncSetAttribute(sk::streamk_gemm_kernel<sk::EpiWuv>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, sk_smem) != cudaSuccess ||
         cudaFuncSetAttribute(sk::streamk_gemm_kernel<sk::EpiWo>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, sk_smem) != cudaSuccess ||
+        cudaFuncSetAttribute(sk::streamk_gemm_kernel<sk::EpiAppendWq>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, sk_smem) != cudaSuccess)
       return MLA_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
@@ -146,6 +154,11 @@ struct GemmShape {
 GemmShape shape_append(const mla_dims* d) {
   return {kRowN, 5, d->d_model, 1, round16(d->batch), 0};
 }
+// cache append and W_Q in one product: 5 append tiles (W_DKV, W_KR) then W_Q's
+GemmShape shape_append_wq(const mla_dims* d) {
+  const int m = d->n_heads * (kDn + kDr);
+  return {sk::EpiAppendWq::kSplitRow + m, 5 + m / 128, d->d_model, 1, round16(d->batch), 0};
+}
 GemmShape shape_wq(const mla_dims* d) {
   const int m = d->n_heads * (kDn + kDr);
   return {m, m / 128, d->d_model, 1, round16(d->batch), 0};
@@ -168,16 +181,16 @@ struct SkPlan {
   size_t smem = 0, partial_bytes = 0;
 };
 
-SkPlan sk_plan(const GemmShape& s, bool rope, int n_out, int sms) {
+SkPlan sk_plan(const GemmShape& s, size_t epi_bytes, int sms) {
   SkPlan q;
   q.tiles = s.m_tiles * s.groups;
-  const size_t tab = rope ? (static_cast<size_t>(n_out) * sk::kRopePairs * 8 + 15) / 16 * 16 : 0;
-  const size_t fixed = 1024 + tab + 256;  // alignment slack, RoPE table, barriers and flags
+  const size_t fixed = 1024 + (epi_bytes + 15) / 16 * 16 + 256;  // alignment, tables, barriers
   const size_t budget = kSmemPerBlockMax - fixed;
-  // Large TMA boxes (several K blocks of 128 weight rows) keep HBM streaming efficient.
-  q.kbs = 4;
-  while (q.kbs > 1 && (q.kbs > s.k_blocks() || 2 * sk::stage_bytes(s.n_pad, q.kbs) > budget))
-    q.kbs /= 2;
+  // Large TMA boxes (several K blocks of 128 weight rows) stream HBM more efficiently: the
+  // largest box (up to 4 K blocks) that still leaves a double-buffered ring.
+  q.kbs = 1;
+  for (int kbs = 2; kbs <= 4 && kbs <= s.k_blocks(); kbs *= 2)
+    if (budget / sk::stage_bytes(s.n_pad, kbs) >= 2) q.kbs = kbs;
   q.units = (s.k_blocks() + q.kbs - 1) / q.kbs;
   q.iters = static_cast<long long>(q.tiles) * q.units;
   long long P = std::min<long long>(sms, (q.iters + kSkMinUnits - 1) / kSkMinUnits);
@@ -218,10 +231,13 @@ Workspace layout(const mla_dims* d, int num_parts, int sms) {
   const size_t B = d->batch, H = d->n_heads, Bp = round16(d->batch);
   size_t part = 0, ctr = 0;
   if (d->dtype == MLA_BF16) {
-    const GemmShape shapes[5] = {shape_append(d), shape_wq(d), shape_wuk(d), shape_wuv(d),
-                                 shape_wo(d)};
-    for (const GemmShape& s : shapes) {
-      const SkPlan q = sk_plan(s, true, d->batch, sms);
+    // the same (shape, epilogue table size) pairs the launches use
+    const GemmShape shapes[6] = {shape_append(d), shape_wq(d), shape_wuk(d), shape_wuv(d),
+                                 shape_wo(d), shape_append_wq(d)};
+    const size_t epi[6] = {sk::EpiAppend::smem_bytes(d->batch), sk::EpiWq::smem_bytes(d->batch),
+                           0, 0, 0, sk::EpiAppendWq::smem_bytes(d->batch)};
+    for (int i = 0; i < 6; ++i) {
+      const SkPlan q = sk_plan(shapes[i], epi[i], sms);
       part = std::max(part, q.partial_bytes);
       ctr = std::max(ctr, static_cast<size_t>(q.tiles) * 8);
     }
@@ -330,12 +346,13 @@ int run_streamk(const DevCtx* c, const GemmShape& s, const SkPlan& q, int n_out,
                 const int32_t* positions, float theta, const CUtensorMap& a0,
                 const CUtensorMap& a1, int a1_tile_start, int a_mn_major,
                 const CUtensorMap& xmap, char* ws, const Workspace& w, const Epi& epi,
-                cudaStream_t st) {
+                cudaStream_t st, const CUtensorMap* a2 = nullptr, int a2_tile_start = 1 << 30) {
   sk::Params p{};
   p.m_total = s.m_total;
   p.m_tiles = s.m_tiles;
   p.groups = s.groups;
   p.a1_tile_start = a1_tile_start;
+  p.a2_tile_start = a2_tile_start;
   p.k_blocks = s.k_blocks();
   p.kbs = q.kbs;
   p.units = q.units;
@@ -353,8 +370,29 @@ int run_streamk(const DevCtx* c, const GemmShape& s, const SkPlan& q, int n_out,
   p.rope_theta = theta;
   p.status = c->status;
   p.wait_ns = kDefaultWaitNs;
-  sk::streamk_gemm_kernel<Epi><<<q.ctas, sk::kThreads, q.smem, st>>>(a0, a1, xmap, p, epi);
+  sk::streamk_gemm_kernel<Epi><<<q.ctas, sk::kThreads, q.smem, st>>>(a0, a1, a2 ? *a2 : a1,
+                                                                      xmap, p, epi);
   return last_launch();
+}
+
+// q_lat_h = W_UK_h^T [q_nope_hi | q_nope_lo] into q_cat[..., :512] (+ q_lo), bf16 path; the
+// q_nope hi/lo planes are in the workspace (written by the W_Q product).  A is MN-major: the
+// rows of W_UK are the K side.
+int run_wuk(const DevCtx* c, const mla_dims* dims, const void* w_uk, char* ws,
+            const Workspace& w, __nv_bfloat16* qc, __nv_bfloat16* ql, cudaStream_t st) {
+  const int B = dims->batch, H = dims->n_heads;
+  const GemmShape s2 = shape_wuk(dims);
+  const int Bp = s2.n_lo;
+  const SkPlan q2 = sk_plan(s2, 0, c->sms);
+  CUtensorMap a2, b2;
+  int rc;
+  if ((rc = map3(&a2, w_uk, kDc, kDn, H, kDc * 2ull, kDc * 2ull * kDn, 64, 64 * q2.kbs, 1)))
+    return rc;
+  if ((rc = map_acts(&b2, ws + w.qn, H, 2 * Bp, kDn, kDn * 2ull, kDn * 2ull * H, s2.n_pad,
+                     q2.kbs)))
+    return rc;
+  sk::EpiWuk e2{H, qc, ql};
+  return run_streamk(c, s2, q2, B, nullptr, 0.f, a2, a2, 1 << 30, 1, b2, ws, w, e2, st);
 }
 
 }  // namespace
@@ -418,13 +456,13 @@ int mla_cache_append(const mla_dims* dims, const void* h, const void* w_dkv, con
   float* part = reinterpret_cast<float*>(ws + w.partial);
   if (dims->dtype == MLA_BF16) {
     const GemmShape s = shape_append(dims);
-    const SkPlan q = sk_plan(s, true, B, c->sms);
+    const SkPlan q = sk_plan(s, sk::EpiAppend::smem_bytes(B), c->sms);
     CUtensorMap a0, a1, bm;
     if ((rc = map_weights(&a0, w_dkv, kDc, 1, D, q.kbs))) return rc;
     if ((rc = map_weights(&a1, w_kr, kDr, 1, D, q.kbs))) return rc;
     if ((rc = map_acts(&bm, h, 1, B, D, D * 2ull, D * 2ull, s.n_pad, q.kbs))) return rc;
     sk::EpiAppend e{positions, page_table, max_pages, static_cast<__nv_bfloat16*>(cache_pool),
-                    num_pages, c->status};
+                    num_pages, c->status, dims->rope_theta};
     return run_streamk(c, s, q, B, positions, dims->rope_theta, a0, a1, kDc / 128, 0, bm, ws, w,
                        e, st);
   } else {
@@ -472,24 +510,15 @@ int mla_absorb_q(const mla_dims* dims, const void* h, const void* w_q, const voi
     // q = W_Q h -> q_nope hi/lo planes [2][Bp][H][128] and RoPE(q_rope) into q_cat
     const GemmShape s1 = shape_wq(dims);
     const int Bp = s1.n_pad;
-    const SkPlan q1 = sk_plan(s1, true, B, c->sms);
+    const SkPlan q1 = sk_plan(s1, sk::EpiWq::smem_bytes(B), c->sms);
     CUtensorMap a, bm;
     if ((rc = map_weights(&a, w_q, s1.m_total, 1, D, q1.kbs))) return rc;
     if ((rc = map_acts(&bm, h, 1, B, D, D * 2ull, D * 2ull, s1.n_pad, q1.kbs))) return rc;
     __nv_bfloat16* qnb = static_cast<__nv_bfloat16*>(qn);
-    sk::EpiWq e1{H, Bp, qc, ql, qnb};
+    sk::EpiWq e1{H, Bp, qc, ql, qnb, positions, theta};
     if ((rc = run_streamk(c, s1, q1, B, positions, theta, a, a, 1 << 30, 0, bm, ws, w, e1, st)))
       return rc;
-    // q_lat_h = W_UK_h^T [q_nope_hi | q_nope_lo]   (A MN-major: W_UK rows are the K side)
-    const GemmShape s2 = shape_wuk(dims);
-    const SkPlan q2 = sk_plan(s2, false, B, c->sms);
-    CUtensorMap a2, b2;
-    if ((rc = map3(&a2, w_uk, kDc, kDn, H, kDc * 2ull, kDc * 2ull * kDn, 64, 64 * q2.kbs, 1)))
-      return rc;
-    if ((rc = map_acts(&b2, qn, H, 2 * Bp, kDn, kDn * 2ull, kDn * 2ull * H, s2.n_pad, q2.kbs)))
-      return rc;
-    sk::EpiWuk e2{H, qc, ql};
-    return run_streamk(c, s2, q2, B, nullptr, theta, a2, a2, 1 << 30, 1, b2, ws, w, e2, st);
+    return run_wuk(c, dims, w_uk, ws, w, qc, ql, st);
   } else {
     float* qc = static_cast<float*>(q_cat);
     const int M = H * (kDn + kDr);
@@ -508,6 +537,61 @@ int mla_absorb_q(const mla_dims* dims, const void* h, const void* w_q, const voi
     wuk_epilogue_kernel<float, false><<<dim3(H, B), 128, 0, st>>>(part, B, B, H, qc, nullptr);
   }
   return last_launch();
+}
+
+int mla_append_absorb(const mla_dims* dims, const void* h, const void* w_dkv, const void* w_kr,
+                      const void* w_q, const void* w_uk, const int32_t* positions,
+                      const int32_t* page_table, int32_t max_pages, void* cache_pool,
+                      int32_t num_pages, void* q_cat, void* q_lo, void* workspace,
+                      size_t workspace_bytes, mla_stream_t stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (!h || !w_dkv || !w_kr || !w_q || !w_uk || !positions || !page_table || !cache_pool ||
+      !q_cat)
+    return MLA_ERR_NULL_ARG;
+  if (!workspace) return MLA_ERR_WORKSPACE;
+  if (max_pages < 1 || num_pages < 1) return MLA_ERR_ARG;
+  if (q_lo && dims->dtype != MLA_BF16) return MLA_ERR_ARG;
+  if (!aligned(h, 16) || !aligned(w_dkv, 16) || !aligned(w_kr, 16) || !aligned(w_q, 16) ||
+      !aligned(w_uk, 16) || !aligned(cache_pool, 16) || !aligned(q_cat, 16) ||
+      (q_lo && !aligned(q_lo, 16)) || !aligned(positions, 4) || !aligned(page_table, 4))
+    return MLA_ERR_ALIGN;
+  if (!aligned(workspace, 256)) return MLA_ERR_ALIGN;
+  if (dims->dtype != MLA_BF16) {
+    // fp32 path: the two calls in order
+    if ((rc = mla_cache_append(dims, h, w_dkv, w_kr, positions, page_table, max_pages,
+                               cache_pool, num_pages, workspace, workspace_bytes, stream)))
+      return rc;
+    return mla_absorb_q(dims, h, w_q, w_uk, positions, q_cat, q_lo, workspace, workspace_bytes,
+                        stream);
+  }
+  DevCtx* c = nullptr;
+  if ((rc = device_ctx(&c))) return rc;
+  const Workspace w = layout(dims, resolve_parts(0, c), c->sms);
+  if (workspace_bytes < w.total) return MLA_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int B = dims->batch, D = dims->d_model, H = dims->n_heads;
+  char* ws = static_cast<char*>(workspace);
+  __nv_bfloat16* qc = static_cast<__nv_bfloat16*>(q_cat);
+  __nv_bfloat16* ql = static_cast<__nv_bfloat16*>(q_lo);
+  // [W_DKV; W_KR; W_Q] h in one stream-K product: cache rows + q_nope planes + RoPE(q_rope)
+  const GemmShape s = shape_append_wq(dims);
+  const SkPlan q = sk_plan(s, sk::EpiAppendWq::smem_bytes(B), c->sms);
+  CUtensorMap a0, a1, a2, bm;
+  if ((rc = map_weights(&a0, w_dkv, kDc, 1, D, q.kbs))) return rc;
+  if ((rc = map_weights(&a1, w_kr, kDr, 1, D, q.kbs))) return rc;
+  if ((rc = map_weights(&a2, w_q, static_cast<uint64_t>(H) * (kDn + kDr), 1, D, q.kbs)))
+    return rc;
+  if ((rc = map_acts(&bm, h, 1, B, D, D * 2ull, D * 2ull, s.n_pad, q.kbs))) return rc;
+  sk::EpiAppendWq e{
+      sk::EpiAppend{positions, page_table, max_pages, static_cast<__nv_bfloat16*>(cache_pool),
+                    num_pages, c->status, dims->rope_theta},
+      sk::EpiWq{H, s.n_pad, qc, ql, reinterpret_cast<__nv_bfloat16*>(ws + w.qn), positions,
+                dims->rope_theta}};
+  if ((rc = run_streamk(c, s, q, B, positions, dims->rope_theta, a0, a1, kDc / 128, 0, bm, ws, w,
+                        e, st, &a2, sk::EpiAppendWq::kSplitRow / 128)))
+    return rc;
+  return run_wuk(c, dims, w_uk, ws, w, qc, ql, st);
 }
 
 int mla_decode_attn(const mla_dims* dims, const void* q_cat, const void* q_lo,
@@ -624,7 +708,7 @@ int mla_out_proj(const mla_dims* dims, const float* o_lat, const void* w_uv, con
                          st>>>(o_lat, n, static_cast<size_t>(Bp) * H * kDc, os);
     if ((rc = last_launch())) return rc;
     // o_h = W_UV_h [o_lat_hi | o_lat_lo]
-    const SkPlan q1 = sk_plan(s1, false, B, c->sms);
+    const SkPlan q1 = sk_plan(s1, 0, c->sms);
     CUtensorMap a, bm;
     if ((rc = map_weights(&a, w_uv, kDv, H, kDc, q1.kbs))) return rc;
     if ((rc = map_acts(&bm, os, H, 2 * Bp, kDc, kDc * 2ull, kDc * 2ull * H, s1.n_pad, q1.kbs)))
@@ -636,7 +720,7 @@ int mla_out_proj(const mla_dims* dims, const float* o_lat, const void* w_uv, con
     if (out) {
       const GemmShape s2 = shape_wo(dims);
       const uint64_t K = static_cast<uint64_t>(H) * kDv;
-      const SkPlan q2 = sk_plan(s2, false, B, c->sms);
+      const SkPlan q2 = sk_plan(s2, 0, c->sms);
       CUtensorMap a2, b2;
       if ((rc = map_weights(&a2, w_o, D, 1, K, q2.kbs))) return rc;
       if ((rc = map_acts(&b2, oh_split, 1, 2 * Bp, K, K * 2, K * 2, s2.n_pad, q2.kbs))) return rc;

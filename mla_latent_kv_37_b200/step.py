@@ -1,7 +1,7 @@
 """One MLA decode step over a stack of layers, driven through the C ABI.
 
 A step, per layer l (each layer has its own weights, paged cache and hidden state h[l]):
-    mla_cache_append -> mla_absorb_q -> mla_decode_attn -> mla_out_proj
+    mla_append_absorb (= mla_cache_append + mla_absorb_q) -> mla_decode_attn -> mla_out_proj
 Everything stays on the device; `run_host` adds the host<->device copies of the step's inputs
 and results (pinned buffers) for end-to-end measurement.  Marshalling only: no arithmetic.
 """
@@ -11,8 +11,7 @@ import dataclasses
 
 import torch
 
-from . import (dims as make_dims, mla_absorb_q, mla_cache_append, mla_decode_attn, mla_out_proj,
-               workspace)
+from . import (dims as make_dims, mla_append_absorb, mla_decode_attn, mla_out_proj, workspace)
 
 
 @dataclasses.dataclass
@@ -46,9 +45,8 @@ class DecodeStep:
         """h [L, B, D] on the device; positions [B] (append slot), seq_lens [B] = positions+1."""
         d = self.dims
         for l, ly in enumerate(self.layers):
-            mla_cache_append(d, h[l], ly.w_dkv, ly.w_kr, positions, ly.page_table, ly.pool,
-                             self.ws, stream=stream)
-            mla_absorb_q(d, h[l], ly.w_q, ly.w_uk, positions, self.q_cat, self.ws, stream=stream)
+            mla_append_absorb(d, h[l], ly.w_dkv, ly.w_kr, ly.w_q, ly.w_uk, positions,
+                              ly.page_table, ly.pool, self.q_cat, self.ws, stream=stream)
             mla_decode_attn(d, self.q_cat, ly.pool, ly.page_table, seq_lens, self.o_lat, self.ws,
                             lse=self.lse, num_splits=self.num_splits, stream=stream)
             mla_out_proj(d, self.o_lat, ly.w_uv, self.ws, w_o=ly.w_o, o_heads=self.o_heads[l],

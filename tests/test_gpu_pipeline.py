@@ -125,3 +125,41 @@ def test_absorbed_query_matches_oracle_projection():
         q_lat = np.stack([w_uk[h * 128:(h + 1) * 128].T @ qn[h] for h in range(128)])
         assert_close(to_np(got["q_cat"][b, :, :512]), q_lat, torch.bfloat16, "q_lat")
         assert_close(to_np(got["q_cat"][b, :, 512:]), qr, torch.bfloat16, "q_rope")
+
+
+@pytest.mark.parametrize("dtype,B,H,D", [(torch.bfloat16, 32, 128, 7168),
+                                         (torch.bfloat16, 5, 16, 1024),
+                                         (torch.bfloat16, 1, 64, 512),
+                                         (torch.float32, 3, 16, 1024)])
+def test_append_absorb_matches_the_two_calls(dtype, B, H, D):
+    """mla_append_absorb (one shared projection launch) gives what mla_cache_append followed
+    by mla_absorb_q give: the same cache rows and absorbed queries within the tolerance (the
+    fp32 sums are split differently), every other pool byte untouched."""
+    import mla_latent_kv_37_b200 as M
+    hist = [(37 * i + 5) % 300 for i in range(B)]
+    wl = Workload(40 + B, B, H, D, hist, dtype=dtype)
+    d = M.dims(B, H, D, dtype)
+    w = wl.w
+    args = dict(h=dev(wl.h), pos=dev(wl.pos), table=dev(wl.cache.page_table))
+    outs = []
+    for fused in (False, True):
+        pool = dev(wl.cache.pool)
+        q = torch.empty(B, H, 576, dtype=dtype, device="cuda")
+        ws = M.workspace(d)
+        if fused:
+            M.mla_append_absorb(d, args["h"], dev(w.w_dkv), dev(w.w_kr), dev(w.w_q), dev(w.w_uk),
+                                args["pos"], args["table"], pool, q, ws)
+        else:
+            M.mla_cache_append(d, args["h"], dev(w.w_dkv), dev(w.w_kr), args["pos"],
+                               args["table"], pool, ws)
+            M.mla_absorb_q(d, args["h"], dev(w.w_q), dev(w.w_uk), args["pos"], q, ws)
+        torch.cuda.synchronize()
+        assert M.mla_get_status() == 0
+        outs.append((pool.cpu(), q.cpu()))
+    (p0, q0), (p1, q1) = outs
+    assert_close(to_np(q1), to_np(q0), dtype, "q_cat")
+    changed = (p0 != wl.cache.pool).any(dim=-1) | (p1 != wl.cache.pool).any(dim=-1)
+    rows0, rows1 = p0[changed], p1[changed]
+    assert changed.sum().item() == B  # one slot per sequence
+    assert_close(to_np(rows1), to_np(rows0), dtype, "appended rows")
+    assert torch.equal(p1[~changed], wl.cache.pool[~changed])
