@@ -55,6 +55,8 @@ def log(*a):
 # distributed plumbing (replicas only: used for the barrier and the max over ranks)
 # ---------------------------------------------------------------------------------------------
 def dist_setup():
+    """One process per GPU under torchrun: NCCL when CUDA is present, gloo otherwise (the
+    replicas exchange nothing but a barrier and the max over ranks of the step time)."""
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     if ws <= 1:
         return 0, 1, 0
@@ -62,9 +64,12 @@ def dist_setup():
     import torch.distributed as dist
     rank = int(os.environ["RANK"])
     local = int(os.environ.get("LOCAL_RANK", rank))
-    torch.cuda.set_device(local)
-    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
-                            device_id=torch.device("cuda", local))
+    if torch.cuda.is_available():
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+    else:
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
     return rank, ws, local
 
 
@@ -78,7 +83,8 @@ def max_over_ranks(x: float, world: int) -> float:
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -308,7 +314,7 @@ def run_reference(args, rank, world):
     per_step = []
     heads_timed = 0
     for i in range(args.warmup + args.steps):
-        budget = max(2.0, min(20.0, 150.0 / max(1, args.warmup + args.steps)))
+        budget = args.ref_seconds or max(2.0, min(20.0, 150.0 / max(1, args.warmup + args.steps)))
         t, heads_timed, wall = time_oracle(w, h, hist, n - 1, H, budget_s=budget)
         if i >= args.warmup:
             per_step.append(t)
@@ -340,11 +346,14 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-check", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--ref-seconds", type=float, default=0.0,
+                    help="reference arm: CPU seconds per timed sample (0 = fit a few minutes)")
     args = ap.parse_args()
-    rank, world, local = dist_setup()
     if args.impl == "reference":
-        run_reference(args, rank, world)
+        # the CPU oracle arm: rank 0 alone runs it; under torchrun the other ranks exit at once
+        run_reference(args, int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")))
         return
+    rank, world, local = dist_setup()
     args.warmup = max(args.warmup, 3)
     from mla_latent_kv_37_b200 import build
     if rank == 0:
