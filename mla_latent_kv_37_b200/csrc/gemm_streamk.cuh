@@ -17,7 +17,9 @@
 // itself on the tile's counter; the one that completes the count adds the slots in slot order
 // (so the result does not depend on arrival order) and runs the epilogue.  Nobody waits for
 // another CTA.  Counters are tagged with a per-launch epoch in their upper 32 bits, so stale
-// counts from earlier launches read as zero and the workspace never needs clearing.
+// counts from earlier launches read as zero and the workspace never needs clearing; the
+// finisher also clears its tile's counter, so a launch replayed with the same epoch (from a
+// CUDA graph) starts from zero too.
 //
 // Roles (192 threads): warp 0 TMA producer, warp 1 MMA issuer + TMEM owner, warps 2-5
 // epilogue (warp w reads TMEM lanes 32*(w%4) .. +31, i.e. tile rows).
@@ -611,6 +613,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (mbar_wait(epi_sync, ph, wc)) {
           const uint32_t n = count_in(&p.counters[t], p.epoch, p.status);
           fin = (n == static_cast<uint32_t>(n_contrib)) ? 1 : 0;
+          if (fin) atomicExch(&p.counters[t], 0ull);  // last user of this counter in the launch
           __threadfence();
         }
         *fin_flag = fin;

@@ -163,3 +163,15 @@ def test_append_absorb_matches_the_two_calls(dtype, B, H, D):
     assert changed.sum().item() == B  # one slot per sequence
     assert_close(to_np(rows1), to_np(rows0), dtype, "appended rows")
     assert torch.equal(p1[~changed], wl.cache.pool[~changed])
+
+
+@pytest.mark.parametrize("B", [128, 100])
+def test_max_and_ragged_batch(B):
+    """The largest batch the bf16 path takes (128: the hi/lo products run the tensor core at
+    N = 256) and a batch that is not a multiple of 16 (100 -> N padded to 112 / 224), against
+    the oracle on sampled sequences; 16 heads and d_model 1024 keep the oracle quick."""
+    hist = [(53 * i + 11) % 257 for i in range(B)]
+    wl = Workload(70 + B, B, 16, 1024, hist)
+    got = wl.run_gpu()
+    assert got["status"] == 0
+    _check_step(wl, got, [0, B // 2, B - 1])
