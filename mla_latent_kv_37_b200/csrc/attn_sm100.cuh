@@ -36,8 +36,9 @@
 // log-sum-exp weights.
 //
 // Roles (384 threads): warps 0-3 softmax + epilogue (thread i owns head row i = TMEM lane i),
-// warps 4-7 send, warp 8 TMA producer, warp 9 MMA issuer, warp 10 bulk-copy sender, warp 11
-// cluster-scope signals.  The online softmax keeps a per-row reference maximum and rescales O
+// warps 4-7 send, warp 8 TMA producer, warp 9 MMA issuer, warp 10 bulk-copy sender (warp 11
+// has no role).  Each softmax warp hands its rows of the receive buffer back to the peer
+// itself once it has decoded them.  The online softmax keeps a per-row reference maximum and rescales O
 // only when the running maximum grows by more than 2^8.
 #pragma once
 #include "ptx_sm100.cuh"
@@ -312,9 +313,9 @@ struct Bars {
   uint64_t staged[2];     // send WG: partial staged in send[i] (128)
   uint64_t p_full;        // softmax WG: P written (128)
   uint64_t pv_done;       // MMA: PV finished, P buffer free (commit, once per page)
-  uint64_t consumed;      // softmax WG: recv read (128)
   uint64_t x_full;        // the peer's partial landed in recv (bulk-copy bytes)
-  uint64_t peer_done[2];  // the peer consumed our partial of a page of parity i (1 remote)
+  uint64_t peer_done[2];  // the peer's 4 softmax warps decoded our partial of a page of
+                          // parity i (4 remote arrivals)
   uint64_t o_free;        // softmax WG: the epilogue drained O (128)
   uint64_t seg_done;      // MMA: every PV of the segment finished (commit, once per segment)
   uint64_t drain;
@@ -349,11 +350,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(&bars->s_full[i], 1);
       mbar_init(&bars->s_free[i], 256);
       mbar_init(&bars->staged[i], 128);
-      mbar_init(&bars->peer_done[i], 1);
+      mbar_init(&bars->peer_done[i], 4);
     }
     mbar_init(&bars->p_full, 128);
     mbar_init(&bars->pv_done, 1);
-    mbar_init(&bars->consumed, 128);
     mbar_init(&bars->x_full, 1);
     mbar_init(&bars->o_free, 128);
     mbar_init(&bars->seg_done, 1);
@@ -515,13 +515,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         mbar_wait(&bars->drain, 0, drain);
       }
     }
-  } else if (warp == 10 || warp == 11) {
-    // =================== exchange: bulk copies out (10), cluster-scope signals (11) ===========
+  } else if (warp == 10) {
+    // =================== exchange: bulk copies out ===================
     if (lane == 0) {
       const uint32_t peer_recv = mapa_shared(recv_base, peer);
       const uint32_t peer_xfull = mapa_shared(smem_u32(&bars->x_full), peer);
-      const uint32_t peer_done_r[2] = {mapa_shared(smem_u32(&bars->peer_done[0]), peer),
-                                       mapa_shared(smem_u32(&bars->peer_done[1]), peer)};
       SegIter it{plan.seq_pages(), plan.seq_prefix(), p.batch, g_begin, g_end, b_begin};
       int seq, p0, p1, t = 0;
       bool ok = true;
@@ -529,24 +527,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int n = p1 - p0;
         for (int tt = t; ok && tt < t + n; ++tt) {
           const int buf = tt & 1;
-          if (warp == 10) {
-            // the page's partial is staged in send[buf] and the peer's (single) receive buffer
-            // has been read for page tt - 1: ship it
-            if (!(ok = mbar_wait(&bars->staged[buf], (tt >> 1) & 1, wc))) break;
-            if (tt >= 1 && !(ok = mbar_wait<true>(&bars->peer_done[(tt - 1) & 1],
-                                                 ((tt - 1) >> 1) & 1, wc)))
-              break;
-            bulk_copy_s2cluster(peer_recv, send_base + buf * kXBytes, kXBytes, peer_xfull);
-          } else {
-            // every softmax row has read recv: re-arm it for page tt + 1, tell the peer
-            if (!(ok = mbar_wait(&bars->consumed, tt & 1, wc))) break;
-            mbar_arrive_expect_tx(&bars->x_full, kXBytes);
-            mbar_arrive_remote(peer_done_r[buf]);
-          }
+          // the page's partial is staged in send[buf] and the peer's (single) receive buffer
+          // has been decoded for page tt - 1: ship it
+          if (!(ok = mbar_wait(&bars->staged[buf], (tt >> 1) & 1, wc))) break;
+          if (tt >= 1 && !(ok = mbar_wait<true>(&bars->peer_done[(tt - 1) & 1],
+                                               ((tt - 1) >> 1) & 1, wc)))
+            break;
+          bulk_copy_s2cluster(peer_recv, send_base + buf * kXBytes, kXBytes, peer_xfull);
         }
         t += n;
       }
     }
+  } else if (warp == 11) {
+    // no role
   } else if (warp >= 4) {
     // =================== send warpgroup (warps 4-7) ===================
     const int row = threadIdx.x - 128;
@@ -609,6 +602,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     const float NEG_INF = -__int_as_float(0x7f800000);
     const bool row_ok = row < p.n_heads;
+    const uint32_t peer_done_r[2] = {mapa_shared(smem_u32(&bars->peer_done[0]), peer),
+                                     mapa_shared(smem_u32(&bars->peer_done[1]), peer)};
     SegIter it{plan.seq_pages(), plan.seq_prefix(), p.batch, g_begin, g_end, b_begin};
     int seq, p0, p1, t = 0, sg = 0;
     bool ok = true;
@@ -676,7 +671,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               s[8 * c + 2 * k + 1] = fmaf(dec_hi(v[k]), dq, s[8 * c + 2 * k + 1]);
             }
           }
-          mbar_arrive(&bars->consumed);
+          // this warp's rows are decoded: warp 0 re-arms recv for the next page (its phase
+          // cannot complete before all four warps have handed their rows back), and every
+          // warp tells the peer its rows may be refilled
+          __syncwarp();
+          if (lane == 0) {
+            if (warp == 0) mbar_arrive_expect_tx(&bars->x_full, kXBytes);
+            mbar_arrive_remote_relaxed(peer_done_r[buf]);
+          }
         }
         // ---- online softmax ----
         const int valid = min(kPage, len - (p0 + i) * kPage);
