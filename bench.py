@@ -346,6 +346,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-check", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch every kernel eagerly instead of replaying a captured step")
     ap.add_argument("--ref-seconds", type=float, default=0.0,
                     help="reference arm: CPU seconds per timed sample (0 = fit a few minutes)")
     args = ap.parse_args()
@@ -373,7 +375,8 @@ def main():
     torch.cuda.synchronize()
     log(f"[bench] rank {rank}: workload ready in {time.time() - t_gen:.1f} s, "
         f"{torch.cuda.memory_allocated() / 1e9:.1f} GB on device")
-    step = DecodeStep(layers, B, H, D, num_splits=args.num_splits, device=dev)
+    graph = not args.no_graph
+    step = DecodeStep(layers, B, H, D, num_splits=args.num_splits, device=dev, graph=graph)
     stream = torch.cuda.current_stream()
     for _ in range(args.warmup):
         step.run(h, pos, lens_dev)
@@ -383,10 +386,22 @@ def main():
         raise RuntimeError(f"device status {st:#x} after warm-up")
 
     # ---------------- timed region (device-resident inputs) ----------------
-    n_prof = args.steps * L
+    # CUDA events around every split-kernel launch, on the stream it runs on.  In graph mode
+    # the events are captured into the step's graph and re-recorded by every replay: after
+    # the timed steps they hold the last step's L launches.
+    n_prof = L if graph else args.steps * L
     ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(n_prof)]
     ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(n_prof)]
-    M.mla_set_profile_events(ev_b, ev_e)
+    if graph:
+        step.capture(h, pos, lens_dev,
+                     before_capture=lambda: M.mla_set_profile_events(ev_b, ev_e))
+        used = M.mla_profile_events_used()
+        M.mla_set_profile_events([], [])
+        for _ in range(2):
+            step.run(h, pos, lens_dev)
+        torch.cuda.synchronize()
+    else:
+        M.mla_set_profile_events(ev_b, ev_e)
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)
@@ -399,11 +414,13 @@ def main():
         step.run(h, pos, lens_dev)
     e1.record(stream)
     torch.cuda.synchronize()
-    launches = M.mla_launch_count() - launches0
+    launches = (step.launches_per_step * args.steps if graph
+                else M.mla_launch_count() - launches0)
     barrier(world)
     clocks = sampler.stop()
-    used = M.mla_profile_events_used()
-    M.mla_set_profile_events([], [])
+    if not graph:
+        used = M.mla_profile_events_used()
+        M.mla_set_profile_events([], [])
     ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
     split_ms = [b.elapsed_time(e) for b, e in zip(ev_b[:used], ev_e[:used])]
     st = M.mla_get_status()
@@ -496,6 +513,7 @@ def main():
                        "d_model": D, "d_c": 512, "d_rope": 64, "page_size": 64,
                        "global_batch": B * world, "parallelism": f"replicas x{world}",
                        "num_splits": args.num_splits or "auto",
+                       "launch": "CUDA graph of the step" if graph else "eager",
                        "l2": "no flush: inputs per step exceed L2 "
                              f"({(tokens_read * ROW_BYTES * L + 0.629e9 * L) / 1e9:.0f} GB vs 0.126 GB)"},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,

@@ -340,6 +340,15 @@ int last_launch(int kernels = 1) {
   return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
+// A profiling event on `st`.  Under stream capture it becomes an external event node, which
+// records a timestamp every time the graph runs (a plain record inside a capture does not).
+cudaError_t record_profile_event(cudaEvent_t ev, cudaStream_t st) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return cudaErrorUnknown;
+  return cudaEventRecordWithFlags(
+      ev, st, cs == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : cudaEventRecordDefault);
+}
+
 // One weight product on the tensor cores, its epilogue fused (stream-K, see gemm_streamk.cuh).
 template <class Epi>
 int run_streamk(const DevCtx* c, const GemmShape& s, const SkPlan& q, int n_out,
@@ -657,12 +666,13 @@ int mla_decode_attn(const mla_dims* dims, const void* q_cat, const void* q_lo,
     p.status = c->status;
     p.wait_ns = kDefaultWaitNs;
     const bool prof = g_prof_next < g_prof_count;
-    if (prof && cudaEventRecord(g_prof_begin[g_prof_next], st) != cudaSuccess) return MLA_ERR_CUDA;
+    if (prof && record_profile_event(g_prof_begin[g_prof_next], st) != cudaSuccess)
+      return MLA_ERR_CUDA;
     attn::split_kernel<<<2 * parts, attn::kThreads, attn::kSmemBytes, st>>>(tc_lat, tc_rope,
                                                                             tq_rope, p);
     if (prof) {
       if ((rc = last_launch())) return rc;
-      if (cudaEventRecord(g_prof_end[g_prof_next++], st) != cudaSuccess) return MLA_ERR_CUDA;
+      if (record_profile_event(g_prof_end[g_prof_next++], st) != cudaSuccess) return MLA_ERR_CUDA;
       g_launches.fetch_sub(1, std::memory_order_relaxed);  // counted again below
     }
   } else {

@@ -11,7 +11,8 @@ import dataclasses
 
 import torch
 
-from . import (dims as make_dims, mla_append_absorb, mla_decode_attn, mla_out_proj, workspace)
+from . import (dims as make_dims, mla_append_absorb, mla_decode_attn, mla_launch_count,
+               mla_out_proj, workspace)
 
 
 @dataclasses.dataclass
@@ -28,7 +29,7 @@ class Layer:
 
 class DecodeStep:
     def __init__(self, layers: list[Layer], batch: int, n_heads: int, d_model: int,
-                 dtype=torch.bfloat16, num_splits: int = 0, device="cuda"):
+                 dtype=torch.bfloat16, num_splits: int = 0, device="cuda", graph: bool = False):
         self.layers = layers
         self.B, self.H, self.D, self.dtype = batch, n_heads, d_model, dtype
         self.dims = make_dims(batch, n_heads, d_model, dtype)
@@ -40,9 +41,44 @@ class DecodeStep:
         self.lse = torch.empty(batch, n_heads, dtype=torch.float32, device=device)
         self.o_heads = torch.empty(L, batch, n_heads, 128, dtype=dtype, device=device)
         self.out = torch.empty(L, batch, d_model, dtype=dtype, device=device)
+        # graph mode: the step's launches are captured once per set of input buffers (a CUDA
+        # graph) and replayed; every launch keeps the arguments it was captured with
+        self.graph = graph
+        self._graphs: dict = {}
+        self.launches_per_step = 0
 
     def run(self, h, positions, seq_lens, stream=None):
         """h [L, B, D] on the device; positions [B] (append slot), seq_lens [B] = positions+1."""
+        if not self.graph:
+            self._run(h, positions, seq_lens, stream)
+            return
+        key = (h.data_ptr(), positions.data_ptr(), seq_lens.data_ptr())
+        g = self._graphs.get(key)
+        if g is None:
+            g = self.capture(h, positions, seq_lens)
+        if stream is None:
+            g.replay()
+        else:
+            with torch.cuda.stream(stream):
+                g.replay()
+
+    def capture(self, h, positions, seq_lens, before_capture=None):
+        """(Re)capture the step for these input buffers.  One eager step first, so that every
+        one-time set-up of the library (device context, kernel attributes) happens outside the
+        capture; `before_capture` runs between the two."""
+        self._run(h, positions, seq_lens)
+        torch.cuda.synchronize()
+        if before_capture is not None:
+            before_capture()
+        g = torch.cuda.CUDAGraph()
+        n0 = mla_launch_count()
+        with torch.cuda.graph(g):
+            self._run(h, positions, seq_lens)
+        self.launches_per_step = mla_launch_count() - n0
+        self._graphs[(h.data_ptr(), positions.data_ptr(), seq_lens.data_ptr())] = g
+        return g
+
+    def _run(self, h, positions, seq_lens, stream=None):
         d = self.dims
         for l, ly in enumerate(self.layers):
             mla_append_absorb(d, h[l], ly.w_dkv, ly.w_kr, ly.w_q, ly.w_uk, positions,
