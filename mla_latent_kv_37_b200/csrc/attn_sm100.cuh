@@ -65,6 +65,8 @@ constexpr uint32_t kOffBar = kOffRecv + kXBytes;
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // barriers + alignment slack
 // TMEM columns
 constexpr uint32_t kTmemO = 0, kTmemQ = 256, kTmemS = 384, kTmemCols = 512;
+constexpr int kAhead = 4;  // pages prefetched into L2 ahead of the TMA ring
+constexpr uint32_t kPageBytes = kPage * kRow * 2;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // Registers per thread the split kernel must be built with when it re-divides them between
 // warpgroups (setmaxnreg); 0 = no re-division.
@@ -81,6 +83,7 @@ struct Params {
   int num_pages;
   int num_parts;  // clusters launched
   const __nv_bfloat16* q_cat;  // [B][H][576]
+  const uint8_t* pool;         // cache pages, [num_pages][64][576] bf16
   const int32_t* page_table;
   const int32_t* seq_lens;
   const int32_t* plan;
@@ -142,6 +145,25 @@ __device__ inline int block_exclusive_scan(int v, int* warp_sums, int* total) {
   return before;
 }
 
+// Pages of sequence b, its length clamped to the cache (a bad length is reported once, by the
+// thread that first reads it).
+__device__ inline int plan_pages(const int32_t* seq_lens, int b, int cap, unsigned int* status) {
+  int len = seq_lens[b];
+  if (len < 0 || len > cap) {
+    if (status) atomicOr(status, MLA_STATUS_BAD_LENGTH);
+    len = len < 0 ? 0 : cap;
+  }
+  return (len + kPage - 1) / kPage;
+}
+
+// The part that holds global page g of the concatenated list (g = -1 gives -1).
+__device__ inline int part_of_page(int64_t g, int C, int P) {
+  return g < 0 ? -1 : static_cast<int>(((g + 1) * C - 1) / P);
+}
+
+// Every value a thread needs comes from its own sequences and two block-wide scans: the parts
+// whose first page lies inside sequence b are written by b's thread, so no thread searches the
+// prefix sums that other threads wrote.
 __global__ void __launch_bounds__(kPlanThreads)
     plan_kernel(const int32_t* __restrict__ seq_lens, int B, int max_pages, int C_req,
                 int min_pages_per_part, int32_t* __restrict__ plan, unsigned int* status) {
@@ -158,70 +180,51 @@ __global__ void __launch_bounds__(kPlanThreads)
   const int chunk = (B + T - 1) / T;
   const int b0 = threadIdx.x * chunk, b1 = min(B, b0 + chunk);
   const int cap = max_pages * kPage;
-  // 1. pages per sequence
+  // 1. pages of this thread's sequences, and their exclusive prefix over the whole batch
   int local = 0;
-  for (int b = b0; b < b1; ++b) {
-    int len = seq_lens[b];
-    if (len < 0 || len > cap) {
-      atomicOr(status, MLA_STATUS_BAD_LENGTH);
-      len = len < 0 ? 0 : cap;
-    }
-    const int n = (len + kPage - 1) / kPage;
-    pg[b] = n;
-    local += n;
-  }
-  // 2. prefix sums
-  int run = block_exclusive_scan(local, warp_sums, &s_total);
-  for (int b = b0; b < b1; ++b) {
-    prefix[b] = run;
-    run += pg[b];
-  }
+  for (int b = b0; b < b1; ++b) local += plan_pages(seq_lens, b, cap, status);
+  const int run0 = block_exclusive_scan(local, warp_sums, &s_total);
   const int P = s_total;
-  if (threadIdx.x == 0) prefix[B] = P;
   int C = 0;
   if (P > 0) C = max(1, min(C_req, (P + min_pages_per_part - 1) / min_pages_per_part));
   if (threadIdx.x == 0) {
     plan[0] = P;
     plan[1] = C;
+    prefix[B] = P;
   }
-  // 3. equal division of the page list
-  for (int c = threadIdx.x; c <= C_req; c += T)
+  // 2. equal division of the page list; parts beyond C are empty and start no sequence
+  for (int c = threadIdx.x; c <= C_req; c += T) {
     pstart[c] = (c <= C && C > 0) ? static_cast<int>((static_cast<int64_t>(c) * P) / C) : P;
-  // 4. parts covering each sequence
-  int nloc = 0;
+    if (c < C_req && c >= C) pseq[c] = B;
+  }
+  // 3. per sequence: its pages, prefix, the parts that cover it, and the parts starting in it
+  int run = run0, nloc = 0;
   for (int b = b0; b < b1; ++b) {
-    const int n = pg[b];
+    const int n = plan_pages(seq_lens, b, cap, nullptr);
+    pg[b] = n;
+    prefix[b] = run;
     if (n == 0) {
       first[b] = 0;
       npart[b] = 0;
       continue;
     }
-    const int64_t g_first = prefix[b], g_last = prefix[b] + n - 1;
-    const int pf = static_cast<int>(((g_first + 1) * C - 1) / P);
-    const int pl = static_cast<int>(((g_last + 1) * C - 1) / P);
+    const int pf = part_of_page(run, C, P);
+    const int pl = part_of_page(static_cast<int64_t>(run) + n - 1, C, P);
     first[b] = pf;
     npart[b] = pl - pf + 1;
     nloc += pl - pf + 1;
+    for (int c = part_of_page(static_cast<int64_t>(run) - 1, C, P) + 1; c <= pl; ++c) pseq[c] = b;
+    run += n;
   }
-  __syncthreads();
+  // 4. where each sequence's partials go
   int srun = block_exclusive_scan(nloc, warp_sums, nullptr);
+  run = run0;
   for (int b = b0; b < b1; ++b) {
+    const int n = plan_pages(seq_lens, b, cap, nullptr);
     slot[b] = srun;
-    srun += npart[b];
-  }
-  // 5. first sequence of each part: last b with prefix[b] <= start
-  for (int c = threadIdx.x; c < C_req; c += T) {
-    if (c >= C) {
-      pseq[c] = B;
-      continue;
-    }
-    const int g0 = static_cast<int>((static_cast<int64_t>(c) * P) / C);
-    int lo = 0, hi = B - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (prefix[mid] <= g0) lo = mid; else hi = mid - 1;
-    }
-    pseq[c] = lo;
+    if (n > 0)
+      srun += part_of_page(static_cast<int64_t>(run) + n - 1, C, P) - part_of_page(run, C, P) + 1;
+    run += n;
   }
 }
 
@@ -412,8 +415,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           atomicOr(p.status, MLA_STATUS_BAD_PAGE);
           my_page = 0;
         }
+        // warm L2 ahead of the ring: each CTA of the pair fetches half of a page's rows
+        if (lane < min(cnt, kAhead))
+          prefetch_l2(p.pool + static_cast<size_t>(my_page) * kPageBytes + rank * (kPageBytes / 2),
+                      kPageBytes / 2);
         for (int j = 0; j < cnt; ++j, ++t) {
           const int page = __shfl_sync(0xffffffffu, my_page, j);
+          const int later = __shfl_sync(0xffffffffu, my_page, min(j + kAhead, 31));
+          if (lane == 0 && j + kAhead < cnt)
+            prefetch_l2(p.pool + static_cast<size_t>(later) * kPageBytes + rank * (kPageBytes / 2),
+                        kPageBytes / 2);
           if (lane == 0) {
             const int s = t % kStages;
             if (t >= kStages) ok = mbar_wait(&bars->empty[s], ((t / kStages) - 1) & 1, wc);
@@ -797,38 +808,64 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 // ------------------------------------------------------------------------------------------
 // Combine: log-sum-exp merge of the parts of sequences split over several ranges.
 // ------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(128)
+constexpr int kCombineWarps = 8;
+
+// One warp per (sequence, head); lane l owns float4 columns l, l + 32, l + 64 and l + 96.  The
+// parts are merged in slot order; every part's loads of a chunk are issued before any is used.
+__global__ void __launch_bounds__(32 * kCombineWarps)
     combine_kernel(const int32_t* __restrict__ plan_words, int B, int C, int H,
                    const float* __restrict__ part_o, const float* __restrict__ part_lse,
                    float* __restrict__ o_lat, float* __restrict__ lse) {
   const PlanView plan(plan_words, B, C);
-  const int h = blockIdx.x, b = blockIdx.y;
+  const int wid = blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (wid >= B * H) return;
+  const int b = wid / H, h = wid - b * H;
   const int n = plan.seq_nparts()[b];
   if (n == 1) return;
   float4* out = reinterpret_cast<float4*>(o_lat + (static_cast<size_t>(b) * H + h) * 512);
+  const float NEG_INF = -__int_as_float(0x7f800000);
   if (n == 0) {
-    out[threadIdx.x] = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (threadIdx.x == 0 && lse) lse[static_cast<size_t>(b) * H + h] = -__int_as_float(0x7f800000);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) out[lane + 32 * k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (lane == 0 && lse) lse[static_cast<size_t>(b) * H + h] = NEG_INF;
     return;
   }
   const int slot0 = plan.seq_slot()[b];
-  float m = -__int_as_float(0x7f800000);
-  for (int s = 0; s < n; ++s) m = fmaxf(m, part_lse[static_cast<size_t>(slot0 + s) * H + h]);
+  float m = NEG_INF;
+  for (int s = lane; s < n; s += 32)
+    m = fmaxf(m, part_lse[static_cast<size_t>(slot0 + s) * H + h]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   float tot = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s = 0; s < n; ++s) {
-    const float w = __expf(part_lse[static_cast<size_t>(slot0 + s) * H + h] - m);
-    tot += w;
-    const float4 v = reinterpret_cast<const float4*>(
-        part_o + (static_cast<size_t>(slot0 + s) * H + h) * 512)[threadIdx.x];
-    acc.x += w * v.x;
-    acc.y += w * v.y;
-    acc.z += w * v.z;
-    acc.w += w * v.w;
+  float4 acc[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s0 = 0; s0 < n; s0 += 32) {
+    const int cnt = min(32, n - s0);
+    const float wl =
+        lane < cnt ? __expf(part_lse[static_cast<size_t>(slot0 + s0 + lane) * H + h] - m) : 0.f;
+#pragma unroll 4
+    for (int j = 0; j < cnt; ++j) {
+      const float w = __shfl_sync(0xffffffffu, wl, j);
+      const float4* src = reinterpret_cast<const float4*>(
+          part_o + (static_cast<size_t>(slot0 + s0 + j) * H + h) * 512);
+      tot += w;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float4 v = src[lane + 32 * k];
+        acc[k].x += w * v.x;
+        acc[k].y += w * v.y;
+        acc[k].z += w * v.z;
+        acc[k].w += w * v.w;
+      }
+    }
   }
   const float inv = 1.f / tot;
-  out[threadIdx.x] = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-  if (threadIdx.x == 0 && lse) lse[static_cast<size_t>(b) * H + h] = m + __logf(tot);
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    out[lane + 32 * k] = make_float4(acc[k].x * inv, acc[k].y * inv, acc[k].z * inv, acc[k].w * inv);
+  if (lane == 0 && lse) lse[static_cast<size_t>(b) * H + h] = m + __logf(tot);
 }
 
 }  // namespace attn

@@ -655,6 +655,7 @@ int mla_decode_attn(const mla_dims* dims, const void* q_cat, const void* q_lo,
     p.num_pages = num_pages;
     p.num_parts = parts;
     p.q_cat = static_cast<const __nv_bfloat16*>(q_cat);
+    p.pool = static_cast<const uint8_t*>(cache_pool);
     p.page_table = page_table;
     p.seq_lens = seq_lens;
     p.plan = plan;
@@ -682,8 +683,10 @@ int mla_decode_attn(const mla_dims* dims, const void* q_cat, const void* q_lo,
         c->status);
   }
   if ((rc = last_launch())) return rc;
-  attn::combine_kernel<<<dim3(H, B), 128, 0, st>>>(plan, B, parts, H, part_o, part_lse, o_lat,
-                                                   lse);
+  attn::combine_kernel<<<static_cast<unsigned>((static_cast<size_t>(B) * H +
+                                                 attn::kCombineWarps - 1) / attn::kCombineWarps),
+                         32 * attn::kCombineWarps, 0, st>>>(plan, B, parts, H, part_o, part_lse,
+                                                            o_lat, lse);
   return last_launch();
 }
 
@@ -714,8 +717,8 @@ int mla_out_proj(const mla_dims* dims, const float* o_lat, const void* w_uv, con
     const GemmShape s1 = shape_wuv(dims);
     const int Bp = s1.n_lo;
     const size_t n = static_cast<size_t>(B) * H * kDc;
-    split_hi_lo_kernel<<<static_cast<unsigned>(std::min<size_t>((n + 255) / 256, 4096)), 256, 0,
-                         st>>>(o_lat, n, static_cast<size_t>(Bp) * H * kDc, os);
+    split_hi_lo_kernel<<<static_cast<unsigned>(std::min<size_t>((n / 8 + 255) / 256, 4096)), 256,
+                         0, st>>>(o_lat, n, static_cast<size_t>(Bp) * H * kDc, os);
     if ((rc = last_launch())) return rc;
     // o_h = W_UV_h [o_lat_hi | o_lat_lo]
     const SkPlan q1 = sk_plan(s1, 0, c->sms);
@@ -918,6 +921,7 @@ extern "C" int mla_decode_attn_static_scratch(const mla_dims* dims, const void* 
     p.num_pages = num_pages;
     p.num_parts = parts;
     p.q_cat = static_cast<const __nv_bfloat16*>(q_cat);
+    p.pool = static_cast<const uint8_t*>(cache_pool);
     p.page_table = page_table;
     p.seq_lens = seq_lens;
     p.plan = plan;
@@ -937,7 +941,9 @@ extern "C" int mla_decode_attn_static_scratch(const mla_dims* dims, const void* 
         c->status);
   }
   if ((rc = last_launch())) return rc;
-  attn::combine_kernel<<<dim3(H, B), 128, 0, st>>>(plan, B, parts, H, part_o, part_lse, o_lat,
-                                                   lse);
+  attn::combine_kernel<<<static_cast<unsigned>((static_cast<size_t>(B) * H +
+                                                 attn::kCombineWarps - 1) / attn::kCombineWarps),
+                         32 * attn::kCombineWarps, 0, st>>>(plan, B, parts, H, part_o, part_lse,
+                                                            o_lat, lse);
   return last_launch();
 }
