@@ -167,6 +167,8 @@ __device__ inline int part_of_page(int64_t g, int C, int P) {
 __global__ void __launch_bounds__(kPlanThreads)
     plan_kernel(const int32_t* __restrict__ seq_lens, int B, int max_pages, int C_req,
                 int min_pages_per_part, int32_t* __restrict__ plan, unsigned int* status) {
+  griddep_launch_dependents();
+  griddep_wait();
   __shared__ int warp_sums[32];
   __shared__ int s_total;
   int32_t* pg = plan + 4;
@@ -375,6 +377,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
   WaitCtx wc{&bars->abort_flag, p.status, p.wait_ns};
+  // everything below reads what the preceding kernels wrote (plan, q_cat, the appended rows)
+  griddep_launch_dependents();
+  griddep_wait();
 
   const PlanView plan(p.plan, p.batch, p.num_parts);
   const int n_parts = plan.parts();
@@ -816,6 +821,8 @@ __global__ void __launch_bounds__(32 * kCombineWarps)
     combine_kernel(const int32_t* __restrict__ plan_words, int B, int C, int H,
                    const float* __restrict__ part_o, const float* __restrict__ part_lse,
                    float* __restrict__ o_lat, float* __restrict__ lse) {
+  griddep_launch_dependents();
+  griddep_wait();
   const PlanView plan(plan_words, B, C);
   const int wid = blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;

@@ -153,6 +153,8 @@ __global__ void wuk_epilogue_kernel(const float* __restrict__ part, int n_pad, i
 // 32-byte load and two 16-byte stores.
 __global__ void split_hi_lo_kernel(const float* __restrict__ x, size_t n, size_t plane,
                                    __nv_bfloat16* __restrict__ out) {
+  griddep_launch_dependents();
+  griddep_wait();
   const size_t n8 = n / 8;
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n8;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {

@@ -438,6 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   WaitCtx wc{abort_flag, p.status, p.wait_ns};
+  griddep_launch_dependents();
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -448,11 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmX);
       const uint64_t pol_w = l2_policy_evict_first();
       const uint64_t pol_x = l2_policy_evict_last();
-      long long issued = 0;
-      for (long long i = i_begin; i < i_end; ++i, ++issued) {
-        const int s = static_cast<int>(issued % p.stages);
-        const uint32_t ph = static_cast<uint32_t>((issued / p.stages) & 1);
-        if (issued >= p.stages && !mbar_wait(&empty_bar[s], ph ^ 1, wc)) break;
+      auto load_a = [&](long long i, int s) {
         const long long t = i / kb;
         const int kb0 = static_cast<int>(i - t * kb) * p.kbs;
         const int g = static_cast<int>(t / p.m_tiles);
@@ -467,8 +464,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           m_row0 = (mt - p.a1_tile_start) * 128;
         }
         uint8_t* a_dst = smem + s * sbytes;
-        uint8_t* x_dst = a_dst + a_bytes;
-        mbar_arrive_expect_tx(&full_bar[s], sbytes);
         if (p.a_mn_major) {
           // [g][k][m] with m contiguous: box (64 m, 64 kbs k) per 64-row half of the tile
           tma_load_3d_hint(a_dst, tmA, &full_bar[s], m_row0, kb0 * 64, g, pol_w);
@@ -478,8 +473,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           // view (64 k, rows, groups, k blocks): box (64, 128, 1, kbs)
           tma_load_4d_hint(a_dst, tmA, &full_bar[s], 0, m_row0, g, kb0, pol_w);
         }
+      };
+      auto load_x = [&](long long i, int s) {
+        const long long t = i / kb;
+        const int kb0 = static_cast<int>(i - t * kb) * p.kbs;
+        const int g = static_cast<int>(t / p.m_tiles);
         // view (64 k, groups, n, k blocks): box (64, 1, n_pad, kbs)
-        tma_load_4d_hint(x_dst, &tmX, &full_bar[s], 0, g, 0, kb0, pol_x);
+        tma_load_4d_hint(smem + s * sbytes + a_bytes, &tmX, &full_bar[s], 0, g, 0, kb0, pol_x);
+      };
+      // The weights never depend on the preceding kernel: the first ring's worth of weight
+      // tiles is requested before waiting for that kernel to finish, the activations after.
+      const long long pre = min(i_end - i_begin, static_cast<long long>(p.stages));
+      for (long long j = 0; j < pre; ++j) {
+        mbar_arrive_expect_tx(&full_bar[j], sbytes);
+        load_a(i_begin + j, static_cast<int>(j));
+      }
+      griddep_wait();
+      for (long long j = 0; j < pre; ++j) load_x(i_begin + j, static_cast<int>(j));
+      long long issued = pre;
+      for (long long i = i_begin + pre; i < i_end; ++i, ++issued) {
+        const int s = static_cast<int>(issued % p.stages);
+        const uint32_t ph = static_cast<uint32_t>((issued / p.stages) & 1);
+        if (!mbar_wait(&empty_bar[s], ph ^ 1, wc)) break;
+        mbar_arrive_expect_tx(&full_bar[s], sbytes);
+        load_a(i, s);
+        load_x(i, s);
       }
       if (*abort_flag) {
         // wait (bounded, ignoring the abort flag) for every copy still landing in the ring
@@ -537,7 +555,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- epilogue ----------------
     const int quarter = warp & 3;
     const int m_local = quarter * 32 + lane;
-    // per-CTA epilogue tables while the first tiles stream in (epilogue warps only)
+    // per-CTA epilogue tables while the first tiles stream in (epilogue warps only), once the
+    // preceding kernel's writes are visible
+    griddep_wait();
     epi.prepare(epi_smem, p.n_out, threadIdx.x - 64, 128);
     asm volatile("bar.sync 1, 128;" ::: "memory");
     const int n_cols = p.n_lo > 0 ? p.n_lo : p.n_pad;  // columns that are outputs

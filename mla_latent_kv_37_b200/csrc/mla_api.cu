@@ -7,9 +7,11 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <atomic>
 #include <mutex>
+#include <utility>
 
 #include "attn_f32.cuh"
 #include "attn_sm100.cuh"
@@ -340,6 +342,34 @@ int last_launch(int kernels = 1) {
   return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
+// The kernels of the bf16 decode path are launched with programmatic stream serialisation:
+// each may be scheduled while its predecessor on the stream drains, and waits for it
+// (griddep_wait) before it touches that kernel's results.  MLA_NO_PDL=1 in the environment
+// launches them as ordinary stream-ordered kernels.  A failure is reported by last_launch().
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("MLA_NO_PDL");
+    return !(e && e[0] == '1');
+  }();
+  return on;
+}
+
+template <typename... KArgs, typename... Args>
+void launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr{};
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  (void)cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // A profiling event on `st`.  Under stream capture it becomes an external event node, which
 // records a timestamp every time the graph runs (a plain record inside a capture does not).
 cudaError_t record_profile_event(cudaEvent_t ev, cudaStream_t st) {
@@ -379,8 +409,8 @@ int run_streamk(const DevCtx* c, const GemmShape& s, const SkPlan& q, int n_out,
   p.rope_theta = theta;
   p.status = c->status;
   p.wait_ns = kDefaultWaitNs;
-  sk::streamk_gemm_kernel<Epi><<<q.ctas, sk::kThreads, q.smem, st>>>(a0, a1, a2 ? *a2 : a1,
-                                                                      xmap, p, epi);
+  launch_pdl(sk::streamk_gemm_kernel<Epi>, dim3(q.ctas), dim3(sk::kThreads), q.smem, st, a0, a1,
+             a2 ? *a2 : a1, xmap, p, epi);
   return last_launch();
 }
 
@@ -633,8 +663,8 @@ int mla_decode_attn(const mla_dims* dims, const void* q_cat, const void* q_lo,
   float* part_lse = reinterpret_cast<float*>(ws + w.part_lse);
   const float scale =
       softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(kDn + kDr));
-  attn::plan_kernel<<<1, attn::kPlanThreads, 0, st>>>(seq_lens, B, max_pages, parts,
-                                                      kMinPagesPerPart, plan, c->status);
+  launch_pdl(attn::plan_kernel, dim3(1), dim3(attn::kPlanThreads), 0, st, seq_lens, B, max_pages,
+             parts, kMinPagesPerPart, plan, c->status);
   if ((rc = last_launch())) return rc;
   if (dims->dtype == MLA_BF16) {
     CUtensorMap tc_lat, tc_rope, tq_rope;
@@ -669,8 +699,8 @@ int mla_decode_attn(const mla_dims* dims, const void* q_cat, const void* q_lo,
     const bool prof = g_prof_next < g_prof_count;
     if (prof && record_profile_event(g_prof_begin[g_prof_next], st) != cudaSuccess)
       return MLA_ERR_CUDA;
-    attn::split_kernel<<<2 * parts, attn::kThreads, attn::kSmemBytes, st>>>(tc_lat, tc_rope,
-                                                                            tq_rope, p);
+    launch_pdl(attn::split_kernel, dim3(2 * parts), dim3(attn::kThreads), attn::kSmemBytes, st,
+               tc_lat, tc_rope, tq_rope, p);
     if (prof) {
       if ((rc = last_launch())) return rc;
       if (record_profile_event(g_prof_end[g_prof_next++], st) != cudaSuccess) return MLA_ERR_CUDA;
@@ -683,10 +713,11 @@ int mla_decode_attn(const mla_dims* dims, const void* q_cat, const void* q_lo,
         c->status);
   }
   if ((rc = last_launch())) return rc;
-  attn::combine_kernel<<<static_cast<unsigned>((static_cast<size_t>(B) * H +
-                                                 attn::kCombineWarps - 1) / attn::kCombineWarps),
-                         32 * attn::kCombineWarps, 0, st>>>(plan, B, parts, H, part_o, part_lse,
-                                                            o_lat, lse);
+  launch_pdl(attn::combine_kernel,
+             dim3(static_cast<unsigned>((static_cast<size_t>(B) * H + attn::kCombineWarps - 1) /
+                                        attn::kCombineWarps)),
+             dim3(32 * attn::kCombineWarps), 0, st, plan, B, parts, H, part_o, part_lse, o_lat,
+             lse);
   return last_launch();
 }
 
@@ -717,8 +748,9 @@ int mla_out_proj(const mla_dims* dims, const float* o_lat, const void* w_uv, con
     const GemmShape s1 = shape_wuv(dims);
     const int Bp = s1.n_lo;
     const size_t n = static_cast<size_t>(B) * H * kDc;
-    split_hi_lo_kernel<<<static_cast<unsigned>(std::min<size_t>((n / 8 + 255) / 256, 4096)), 256,
-                         0, st>>>(o_lat, n, static_cast<size_t>(Bp) * H * kDc, os);
+    launch_pdl(split_hi_lo_kernel,
+               dim3(static_cast<unsigned>(std::min<size_t>((n / 8 + 255) / 256, 4096))), dim3(256),
+               0, st, o_lat, n, static_cast<size_t>(Bp) * H * kDc, os);
     if ((rc = last_launch())) return rc;
     // o_h = W_UV_h [o_lat_hi | o_lat_lo]
     const SkPlan q1 = sk_plan(s1, 0, c->sms);
@@ -899,8 +931,8 @@ extern "C" int mla_decode_attn_static_scratch(const mla_dims* dims, const void* 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const float scale =
       softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(kDn + kDr));
-  attn::plan_kernel<<<1, attn::kPlanThreads, 0, st>>>(seq_lens, B, max_pages, parts,
-                                                      kMinPagesPerPart, plan, c->status);
+  launch_pdl(attn::plan_kernel, dim3(1), dim3(attn::kPlanThreads), 0, st, seq_lens, B, max_pages,
+             parts, kMinPagesPerPart, plan, c->status);
   if ((rc = last_launch())) return rc;
   if (dims->dtype == MLA_BF16) {
     CUtensorMap tc_lat, tc_rope, tq_rope;
@@ -932,8 +964,8 @@ extern "C" int mla_decode_attn_static_scratch(const mla_dims* dims, const void* 
     p.part_lse = part_lse;
     p.status = c->status;
     p.wait_ns = kDefaultWaitNs;
-    attn::split_kernel<<<2 * parts, attn::kThreads, attn::kSmemBytes, st>>>(tc_lat, tc_rope,
-                                                                            tq_rope, p);
+    launch_pdl(attn::split_kernel, dim3(2 * parts), dim3(attn::kThreads), attn::kSmemBytes, st,
+               tc_lat, tc_rope, tq_rope, p);
   } else {
     attn::f32_split_kernel<<<dim3(parts, H), 128, 0, st>>>(
         static_cast<const float*>(q_cat), static_cast<const float*>(cache_pool), page_table,
@@ -941,9 +973,10 @@ extern "C" int mla_decode_attn_static_scratch(const mla_dims* dims, const void* 
         c->status);
   }
   if ((rc = last_launch())) return rc;
-  attn::combine_kernel<<<static_cast<unsigned>((static_cast<size_t>(B) * H +
-                                                 attn::kCombineWarps - 1) / attn::kCombineWarps),
-                         32 * attn::kCombineWarps, 0, st>>>(plan, B, parts, H, part_o, part_lse,
-                                                            o_lat, lse);
+  launch_pdl(attn::combine_kernel,
+             dim3(static_cast<unsigned>((static_cast<size_t>(B) * H + attn::kCombineWarps - 1) /
+                                        attn::kCombineWarps)),
+             dim3(32 * attn::kCombineWarps), 0, st, plan, B, parts, H, part_o, part_lse, o_lat,
+             lse);
   return last_launch();
 }

@@ -123,6 +123,16 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
 // ------------------------------------------------------------------------------------------
 // TMA (tensor copies global -> shared, completion counted on an mbarrier)
 // ------------------------------------------------------------------------------------------
+// Programmatic dependent launch.  A kernel launched with programmatic stream serialisation may
+// start while the preceding kernel on its stream is still running: it must call griddep_wait()
+// before it touches anything that kernel writes (or reads), and griddep_launch_dependents()
+// lets the following kernel be scheduled as soon as every CTA of this one has called it.
+// Both are no-ops when the kernel was launched normally.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Bulk prefetch of a contiguous global range into L2 (address and size multiples of 16 B).
 __device__ __forceinline__ void prefetch_l2(const void* a, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a), "r"(bytes) : "memory");
