@@ -20,6 +20,10 @@
  *     allocates or frees memory and keeps no state between calls other than one device status
  *     word per GPU (see mla_get_status).
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *     The bf16 kernels are launched with programmatic stream serialisation: one may be
+ *     scheduled while the work before it on the stream drains, but it reads and writes nothing
+ *     until that work has completed, so stream order holds exactly as for ordinary launches.
+ *     Setting MLA_NO_PDL=1 in the environment before the first call turns this off.
  *   - Weights are row-major [out_features, in_features] (column-vector form, [TN]):
  *       w_dkv [d_c, D], w_kr [d_rope, D], w_q [H*(d_nope+d_rope), D] (per head d_nope rows then
  *       d_rope rows), w_uk [H*d_nope, d_c], w_uv [H*d_v, d_c], w_o [D, H*d_v].
