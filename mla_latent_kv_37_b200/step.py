@@ -3,7 +3,8 @@
 A step, per layer l (each layer has its own weights, paged cache and hidden state h[l]):
     mla_append_absorb (= mla_cache_append + mla_absorb_q) -> mla_decode_attn -> mla_out_proj
 Everything stays on the device; `run_host` adds the host<->device copies of the step's inputs
-and results (pinned buffers) for end-to-end measurement.  Marshalling only: no arithmetic.
+and results (pinned buffers), overlapped layer by layer with the kernels, for end-to-end use.
+Marshalling only: no arithmetic.
 """
 from __future__ import annotations
 
@@ -46,6 +47,10 @@ class DecodeStep:
         self.graph = graph
         self._graphs: dict = {}
         self.launches_per_step = 0
+        # end-to-end path: one copy stream per direction, one event per layer and direction
+        self._copy_in = self._copy_out = None
+        self._ev_in: list = []
+        self._ev_out: list = []
 
     def run(self, h, positions, seq_lens, stream=None):
         """h [L, B, D] on the device; positions [B] (append slot), seq_lens [B] = positions+1."""
@@ -78,23 +83,64 @@ class DecodeStep:
         self._graphs[(h.data_ptr(), positions.data_ptr(), seq_lens.data_ptr())] = g
         return g
 
+    def _layer(self, l, h_l, positions, seq_lens, stream=None):
+        d, ly = self.dims, self.layers[l]
+        mla_append_absorb(d, h_l, ly.w_dkv, ly.w_kr, ly.w_q, ly.w_uk, positions, ly.page_table,
+                          ly.pool, self.q_cat, self.ws, stream=stream)
+        mla_decode_attn(d, self.q_cat, ly.pool, ly.page_table, seq_lens, self.o_lat, self.ws,
+                        lse=self.lse, num_splits=self.num_splits, stream=stream)
+        mla_out_proj(d, self.o_lat, ly.w_uv, self.ws, w_o=ly.w_o, o_heads=self.o_heads[l],
+                     out=self.out[l] if ly.w_o is not None else None, stream=stream)
+
     def _run(self, h, positions, seq_lens, stream=None):
-        d = self.dims
-        for l, ly in enumerate(self.layers):
-            mla_append_absorb(d, h[l], ly.w_dkv, ly.w_kr, ly.w_q, ly.w_uk, positions,
-                              ly.page_table, ly.pool, self.q_cat, self.ws, stream=stream)
-            mla_decode_attn(d, self.q_cat, ly.pool, ly.page_table, seq_lens, self.o_lat, self.ws,
-                            lse=self.lse, num_splits=self.num_splits, stream=stream)
-            mla_out_proj(d, self.o_lat, ly.w_uv, self.ws, w_o=ly.w_o, o_heads=self.o_heads[l],
-                         out=self.out[l] if ly.w_o is not None else None, stream=stream)
+        for l in range(len(self.layers)):
+            self._layer(l, h[l], positions, seq_lens, stream)
+
+    def _run_layer(self, l, h_l, positions, seq_lens, stream):
+        """Layer l on `stream`: eagerly, or (graph mode) as that layer's own captured graph."""
+        if not self.graph:
+            self._layer(l, h_l, positions, seq_lens, stream)
+            return
+        key = ("layer", l, h_l.data_ptr(), positions.data_ptr(), seq_lens.data_ptr())
+        g = self._graphs.get(key)
+        if g is None:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self._layer(l, h_l, positions, seq_lens)
+            self._graphs[key] = g
+        with torch.cuda.stream(stream):
+            g.replay()
 
     def run_host(self, h_host, pos_host, lens_host, out_host, h_dev, pos_dev, lens_dev,
                  stream=None):
-        """End-to-end: copy the step's inputs from pinned host memory, run, copy `out` back."""
+        """End-to-end: the step's inputs come from pinned host memory and `out` goes back to
+        pinned host memory.  The copies overlap the kernels: every layer's hidden state goes up
+        on one copy stream ahead of that layer, every layer's output comes back on another as
+        soon as the layer has written it, and the step (on `stream`) ends when the last output
+        is on the host.  Only the first layer's input and the last layer's output are exposed.
+        In graph mode each layer is its own captured graph, so that the copies can interleave;
+        the device library must already be set up (one eager or graph step run before)."""
         s = torch.cuda.current_stream() if stream is None else stream
-        with torch.cuda.stream(s):
-            h_dev.copy_(h_host, non_blocking=True)
+        L = len(self.layers)
+        if self._copy_in is None:
+            self._copy_in, self._copy_out = torch.cuda.Stream(), torch.cuda.Stream()
+            self._ev_in = [torch.cuda.Event() for _ in range(L)]
+            self._ev_out = [torch.cuda.Event() for _ in range(L)]
+        cin, cout = self._copy_in, self._copy_out
+        # the device buffers are free once everything already queued on `stream` has run
+        cin.wait_stream(s)
+        cout.wait_stream(s)
+        with torch.cuda.stream(cin):
             pos_dev.copy_(pos_host, non_blocking=True)
             lens_dev.copy_(lens_host, non_blocking=True)
-            self.run(h_dev, pos_dev, lens_dev, stream=s)
-            out_host.copy_(self.out, non_blocking=True)
+            for l in range(L):
+                h_dev[l].copy_(h_host[l], non_blocking=True)
+                self._ev_in[l].record(cin)
+        for l in range(L):
+            s.wait_event(self._ev_in[l])
+            self._run_layer(l, h_dev[l], pos_dev, lens_dev, s)
+            self._ev_out[l].record(s)
+            cout.wait_event(self._ev_out[l])
+            with torch.cuda.stream(cout):
+                out_host[l].copy_(self.out[l], non_blocking=True)
+        s.wait_stream(cout)
