@@ -96,38 +96,15 @@ class DecodeStep:
         for l in range(len(self.layers)):
             self._layer(l, h[l], positions, seq_lens, stream)
 
-    def _run_layer(self, l, h_l, positions, seq_lens, stream):
-        """Layer l on `stream`: eagerly, or (graph mode) as that layer's own captured graph."""
-        if not self.graph:
-            self._layer(l, h_l, positions, seq_lens, stream)
-            return
-        key = ("layer", l, h_l.data_ptr(), positions.data_ptr(), seq_lens.data_ptr())
-        g = self._graphs.get(key)
-        if g is None:
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                self._layer(l, h_l, positions, seq_lens)
-            self._graphs[key] = g
-        with torch.cuda.stream(stream):
-            g.replay()
-
-    def run_host(self, h_host, pos_host, lens_host, out_host, h_dev, pos_dev, lens_dev,
-                 stream=None):
-        """End-to-end: the step's inputs come from pinned host memory and `out` goes back to
-        pinned host memory.  The copies overlap the kernels: every layer's hidden state goes up
-        on one copy stream ahead of that layer, every layer's output comes back on another as
-        soon as the layer has written it, and the step (on `stream`) ends when the last output
-        is on the host.  Only the first layer's input and the last layer's output are exposed.
-        In graph mode each layer is its own captured graph, so that the copies can interleave;
-        the device library must already be set up (one eager or graph step run before)."""
-        s = torch.cuda.current_stream() if stream is None else stream
+    def _host_step(self, h_host, pos_host, lens_host, out_host, h_dev, pos_dev, lens_dev):
+        """Enqueue one host-path step on the current stream, eagerly or under graph capture.
+        Every layer's hidden state goes up on one copy stream ahead of that layer, every
+        layer's output comes back on another as soon as the layer has written it, and the
+        step ends when the last output is on the host."""
+        s = torch.cuda.current_stream()
         L = len(self.layers)
-        if self._copy_in is None:
-            self._copy_in, self._copy_out = torch.cuda.Stream(), torch.cuda.Stream()
-            self._ev_in = [torch.cuda.Event() for _ in range(L)]
-            self._ev_out = [torch.cuda.Event() for _ in range(L)]
         cin, cout = self._copy_in, self._copy_out
-        # the device buffers are free once everything already queued on `stream` has run
+        # the device buffers are free once everything already queued on `s` has run
         cin.wait_stream(s)
         cout.wait_stream(s)
         with torch.cuda.stream(cin):
@@ -138,9 +115,40 @@ class DecodeStep:
                 self._ev_in[l].record(cin)
         for l in range(L):
             s.wait_event(self._ev_in[l])
-            self._run_layer(l, h_dev[l], pos_dev, lens_dev, s)
+            self._layer(l, h_dev[l], pos_dev, lens_dev)
             self._ev_out[l].record(s)
             cout.wait_event(self._ev_out[l])
             with torch.cuda.stream(cout):
                 out_host[l].copy_(self.out[l], non_blocking=True)
         s.wait_stream(cout)
+
+    def run_host(self, h_host, pos_host, lens_host, out_host, h_dev, pos_dev, lens_dev,
+                 stream=None):
+        """End-to-end: the step's inputs come from pinned host memory and `out` goes back to
+        pinned host memory, the copies overlapped with the kernels (only the first layer's
+        input and the last layer's output are exposed).  In graph mode the whole host-path
+        step, copies and both copy streams included, is one graph per set of buffers, captured
+        after one eager run of it."""
+        s = torch.cuda.current_stream() if stream is None else stream
+        if self._copy_in is None:
+            L = len(self.layers)
+            self._copy_in, self._copy_out = torch.cuda.Stream(), torch.cuda.Stream()
+            self._ev_in = [torch.cuda.Event() for _ in range(L)]
+            self._ev_out = [torch.cuda.Event() for _ in range(L)]
+        bufs = (h_host, pos_host, lens_host, out_host, h_dev, pos_dev, lens_dev)
+        if not self.graph:
+            with torch.cuda.stream(s):
+                self._host_step(*bufs)
+            return
+        key = ("host",) + tuple(t.data_ptr() for t in bufs)
+        g = self._graphs.get(key)
+        if g is None:
+            with torch.cuda.stream(s):
+                self._host_step(*bufs)  # one-time library set-up happens outside the capture
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self._host_step(*bufs)
+            self._graphs[key] = g
+        with torch.cuda.stream(s):
+            g.replay()
