@@ -16,6 +16,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import math
 import os
@@ -277,10 +278,13 @@ def parity_sample(layers, h, hist, step, cfg, n_layers=2, n_seqs=2, n_heads=8, s
 # traffic figure from a committed ncu summary, valid only for the exact kernel source
 # ---------------------------------------------------------------------------------------------
 def kernel_source_hash():
+    """Hash of the split kernel's code: its two source files without // comments and blank
+    lines, so that editing a comment does not invalidate the recorded counters."""
     hsh = hashlib.sha256()
     for f in ("attn_sm100.cuh", "ptx_sm100.cuh"):
-        with open(os.path.join(ROOT, "mla_latent_kv_37_b200", "csrc", f), "rb") as fh:
-            hsh.update(fh.read())
+        with open(os.path.join(ROOT, "mla_latent_kv_37_b200", "csrc", f)) as fh:
+            lines = [re.sub(r"//.*$", "", ln).rstrip() for ln in fh.read().splitlines()]
+        hsh.update("\n".join(ln for ln in lines if ln.strip()).encode())
     return hsh.hexdigest()[:16]
 
 

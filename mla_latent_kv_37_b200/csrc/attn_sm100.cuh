@@ -16,6 +16,8 @@
 //     64B swizzle), and so does P (bf16, 128B swizzle, A operand of PV), so an S buffer is
 //     free again as soon as it has been drained and QK runs two pages ahead of the softmax.
 //   * Pages arrive by TMA (128B/64B swizzle) into a 4-stage ring; each byte leaves HBM once.
+//     Four pages ahead of the ring each CTA issues a bulk L2 prefetch of half of the page's
+//     rows, so the ring's loads find their lines in L2.
 //   * S_r = Q_r C_r^T is a partial score; the pair exchanges partials.  Distributed shared
 //     memory moves ~16 B/clk per SM, so a partial travels as 16-bit fixed point relative to
 //     its row's largest magnitude (error <= 2^-16 of it, ~1e-4 in the softmax logit), staged
