@@ -301,6 +301,82 @@ def committed_traffic(config_name):
 
 
 # ---------------------------------------------------------------------------------------------
+# single-layer attention sweep: mla_decode_attn alone over batch x context
+# ---------------------------------------------------------------------------------------------
+SWEEP_BATCH = (32, 64, 128)
+SWEEP_CONTEXT = (8192, 16384, 32768)
+
+
+def run_sweep(args):
+    """mla_decode_attn (plan + split + combine) on one layer for every batch x context of the
+    sweep, 128 heads, full pages, random page placement: `--sweep-warmup` untimed and
+    `--sweep-iters` timed calls per shape, the L2 flushed (a 256 MB write) before every timed
+    call, CUDA events around each call.  One JSON line per shape: median / p10 / p90 time and the
+    fraction of the roofline, against the burst peaks (the call is timed alone)."""
+    import json as _json
+
+    import mla_inputs as I
+    import mla_latent_kv_37_b200 as M
+    from mla_latent_kv_37_b200 import build
+    build.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks = {}
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peaks = _json.load(f)
+    except Exception:
+        pass
+    hbm_peak = peaks.get("hbm_gbs", 6650.0)
+    tc_peak = peaks.get("bf16_tflops", 1590.0)
+    src = "of measured" if peaks else "of fallback"
+    H = 128
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for B in SWEEP_BATCH:
+        for N in SWEEP_CONTEXT:
+            q = I.query_cat(7, B, H, device=dev)
+            cache = I.paged_cache(8, [N] * B, [N] * B, device=dev)
+            lens = torch.full((B,), N, dtype=torch.int32, device=dev)
+            d = M.dims(B, H, 7168)
+            ws = M.workspace(d, 0, dev)
+            o = torch.empty(B, H, 512, dtype=torch.float32, device=dev)
+            lse = torch.empty(B, H, dtype=torch.float32, device=dev)
+            for _ in range(args.sweep_warmup):
+                M.mla_decode_attn(d, q, cache.pool, cache.page_table, lens, o, ws, lse=lse)
+            torch.cuda.synchronize()
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.sweep_iters)]
+            for i, (e0, e1) in enumerate(ev):
+                flush.fill_(i & 0xFF)
+                e0.record()
+                M.mla_decode_attn(d, q, cache.pool, cache.page_table, lens, o, ws, lse=lse)
+                e1.record()
+            torch.cuda.synchronize()
+            st = M.mla_get_status()
+            if st:
+                raise RuntimeError(f"device status {st:#x} in the sweep (B={B}, N={N})")
+            us = sorted(e0.elapsed_time(e1) * 1e3 for e0, e1 in ev)
+            pick = lambda f: us[min(len(us) - 1, int(f * (len(us) - 1) + 0.5))]
+            med = pick(0.5)
+            tokens = B * N
+            nbytes = tokens * ROW_BYTES + B * H * 576 * 2 + B * H * 512 * 4
+            flops = tokens * H * FLOP_PER_TOKEN_HEAD
+            t_hbm = nbytes / (hbm_peak * 1e9) * 1e6
+            t_tc = flops / (tc_peak * 1e12) * 1e6
+            print(_json.dumps({
+                "metric": "mla_decode_attn, one layer (plan + split + combine)",
+                "batch": B, "context": N, "heads": H, "us_median": med, "us_p10": pick(0.1),
+                "us_p90": pick(0.9), "tflops": flops / (med * 1e-6) / 1e12,
+                "gbs": nbytes / (med * 1e-6) / 1e9, "bound": "hbm" if t_hbm >= t_tc else "tensor",
+                "roofline_us": max(t_hbm, t_tc), "frac": max(t_hbm, t_tc) / med,
+                "peaks": {"hbm_gbs": hbm_peak, "bf16_tflops": tc_peak, "source": src + " (burst)"},
+                "warmup": args.sweep_warmup, "timed": args.sweep_iters,
+                "l2": "flushed by a 256 MB write before every timed call"}), flush=True)
+            del q, cache, lens, ws, o, lse
+            torch.cuda.empty_cache()
+
+
+# ---------------------------------------------------------------------------------------------
 def run_reference(args, rank, world):
     """The oracle arm: times the fp64 CPU oracle on bounded samples of the same workload."""
     if rank != 0:
@@ -354,7 +430,15 @@ def main():
                     help="launch every kernel eagerly instead of replaying a captured step")
     ap.add_argument("--ref-seconds", type=float, default=0.0,
                     help="reference arm: CPU seconds per timed sample (0 = fit a few minutes)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time mla_decode_attn alone on one layer over batch {32,64,128} x "
+                         "context {8K,16K,32K} (one JSON line per shape) instead of the step")
+    ap.add_argument("--sweep-warmup", type=int, default=10)
+    ap.add_argument("--sweep-iters", type=int, default=50)
     args = ap.parse_args()
+    if args.sweep:
+        run_sweep(args)
+        return
     if args.impl == "reference":
         # the CPU oracle arm: rank 0 alone runs it; under torchrun the other ranks exit at once
         run_reference(args, int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")))
