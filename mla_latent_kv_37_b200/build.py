@@ -2,7 +2,6 @@
 from __future__ import annotations
 
 import os
-import re
 import shutil
 import subprocess
 import sys
@@ -35,43 +34,16 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(d) <= t for d in DEPS)
 
 
-# When the decode split kernel re-divides its registers between warpgroups (setmaxnreg), the
-# division assumes it is compiled to exactly kLaunchRegs registers per thread.
-SPLIT_KERNEL = "_ZN3mla4attn12split_kernel"
-
-
-def split_kernel_regs() -> int:
-    with open(os.path.join(HERE, "csrc", "attn_sm100.cuh")) as f:
-        m = re.search(r"constexpr int kLaunchRegs = (\d+);", f.read())
-    return int(m.group(1)) if m else 0
-
-
-def check_split_kernel_regs(ptxas_log: str) -> None:
-    want = split_kernel_regs()
-    if want == 0:
-        return
-    lines = ptxas_log.splitlines()
-    for i, ln in enumerate(lines):
-        if "Function properties for" in ln and SPLIT_KERNEL in ln:
-            for nxt in lines[i + 1:i + 4]:
-                m = re.search(r"Used (\d+) registers", nxt)
-                if m:
-                    if int(m.group(1)) != want:
-                        raise RuntimeError(f"split_kernel compiled to {m.group(1)} registers per "
-                                           f"thread, expected {want}")
-                    return
-    raise RuntimeError("ptxas did not report the register count of split_kernel")
-
-
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and up_to_date():
         return LIB
     tmp = LIB + ".tmp"
-    cmd = command(tmp, extra=("-Xptxas", "-v"))
+    cmd = command(tmp, extra=("-Xptxas", "-v") if verbose else ())
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     res = subprocess.run(cmd, check=True, capture_output=True, text=True)
-    check_split_kernel_regs(res.stdout + res.stderr)
+    if verbose:
+        print(res.stdout + res.stderr, file=sys.stderr)
     os.replace(tmp, LIB)
     return LIB
 

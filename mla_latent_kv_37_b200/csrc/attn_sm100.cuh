@@ -70,9 +70,6 @@ constexpr uint32_t kTmemO = 0, kTmemQ = 256, kTmemS = 384, kTmemCols = 512;
 constexpr int kAhead = 4;  // pages prefetched into L2 ahead of the TMA ring
 constexpr uint32_t kPageBytes = kPage * kRow * 2;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-// Registers per thread the split kernel must be built with when it re-divides them between
-// warpgroups (setmaxnreg); 0 = no re-division.
-constexpr int kLaunchRegs = 0;
 
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 static_assert(kTmemS + 2 * 64 == kTmemCols, "tensor memory budget");

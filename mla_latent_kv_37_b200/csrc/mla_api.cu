@@ -98,12 +98,6 @@ int device_ctx(DevCtx** out) {
       g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     }
     // kernel attributes (once per device)
-    // The split kernel re-divides its registers between warpgroups (setmaxnreg); that is only
-    // sound if it was built with exactly the per-thread count the division assumes.
-    cudaFuncAttributes fa{};
-    if (cudaFuncGetAttributes(&fa, attn::split_kernel) != cudaSuccess ||
-        (attn::kLaunchRegs != 0 && fa.numRegs != attn::kLaunchRegs))
-      return MLA_ERR_CUDA;
     const int attn_smem = static_cast<int>(attn::kSmemBytes);
     if (cudaFuncSetAttribute(attn::split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              attn_smem) != cudaSuccess)
