@@ -121,7 +121,8 @@ int mla_cache_append(const mla_dims* dims, const void* h, const void* w_dkv, con
  *   q_cat    [B, H, d_c + d_rope] (dims.dtype)
  *   q_lo     nullable; bf16 only: [B, H, d_c + d_rope] receives the rounding remainder
  *            q - bf16(q) of every element, so that q_cat + q_lo carries ~16 significant bits.
- *            Pass it on to mla_decode_attn when score logits are large (|logit| >> 10).
+ *            It is meant for large score logits (|logit| >> 10), where the bf16 rounding of
+ *            q_cat alone costs accuracy; mla_decode_attn does not consume it yet (see there).
  * q_nope is kept at ~16 bits (bf16 hi + lo) through the W_UK product; accumulation is fp32.
  */
 int mla_absorb_q(const mla_dims* dims, const void* h, const void* w_q, const void* w_uk,
@@ -147,7 +148,9 @@ int mla_append_absorb(const mla_dims* dims, const void* h, const void* w_dkv, co
  * cached row since the query is the newest token), in latent space:
  *   s_j = scale * (q_lat . c_j + q_rope . k_R,j),  j < seq_lens[b];   p = softmax(s);
  *   o_lat[b][h] = sum_j p_j c_j (d_c wide),   lse[b][h] = log sum_j exp(s_j).
- *   q_cat    [B, H, d_c + d_rope] (dims.dtype); q_lo nullable (bf16, see mla_absorb_q).
+ *   q_cat    [B, H, d_c + d_rope] (dims.dtype).
+ *   q_lo     must be NULL: the decode kernel does not consume the query's rounding remainder
+ *            yet (its tensor memory is fully in use), and a non-NULL q_lo returns MLA_ERR_ARG.
  *   seq_lens [B] int32 (rows to attend, including the token just appended); 0 is allowed
  *            and yields o_lat = 0, lse = -inf.
  *   softmax_scale: 0 selects 1/sqrt(d_nope + d_rope).
@@ -180,9 +183,10 @@ int mla_out_proj(const mla_dims* dims, const float* o_lat, const void* w_uv, con
  * A process whose memory manager already owns all of the GPU's memory, or a code path where a
  * cudaMalloc -- which may synchronise the device or fail under memory pressure -- is not
  * acceptable, cannot provide the workspace mla_decode_attn needs.  This entry point takes the
- * same arguments minus the workspace and keeps the split-KV scratch (page plan and per-part
- * partial results) in a fixed array of MLA_STATIC_SCRATCH_BYTES in the library's own device
- * data, which every GPU that loads the library holds until the process exits.  It allocates
+ * same arguments minus the workspace (q_lo must be NULL here too) and keeps the split-KV
+ * scratch (page plan and per-part partial results) in a fixed array of
+ * MLA_STATIC_SCRATCH_BYTES in the library's own device data, which every GPU that loads the
+ * library holds until the process exits.  It allocates
  * nothing.  Results equal mla_decode_attn's for the same arguments.
  *   - The scratch needed is about (batch + parts) * n_heads * 2 KiB (parts = num_splits, or
  *     the automatic choice); calls needing more than MLA_STATIC_SCRATCH_BYTES return
