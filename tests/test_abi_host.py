@@ -94,6 +94,18 @@ def test_null_and_alignment_errors(M):
     assert L.mla_out_proj(ctypes.byref(d), f, f, None, None, None, f, 1 << 30, None) == -1
 
 
+def test_decode_calls_reject_q_lo(M):
+    # Both decode entry points document q_lo as "must be NULL" (the kernel does not consume the
+    # query's rounding remainder): a non-NULL q_lo is an argument error, found on the host.
+    d = _d(M)
+    L = M.lib()
+    f = ctypes.c_void_p(0x10000)
+    assert L.mla_decode_attn(ctypes.byref(d), f, f, f, 10, f, 4, f, 0.0, 0, f, 1 << 30, f, None,
+                             None) == -5
+    assert L.mla_decode_attn_static_scratch(ctypes.byref(d), f, f, f, 10, f, 4, f, 0.0, 0, f,
+                                            None, None) == -5
+
+
 def test_valid_call_without_gpu_fails_loudly(M):
     import torch
     if torch.cuda.is_available():
