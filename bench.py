@@ -94,13 +94,19 @@ def max_over_ranks(x: float, world: int) -> float:
 # clocks sampled during the timed region
 # ---------------------------------------------------------------------------------------------
 class ClockSampler:
+    """nvidia-smi clock and throttle-reason samples, every `interval_ms`, each stamped with the
+    host time it arrived.  stop(t0, t1) summarises the samples that arrived inside the timed
+    window [t0, t1] (host seconds); if none did (a window shorter than the interval), the
+    sample nearest to the window's middle is used."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, interval_ms: int = 200):
         self.gpu = gpu_index
-        self.lines = []
+        self.interval_ms = interval_ms
+        self.lines = []  # (host time, csv line)
         self.proc = None
         self.thread = None
 
@@ -108,7 +114,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200", "-i", str(self.gpu)], stdout=subprocess.PIPE,
+                 "-lms", str(self.interval_ms), "-i", str(self.gpu)], stdout=subprocess.PIPE,
                 stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
@@ -118,9 +124,23 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.time(), line.strip()))
 
-    def stop(self):
+    @staticmethod
+    def parse(line):
+        """(sm MHz, max sm MHz, active reasons) of one csv line, or None."""
+        parts = [p.strip() for p in line.split(",")]
+        if len(parts) < 9:
+            return None
+        try:
+            sm, mx = float(parts[1]), float(parts[2])
+        except ValueError:
+            return None
+        active = {n for n, v in zip(ClockSampler.REASONS, parts[5:9])
+                  if v.lower().startswith("active")}
+        return sm, mx, active
+
+    def stop(self, t0=None, t1=None):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
@@ -130,24 +150,24 @@ class ClockSampler:
             self.proc.kill()
         if self.thread:
             self.thread.join(timeout=2)
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        sm.sort()
-        med = sm[len(sm) // 2] if sm else None
-        return {"sm_mhz": med, "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return self.summarise(self.lines, t0, t1)
+
+    @staticmethod
+    def summarise(lines, t0, t1, slack=0.0):
+        samples = [(t, r) for t, r in ((t, ClockSampler.parse(ln)) for t, ln in lines) if r]
+        if t0 is not None and t1 is not None and samples:
+            inside = [(t, r) for t, r in samples if t0 - slack <= t <= t1 + slack]
+            if not inside:
+                mid = 0.5 * (t0 + t1)
+                inside = [min(samples, key=lambda s: abs(s[0] - mid))]
+            samples = inside
+        sm = sorted(r[0] for _, r in samples)
+        reasons = set()
+        for _, r in samples:
+            reasons |= r[2]
+        return {"sm_mhz": sm[len(sm) // 2] if sm else None,
+                "sm_max_mhz": samples[-1][1][1] if samples else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
 
 
 # ---------------------------------------------------------------------------------------------
@@ -416,7 +436,7 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--config", default="full_61", choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -497,15 +517,17 @@ def main():
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     launches0 = M.mla_launch_count()
+    t_wall0 = time.time()
     e0.record(stream)
     for _ in range(args.steps):
         step.run(h, pos, lens_dev)
     e1.record(stream)
     torch.cuda.synchronize()
+    t_wall1 = time.time()
     launches = (step.launches_per_step * args.steps if graph
                 else M.mla_launch_count() - launches0)
     barrier(world)
-    clocks = sampler.stop()
+    clocks = sampler.stop(t_wall0, t_wall1)
     if not graph:
         used = M.mla_profile_events_used()
         M.mla_set_profile_events([], [])
