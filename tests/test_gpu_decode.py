@@ -108,6 +108,16 @@ def test_long_context(scale):
     _check(q, cache, lens, o, l)
 
 
+def test_headline_shape():
+    """The attention of one layer of the full decode step: batch 32 x 32768 tokens, 128 heads,
+    the automatic split (every sequence spread over several parts), every sequence checked."""
+    lens = [32768] * 32
+    q, cache = _case(5, lens, 128)
+    o, l, st = _run(q, cache, lens, 128)
+    assert st == 0
+    _check(q, cache, lens, o, l)
+
+
 def test_fp32_path():
     lens = [256, 100, 1]
     q, cache = _case(11, lens, 16, dtype=torch.float32)
