@@ -24,6 +24,11 @@
 // Roles (192 threads): warp 0 TMA producer, warp 1 MMA issuer + TMEM owner, warps 2-5
 // epilogue (warp w reads TMEM lanes 32*(w%4) .. +31, i.e. tile rows).
 //
+// Launched with programmatic stream serialisation: the kernel may start while the previous
+// kernel on its stream drains.  The producer requests its first ring of weight tiles at once
+// (weights never depend on an earlier kernel), then waits for that kernel (griddepcontrol.wait)
+// before it loads any activation; the epilogue warps wait before they touch global memory.
+//
 // Operand layouts in shared memory (128-byte swizzle, filled by TMA):
 //   A K-major : box (64 k, 128 m)   -> [128 rows][128 B], SBO = 1024 B
 //   A MN-major: 2 boxes (64 m, 64 k) -> [64 k rows][128 B] per 64-m half, LBO = 8 KiB
