@@ -122,7 +122,7 @@ int mla_cache_append(const mla_dims* dims, const void* h, const void* w_dkv, con
  *   q_lo     nullable; bf16 only: [B, H, d_c + d_rope] receives the rounding remainder
  *            q - bf16(q) of every element, so that q_cat + q_lo carries ~16 significant bits.
  *            It is meant for large score logits (|logit| >> 10), where the bf16 rounding of
- *            q_cat alone costs accuracy; mla_decode_attn does not consume it yet (see there).
+ *            q_cat alone costs accuracy; pass it on to mla_decode_attn.
  * q_nope is kept at ~16 bits (bf16 hi + lo) through the W_UK product; accumulation is fp32.
  */
 int mla_absorb_q(const mla_dims* dims, const void* h, const void* w_q, const void* w_uk,
@@ -149,14 +149,19 @@ int mla_append_absorb(const mla_dims* dims, const void* h, const void* w_dkv, co
  *   s_j = scale * (q_lat . c_j + q_rope . k_R,j),  j < seq_lens[b];   p = softmax(s);
  *   o_lat[b][h] = sum_j p_j c_j (d_c wide),   lse[b][h] = log sum_j exp(s_j).
  *   q_cat    [B, H, d_c + d_rope] (dims.dtype).
- *   q_lo     must be NULL: the decode kernel does not consume the query's rounding remainder
- *            yet (its tensor memory is fully in use), and a non-NULL q_lo returns MLA_ERR_ARG.
+ *   q_lo     nullable; bf16 only: [B, H, d_c + d_rope], the query's rounding remainder as
+ *            written by mla_absorb_q.  When given, the scores use q_cat + q_lo (~16 significant
+ *            bits instead of 8), for inputs whose logits are large enough (spread >> 10) that
+ *            the bf16 rounding of the query alone moves the output by more than ~1e-3.  It
+ *            costs about twice the tensor work (each cluster then handles 64 heads) and reads
+ *            the same cache bytes.  The workspace size does not change.
  *   seq_lens [B] int32 (rows to attend, including the token just appended); 0 is allowed
  *            and yields o_lat = 0, lse = -inf.
  *   softmax_scale: 0 selects 1/sqrt(d_nope + d_rope).
  *   num_splits: number of parts the concatenated page list of all sequences is divided into
- *            (split-KV); 0 = automatic (about one part per pair of SMs).  Must not exceed the
- *            value used for mla_workspace_size.
+ *            (split-KV); 0 = automatic (about one part per pair of SMs, or per four SMs with
+ *            q_lo).  At most 65536, and not more than the value used for mla_workspace_size.
+ *   num_pages * page_size and max_pages * page_size must fit in int32 (MLA_ERR_ARG).
  *   o_lat    [B, H, d_c] fp32;  lse [B, H] fp32, nullable.
  */
 int mla_decode_attn(const mla_dims* dims, const void* q_cat, const void* q_lo,

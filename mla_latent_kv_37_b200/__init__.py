@@ -213,7 +213,7 @@ def mla_decode_attn(d: mla_dims, q_cat, cache_pool, page_table, seq_lens, o_lat,
     _need(seq_lens, "seq_lens", torch.int32, (d.batch,))
     _need(o_lat, "o_lat", torch.float32, (d.batch, H, d.d_c))
     _need(lse, "lse", torch.float32, (d.batch, H))
-    _need(q_lo, "q_lo", torch.bfloat16)
+    _need(q_lo, "q_lo", torch.bfloat16, (d.batch, H, d.d_c + d.d_rope))
     _need(ws, "workspace", torch.uint8)
     rc = lib().mla_decode_attn(ctypes.byref(d), _ptr(q_cat), _ptr(q_lo), _ptr(cache_pool),
                                cache_pool.shape[0], _ptr(page_table), page_table.shape[1],

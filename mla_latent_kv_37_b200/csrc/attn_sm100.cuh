@@ -37,6 +37,18 @@
 // split over several ranges gets normalised partials that the combine kernel merges with
 // log-sum-exp weights.
 //
+// Extended-precision query.  Rounding the absorbed query to bf16 perturbs every logit by about
+// 2^-9 of its size; with large logits (inputs scaled x4 give a logit spread of ~16) that is
+// enough to move the output by ~1e-2.  When the caller passes the rounding remainder q_lo as
+// well (q = q_cat + q_lo to ~16 bits), each cluster takes 64 heads instead of 128 and stacks,
+// for each of them, a row of q_cat and a row of q_lo in the 128 rows of the MMA: in every
+// quarter of the rows (one warp's TMEM lanes), rows 0-15 hold heads 16w..16w+15 of the group
+// from q_cat and rows 16-31 the same heads from q_lo.  The score of a head is then the sum of
+// its two rows (one shuffle), the softmax runs identically on both rows, O gets the same P in
+// both, and only the q_cat row is written out.  Launch: `groups` = ceil(H/64) clusters per
+// part, so the tensor work per token doubles; the page bytes are read by the part's clusters
+// at about the same time and mostly come from L2 the second time.
+//
 // Roles (384 threads): warps 0-3 softmax + epilogue (thread i owns head row i = TMEM lane i),
 // warps 4-7 send, warp 8 TMA producer, warp 9 MMA issuer, warp 10 bulk-copy sender (warp 11
 // has no role).  Each softmax warp hands its rows of the receive buffer back to the peer
@@ -80,8 +92,10 @@ struct Params {
   int n_heads;
   int max_pages;
   int num_pages;
-  int num_parts;  // clusters launched
+  int num_parts;  // ranges of the page list (the plan's parts)
+  int groups;     // clusters per part: 1, or ceil(H / 64) with the query remainder (q_lo)
   const __nv_bfloat16* q_cat;  // [B][H][576]
+  const __nv_bfloat16* q_lo;   // [B][H][576] rounding remainder of the query, or null
   const uint8_t* pool;         // cache pages, [num_pages][64][576] bf16
   const int32_t* page_table;
   const int32_t* seq_lens;
@@ -331,7 +345,8 @@ static_assert(sizeof(Bars) <= 256, "barrier block");
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     split_kernel(const __grid_constant__ CUtensorMap tm_c_lat,
                  const __grid_constant__ CUtensorMap tm_c_rope,
-                 const __grid_constant__ CUtensorMap tm_q_rope, const Params p) {
+                 const __grid_constant__ CUtensorMap tm_q_rope,
+                 const __grid_constant__ CUtensorMap tm_ql_rope, const Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -340,7 +355,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const uint32_t peer = rank ^ 1u;
-  const int part = blockIdx.x >> 1;
+  // clusters of one part are adjacent, so they stream the same pages at about the same time
+  const int part = static_cast<int>(blockIdx.x >> 1) / p.groups;
+  const int group = static_cast<int>(blockIdx.x >> 1) - part * p.groups;
+  const bool hi_lo = p.q_lo != nullptr;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -401,13 +419,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_c_lat);
       tma_prefetch_desc(&tm_c_rope);
       tma_prefetch_desc(&tm_q_rope);
+      if (hi_lo) tma_prefetch_desc(&tm_ql_rope);
     }
     while (ok && it.next(seq, p0, p1)) {
       if (lane == 0) {
         if (sg > 0) ok = mbar_wait(&bars->q_empty, (sg - 1) & 1, wc);
         if (ok) {
           mbar_arrive_expect_tx(&bars->q_full, kQRopeBytes);
-          tma_load_3d(sQRope, &tm_q_rope, &bars->q_full, 512 + 32 * rank, 0, seq);
+          if (!hi_lo) {
+            tma_load_3d(sQRope, &tm_q_rope, &bars->q_full, 512 + 32 * rank, 0, seq);
+          } else {
+            // 16-row boxes: rows 32w..32w+15 from q_cat, rows 32w+16..32w+31 from q_lo, both
+            // for heads 64 group + 16w .. +15 (rows past H are zero-filled by the copy)
+#pragma unroll
+            for (int w4 = 0; w4 < 4; ++w4) {
+              const int h0 = 64 * group + 16 * w4;
+              tma_load_3d(sQRope + (32 * w4) * 64, &tm_q_rope, &bars->q_full, 512 + 32 * rank,
+                          h0, seq);
+              tma_load_3d(sQRope + (32 * w4 + 16) * 64, &tm_ql_rope, &bars->q_full,
+                          512 + 32 * rank, h0, seq);
+            }
+          }
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -616,7 +648,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int row = threadIdx.x;  // head row = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     const float NEG_INF = -__int_as_float(0x7f800000);
-    const bool row_ok = row < p.n_heads;
+    // the head this row computes, and whether it carries the query's remainder (q_lo)
+    const int head = hi_lo ? 64 * group + 16 * warp + (lane & 15) : row;
+    const bool lo_row = hi_lo && (lane & 16);
+    const bool row_ok = head < p.n_heads;
+    const bool row_out = row_ok && !lo_row;  // rows whose result is written
     const uint32_t peer_done_r[2] = {mapa_shared(smem_u32(&bars->peer_done[0]), peer),
                                      mapa_shared(smem_u32(&bars->peer_done[1]), peer)};
     SegIter it{plan.seq_pages(), plan.seq_prefix(), p.batch, g_begin, g_end, b_begin};
@@ -628,7 +664,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // ---- this CTA's latent half of the query row -> TMEM (A operand of QK) ----
       {
         const uint4* src = reinterpret_cast<const uint4*>(
-            p.q_cat + (static_cast<size_t>(seq) * p.n_heads + (row_ok ? row : 0)) * kRow);
+            (lo_row ? p.q_lo : p.q_cat) +
+            (static_cast<size_t>(seq) * p.n_heads + (row_ok ? head : 0)) * kRow);
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t r[32];
@@ -694,6 +731,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (warp == 0) mbar_arrive_expect_tx(&bars->x_full, kXBytes);
             mbar_arrive_remote_relaxed(peer_done_r[buf]);
           }
+        }
+        // ---- extended-precision query: a head's score is the sum of its q_cat and q_lo rows
+        // (lanes l and l ^ 16 of this warp); both rows continue with the same scores ----
+        if (hi_lo) {
+#pragma unroll
+          for (int k = 0; k < 64; ++k) s[k] += __shfl_xor_sync(0xffffffffu, s[k], 16);
         }
         // ---- online softmax ----
         const int valid = min(kPage, len - (p0 + i) * kPage);
@@ -763,19 +806,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       float* dst;
       float* dst_lse;
       if (nparts == 1) {
-        dst = p.o_lat + (static_cast<size_t>(seq) * p.n_heads + row) * 512 + 256 * rank;
-        dst_lse = p.lse ? p.lse + static_cast<size_t>(seq) * p.n_heads + row : nullptr;
+        dst = p.o_lat + (static_cast<size_t>(seq) * p.n_heads + head) * 512 + 256 * rank;
+        dst_lse = p.lse ? p.lse + static_cast<size_t>(seq) * p.n_heads + head : nullptr;
       } else {
         const int slot = plan.seq_slot()[seq] + (part - plan.seq_first_part()[seq]);
-        dst = p.part_o + (static_cast<size_t>(slot) * p.n_heads + row) * 512 + 256 * rank;
-        dst_lse = p.part_lse + static_cast<size_t>(slot) * p.n_heads + row;
+        dst = p.part_o + (static_cast<size_t>(slot) * p.n_heads + head) * 512 + 256 * rank;
+        dst_lse = p.part_lse + static_cast<size_t>(slot) * p.n_heads + head;
       }
 #pragma unroll 1
       for (int c = 0; c < 256; c += 32) {
         uint32_t r[32];
         tmem_ld32(tmem + kTmemO + c + lane_off, r);
         tmem_wait_ld();
-        if (row_ok) {
+        if (row_out) {
           float4* d4 = reinterpret_cast<float4*>(dst + c);
 #pragma unroll
           for (int k = 0; k < 8; ++k)
@@ -785,7 +828,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                 __uint_as_float(r[4 * k + 3]) * inv_l);
         }
       }
-      if (row_ok && rank == 0 && dst_lse) *dst_lse = lse_nat;
+      if (row_out && rank == 0 && dst_lse) *dst_lse = lse_nat;
       tc_fence_before();
       mbar_arrive(&bars->o_free);
       t += n;

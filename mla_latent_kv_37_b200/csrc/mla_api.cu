@@ -27,6 +27,7 @@ namespace {
 constexpr int kDc = 512, kDr = 64, kDn = 128, kDv = 128, kRowN = 576, kPageN = 64;
 constexpr uint64_t kDefaultWaitNs = 2000000000ull;  // 2 s per bounded wait
 constexpr int kMinPagesPerPart = 4;
+constexpr int kMaxParts = 1 << 16;  // upper bound on num_splits (host check before any arithmetic)
 constexpr int kSkMinUnits = 2;    // fewest stages' worth of weights a stream-K CTA streams
 constexpr int kSkMaxContrib = 4;  // aim for at most this many CTAs sharing one tile
 constexpr int kSkMaxStages = 12;
@@ -261,8 +262,11 @@ Workspace layout(const mla_dims* d, int num_parts, int sms) {
   return w;
 }
 
-int resolve_parts(int num_splits, const DevCtx* c) {
-  return num_splits > 0 ? num_splits : default_parts(c ? c->sms : 148, c ? c->max_clusters : 74);
+// Parts of the page list: num_splits, or about one cluster per co-resident cluster slot, shared
+// by the `groups` clusters that each part runs on (2 for 128 heads with the query remainder).
+int resolve_parts(int num_splits, const DevCtx* c, int groups = 1) {
+  if (num_splits > 0) return num_splits;
+  return std::max(1, default_parts(c ? c->sms : 148, c ? c->max_clusters : 74) / groups);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -428,6 +432,114 @@ int run_wuk(const DevCtx* c, const mla_dims* dims, const void* w_uk, char* ws,
   return run_streamk(c, s2, q2, B, nullptr, 0.f, a2, a2, 1 << 30, 1, b2, ws, w, e2, st);
 }
 
+
+// Host checks shared by both decode entry points (everything but the workspace).
+int check_decode_args(const mla_dims* dims, const void* q_cat, const void* q_lo,
+                      const void* cache_pool, int32_t num_pages, const int32_t* page_table,
+                      int32_t max_pages, const int32_t* seq_lens, float softmax_scale,
+                      int32_t num_splits, const float* o_lat, const float* lse) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (!q_cat || !cache_pool || !page_table || !seq_lens || !o_lat) return MLA_ERR_NULL_ARG;
+  if (num_pages < 1 || max_pages < 1 || num_splits < 0 || num_splits > kMaxParts)
+    return MLA_ERR_ARG;
+  if (q_lo && dims->dtype != MLA_BF16) return MLA_ERR_ARG;
+  if (!(softmax_scale >= 0.f) || !std::isfinite(softmax_scale)) return MLA_ERR_ARG;
+  if (!aligned(q_cat, 16) || !aligned(cache_pool, 16) || !aligned(o_lat, 16) ||
+      (q_lo && !aligned(q_lo, 16)) || !aligned(page_table, 4) || !aligned(seq_lens, 4) ||
+      (lse && !aligned(lse, 4)))
+    return MLA_ERR_ALIGN;
+  // page ids and lengths are int32 token counts on the device
+  if (static_cast<int64_t>(num_pages) * kPageN > INT32_MAX ||
+      static_cast<int64_t>(max_pages) * kPageN > INT32_MAX)
+    return MLA_ERR_ARG;
+  return MLA_OK;
+}
+
+// Clusters per part: 1, or one per 64 heads when the query remainder q_lo is given.
+int decode_groups(const mla_dims* dims, const void* q_lo) {
+  return (q_lo && dims->dtype == MLA_BF16) ? (dims->n_heads + 63) / 64 : 1;
+}
+
+// plan -> split-KV attention -> combine, on `st`, with the scratch the caller placed.
+int enqueue_decode(const DevCtx* c, const mla_dims* dims, const void* q_cat, const void* q_lo,
+                   const void* cache_pool, int32_t num_pages, const int32_t* page_table,
+                   int32_t max_pages, const int32_t* seq_lens, float softmax_scale, int parts,
+                   int32_t* plan, float* part_o, float* part_lse, float* o_lat, float* lse,
+                   cudaStream_t st) {
+  int rc;
+  const int B = dims->batch, H = dims->n_heads;
+  const int groups = decode_groups(dims, q_lo);
+  const float scale =
+      softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(kDn + kDr));
+  launch_pdl(attn::plan_kernel, dim3(1), dim3(attn::kPlanThreads), 0, st, seq_lens, B, max_pages,
+             parts, kMinPagesPerPart, plan, c->status);
+  if ((rc = last_launch())) return rc;
+  if (dims->dtype == MLA_BF16) {
+    CUtensorMap tc_lat, tc_rope, tq_rope, tql_rope;
+    const uint64_t rows = static_cast<uint64_t>(num_pages) * kPageN;
+    // query RoPE halves: one 128-head box, or 16-head boxes from q_cat and q_lo
+    const uint32_t qbox = q_lo ? 16 : 128;
+    if ((rc = map3(&tq_rope, q_cat, kRowN, H, B, kRowN * 2ull, kRowN * 2ull * H, 32, qbox, 1,
+                   CU_TENSOR_MAP_SWIZZLE_64B)))
+      return rc;
+    if (q_lo) {
+      if ((rc = map3(&tql_rope, q_lo, kRowN, H, B, kRowN * 2ull, kRowN * 2ull * H, 32, qbox, 1,
+                     CU_TENSOR_MAP_SWIZZLE_64B)))
+        return rc;
+    } else {
+      tql_rope = tq_rope;
+    }
+    if ((rc = map2(&tc_lat, cache_pool, kRowN, rows, kRowN * 2ull, 64, 64,
+                   CU_TENSOR_MAP_SWIZZLE_128B)))
+      return rc;
+    if ((rc = map2(&tc_rope, cache_pool, kRowN, rows, kRowN * 2ull, 32, 64,
+                   CU_TENSOR_MAP_SWIZZLE_64B)))
+      return rc;
+    attn::Params p{};
+    p.batch = B;
+    p.n_heads = H;
+    p.max_pages = max_pages;
+    p.num_pages = num_pages;
+    p.num_parts = parts;
+    p.groups = groups;
+    p.q_cat = static_cast<const __nv_bfloat16*>(q_cat);
+    p.q_lo = static_cast<const __nv_bfloat16*>(q_lo);
+    p.pool = static_cast<const uint8_t*>(cache_pool);
+    p.page_table = page_table;
+    p.seq_lens = seq_lens;
+    p.plan = plan;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.o_lat = o_lat;
+    p.lse = lse;
+    p.part_o = part_o;
+    p.part_lse = part_lse;
+    p.status = c->status;
+    p.wait_ns = kDefaultWaitNs;
+    const bool prof = g_prof_next < g_prof_count;
+    if (prof && record_profile_event(g_prof_begin[g_prof_next], st) != cudaSuccess)
+      return MLA_ERR_CUDA;
+    launch_pdl(attn::split_kernel, dim3(2 * parts * groups), dim3(attn::kThreads),
+               attn::kSmemBytes, st, tc_lat, tc_rope, tq_rope, tql_rope, p);
+    if (prof) {
+      if ((rc = last_launch())) return rc;
+      if (record_profile_event(g_prof_end[g_prof_next++], st) != cudaSuccess) return MLA_ERR_CUDA;
+      g_launches.fetch_sub(1, std::memory_order_relaxed);  // counted again below
+    }
+  } else {
+    attn::f32_split_kernel<<<dim3(parts, H), 128, 0, st>>>(
+        static_cast<const float*>(q_cat), static_cast<const float*>(cache_pool), page_table,
+        max_pages, num_pages, seq_lens, plan, B, parts, H, scale, o_lat, lse, part_o, part_lse,
+        c->status);
+  }
+  if ((rc = last_launch())) return rc;
+  launch_pdl(attn::combine_kernel,
+             dim3(static_cast<unsigned>((static_cast<size_t>(B) * H + attn::kCombineWarps - 1) /
+                                        attn::kCombineWarps)),
+             dim3(32 * attn::kCombineWarps), 0, st, plan, B, parts, H, part_o, part_lse, o_lat,
+             lse);
+  return last_launch();
+}
 }  // namespace
 }  // namespace mla
 
@@ -439,7 +551,7 @@ using namespace mla;
 extern "C" {
 
 size_t mla_workspace_size(const mla_dims* dims, int32_t num_splits) {
-  if (check_dims(dims) != MLA_OK || num_splits < 0) return 0;
+  if (check_dims(dims) != MLA_OK || num_splits < 0 || num_splits > kMaxParts) return 0;
   DevCtx* c = nullptr;
   const bool have = device_ctx(&c) == MLA_OK;
   const int sms = have ? c->sms : 148;
@@ -632,87 +744,22 @@ int mla_decode_attn(const mla_dims* dims, const void* q_cat, const void* q_lo,
                     int32_t max_pages, const int32_t* seq_lens, float softmax_scale,
                     int32_t num_splits, void* workspace, size_t workspace_bytes, float* o_lat,
                     float* lse, mla_stream_t stream) {
-  int rc = check_dims(dims);
+  int rc = check_decode_args(dims, q_cat, q_lo, cache_pool, num_pages, page_table, max_pages,
+                             seq_lens, softmax_scale, num_splits, o_lat, lse);
   if (rc) return rc;
-  if (!q_cat || !cache_pool || !page_table || !seq_lens || !o_lat) return MLA_ERR_NULL_ARG;
   if (!workspace) return MLA_ERR_WORKSPACE;
-  if (num_pages < 1 || max_pages < 1 || num_splits < 0) return MLA_ERR_ARG;
-  if (q_lo) return MLA_ERR_ARG;  // extended-precision query input: not supported yet
-  if (!(softmax_scale >= 0.f) || !std::isfinite(softmax_scale)) return MLA_ERR_ARG;
-  if (!aligned(q_cat, 16) || !aligned(cache_pool, 16) || !aligned(o_lat, 16) ||
-      !aligned(page_table, 4) || !aligned(seq_lens, 4) || (lse && !aligned(lse, 4)))
-    return MLA_ERR_ALIGN;
   if (!aligned(workspace, 256)) return MLA_ERR_ALIGN;
-  if (static_cast<int64_t>(num_pages) * kPageN > INT32_MAX) return MLA_ERR_ARG;
   DevCtx* c = nullptr;
   if ((rc = device_ctx(&c))) return rc;
-  const int parts = resolve_parts(num_splits, c);
+  const int parts = resolve_parts(num_splits, c, decode_groups(dims, q_lo));
   const Workspace w = layout(dims, parts, c->sms);
   if (workspace_bytes < w.total) return MLA_ERR_WORKSPACE;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int B = dims->batch, H = dims->n_heads;
   char* ws = static_cast<char*>(workspace);
-  int32_t* plan = reinterpret_cast<int32_t*>(ws + w.plan);
-  float* part_o = reinterpret_cast<float*>(ws + w.part_o);
-  float* part_lse = reinterpret_cast<float*>(ws + w.part_lse);
-  const float scale =
-      softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(kDn + kDr));
-  launch_pdl(attn::plan_kernel, dim3(1), dim3(attn::kPlanThreads), 0, st, seq_lens, B, max_pages,
-             parts, kMinPagesPerPart, plan, c->status);
-  if ((rc = last_launch())) return rc;
-  if (dims->dtype == MLA_BF16) {
-    CUtensorMap tc_lat, tc_rope, tq_rope;
-    const uint64_t rows = static_cast<uint64_t>(num_pages) * kPageN;
-    if ((rc = map3(&tq_rope, q_cat, kRowN, H, B, kRowN * 2ull, kRowN * 2ull * H, 32, 128, 1,
-                   CU_TENSOR_MAP_SWIZZLE_64B)))
-      return rc;
-    if ((rc = map2(&tc_lat, cache_pool, kRowN, rows, kRowN * 2ull, 64, 64,
-                   CU_TENSOR_MAP_SWIZZLE_128B)))
-      return rc;
-    if ((rc = map2(&tc_rope, cache_pool, kRowN, rows, kRowN * 2ull, 32, 64,
-                   CU_TENSOR_MAP_SWIZZLE_64B)))
-      return rc;
-    attn::Params p{};
-    p.batch = B;
-    p.n_heads = H;
-    p.max_pages = max_pages;
-    p.num_pages = num_pages;
-    p.num_parts = parts;
-    p.q_cat = static_cast<const __nv_bfloat16*>(q_cat);
-    p.pool = static_cast<const uint8_t*>(cache_pool);
-    p.page_table = page_table;
-    p.seq_lens = seq_lens;
-    p.plan = plan;
-    p.scale_log2 = scale * 1.4426950408889634f;
-    p.o_lat = o_lat;
-    p.lse = lse;
-    p.part_o = part_o;
-    p.part_lse = part_lse;
-    p.status = c->status;
-    p.wait_ns = kDefaultWaitNs;
-    const bool prof = g_prof_next < g_prof_count;
-    if (prof && record_profile_event(g_prof_begin[g_prof_next], st) != cudaSuccess)
-      return MLA_ERR_CUDA;
-    launch_pdl(attn::split_kernel, dim3(2 * parts), dim3(attn::kThreads), attn::kSmemBytes, st,
-               tc_lat, tc_rope, tq_rope, p);
-    if (prof) {
-      if ((rc = last_launch())) return rc;
-      if (record_profile_event(g_prof_end[g_prof_next++], st) != cudaSuccess) return MLA_ERR_CUDA;
-      g_launches.fetch_sub(1, std::memory_order_relaxed);  // counted again below
-    }
-  } else {
-    attn::f32_split_kernel<<<dim3(parts, H), 128, 0, st>>>(
-        static_cast<const float*>(q_cat), static_cast<const float*>(cache_pool), page_table,
-        max_pages, num_pages, seq_lens, plan, B, parts, H, scale, o_lat, lse, part_o, part_lse,
-        c->status);
-  }
-  if ((rc = last_launch())) return rc;
-  launch_pdl(attn::combine_kernel,
-             dim3(static_cast<unsigned>((static_cast<size_t>(B) * H + attn::kCombineWarps - 1) /
-                                        attn::kCombineWarps)),
-             dim3(32 * attn::kCombineWarps), 0, st, plan, B, parts, H, part_o, part_lse, o_lat,
-             lse);
-  return last_launch();
+  return enqueue_decode(c, dims, q_cat, q_lo, cache_pool, num_pages, page_table, max_pages,
+                        seq_lens, softmax_scale, parts, reinterpret_cast<int32_t*>(ws + w.plan),
+                        reinterpret_cast<float*>(ws + w.part_o),
+                        reinterpret_cast<float*>(ws + w.part_lse), o_lat, lse,
+                        reinterpret_cast<cudaStream_t>(stream));
 }
 
 int mla_out_proj(const mla_dims* dims, const float* o_lat, const void* w_uv, const void* w_o,
@@ -885,8 +932,8 @@ DecodeScratch decode_scratch_layout(int B, int H, int parts) {
     return o;
   };
   d.plan = take(attn::PlanView::words(B, parts) * 4);
-  d.part_o = take(static_cast<size_t>(B + parts) * H * kDc * 4);
-  d.part_lse = take(static_cast<size_t>(B + parts) * H * 4);
+  d.part_o = take((static_cast<size_t>(B) + static_cast<size_t>(parts)) * H * kDc * 4);
+  d.part_lse = take((static_cast<size_t>(B) + static_cast<size_t>(parts)) * H * 4);
   d.total = off;
   return d;
 }
@@ -898,16 +945,10 @@ extern "C" int mla_decode_attn_static_scratch(const mla_dims* dims, const void* 
                                               int32_t max_pages, const int32_t* seq_lens,
                                               float softmax_scale, int32_t num_splits,
                                               float* o_lat, float* lse, mla_stream_t stream) {
-  int rc = check_dims(dims);
+  int rc = check_decode_args(dims, q_cat, q_lo, cache_pool, num_pages, page_table, max_pages,
+                             seq_lens, softmax_scale, num_splits, o_lat, lse);
   if (rc) return rc;
-  if (!q_cat || !cache_pool || !page_table || !seq_lens || !o_lat) return MLA_ERR_NULL_ARG;
-  if (num_pages < 1 || max_pages < 1 || num_splits < 0) return MLA_ERR_ARG;
-  if (q_lo) return MLA_ERR_ARG;
-  if (!(softmax_scale >= 0.f) || !std::isfinite(softmax_scale)) return MLA_ERR_ARG;
-  if (!aligned(q_cat, 16) || !aligned(cache_pool, 16) || !aligned(o_lat, 16) ||
-      !aligned(page_table, 4) || !aligned(seq_lens, 4) || (lse && !aligned(lse, 4)))
-    return MLA_ERR_ALIGN;
-  if (static_cast<int64_t>(num_pages) * kPageN > INT32_MAX) return MLA_ERR_ARG;
+  if (q_lo) return MLA_ERR_ARG;  // this entry point takes the bf16 query alone
   DevCtx* c = nullptr;
   if ((rc = device_ctx(&c))) return rc;
   const int B = dims->batch, H = dims->n_heads;
@@ -919,58 +960,9 @@ extern "C" int mla_decode_attn_static_scratch(const mla_dims* dims, const void* 
   // Nothing in the scratch has to start at zero: the plan kernel writes every plan word and
   // the split kernel writes every partial slot before the combine kernel reads it.
   char* ws = static_cast<char*>(scratch);
-  int32_t* plan = reinterpret_cast<int32_t*>(ws + w.plan);
-  float* part_o = reinterpret_cast<float*>(ws + w.part_o);
-  float* part_lse = reinterpret_cast<float*>(ws + w.part_lse);
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const float scale =
-      softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(kDn + kDr));
-  launch_pdl(attn::plan_kernel, dim3(1), dim3(attn::kPlanThreads), 0, st, seq_lens, B, max_pages,
-             parts, kMinPagesPerPart, plan, c->status);
-  if ((rc = last_launch())) return rc;
-  if (dims->dtype == MLA_BF16) {
-    CUtensorMap tc_lat, tc_rope, tq_rope;
-    const uint64_t rows = static_cast<uint64_t>(num_pages) * kPageN;
-    if ((rc = map3(&tq_rope, q_cat, kRowN, H, B, kRowN * 2ull, kRowN * 2ull * H, 32, 128, 1,
-                   CU_TENSOR_MAP_SWIZZLE_64B)))
-      return rc;
-    if ((rc = map2(&tc_lat, cache_pool, kRowN, rows, kRowN * 2ull, 64, 64,
-                   CU_TENSOR_MAP_SWIZZLE_128B)))
-      return rc;
-    if ((rc = map2(&tc_rope, cache_pool, kRowN, rows, kRowN * 2ull, 32, 64,
-                   CU_TENSOR_MAP_SWIZZLE_64B)))
-      return rc;
-    attn::Params p{};
-    p.batch = B;
-    p.n_heads = H;
-    p.max_pages = max_pages;
-    p.num_pages = num_pages;
-    p.num_parts = parts;
-    p.q_cat = static_cast<const __nv_bfloat16*>(q_cat);
-    p.pool = static_cast<const uint8_t*>(cache_pool);
-    p.page_table = page_table;
-    p.seq_lens = seq_lens;
-    p.plan = plan;
-    p.scale_log2 = scale * 1.4426950408889634f;
-    p.o_lat = o_lat;
-    p.lse = lse;
-    p.part_o = part_o;
-    p.part_lse = part_lse;
-    p.status = c->status;
-    p.wait_ns = kDefaultWaitNs;
-    launch_pdl(attn::split_kernel, dim3(2 * parts), dim3(attn::kThreads), attn::kSmemBytes, st,
-               tc_lat, tc_rope, tq_rope, p);
-  } else {
-    attn::f32_split_kernel<<<dim3(parts, H), 128, 0, st>>>(
-        static_cast<const float*>(q_cat), static_cast<const float*>(cache_pool), page_table,
-        max_pages, num_pages, seq_lens, plan, B, parts, H, scale, o_lat, lse, part_o, part_lse,
-        c->status);
-  }
-  if ((rc = last_launch())) return rc;
-  launch_pdl(attn::combine_kernel,
-             dim3(static_cast<unsigned>((static_cast<size_t>(B) * H + attn::kCombineWarps - 1) /
-                                        attn::kCombineWarps)),
-             dim3(32 * attn::kCombineWarps), 0, st, plan, B, parts, H, part_o, part_lse, o_lat,
-             lse);
-  return last_launch();
+  return enqueue_decode(c, dims, q_cat, nullptr, cache_pool, num_pages, page_table, max_pages,
+                        seq_lens, softmax_scale, parts, reinterpret_cast<int32_t*>(ws + w.plan),
+                        reinterpret_cast<float*>(ws + w.part_o),
+                        reinterpret_cast<float*>(ws + w.part_lse), o_lat, lse,
+                        reinterpret_cast<cudaStream_t>(stream));
 }

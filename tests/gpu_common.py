@@ -76,7 +76,10 @@ class Workload:
         self.pos = torch.tensor(history, dtype=torch.int32)
         self.lens = self.pos + 1
 
-    def run_gpu(self, num_splits=0, want_out=True):
+    def run_gpu(self, num_splits=0, want_out=True, fused=False, query_remainder=False):
+        """One decode step through the C ABI: cache append and absorbed query (two calls, or
+        the fused mla_append_absorb), attention, output projection.  `query_remainder` also
+        carries the query's bf16 rounding remainder from the projection to the attention."""
         import mla_latent_kv_37_b200 as M
         B, H, D = self.B, self.H, self.D
         d = M.dims(B, H, D, self.dtype)
@@ -84,15 +87,23 @@ class Workload:
         pool = dev(self.cache.pool)
         table = dev(self.cache.page_table)
         q_cat = torch.empty(B, H, 576, dtype=self.dtype, device="cuda")
+        q_lo = (torch.empty(B, H, 576, dtype=torch.bfloat16, device="cuda")
+                if query_remainder else None)
         o_lat = torch.empty(B, H, 512, dtype=torch.float32, device="cuda")
         lse = torch.empty(B, H, dtype=torch.float32, device="cuda")
         o_heads = torch.empty(B, H, 128, dtype=self.dtype, device="cuda")
         out = torch.empty(B, D, dtype=self.dtype, device="cuda") if want_out else None
         w = self.w
-        M.mla_cache_append(d, dev(self.h), dev(w.w_dkv), dev(w.w_kr), dev(self.pos), table, pool, ws)
-        M.mla_absorb_q(d, dev(self.h), dev(w.w_q), dev(w.w_uk), dev(self.pos), q_cat, ws)
+        if fused:
+            M.mla_append_absorb(d, dev(self.h), dev(w.w_dkv), dev(w.w_kr), dev(w.w_q),
+                                dev(w.w_uk), dev(self.pos), table, pool, q_cat, ws, q_lo=q_lo)
+        else:
+            M.mla_cache_append(d, dev(self.h), dev(w.w_dkv), dev(w.w_kr), dev(self.pos), table,
+                               pool, ws)
+            M.mla_absorb_q(d, dev(self.h), dev(w.w_q), dev(w.w_uk), dev(self.pos), q_cat, ws,
+                           q_lo=q_lo)
         M.mla_decode_attn(d, q_cat, pool, table, dev(self.lens), o_lat, ws, lse=lse,
-                          num_splits=num_splits)
+                          q_lo=q_lo, num_splits=num_splits)
         M.mla_out_proj(d, o_lat, dev(w.w_uv), ws, w_o=dev(w.w_o) if want_out else None,
                        o_heads=o_heads, out=out)
         status = M.mla_get_status()

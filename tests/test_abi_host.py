@@ -94,16 +94,40 @@ def test_null_and_alignment_errors(M):
     assert L.mla_out_proj(ctypes.byref(d), f, f, None, None, None, f, 1 << 30, None) == -1
 
 
-def test_decode_calls_reject_q_lo(M):
-    # Both decode entry points document q_lo as "must be NULL" (the kernel does not consume the
-    # query's rounding remainder): a non-NULL q_lo is an argument error, found on the host.
+def test_query_remainder_arguments(M):
+    # mla_decode_attn takes the query's rounding remainder on the bf16 path only; the
+    # static-scratch entry point takes the bf16 query alone.  Both are host-side checks.
+    import torch
     d = _d(M)
     L = M.lib()
     f = ctypes.c_void_p(0x10000)
-    assert L.mla_decode_attn(ctypes.byref(d), f, f, f, 10, f, 4, f, 0.0, 0, f, 1 << 30, f, None,
-                             None) == -5
+    odd = ctypes.c_void_p(0x10008)
+    d32 = M.dims(4, 16, 1024, dtype=torch.float32)
+    assert L.mla_decode_attn(ctypes.byref(d32), f, f, f, 10, f, 4, f, 0.0, 0, f, 1 << 30, f,
+                             None, None) == -5
+    assert L.mla_decode_attn(ctypes.byref(d), f, odd, f, 10, f, 4, f, 0.0, 0, f, 1 << 30, f,
+                             None, None) == -3
     assert L.mla_decode_attn_static_scratch(ctypes.byref(d), f, f, f, 10, f, 4, f, 0.0, 0, f,
                                             None, None) == -5
+    if not torch.cuda.is_available():  # the host checks pass; then the missing device shows
+        rc = L.mla_decode_attn(ctypes.byref(d), f, f, f, 10, f, 4, f, 0.0, 0, f, 1 << 30, f,
+                               None, None)
+        assert rc in (-6, -7)
+
+
+def test_split_count_and_page_bounds(M):
+    # num_splits above 65536 and page counts whose token count overflows int32 are rejected
+    # before any arithmetic on them
+    d = _d(M)
+    L = M.lib()
+    f = ctypes.c_void_p(0x10000)
+    assert M.mla_workspace_size(d, 65537) == 0
+    assert M.mla_workspace_size(d, 65536) > 0
+    for fn in (lambda *a: L.mla_decode_attn(*a[:10], f, 1 << 40, f, None, None),
+               lambda *a: L.mla_decode_attn_static_scratch(*a, f, None, None)):
+        assert fn(ctypes.byref(d), f, None, f, 10, f, 4, f, 0.0, 65537) == -5
+        assert fn(ctypes.byref(d), f, None, f, 10, f, 1 << 25, f, 0.0, 0) == -5
+        assert fn(ctypes.byref(d), f, None, f, 1 << 25, f, 4, f, 0.0, 0) == -5
 
 
 def test_valid_call_without_gpu_fails_loudly(M):

@@ -141,3 +141,63 @@ def test_bad_length_sets_status():
     q, cache = _case(13, lens, 128)
     _, _, st = _run(q, cache, [100, 10_000], 128)
     assert st & M.STATUS_BAD_LENGTH
+
+
+# ---------------------------------------------------------------------------------------------
+# Query carried as bf16 hi + lo (q_lo): the scores use ~16 significant bits of the query.
+# ---------------------------------------------------------------------------------------------
+def _split_query(seed, B, H, scale):
+    """An fp32 absorbed query and its bf16 hi/lo split; the oracle gets hi + lo exactly."""
+    q = I.query_cat(seed, B, H, scale, torch.float32)
+    hi = q.to(torch.bfloat16)
+    lo = (q - hi.float()).to(torch.bfloat16)
+    exact = hi.double() + lo.double()
+    return hi, lo, exact
+
+
+def _run_lo(hi, lo, cache, lens, H, num_splits=0):
+    import mla_latent_kv_37_b200 as M
+    B = hi.shape[0]
+    d = M.dims(B, H, 1024)
+    ws = M.workspace(d, num_splits)
+    o_lat = torch.full((B, H, 512), float("nan"), dtype=torch.float32, device="cuda")
+    lse = torch.full((B, H), float("nan"), dtype=torch.float32, device="cuda")
+    M.mla_decode_attn(d, dev(hi), dev(cache.pool), dev(cache.page_table),
+                      dev(torch.tensor(lens, dtype=torch.int32)), o_lat, ws, lse=lse,
+                      q_lo=dev(lo), num_splits=num_splits)
+    st = M.mla_get_status()
+    return o_lat.cpu(), lse.cpu(), st
+
+
+@pytest.mark.parametrize("H,lens,splits", [(128, [5, 64, 200, 3], 0), (96, [300, 65], 0),
+                                           (16, [129, 1], 2), (64, [0, 700, 63], 3),
+                                           (128, [900, 333, 64, 1], 7)])
+def test_query_remainder(H, lens, splits):
+    hi, lo, exact = _split_query(40 + H, len(lens), H, 4.0)
+    cache = I.paged_cache(41 + H, lens, lens, 4.0)
+    o, l, st = _run_lo(hi, lo, cache, lens, H, splits)
+    assert st == 0
+    _check(exact, cache, lens, o, l)
+
+
+def test_query_remainder_long_context_scaled():
+    """Long context (4 x 131072) at inputs x4 (logit spread ~16): with the remainder the
+    attention output is within tolerance of the oracle fed the ~16-bit query."""
+    lens = [131072] * 4
+    hi, lo, exact = _split_query(3, 4, 128, 4.0)
+    cache = I.paged_cache(4, lens, lens, 4.0)
+    o, l, st = _run_lo(hi, lo, cache, lens, 128)
+    assert st == 0
+    _check(exact, cache, lens, o, l)
+
+
+def test_query_remainder_zero_matches_plain_call():
+    """A zero remainder gives the plain call's result to within the split's rounding."""
+    lens = [777, 64]
+    q, cache = _case(14, lens, 128)
+    o1, l1, _ = _run(q, cache, lens, 128, num_splits=4)
+    o2, l2, st = _run_lo(q, torch.zeros_like(q), cache, lens, 128, num_splits=4)
+    assert st == 0
+    rel, _ = errors(o2.numpy(), o1.numpy())
+    assert rel < 1e-3
+    np.testing.assert_allclose(l2.numpy(), l1.numpy(), rtol=1e-4, atol=1e-4)
