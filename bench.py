@@ -45,7 +45,15 @@ CONFIGS = {
                       workload="batched paged MLA decode, batch 64, context U[1024,8192]"),
     "long_128k": dict(batch=4, context=131072, layers=1, heads=128, d_model=7168,
                       workload="long-context split-KV MLA decode, batch 4 x 131072"),
+    "long_128k_x4": dict(batch=4, context=131072, layers=1, heads=128, d_model=7168, scale=4.0,
+                         remainder=True,
+                         workload="long-context split-KV MLA decode, batch 4 x 131072, inputs x4"
+                                  " (query carried as bf16 hi + lo)"),
 }
+# the single-layer configurations reported beside the headline: (name, sequences, heads) sampled
+# for the parity check against the oracle
+EXTRA_CONFIGS = (("v3_single", 1, 8), ("paged_b64", 2, 4), ("long_128k", 1, 4),
+                 ("long_128k_x4", 1, 4))
 
 
 def log(*a):
@@ -182,7 +190,7 @@ def context_lengths(cfg, seed):
 
 def make_workload(cfg, device, seed=4):
     """Per-layer weights, paged cache (history = context - 1 rows) and hidden states, drawn on
-    the device with seeded generators."""
+    the device with seeded generators; hidden states and history are scaled by cfg["scale"]."""
     import mla_inputs as I
     from mla_latent_kv_37_b200.step import Layer
     B, H, D, L = cfg["batch"], cfg["heads"], cfg["d_model"], cfg["layers"]
@@ -191,12 +199,13 @@ def make_workload(cfg, device, seed=4):
     layers = []
     for l in range(L):
         w = I.weights(seed * 1000 + l, H, D, torch.bfloat16, device)
-        c = I.paged_cache(seed * 1000 + 500 + l, lens, hist, 1.0, torch.bfloat16, device)
+        c = I.paged_cache(seed * 1000 + 500 + l, lens, hist, cfg.get("scale", 1.0),
+                          torch.bfloat16, device)
         layers.append(Layer(w.w_dkv, w.w_kr, w.w_q, w.w_uk, w.w_uv, w.w_o, c.pool, c.page_table))
         if l == 0 or (l + 1) % 10 == 0:
             log(f"[bench] generated layer {l + 1}/{L}")
-    h = torch.stack([I.hidden(seed * 1000 + 900 + l, B, D, 1.0, torch.bfloat16, device)
-                     for l in range(L)])
+    h = torch.stack([I.hidden(seed * 1000 + 900 + l, B, D, cfg.get("scale", 1.0),
+                              torch.bfloat16, device) for l in range(L)])
     pos = torch.tensor(hist, dtype=torch.int32, device=device)
     return layers, h, pos, pos + 1, lens
 
@@ -327,73 +336,170 @@ SWEEP_BATCH = (32, 64, 128)
 SWEEP_CONTEXT = (8192, 16384, 32768)
 
 
-def run_sweep(args):
-    """mla_decode_attn (plan + split + combine) on one layer for every batch x context of the
-    sweep, 128 heads, full pages, random page placement: `--sweep-warmup` untimed and
-    `--sweep-iters` timed calls per shape, the L2 flushed (a 256 MB write) before every timed
-    call, CUDA events around each call.  One JSON line per shape: median / p10 / p90 time and the
-    fraction of the roofline, against the burst peaks (the call is timed alone)."""
-    import json as _json
+def load_peaks():
+    """MEASURED_PEAKS.json (written on the GPU machine) or {} when it is absent."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f)
+    except Exception:
+        return {}
 
+
+def attention_roofline(tokens, B, H, seconds, peaks, sustained):
+    """Roofline numbers of one mla_decode_attn call over `tokens` cached tokens: algorithmic
+    bytes (cache rows + query + o_lat) and flops, against the HBM and bf16 tensor peaks (the
+    sustained GEMM rate for a kernel timed inside a long step, the burst rate for one timed
+    alone); bound = the slower of the two."""
+    hbm = peaks.get("hbm_gbs", 6650.0)
+    tc_burst = peaks.get("bf16_tflops", 1590.0)
+    tc = peaks.get("bf16_tflops_sustained", 1400.0) if sustained else tc_burst
+    nbytes = tokens * ROW_BYTES + B * H * 576 * 2 + B * H * 512 * 4
+    flops = tokens * H * FLOP_PER_TOKEN_HEAD
+    t_hbm, t_tc = nbytes / (hbm * 1e9), flops / (tc * 1e12)
+    gbs, tfs = nbytes / seconds / 1e9, flops / seconds / 1e12
+    return {"bound": "hbm" if t_hbm >= t_tc else "tensor", "us": seconds * 1e6,
+            "roofline_us": max(t_hbm, t_tc) * 1e6, "frac": max(t_hbm, t_tc) / seconds,
+            "gbs": gbs, "hbm_frac": gbs / hbm, "tflops": tfs,
+            "tensor_frac_burst": tfs / tc_burst,
+            "tensor_frac_sustained": tfs / peaks.get("bf16_tflops_sustained", 1400.0),
+            "bytes": nbytes, "flops": flops}
+
+
+def sweep_shape(B, N, warmup, iters, peaks, dev, flush, H=128):
+    """mla_decode_attn (plan + split + combine) alone on one layer: B sequences of N tokens in
+    full pages at random places, the L2 flushed (a 256 MB write) before every timed call, CUDA
+    events around each call; median / p10 / p90 and the roofline fraction at the median against
+    the burst peaks (the call is timed alone)."""
     import mla_inputs as I
     import mla_latent_kv_37_b200 as M
+    q = I.query_cat(7, B, H, device=dev)
+    cache = I.paged_cache(8, [N] * B, [N] * B, device=dev)
+    lens = torch.full((B,), N, dtype=torch.int32, device=dev)
+    d = M.dims(B, H, 7168)
+    ws = M.workspace(d, 0, dev)
+    o = torch.empty(B, H, 512, dtype=torch.float32, device=dev)
+    lse = torch.empty(B, H, dtype=torch.float32, device=dev)
+    for _ in range(warmup):
+        M.mla_decode_attn(d, q, cache.pool, cache.page_table, lens, o, ws, lse=lse)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(iters)]
+    for i, (e0, e1) in enumerate(ev):
+        flush.fill_(i & 0xFF)
+        e0.record()
+        M.mla_decode_attn(d, q, cache.pool, cache.page_table, lens, o, ws, lse=lse)
+        e1.record()
+    torch.cuda.synchronize()
+    st = M.mla_get_status()
+    if st:
+        raise RuntimeError(f"device status {st:#x} in the sweep (B={B}, N={N})")
+    us = sorted(e0.elapsed_time(e1) * 1e3 for e0, e1 in ev)
+    pick = lambda f: us[min(len(us) - 1, int(f * (len(us) - 1) + 0.5))]
+    r = attention_roofline(B * N, B, H, pick(0.5) * 1e-6, peaks, sustained=False)
+    del q, cache, lens, ws, o, lse
+    torch.cuda.empty_cache()
+    return {"batch": B, "context": N, "heads": H, "us_median": pick(0.5), "us_p10": pick(0.1),
+            "us_p90": pick(0.9), "frac": r["frac"], "bound": r["bound"], "gbs": r["gbs"],
+            "tflops": r["tflops"], "hbm_frac": r["hbm_frac"],
+            "tensor_frac_burst": r["tensor_frac_burst"]}
+
+
+def run_sweep(args):
+    """`--sweep`: every batch x context of SWEEP_BATCH x SWEEP_CONTEXT, one JSON line each."""
     from mla_latent_kv_37_b200 import build
     build.build()
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    peaks = {}
-    try:
-        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-            peaks = _json.load(f)
-    except Exception:
-        pass
-    hbm_peak = peaks.get("hbm_gbs", 6650.0)
-    tc_peak = peaks.get("bf16_tflops", 1590.0)
+    peaks = load_peaks()
     src = "of measured" if peaks else "of fallback"
-    H = 128
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     for B in SWEEP_BATCH:
         for N in SWEEP_CONTEXT:
-            q = I.query_cat(7, B, H, device=dev)
-            cache = I.paged_cache(8, [N] * B, [N] * B, device=dev)
-            lens = torch.full((B,), N, dtype=torch.int32, device=dev)
-            d = M.dims(B, H, 7168)
-            ws = M.workspace(d, 0, dev)
-            o = torch.empty(B, H, 512, dtype=torch.float32, device=dev)
-            lse = torch.empty(B, H, dtype=torch.float32, device=dev)
-            for _ in range(args.sweep_warmup):
-                M.mla_decode_attn(d, q, cache.pool, cache.page_table, lens, o, ws, lse=lse)
-            torch.cuda.synchronize()
-            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                  for _ in range(args.sweep_iters)]
-            for i, (e0, e1) in enumerate(ev):
-                flush.fill_(i & 0xFF)
-                e0.record()
-                M.mla_decode_attn(d, q, cache.pool, cache.page_table, lens, o, ws, lse=lse)
-                e1.record()
-            torch.cuda.synchronize()
-            st = M.mla_get_status()
-            if st:
-                raise RuntimeError(f"device status {st:#x} in the sweep (B={B}, N={N})")
-            us = sorted(e0.elapsed_time(e1) * 1e3 for e0, e1 in ev)
-            pick = lambda f: us[min(len(us) - 1, int(f * (len(us) - 1) + 0.5))]
-            med = pick(0.5)
-            tokens = B * N
-            nbytes = tokens * ROW_BYTES + B * H * 576 * 2 + B * H * 512 * 4
-            flops = tokens * H * FLOP_PER_TOKEN_HEAD
-            t_hbm = nbytes / (hbm_peak * 1e9) * 1e6
-            t_tc = flops / (tc_peak * 1e12) * 1e6
-            print(_json.dumps({
-                "metric": "mla_decode_attn, one layer (plan + split + combine)",
-                "batch": B, "context": N, "heads": H, "us_median": med, "us_p10": pick(0.1),
-                "us_p90": pick(0.9), "tflops": flops / (med * 1e-6) / 1e12,
-                "gbs": nbytes / (med * 1e-6) / 1e9, "bound": "hbm" if t_hbm >= t_tc else "tensor",
-                "roofline_us": max(t_hbm, t_tc), "frac": max(t_hbm, t_tc) / med,
-                "peaks": {"hbm_gbs": hbm_peak, "bf16_tflops": tc_peak, "source": src + " (burst)"},
-                "warmup": args.sweep_warmup, "timed": args.sweep_iters,
-                "l2": "flushed by a 256 MB write before every timed call"}), flush=True)
-            del q, cache, lens, ws, o, lse
-            torch.cuda.empty_cache()
+            line = sweep_shape(B, N, args.sweep_warmup, args.sweep_iters, peaks, dev, flush)
+            line.update({"metric": "mla_decode_attn, one layer (plan + split + combine)",
+                         "peaks": {"hbm_gbs": peaks.get("hbm_gbs", 6650.0),
+                                   "bf16_tflops": peaks.get("bf16_tflops", 1590.0),
+                                   "source": src + " (burst)"},
+                         "warmup": args.sweep_warmup, "timed": args.sweep_iters,
+                         "l2": "flushed by a 256 MB write before every timed call"})
+            print(json.dumps(line), flush=True)
+
+
+# the attention sweep carried in the default JSON line (batch >= 32, context >= 8K)
+COMPACT_SWEEP = ((32, 8192), (32, 32768), (64, 8192), (64, 32768), (128, 8192), (128, 32768))
+
+
+def compact_sweep(dev, peaks, warmup=5, iters=20):
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    shapes = [sweep_shape(B, N, warmup, iters, peaks, dev, flush) for B, N in COMPACT_SWEEP]
+    del flush
+    torch.cuda.empty_cache()
+    fr = [x["frac"] for x in shapes]
+    return {"what": "mla_decode_attn alone (plan + split + combine), one layer, 128 heads, "
+                    f"{warmup} warm-up + {iters} timed calls per shape, L2 flushed before each, "
+                    "median; roofline against the burst peaks",
+            "shapes": [{k: (round(v, 4) if isinstance(v, float) else v) for k, v in x.items()}
+                       for x in shapes],
+            "min_frac": min(fr), "max_frac": max(fr), "target_frac": 0.7,
+            "meets_target": min(fr) >= 0.7}
+
+
+def run_extra_configs(dev, peaks, steps=10):
+    """The single-layer configurations beside the headline: each one decode step (append +
+    absorbed query + attention + W_UV/W_O) timed over `steps` eager steps, its split-KV kernel
+    timed by CUDA events on its stream, and a parity sample against the oracle."""
+    import mla_latent_kv_37_b200 as M
+    from mla_latent_kv_37_b200.step import DecodeStep
+    out = {}
+    for name, n_seqs, n_heads in EXTRA_CONFIGS:
+        cfg = dict(CONFIGS[name])
+        B, H, D = cfg["batch"], cfg["heads"], cfg["d_model"]
+        layers, h, pos, lens_dev, lens = make_workload(cfg, dev, seed=7)
+        step = DecodeStep(layers, B, H, D, device=dev, graph=False,
+                          query_remainder=cfg.get("remainder", False))
+        for _ in range(3):
+            step.run(h, pos, lens_dev)
+        torch.cuda.synchronize()
+        ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        M.mla_set_profile_events(ev_b, ev_e)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            step.run(h, pos, lens_dev)
+        e1.record()
+        torch.cuda.synchronize()
+        used = M.mla_profile_events_used()
+        M.mla_set_profile_events([], [])
+        st = M.mla_get_status()
+        if st:
+            raise RuntimeError(f"device status {st:#x} in config {name}")
+        ms = e0.elapsed_time(e1) / steps
+        split_s = sorted(b.elapsed_time(e) for b, e in zip(ev_b[:used], ev_e[:used]))
+        split_s = split_s[len(split_s) // 2] / 1e3
+        r = attention_roofline(sum(lens), B, H, split_s, peaks, sustained=False)
+        par = parity_sample(layers, h, [n - 1 for n in lens], step, cfg, n_layers=1,
+                            n_seqs=n_seqs, n_heads=n_heads, seed=1)
+        out[name] = {"workload": cfg["workload"], "batch": B, "tokens_read": sum(lens),
+                     "ms_per_step": ms, "tokens_per_s": B / (ms / 1e3),
+                     "attention": {k: r[k] for k in ("us", "roofline_us", "frac", "bound",
+                                                     "gbs", "tflops")},
+                     "query_remainder": bool(cfg.get("remainder", False)), "parity": par}
+        del layers, h, pos, lens_dev, step
+        torch.cuda.empty_cache()
+    return out
+
+
+def config_block(cfg, lens, world):
+    """The workload description both arms print (identical for the same configuration)."""
+    B, L = cfg["batch"], cfg["layers"]
+    tokens = sum(lens)
+    return {"workload": cfg["workload"], "batch": B,
+            "context": lens[0] if cfg["context"] else "U[1024,8192]", "layers": L,
+            "heads": cfg["heads"], "d_model": cfg["d_model"], "d_c": 512, "d_rope": 64,
+            "page_size": 64, "global_batch": B * world, "parallelism": f"replicas x{world}",
+            "l2": "no flush: inputs per step exceed L2 "
+                  f"({(tokens * ROW_BYTES * L + 0.629e9 * L) / 1e9:.0f} GB vs 0.126 GB)"}
 
 
 # ---------------------------------------------------------------------------------------------
@@ -425,8 +531,7 @@ def run_reference(args, rank, world):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": cfg["workload"], "batch": B, "context": n,
-                       "layers": cfg["layers"], "heads": H, "d_model": D},
+            "config": config_block(cfg, lens, world),
             "cpu_baseline": cb,
             "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -446,6 +551,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-check", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the other single-layer configurations and the attention sweep")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch every kernel eagerly instead of replaying a captured step")
     ap.add_argument("--ref-seconds", type=float, default=0.0,
@@ -540,41 +647,35 @@ def main():
     value = tokens_per_step / (ms / 1e3)
 
     # ---------------- roofline of the dominant kernel (split-KV decode) ----------------
-    import json as _json
-    peaks = {}
-    try:
-        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-            peaks = _json.load(f)
-    except Exception:
-        pass
-    hbm_peak = peaks.get("hbm_gbs", 6650.0)
-    tc_peak = peaks.get("bf16_tflops_sustained", 1400.0)
+    peaks = load_peaks()
     peak_src = "of measured" if peaks else "of fallback"
     tokens_read = sum(lens)
-    bytes_per_launch = tokens_read * ROW_BYTES + B * H * 576 * 2 + B * H * 512 * 4
-    flops_per_launch = tokens_read * H * FLOP_PER_TOKEN_HEAD
     avg_split_s = (sum(split_ms) / len(split_ms)) / 1e3 if split_ms else float("nan")
-    gbs = bytes_per_launch / avg_split_s / 1e9
-    tfs = flops_per_launch / avg_split_s / 1e12
-    t_hbm = bytes_per_launch / (hbm_peak * 1e9)
-    t_tc = flops_per_launch / (tc_peak * 1e12)
-    bound = "hbm" if t_hbm >= t_tc else "tensor"
+    # the kernel runs inside a long step: the sustained tensor rate is its ceiling
+    r = attention_roofline(tokens_read, B, H, avg_split_s, peaks, sustained=True)
     traffic = committed_traffic(args.config)
-    roofline = {"bound": bound,
-                "achieved": gbs if bound == "hbm" else tfs,
-                "peak": hbm_peak if bound == "hbm" else tc_peak,
-                "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
-                "frac": (gbs / hbm_peak) if bound == "hbm" else (tfs / tc_peak),
+    hbm_peak = peaks.get("hbm_gbs", 6650.0)
+    tc_peak = peaks.get("bf16_tflops_sustained", 1400.0)
+    roofline = {"bound": r["bound"],
+                "achieved": r["gbs"] if r["bound"] == "hbm" else r["tflops"],
+                "peak": hbm_peak if r["bound"] == "hbm" else tc_peak,
+                "unit": "GB/s" if r["bound"] == "hbm" else "TFLOP/s",
+                "frac": r["frac"],
                 "traffic": traffic,
                 "kernel": "mla::attn::split_kernel",
-                "peak_source": peak_src + (" (HBM copy)" if bound == "hbm" else
+                "peak_source": peak_src + (" (HBM copy)" if r["bound"] == "hbm" else
                                            " (sustained bf16 GEMM)"),
-                "us_per_launch": avg_split_s * 1e6,
-                "hbm_gbs": gbs, "hbm_frac": gbs / hbm_peak,
-                "tflops": tfs, "tensor_frac": tfs / tc_peak,
-                "bytes_per_launch": bytes_per_launch, "flops_per_launch": flops_per_launch,
-                "roofline_us": max(t_hbm, t_tc) * 1e6,
-                "frac_of_roofline_time": max(t_hbm, t_tc) / avg_split_s}
+                "us_per_launch": r["us"],
+                "hbm_gbs": r["gbs"], "hbm_frac": r["hbm_frac"],
+                "tflops": r["tflops"],
+                "tensor_frac": r["tensor_frac_sustained"],
+                "tensor_frac_label": "achieved TFLOP/s / measured sustained bf16 GEMM rate",
+                "tensor_frac_burst": r["tensor_frac_burst"],
+                "tensor_frac_burst_label": "achieved TFLOP/s / measured burst bf16 dense GEMM "
+                                           "rate (the dense peak a kernel timed alone reaches)",
+                "bytes_per_launch": r["bytes"], "flops_per_launch": r["flops"],
+                "roofline_us": r["roofline_us"],
+                "frac_of_roofline_time": r["frac"]}
 
     # ---------------- end-to-end through the API with host buffers ----------------
     e2e = None
@@ -611,6 +712,15 @@ def main():
         sec, heads_timed, wall = time_oracle(w, hb, rows, lens[0] - 1, H)
         cpu = cpu_baseline_from(sec, cfg, heads_timed, wall)
 
+    # ---------------- the other configurations and the attention sweep (one GPU) ----------
+    configs = sweep = None
+    if rank == 0 and world == 1 and not args.no_extras:
+        del layers, h, step
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        configs = run_extra_configs(dev, peaks)
+        sweep = compact_sweep(dev, peaks)
+
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -618,17 +728,13 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded: N(0,1) hidden states and cache history, "
                     "N(0,1/fan_in) weights, random page placement)",
-            "config": {"workload": cfg["workload"], "batch": B, "context": lens[0]
-                       if cfg["context"] else "U[1024,8192]", "layers": L, "heads": H,
-                       "d_model": D, "d_c": 512, "d_rope": 64, "page_size": 64,
-                       "global_batch": B * world, "parallelism": f"replicas x{world}",
-                       "num_splits": args.num_splits or "auto",
-                       "launch": "CUDA graph of the step" if graph else "eager",
-                       "l2": "no flush: inputs per step exceed L2 "
-                             f"({(tokens_read * ROW_BYTES * L + 0.629e9 * L) / 1e9:.0f} GB vs 0.126 GB)"},
+            "config": config_block(cfg, lens, world),
+            "launch": "CUDA graph of the step" if graph else "eager",
+            "num_splits": args.num_splits or "auto",
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": int(launches), "clocks": clocks, "parity": parity,
             "attention_us_per_layer": roofline["us_per_launch"],
+            "configs": configs, "attention_sweep": sweep,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -218,6 +218,11 @@ int mla_get_status(mla_stream_t stream);
 /* Static description of a return code or status bit set. */
 const char* mla_error_string(int code);
 
+/* The CUDA error behind the last MLA_ERR_CUDA returned to the calling thread: the failing
+ * call, the error's name and its description ("" if there was none).  The string belongs to
+ * the library and stays valid until the thread's next call into it. */
+const char* mla_error_detail(void);
+
 /* Library build string (for logs). */
 const char* mla_version(void);
 

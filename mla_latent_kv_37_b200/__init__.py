@@ -33,7 +33,9 @@ ERRORS = {
 class MlaError(RuntimeError):
     def __init__(self, code: int, where: str):
         self.code = code
-        super().__init__(f"{where}: {ERRORS.get(code, code)} ({_error_string(code)})")
+        detail = _error_detail() if code == -6 else ""
+        super().__init__(f"{where}: {ERRORS.get(code, code)} ({_error_string(code)})"
+                         + (f": {detail}" if detail else ""))
 
 
 class mla_dims(ctypes.Structure):
@@ -70,6 +72,7 @@ _SIGS = {
                                                       _P]),
     "mla_get_status": (ctypes.c_int, [_P]),
     "mla_error_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "mla_error_detail": (ctypes.c_char_p, []),
     "mla_version": (ctypes.c_char_p, []),
     "mla_launch_count": (ctypes.c_uint64, []),
     "mla_set_profile_events": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p),
@@ -99,6 +102,13 @@ def _error_string(code: int) -> str:
         return lib().mla_error_string(code).decode()
     except Exception:  # pragma: no cover
         return "?"
+
+
+def _error_detail() -> str:
+    try:
+        return lib().mla_error_detail().decode()
+    except Exception:  # pragma: no cover
+        return ""
 
 
 def _ptr(t):

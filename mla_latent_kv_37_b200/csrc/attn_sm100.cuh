@@ -11,25 +11,32 @@
 // ([128 x 64] x [64 x 512]).  O (128 x 512 fp32) alone would fill a whole SM's tensor memory,
 // so each work unit runs on a CLUSTER OF TWO CTAs that split the 576 columns of every row:
 // CTA r owns latent columns [256r, 256r+256) and RoPE columns [512+32r, 512+32r+32).
-//   * TMEM (512 columns): O half 256 | query latent half 128 (A operand of QK) | two S
-//     buffers of 64.  The 32 RoPE columns of the query half sit in shared memory (A operand,
-//     64B swizzle), and so does P (bf16, 128B swizzle, A operand of PV), so an S buffer is
-//     free again as soon as it has been drained and QK runs two pages ahead of the softmax.
-//   * Pages arrive by TMA (128B/64B swizzle) into a 4-stage ring; each byte leaves HBM once.
-//     Four pages ahead of the ring each CTA issues a bulk L2 prefetch of half of the page's
-//     rows, so the ring's loads find their lines in L2.
-//   * S_r = Q_r C_r^T is a partial score; the pair exchanges partials.  Distributed shared
-//     memory moves ~16 B/clk per SM, so a partial travels as 16-bit fixed point relative to
-//     its row's largest magnitude (error <= 2^-16 of it, ~1e-4 in the softmax logit), staged
-//     in shared memory and sent with ONE bulk copy (cp.async.bulk, completion counted in bytes
-//     on the peer's mbarrier).
-//   * Two warpgroups share the per-page softmax work: the "send" warpgroup drains S_t,
-//     quantises and stages it; the "softmax" warpgroup drains S_t again, adds the peer's
-//     decoded partial, runs the online softmax and writes P_t.  With S double-buffered, QK of
-//     page t+1 and the exchange of page t+1 run while page t is being softmaxed.
-//   * Each CTA normalises its own half of O with its own running sum (its copy of the scores
-//     differs from the peer's only by the 16-bit rounding of the received half), so the halves
-//     need no further agreement.
+//   * TMEM (512 columns): O half 256 | query latent half 128 (A operand of QK) | S 128, the
+//     scores of a pair of pages.  QK runs once per page pair (N = 128; the tensor core needs
+//     N >= 128 for its full rate), PV once per page (N = 256).
+//   * Pages arrive by TMA into a 4-slot ring laid out box-major, so the rows of two adjacent
+//     slots form one N = 128 operand.  Four pages ahead of the ring each CTA issues a bulk L2
+//     prefetch of half of the page's rows, so the ring's loads find their lines in L2.
+//   * S_r = Q_r C_r^T is a partial score, and the softmax of a row needs both CTAs' partials.
+//     CTA r runs the softmax for half of the rows only (in every warp's 32 TMEM lanes, the 16
+//     lanes 16r .. 16r+15), two threads per row, 32 columns each (the 16x32bx2 TMEM load), so
+//     each SM does half the exponentials.  Per page:
+//       - the send warps read the PEER's rows of S, quantise them to 16-bit fixed point
+//         relative to the row's largest magnitude (error <= 2^-16 of it, ~1e-4 in a logit) and
+//         store them straight from registers into the peer's receive buffer (st.async,
+//         completion counted in bytes on the peer's mbarrier; double-buffered by page);
+//       - the softmax warps add the peer's partial to their own rows, run the online softmax,
+//         and write their rows of P both into their own P buffer and into the peer's, with each
+//         row's rescale factor;
+//       - once the peer's rows of P have landed, PV runs; its completion is committed to both
+//         CTAs' barriers (multicast commit), which frees the P buffers on both sides.
+//     A row's running maximum and sum live with the CTA that owns the row; the other CTA gets
+//     the factor whenever the maximum moves (to rescale its half of O) and the final (max, sum)
+//     at the end of a segment (to normalise its half of O).
+//   * The MMA warp issues from an event loop: each page group's QK as soon as its pages have
+//     landed and S is free, each page's PV as soon as P is complete, whichever comes first.
+//   * The next segment's query half goes into TMEM as soon as the last QK of the previous one
+//     has run, before that segment's epilogue, so a sequence boundary costs no pipeline drain.
 //
 // The concatenated page list of all sequences is cut into `num_parts` contiguous ranges of
 // (nearly) equal length, one per cluster; a range may end inside a sequence and may span
@@ -40,43 +47,52 @@
 // Extended-precision query.  Rounding the absorbed query to bf16 perturbs every logit by about
 // 2^-9 of its size; with large logits (inputs scaled x4 give a logit spread of ~16) that is
 // enough to move the output by ~1e-2.  When the caller passes the rounding remainder q_lo as
-// well (q = q_cat + q_lo to ~16 bits), each cluster takes 64 heads instead of 128 and stacks,
-// for each of them, a row of q_cat and a row of q_lo in the 128 rows of the MMA: in every
-// quarter of the rows (one warp's TMEM lanes), rows 0-15 hold heads 16w..16w+15 of the group
-// from q_cat and rows 16-31 the same heads from q_lo.  The score of a head is then the sum of
-// its two rows (one shuffle), the softmax runs identically on both rows, O gets the same P in
-// both, and only the q_cat row is written out.  Launch: `groups` = ceil(H/64) clusters per
-// part, so the tensor work per token doubles; the page bytes are read by the part's clusters
-// at about the same time and mostly come from L2 the second time.
+// well (q = q_cat + q_lo to ~16 bits), each cluster takes 64 heads instead of 128 and puts, for
+// each of them, a row of q_cat and a row of q_lo in the same 16-lane half of a warp's TMEM
+// lanes (see RowMap).  The score of a head is then the sum of its two rows (one shuffle), the
+// softmax runs identically on both rows, O gets the same P in both, and only the q_cat row is
+// written out.  Launch: `groups` = ceil(H/64) clusters per part, so the tensor work per token
+// doubles; the page bytes are read by the part's clusters at about the same time and mostly
+// come from L2 the second time.
 //
-// Roles (384 threads): warps 0-3 softmax + epilogue (thread i owns head row i = TMEM lane i),
-// warps 4-7 send, warp 8 TMA producer, warp 9 MMA issuer, warp 10 bulk-copy sender (warp 11
-// has no role).  Each softmax warp hands its rows of the receive buffer back to the peer
-// itself once it has decoded them.  The online softmax keeps a per-row reference maximum and rescales O
-// only when the running maximum grows by more than 2^8.
+// Roles (320 threads): warps 0-3 softmax (own rows), query load, O rescale and epilogue;
+// warps 4-7 send; warp 8 TMA producer; warp 9 MMA issuer and TMEM owner.  The online softmax
+// keeps a per-row reference maximum and rescales O only when the running maximum grows by
+// more than 2^8.
 #pragma once
 #include "ptx_sm100.cuh"
 
 namespace mla {
 namespace attn {
 
-constexpr int kThreads = 384;
+constexpr int kThreads = 480;  // 15 warps: 8 softmax, 4 send + finish, TMA, MMA, P copy
 constexpr int kPage = 64;
 constexpr int kRow = 576;
-constexpr int kStages = 4;
-constexpr uint32_t kCLatBox = 64 * 128;                   // 64 rows x 64 bf16
-constexpr uint32_t kStageBytes = 4 * kCLatBox + 64 * 64;  // + rope box 64 rows x 32 bf16
-constexpr uint32_t kXPayload = 128 * 128;                 // 128 rows x 64 x 16-bit
-constexpr uint32_t kXBytes = kXPayload + 128 * 4;         // + one fp32 step per row
-constexpr uint32_t kQRopeBytes = 128 * 64;                // 128 rows x 32 bf16
-constexpr uint32_t kPBytes = 128 * 128;                   // P: 128 rows x 64 bf16
-constexpr uint32_t kOffStage = 0;
-constexpr uint32_t kOffP = kOffStage + kStages * kStageBytes;  // one P buffer
-constexpr uint32_t kOffQRope = kOffP + kPBytes;
-constexpr uint32_t kOffSend = kOffQRope + kQRopeBytes;  // two send buffers
-constexpr uint32_t kOffRecv = kOffSend + 2 * kXBytes;   // one receive buffer
-constexpr uint32_t kOffBar = kOffRecv + kXBytes;
-constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // barriers + alignment slack
+constexpr int kSlots = 4;  // page slots of the ring
+constexpr uint32_t kBoxBytes = 64 * 128;      // one page's 64 rows x 64 latent columns (bf16)
+constexpr uint32_t kRopeBoxBytes = 64 * 64;   // one page's 64 rows x 32 RoPE columns (bf16)
+constexpr uint32_t kSlotBytes = 4 * kBoxBytes + kRopeBoxBytes;  // this CTA's half of a page
+// The ring is box-major: latent box i of slot s at i * kSlots * kBoxBytes + s * kBoxBytes, so
+// the rows of slots s and s + 1 are contiguous in every box (one N = 128 operand for a page
+// pair); the RoPE boxes of the slots follow, contiguous in slot order.
+constexpr uint32_t kOffRing = 0;
+constexpr uint32_t kBoxStride = kSlots * kBoxBytes;
+constexpr uint32_t kOffRope = kOffRing + 4 * kBoxStride;
+constexpr uint32_t kPBytes = 128 * 128;  // P of one page: 128 rows x 64 bf16
+constexpr uint32_t kOffP = kOffRope + kSlots * kRopeBoxBytes;  // two P buffers (page parity)
+constexpr uint32_t kQRopeBytes = 128 * 64;                    // 128 rows x 32 bf16
+constexpr uint32_t kOffQRope = kOffP + 2 * kPBytes;
+constexpr uint32_t kXPayload = 64 * 128;          // 64 rows x 64 partial scores x 16 bits
+constexpr uint32_t kXBytes = kXPayload + 64 * 4;  // + one fp32 step per row
+constexpr uint32_t kOffX = kOffQRope + kQRopeBytes;  // two receive buffers (page parity)
+constexpr uint32_t kOffAlphaIn = kOffX + 2 * kXBytes;     // the peer's rescale factors [2][64]
+constexpr uint32_t kOffAlphaOwn = kOffAlphaIn + 2 * 256;  // our rows' factors [2][64]
+constexpr uint32_t kOffStats = kOffAlphaOwn + 2 * 256;    // the peer's (max, sum) per row [64]
+constexpr uint32_t kOffMaxX = kOffStats + 512;            // row maxima of the column halves [2][2][64]
+constexpr uint32_t kOffLPart = kOffMaxX + 1024;  // row sums of the column halves [2][2][64]
+constexpr uint32_t kOffBar = kOffLPart + 1024;
+constexpr uint32_t kSmemBytes = kOffBar + 512 + 1024;  // barriers + alignment slack
+constexpr uint32_t kPMsgBytes = 64 * 128 + 64 * 4;     // P rows sent to the peer + factors
 // TMEM columns
 constexpr uint32_t kTmemO = 0, kTmemQ = 256, kTmemS = 384, kTmemCols = 512;
 constexpr int kAhead = 4;  // pages prefetched into L2 ahead of the TMA ring
@@ -84,8 +100,11 @@ constexpr uint32_t kPageBytes = kPage * kRow * 2;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 static_assert(kSmemBytes <= 232448, "shared memory budget");
-static_assert(kTmemS + 2 * 64 == kTmemCols, "tensor memory budget");
-static_assert(kXBytes % 16 == 0 && kOffP % 1024 == 0 && kOffQRope % 1024 == 0, "alignment");
+static_assert(kTmemS + 128 == kTmemCols, "tensor memory budget");
+static_assert(kXBytes % 16 == 0 && kOffP % 1024 == 0 && kOffQRope % 1024 == 0 &&
+                  kOffRope % 1024 == 0 && kOffX % 16 == 0 && kOffAlphaIn % 16 == 0 &&
+                  kOffAlphaOwn % 16 == 0 && kOffBar % 8 == 0,
+              "alignment");
 
 struct Params {
   int batch;
@@ -272,27 +291,6 @@ __device__ __forceinline__ uint32_t xrow_off(int row, int chunk) {
   return static_cast<uint32_t>(row) * 128u + static_cast<uint32_t>((chunk ^ (row & 7)) * 16);
 }
 
-// Reductions over a row's 64 values as 8 independent chains (a single 64-long chain of
-// dependent instructions would dominate a page's softmax time).
-__device__ __forceinline__ float max64(const float* s) {
-  float m[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) m[j] = s[j];
-#pragma unroll
-  for (int k = 8; k < 64; ++k) m[k & 7] = fmaxf(m[k & 7], s[k]);
-  return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])),
-               fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
-}
-__device__ __forceinline__ float maxabs64(const float* s) {
-  float m[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) m[j] = fabsf(s[j]);
-#pragma unroll
-  for (int k = 8; k < 64; ++k) m[k & 7] = fmaxf(m[k & 7], fabsf(s[k]));
-  return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])),
-               fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
-}
-
 // 16-bit fixed point (offset binary: u = q + 32768 for q in [-32767, 32767]) without the
 // quarter-rate int<->float conversion instructions.  Encoding: fma(x, 1/step, 1.5*2^23 + 32768)
 // rounds to nearest even and leaves u in the low 16 mantissa bits.  Decoding: the bits
@@ -317,32 +315,92 @@ __device__ __forceinline__ float dec_hi(uint32_t v) {
 // ------------------------------------------------------------------------------------------
 // The split kernel
 // ------------------------------------------------------------------------------------------
+// TMEM lanes (MMA rows) and heads.  Without the query remainder, lane L computes head L.  With
+// it, in quarter q of the lanes (one warp's 32) lanes 16h + 8k + j (h, k in {0, 1}, j < 8)
+// compute head 64 group + 16q + 8h + j, from q_cat for k = 0 and from q_lo for k = 1, so that
+// the two rows of a head sit in the same 16-lane half of the quarter.
+struct RowMap {
+  bool hi_lo;
+  int group;
+  __device__ int head(int L) const {
+    return hi_lo ? 64 * group + 16 * (L >> 5) + 8 * ((L >> 4) & 1) + (L & 7) : L;
+  }
+  __device__ bool lo(int L) const { return hi_lo && ((L >> 3) & 1); }
+};
+
 // Every mbarrier below completes one phase per use and is waited phase by phase, never more
 // than one phase behind its current state (buffers that could run two pages ahead of their
-// waiter have one barrier per buffer), so parity waits cannot alias.
+// waiter have one barrier per buffer), so parity waits cannot alias.  Barriers marked "bytes"
+// complete when the stated number of bytes has landed (TMA, bulk copy or st.async from the
+// peer CTA); the ones the peer writes are armed here, one use ahead.
 struct Bars {
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
-  uint64_t q_full;        // TMA: the segment's query RoPE half landed in shared memory
-  uint64_t q_empty;       // MMA: the segment's last QK finished (commit)
-  uint64_t q_ready;       // softmax WG: the segment's query latent half is in TMEM (128)
-  uint64_t s_full[2];     // MMA: S buffer i written (commit)
-  uint64_t s_free[2];     // both warpgroups drained S buffer i (256)
-  uint64_t staged[2];     // send WG: partial staged in send[i] (128)
-  uint64_t p_full;        // softmax WG: P written (128)
-  uint64_t pv_done;       // MMA: PV finished, P buffer free (commit, once per page)
-  uint64_t x_full;        // the peer's partial landed in recv (bulk-copy bytes)
-  uint64_t peer_done[2];  // the peer's 4 softmax warps decoded our partial of a page of
-                          // parity i (4 remote arrivals)
-  uint64_t o_free;        // softmax WG: the epilogue drained O (128)
-  uint64_t seg_done;      // MMA: every PV of the segment finished (commit, once per segment)
-  uint64_t drain;
+  uint64_t full[kSlots];   // TMA: the page slot is filled (bytes)
+  uint64_t empty[kSlots];  // MMA: the PV that read the slot finished (commit)
+  uint64_t q_full;         // TMA: the segment's query RoPE half landed (bytes)
+  uint64_t q_empty;        // MMA: the segment's last QK finished (commit)
+  uint64_t q_ready;        // softmax warps 0-3: the query latent half is in TMEM (4)
+  uint64_t s_full;         // MMA: S of a page group is written (commit)
+  uint64_t s_free;         // the 8 softmax and 4 send warps drained S (12)
+  uint64_t x_full[2];      // the peer's partial scores for our rows landed (bytes)
+  uint64_t x_free[2];      // the peer's softmax warps decoded our partials of a page (8 remote)
+  uint64_t p_own[2];       // softmax warps: our rows of P and their factors are written (8)
+  uint64_t p_peer[2];      // the peer's rows of P and their factors landed (bytes)
+  uint64_t p_ready[2];     // send warps: P complete, O rescaled, PV may run (4)
+  uint64_t p_free[2];      // our PV of the page finished (commit) and the copy of our rows to
+                           // the peer has read them (1 arrival): the buffer may be rewritten
+  uint64_t pv_done[2];     // PV of the page finished in both CTAs (2 commits)
+  uint64_t seg_done;       // MMA: every PV of the segment finished (commit)
+  uint64_t o_free;         // softmax warps: the epilogue drained O (8)
+  uint64_t st_full;        // the peer's row statistics for the segment landed (bytes)
+  uint64_t mx_bar[4][2];   // the two softmax warps of quarter q posted their row maxima (2)
+  uint64_t ls_bar[2];      // the 8 softmax warps posted their row sums of a segment (8)
+  uint64_t drain;          // MMA: final drain after an abort
   uint32_t tmem_base;
   int abort_flag;
 };
-static_assert(sizeof(Bars) <= 256, "barrier block");
+static_assert(sizeof(Bars) <= 512, "barrier block");
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+constexpr uint64_t kDrainNs = 200000000ull;  // waits for copies and MMAs already in flight
+constexpr uint32_t kFull = 0xffffffffu;
+
+__device__ __forceinline__ float max16(const float* s) {
+  float m[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) m[j] = s[j];
+#pragma unroll
+  for (int k = 4; k < 16; ++k) m[k & 3] = fmaxf(m[k & 3], s[k]);
+  return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+}
+__device__ __forceinline__ float maxabs32(const float* s) {
+  float m[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) m[j] = fabsf(s[j]);
+#pragma unroll
+  for (int k = 8; k < 32; ++k) m[k & 7] = fmaxf(m[k & 7], fabsf(s[k]));
+  return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])),
+               fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
+}
+
+__device__ __forceinline__ void spin_ns(uint64_t ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (globaltimer_ns() - t0 < ns) {
+  }
+}
+
+// One lane tests, the warp gets the answer (a warp-uniform decision for an event loop).
+__device__ __forceinline__ bool warp_test(uint64_t* bar, uint32_t parity) {
+  bool ok = false;
+  if ((threadIdx.x & 31) == 0) ok = mbar_test(bar, parity);
+  return __shfl_sync(kFull, ok ? 1 : 0, 0) != 0;
+}
+
+// Advance the start-address field (bits 0-13, in 16-byte units) of a shared-memory matrix
+// descriptor by `bytes` (addresses stay below 256 KiB, so the field cannot overflow).
+__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) {
+  return d + static_cast<uint64_t>(bytes >> 4);
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
     split_kernel(const __grid_constant__ CUtensorMap tm_c_lat,
                  const __grid_constant__ CUtensorMap tm_c_rope,
                  const __grid_constant__ CUtensorMap tm_q_rope,
@@ -358,33 +416,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   // clusters of one part are adjacent, so they stream the same pages at about the same time
   const int part = static_cast<int>(blockIdx.x >> 1) / p.groups;
   const int group = static_cast<int>(blockIdx.x >> 1) - part * p.groups;
-  const bool hi_lo = p.q_lo != nullptr;
+  const RowMap rows{p.q_lo != nullptr, group};
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kSlots; ++s) {
       mbar_init(&bars->full[s], 1);
       mbar_init(&bars->empty[s], 1);
     }
     mbar_init(&bars->q_full, 1);
     mbar_init(&bars->q_empty, 1);
-    mbar_init(&bars->q_ready, 128);
+    mbar_init(&bars->q_ready, 4);
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->s_free, 12);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars->s_full[i], 1);
-      mbar_init(&bars->s_free[i], 256);
-      mbar_init(&bars->staged[i], 128);
-      mbar_init(&bars->peer_done[i], 4);
+      mbar_init(&bars->x_full[i], 1);
+      mbar_init(&bars->x_free[i], 8);
+      mbar_init(&bars->p_own[i], 8);
+      mbar_init(&bars->p_peer[i], 1);
+      mbar_init(&bars->p_ready[i], 4);
+      mbar_init(&bars->p_free[i], 2);
+      mbar_init(&bars->pv_done[i], 2);
     }
-    mbar_init(&bars->p_full, 128);
-    mbar_init(&bars->pv_done, 1);
-    mbar_init(&bars->x_full, 1);
-    mbar_init(&bars->o_free, 128);
     mbar_init(&bars->seg_done, 1);
+    mbar_init(&bars->o_free, 8);
+    mbar_init(&bars->st_full, 1);
+    for (int i = 0; i < 8; ++i) mbar_init(&bars->mx_bar[i >> 1][i & 1], 2);
+    mbar_init(&bars->ls_bar[0], 8);
+    mbar_init(&bars->ls_bar[1], 8);
     mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
     fence_mbar_init_cluster();
-    mbar_arrive_expect_tx(&bars->x_full, kXBytes);  // armed for page 0
+    // receive-side barriers, armed for their first use
+    for (int i = 0; i < 2; ++i) {
+      mbar_arrive_expect_tx(&bars->x_full[i], kXBytes);
+      mbar_arrive_expect_tx(&bars->p_peer[i], kPMsgBytes);
+    }
+    mbar_arrive_expect_tx(&bars->st_full, 512);
   }
-  if (warp == 9) {
+  if (warp == 13) {
     tmem_alloc(&bars->tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -404,12 +473,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int g_begin = active ? plan.part_start()[part] : 0;
   const int g_end = active ? plan.part_start()[part + 1] : 0;
   const int b_begin = active ? plan.part_seq()[part] : p.batch;
-  uint8_t* sStage = smem + kOffStage;
   uint8_t* sQRope = smem + kOffQRope;
-  const uint32_t send_base = smem_u32(smem + kOffSend);
-  const uint32_t recv_base = smem_u32(smem + kOffRecv);
+  volatile int never = 0;
+  const WaitCtx drain_ctx{&never, p.status, kDrainNs};
 
-  if (warp == 8) {
+  if (warp == 12) {
     // =================== TMA producer: page ring + query RoPE half ===================
     SegIter it{plan.seq_pages(), plan.seq_prefix(), p.batch, g_begin, g_end, b_begin};
     int seq, p0, p1, t = 0, sg = 0, issued = 0;
@@ -419,30 +487,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_c_lat);
       tma_prefetch_desc(&tm_c_rope);
       tma_prefetch_desc(&tm_q_rope);
-      if (hi_lo) tma_prefetch_desc(&tm_ql_rope);
+      if (rows.hi_lo) tma_prefetch_desc(&tm_ql_rope);
     }
     while (ok && it.next(seq, p0, p1)) {
       if (lane == 0) {
         if (sg > 0) ok = mbar_wait(&bars->q_empty, (sg - 1) & 1, wc);
         if (ok) {
           mbar_arrive_expect_tx(&bars->q_full, kQRopeBytes);
-          if (!hi_lo) {
+          if (!rows.hi_lo) {
             tma_load_3d(sQRope, &tm_q_rope, &bars->q_full, 512 + 32 * rank, 0, seq);
           } else {
-            // 16-row boxes: rows 32w..32w+15 from q_cat, rows 32w+16..32w+31 from q_lo, both
-            // for heads 64 group + 16w .. +15 (rows past H are zero-filled by the copy)
+            // 8-row boxes in the lane order of RowMap (rows past H are zero-filled)
 #pragma unroll
-            for (int w4 = 0; w4 < 4; ++w4) {
-              const int h0 = 64 * group + 16 * w4;
-              tma_load_3d(sQRope + (32 * w4) * 64, &tm_q_rope, &bars->q_full, 512 + 32 * rank,
-                          h0, seq);
-              tma_load_3d(sQRope + (32 * w4 + 16) * 64, &tm_ql_rope, &bars->q_full,
-                          512 + 32 * rank, h0, seq);
-            }
+            for (int qq = 0; qq < 4; ++qq)
+#pragma unroll
+              for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                for (int k = 0; k < 2; ++k)
+                  tma_load_3d(sQRope + (32 * qq + 16 * hh + 8 * k) * 64,
+                              k ? &tm_ql_rope : &tm_q_rope, &bars->q_full, 512 + 32 * rank,
+                              64 * group + 16 * qq + 8 * hh, seq);
           }
         }
       }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
+      ok = __shfl_sync(kFull, ok, 0);
       const int32_t* pt = p.page_table + static_cast<size_t>(seq) * p.max_pages;
       for (int pb = p0; ok && pb < p1; pb += 32) {
         const int cnt = min(32, p1 - pb);
@@ -456,396 +524,579 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           prefetch_l2(p.pool + static_cast<size_t>(my_page) * kPageBytes + rank * (kPageBytes / 2),
                       kPageBytes / 2);
         for (int j = 0; j < cnt; ++j, ++t) {
-          const int page = __shfl_sync(0xffffffffu, my_page, j);
-          const int later = __shfl_sync(0xffffffffu, my_page, min(j + kAhead, 31));
+          const int page = __shfl_sync(kFull, my_page, j);
+          const int later = __shfl_sync(kFull, my_page, min(j + kAhead, 31));
           if (lane == 0 && j + kAhead < cnt)
             prefetch_l2(p.pool + static_cast<size_t>(later) * kPageBytes + rank * (kPageBytes / 2),
                         kPageBytes / 2);
           if (lane == 0) {
-            const int s = t % kStages;
-            if (t >= kStages) ok = mbar_wait(&bars->empty[s], ((t / kStages) - 1) & 1, wc);
+            const int s = t % kSlots;
+            if (t >= kSlots) ok = mbar_wait(&bars->empty[s], ((t / kSlots) - 1) & 1, wc);
             if (ok) {
-              uint8_t* dst = sStage + s * kStageBytes;
-              mbar_arrive_expect_tx(&bars->full[s], kStageBytes);
+              mbar_arrive_expect_tx(&bars->full[s], kSlotBytes);
               const int y = page * kPage;
 #pragma unroll
               for (int i = 0; i < 4; ++i)
-                tma_load_2d_hint(dst + i * kCLatBox, &tm_c_lat, &bars->full[s],
-                                 256 * rank + 64 * i, y, pol_stream);
-              tma_load_2d_hint(dst + 4 * kCLatBox, &tm_c_rope, &bars->full[s], 512 + 32 * rank,
-                               y, pol_stream);
+                tma_load_2d_hint(smem + kOffRing + i * kBoxStride + s * kBoxBytes, &tm_c_lat,
+                                 &bars->full[s], 256 * rank + 64 * i, y, pol_stream);
+              tma_load_2d_hint(smem + kOffRope + s * kRopeBoxBytes, &tm_c_rope, &bars->full[s],
+                               512 + 32 * rank, y, pol_stream);
               issued = t + 1;
             }
           }
-          ok = __shfl_sync(0xffffffffu, ok, 0);
+          ok = __shfl_sync(kFull, ok, 0);
           if (!ok) break;
         }
       }
       ++sg;
     }
-    if (lane == 0 && bars->abort_flag) {
-      volatile int never = 0;
-      WaitCtx drain{&never, p.status, p.wait_ns};
-      for (int i = max(0, issued - kStages); i < issued; ++i)
-        mbar_wait(&bars->full[i % kStages], (i / kStages) & 1, drain);
-      if (sg > 0) mbar_wait(&bars->q_full, (sg - 1) & 1, drain);
+    if (lane == 0 && bars->abort_flag) {  // no copy may still be landing when the CTA exits
+      for (int i = max(0, issued - kSlots); i < issued; ++i)
+        mbar_wait(&bars->full[i % kSlots], (i / kSlots) & 1, drain_ctx);
+      if (sg > 0) mbar_wait(&bars->q_full, (sg - 1) & 1, drain_ctx);
     }
-  } else if (warp == 9) {
-    // =================== MMA issuer ===================
+  } else if (warp == 13) {
+    // =================== MMA issuer: QK per page group, PV per page, as each is ready ========
     if (lane == 0) {
-      const uint32_t idesc_qk = idesc_bf16(128, 64, 0, 0);
+      const uint32_t idesc_qk128 = idesc_bf16(128, 128, 0, 0);
+      const uint32_t idesc_qk64 = idesc_bf16(128, 64, 0, 0);
       const uint32_t idesc_pv = idesc_bf16(128, 256, 0, 1);
-      const uint32_t qrope = smem_u32(sQRope);
-      SegIter it{plan.seq_pages(), plan.seq_prefix(), p.batch, g_begin, g_end, b_begin};
-      int seq, p0, p1, t = 0, sg = 0;
-      bool ok = true;
-      // S_tt = Q_r C_r^T into S buffer tt & 1: latent half A from TMEM, RoPE half A from smem
-      auto issue_qk = [&](int tt, bool last_of_seg) -> bool {
-        const int s = tt % kStages;
-        if (!mbar_wait(&bars->full[s], (tt / kStages) & 1, wc)) return false;
-        tc_fence_after();
-        const uint32_t st = smem_u32(sStage + s * kStageBytes);
-        const uint32_t d = tmem + kTmemS + (tt & 1) * 64;
+      // descriptors at the buffers' starts; every operand below is one of these advanced
+      const uint64_t d_ring = smem_desc(smem_u32(smem + kOffRing), 16, 1024, kSwizzle128B);
+      const uint64_t d_rope = smem_desc(smem_u32(smem + kOffRope), 16, 512, kSwizzle64B);
+      const uint64_t d_qrope = smem_desc(smem_u32(sQRope), 16, 512, kSwizzle64B);
+      const uint64_t d_p = smem_desc(smem_u32(smem + kOffP), 16, 1024, kSwizzle128B);
+      const uint64_t d_pv_b = smem_desc(smem_u32(smem + kOffRing), kBoxStride, 1024, kSwizzle128B);
+      // S = Q_r C_r^T for the npg (1 or 2) pages from global page t on: one N = 128 product
+      // when the two slots are adjacent in the ring, else one N = 64 product per page
+      auto issue_qk = [&](int t, int npg) {
+        const int s0 = t % kSlots;
+        const int runs = (npg == 2 && s0 + 1 < kSlots) ? 1 : npg;
+        const uint32_t idesc = (npg == 2 && runs == 1) ? idesc_qk128 : idesc_qk64;
+        for (int u = 0; u < runs; ++u) {
+          const uint32_t s = static_cast<uint32_t>((s0 + u) % kSlots);
+          const uint32_t d = tmem + kTmemS + 64 * u;
+          const uint64_t b0 = desc_add(d_ring, s * kBoxBytes);
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          mma_ts(d, tmem + kTmemQ + 8 * j,
-                 smem_desc(st + (j >> 2) * kCLatBox + (j & 3) * 32, 16, 1024, kSwizzle128B),
-                 idesc_qk, j > 0 ? 1u : 0u);
-#pragma unroll
-        for (int j = 0; j < 2; ++j)
-          mma_ss(d, smem_desc(qrope + j * 32, 16, 512, kSwizzle64B),
-                 smem_desc(st + 4 * kCLatBox + j * 32, 16, 512, kSwizzle64B), idesc_qk, 1u);
-        mma_commit(&bars->s_full[tt & 1]);
-        if (last_of_seg) mma_commit(&bars->q_empty);
-        return true;
+          for (int j = 0; j < 16; ++j)
+            mma_ts(d, tmem + kTmemQ + 8 * j,
+                   desc_add(b0, (j >> 2) * kBoxStride + (j & 3) * 32), idesc, j > 0 ? 1u : 0u);
+          const uint64_t r0 = desc_add(d_rope, s * kRopeBoxBytes);
+          mma_ss(d, d_qrope, r0, idesc, 1u);
+          mma_ss(d, desc_add(d_qrope, 32), desc_add(r0, 32), idesc, 1u);
+        }
+        mma_commit(&bars->s_full);
       };
-      // O += P_tt C_lat: A = P (bf16, shared memory), B = the page's latent half
-      const uint32_t p_base = smem_u32(smem + kOffP);
-      auto issue_pv = [&](int tt, bool first_of_seg) -> bool {
-        if (first_of_seg && sg > 0 && !mbar_wait(&bars->o_free, (sg - 1) & 1, wc)) return false;
-        if (!mbar_wait(&bars->p_full, tt & 1, wc)) return false;
-        tc_fence_after();
-        const uint32_t st = smem_u32(sStage + (tt % kStages) * kStageBytes);
-        const uint32_t pa = p_base;
+      // O += P_t C_lat,t: A = P (bf16, shared memory), B = the page's latent half (MN-major)
+      auto issue_pv = [&](int t, bool first) {
+        const uint32_t s = static_cast<uint32_t>(t % kSlots);
+        const uint64_t a0 = desc_add(d_p, (t & 1) * kPBytes);
+        const uint64_t b0 = desc_add(d_pv_b, s * kBoxBytes);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_ss(tmem + kTmemO, smem_desc(pa + kk * 32, 16, 1024, kSwizzle128B),
-                 smem_desc(st + kk * 2048, 8192, 1024, kSwizzle128B), idesc_pv,
-                 (first_of_seg && kk == 0) ? 0u : 1u);
-        mma_commit(&bars->pv_done);
-        mma_commit(&bars->empty[tt % kStages]);
-        return true;
+          mma_ss(tmem + kTmemO, desc_add(a0, kk * 32), desc_add(b0, kk * 2048), idesc_pv,
+                 (first && kk == 0) ? 0u : 1u);
+        mma_commit(&bars->p_free[t & 1]);
+        mma_commit_cluster(&bars->pv_done[t & 1], 0x3);  // both CTAs learn that P_t is read
+        mma_commit(&bars->empty[s]);
       };
-      // S buffer of page tt (tt >= 2) is free once both warpgroups drained page tt - 2
-      auto s_ready = [&](int tt) -> bool {
-        return tt < 2 || mbar_wait(&bars->s_free[tt & 1], ((tt >> 1) - 1) & 1, wc);
-      };
-      while (ok && it.next(seq, p0, p1)) {
-        const int n = p1 - p0, t0 = t;
-        ok = mbar_wait(&bars->q_ready, sg & 1, wc) && mbar_wait(&bars->q_full, sg & 1, wc);
-        if (ok) ok = s_ready(t0) && issue_qk(t0, n == 1);
-        if (ok && n > 1) ok = s_ready(t0 + 1) && issue_qk(t0 + 1, n == 2);
-        // softmax order per page: drain S_i (s_free) ... write P_i (p_full)
-        for (int i = 0; ok && i < n; ++i) {
-          const int tt = t0 + i;
-          if (i + 2 < n && !(ok = s_ready(tt + 2) && issue_qk(tt + 2, i + 3 == n))) break;
-          if (!(ok = issue_pv(tt, i == 0))) break;
-        }
-        if (ok) mma_commit(&bars->seg_done);
-        t += n;
-        ++sg;
-      }
-      if (bars->abort_flag) {  // no MMA may be in flight when TMEM is released
-        mma_commit(&bars->drain);
-        volatile int never = 0;
-        WaitCtx drain{&never, p.status, p.wait_ns};
-        mbar_wait(&bars->drain, 0, drain);
-      }
-    }
-  } else if (warp == 10) {
-    // =================== exchange: bulk copies out ===================
-    if (lane == 0) {
-      const uint32_t peer_recv = mapa_shared(recv_base, peer);
-      const uint32_t peer_xfull = mapa_shared(smem_u32(&bars->x_full), peer);
-      SegIter it{plan.seq_pages(), plan.seq_prefix(), p.batch, g_begin, g_end, b_begin};
-      int seq, p0, p1, t = 0;
+      SegIter itq{plan.seq_pages(), plan.seq_prefix(), p.batch, g_begin, g_end, b_begin};
+      SegIter itv = itq;
+      int qs, q0, q1, vs, v0, v1;
+      bool q_more = itq.next(qs, q0, q1), v_more = itv.next(vs, v0, v1);
+      int q_i = 0, q_t = 0, q_g = 0, q_sg = 0;  // QK: page in segment, global page, group, seg
+      int v_i = 0, v_t = 0, v_sg = 0;           // PV: page in segment, global page, segment
+      uint64_t idle_since = 0;
+      uint32_t spins = 0;
       bool ok = true;
-      while (ok && it.next(seq, p0, p1)) {
-        const int n = p1 - p0;
-        for (int tt = t; ok && tt < t + n; ++tt) {
-          const int buf = tt & 1;
-          // the page's partial is staged in send[buf] and the peer's (single) receive buffer
-          // has been decoded for page tt - 1: ship it
-          if (!(ok = mbar_wait(&bars->staged[buf], (tt >> 1) & 1, wc))) break;
-          if (tt >= 1 && !(ok = mbar_wait<true>(&bars->peer_done[(tt - 1) & 1],
-                                               ((tt - 1) >> 1) & 1, wc)))
-            break;
-          bulk_copy_s2cluster(peer_recv, send_base + buf * kXBytes, kXBytes, peer_xfull);
-        }
-        t += n;
-      }
-    }
-  } else if (warp == 11) {
-    // no role
-  } else if (warp >= 4) {
-    // =================== send warpgroup (warps 4-7) ===================
-    const int row = threadIdx.x - 128;
-    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    SegIter it{plan.seq_pages(), plan.seq_prefix(), p.batch, g_begin, g_end, b_begin};
-    int seq, p0, p1, t = 0;
-    bool ok = true;
-    while (ok && it.next(seq, p0, p1)) {
-      const int n = p1 - p0;
-      const int len = min(p.seq_lens[seq], p.max_pages * kPage);
-      for (int i = 0; i < n; ++i) {
-        const int tt = t + i, buf = tt & 1;
-        if (!(ok = warp_wait(&bars->s_full[buf], (tt >> 1) & 1, wc))) break;
-        tc_fence_after();
-        float s[64];
-        {
-          uint32_t r[32];
-          tmem_ld32(tmem + kTmemS + buf * 64 + lane_off, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int k = 0; k < 32; ++k) s[k] = __uint_as_float(r[k]);
-          tmem_ld32(tmem + kTmemS + buf * 64 + 32 + lane_off, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int k = 0; k < 32; ++k) s[32 + k] = __uint_as_float(r[k]);
-        }
-        tc_fence_before();
-        mbar_arrive(&bars->s_free[buf]);
-        const int valid = min(kPage, len - (p0 + i) * kPage);
-        if (valid < kPage) {
-#pragma unroll
-          for (int k = 0; k < 64; ++k) s[k] = k < valid ? s[k] : 0.f;  // never sent
-        }
-        const float mabs = maxabs64(s);
-        const float inv = mabs > 0.f ? 32767.f / mabs : 0.f;
-        if (tt >= 2 && !(ok = warp_wait<true>(&bars->peer_done[buf], ((tt >> 1) - 1) & 1, wc)))
-          break;
-        const uint32_t base = send_base + buf * kXBytes;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint32_t a = enc_u16x2(s[8 * c], s[8 * c + 1], inv);
-          const uint32_t b = enc_u16x2(s[8 * c + 2], s[8 * c + 3], inv);
-          const uint32_t cc = enc_u16x2(s[8 * c + 4], s[8 * c + 5], inv);
-          const uint32_t d = enc_u16x2(s[8 * c + 6], s[8 * c + 7], inv);
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(base + xrow_off(row, c)),
-                       "r"(a), "r"(b), "r"(cc), "r"(d)
-                       : "memory");
-        }
-        asm volatile("st.shared.f32 [%0], %1;" ::"r"(base + kXPayload + row * 4),
-                     "f"(mabs * (1.f / 32767.f))
-                     : "memory");
-        fence_proxy_async_smem();  // generic-proxy writes -> visible to the bulk copy
-        mbar_arrive(&bars->staged[buf]);
-      }
-      t += n;
-    }
-  } else {
-    // =================== softmax warpgroup (warps 0-3) + epilogue ===================
-    const int row = threadIdx.x;  // head row = TMEM lane
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const float NEG_INF = -__int_as_float(0x7f800000);
-    // the head this row computes, and whether it carries the query's remainder (q_lo)
-    const int head = hi_lo ? 64 * group + 16 * warp + (lane & 15) : row;
-    const bool lo_row = hi_lo && (lane & 16);
-    const bool row_ok = head < p.n_heads;
-    const bool row_out = row_ok && !lo_row;  // rows whose result is written
-    const uint32_t peer_done_r[2] = {mapa_shared(smem_u32(&bars->peer_done[0]), peer),
-                                     mapa_shared(smem_u32(&bars->peer_done[1]), peer)};
-    SegIter it{plan.seq_pages(), plan.seq_prefix(), p.batch, g_begin, g_end, b_begin};
-    int seq, p0, p1, t = 0, sg = 0;
-    bool ok = true;
-    while (ok && it.next(seq, p0, p1)) {
-      const int n = p1 - p0, t0 = t;
-      const int len = min(p.seq_lens[seq], p.max_pages * kPage);
-      // ---- this CTA's latent half of the query row -> TMEM (A operand of QK) ----
-      {
-        const uint4* src = reinterpret_cast<const uint4*>(
-            (lo_row ? p.q_lo : p.q_cat) +
-            (static_cast<size_t>(seq) * p.n_heads + (row_ok ? head : 0)) * kRow);
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const uint4 v = row_ok ? __ldg(src + (256 * rank + 64 * c) / 8 + k)
-                                   : make_uint4(0u, 0u, 0u, 0u);
-            r[4 * k] = v.x;
-            r[4 * k + 1] = v.y;
-            r[4 * k + 2] = v.z;
-            r[4 * k + 3] = v.w;
+      while (ok && (q_more || v_more)) {
+        bool progress = false;
+        // PV first: it frees the ring slots and the P buffers the rest of the pipe waits for
+        if (v_more && mbar_test(&bars->p_ready[v_t & 1], (v_t >> 1) & 1) &&
+            (v_i > 0 || v_sg == 0 || mbar_test(&bars->o_free, (v_sg - 1) & 1))) {
+          tc_fence_after();
+          issue_pv(v_t, v_i == 0);
+          ++v_i;
+          ++v_t;
+          if (v_i == v1 - v0) {
+            mma_commit(&bars->seg_done);
+            ++v_sg;
+            v_i = 0;
+            v_more = itv.next(vs, v0, v1);
           }
-          tmem_st32(tmem + kTmemQ + 32 * c + lane_off, r);
+          progress = true;
         }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&bars->q_ready);
-      }
-      float m_ref = NEG_INF, l_sum = 0.f;
-      for (int i = 0; i < n; ++i) {
-        const int tt = t0 + i, buf = tt & 1;
-        const bool first = i == 0;
-        // ---- own exact partial ----
-        if (!(ok = warp_wait(&bars->s_full[buf], (tt >> 1) & 1, wc))) break;
-        tc_fence_after();
-        float s[64];
-        {
-          uint32_t r[32];
-          tmem_ld32(tmem + kTmemS + buf * 64 + lane_off, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int k = 0; k < 32; ++k) s[k] = __uint_as_float(r[k]);
-          tmem_ld32(tmem + kTmemS + buf * 64 + 32 + lane_off, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int k = 0; k < 32; ++k) s[32 + k] = __uint_as_float(r[k]);
+        if (q_more) {
+          const int n = q1 - q0, npg = min(2, n - q_i);
+          if ((q_i > 0 ||
+               (mbar_test(&bars->q_ready, q_sg & 1) && mbar_test(&bars->q_full, q_sg & 1))) &&
+              (q_g == 0 || mbar_test(&bars->s_free, (q_g - 1) & 1)) &&
+              mbar_test(&bars->full[q_t % kSlots], (q_t / kSlots) & 1) &&
+              (npg == 1 ||
+               mbar_test(&bars->full[(q_t + 1) % kSlots], ((q_t + 1) / kSlots) & 1))) {
+            tc_fence_after();
+            issue_qk(q_t, npg);
+            q_i += npg;
+            q_t += npg;
+            ++q_g;
+            if (q_i == n) {
+              mma_commit(&bars->q_empty);
+              ++q_sg;
+              q_i = 0;
+              q_more = itq.next(qs, q0, q1);
+            }
+            progress = true;
+          }
         }
-        tc_fence_before();
-        mbar_arrive(&bars->s_free[buf]);
-        // ---- plus the peer's decoded partial ----
-        if (!(ok = warp_wait<true>(&bars->x_full, tt & 1, wc))) break;
-        {
-          const uint32_t base = recv_base;
-          float dq;
-          asm volatile("ld.shared.f32 %0, [%1];" : "=f"(dq) : "r"(base + kXPayload + row * 4));
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            uint32_t v[4];
-            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                         : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
-                         : "r"(base + xrow_off(row, c)));
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              s[8 * c + 2 * k] = fmaf(dec_lo(v[k]), dq, s[8 * c + 2 * k]);
-              s[8 * c + 2 * k + 1] = fmaf(dec_hi(v[k]), dq, s[8 * c + 2 * k + 1]);
+        if (progress) {
+          idle_since = 0;
+          spins = 0;
+        } else if ((++spins & 63) == 0) {
+          if (bars->abort_flag) {
+            ok = false;
+          } else {
+            const uint64_t now = globaltimer_ns();
+            if (idle_since == 0) {
+              idle_since = now;
+            } else if (now - idle_since > p.wait_ns) {
+              bars->abort_flag = 1;
+              atomicOr(p.status, MLA_STATUS_TIMEOUT);
+              ok = false;
             }
           }
-          // this warp's rows are decoded: warp 0 re-arms recv for the next page (its phase
-          // cannot complete before all four warps have handed their rows back), and every
-          // warp tells the peer its rows may be refilled
-          __syncwarp();
-          if (lane == 0) {
-            if (warp == 0) mbar_arrive_expect_tx(&bars->x_full, kXBytes);
-            mbar_arrive_remote_relaxed(peer_done_r[buf]);
-          }
         }
-        // ---- extended-precision query: a head's score is the sum of its q_cat and q_lo rows
-        // (lanes l and l ^ 16 of this warp); both rows continue with the same scores ----
-        if (hi_lo) {
+      }
+      if (!ok) {  // no MMA may be in flight when TMEM is released
+        mma_commit(&bars->drain);
+        mbar_wait(&bars->drain, 0, drain_ctx);
+      }
+    }
+  } else if (warp == 14) {
+    // =================== P copy: our rows of P and their factors into the peer ================
+    if (lane == 0) {
+      const uint32_t p_loc = smem_u32(smem + kOffP);
+      const uint32_t p_rem = mapa_shared(p_loc, peer);
+      const uint32_t a_loc = smem_u32(smem + kOffAlphaOwn);
+      const uint32_t a_rem = mapa_shared(smem_u32(smem + kOffAlphaIn), peer);
+      const uint32_t ppeer_rem[2] = {mapa_shared(smem_u32(&bars->p_peer[0]), peer),
+                                     mapa_shared(smem_u32(&bars->p_peer[1]), peer)};
+      int total = 0;
+      SegIter it{plan.seq_pages(), plan.seq_prefix(), p.batch, g_begin, g_end, b_begin};
+      int seq, p0, p1;
+      while (it.next(seq, p0, p1)) total += p1 - p0;
+      bool ok = true;
+      for (int t = 0; ok && t < total; ++t) {
+        const int pb = t & 1;
+        if (!(ok = mbar_wait(&bars->p_own[pb], (t >> 1) & 1, wc))) break;
+        // the peer's buffer pb is free once PV(t - 2) has run in both CTAs
+        if (t >= 2 && !(ok = mbar_wait<true>(&bars->pv_done[pb], ((t >> 1) - 1) & 1, wc))) break;
 #pragma unroll
-          for (int k = 0; k < 64; ++k) s[k] += __shfl_xor_sync(0xffffffffu, s[k], 16);
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t off = pb * kPBytes + (32 * q + 16 * rank) * 128;
+          bulk_copy_s2cluster(p_rem + off, p_loc + off, 16 * 128, ppeer_rem[pb]);
         }
-        // ---- online softmax ----
-        const int valid = min(kPage, len - (p0 + i) * kPage);
-        if (valid < kPage) {
-#pragma unroll
-          for (int k = 0; k < 64; ++k) s[k] = k < valid ? s[k] : NEG_INF;
-        }
-        float mx = max64(s);
-        mx *= p.scale_log2;  // log2 units (scale > 0 keeps the arg max)
-        float alpha = 1.f;
-        bool rescale = false;
-        if (first) {
-          m_ref = mx;
-        } else if (mx > m_ref + kRescaleThreshold) {
-          alpha = ex2_approx(m_ref - mx);
-          m_ref = mx;
-          rescale = true;
-        }
-        float rsum[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        uint32_t pk[32];
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          const float e0 = ex2_approx(fmaf(s[2 * k], p.scale_log2, -m_ref));
-          const float e1 = ex2_approx(fmaf(s[2 * k + 1], p.scale_log2, -m_ref));
-          rsum[k & 7] += e0 + e1;
-          pk[k] = pack_bf16x2(e0, e1);
-        }
-        const float rs = ((rsum[0] + rsum[1]) + (rsum[2] + rsum[3])) +
-                         ((rsum[4] + rsum[5]) + (rsum[6] + rsum[7]));
-        l_sum = l_sum * alpha + rs;
-        if (!first && __any_sync(0xffffffffu, rescale)) {
-          // O must hold PV of the previous page before it is rescaled
-          if (!(ok = warp_wait(&bars->pv_done, (tt - 1) & 1, wc))) break;
+        bulk_copy_s2cluster(a_rem + pb * 256, a_loc + pb * 256, 256, ppeer_rem[pb]);
+        bulk_commit_group();
+        bulk_wait_read_all();
+        mbar_arrive(&bars->p_free[pb]);
+      }
+      if (!ok) bulk_wait_read_all();
+    }
+  } else if (warp >= 8) {
+    // =================== send warps: partials out; P completion and O rescale ================
+    // Sending: 16x32bx2 view, thread (j, h) = (lane & 15, lane >> 4) reads row 32q + 16 peer + j,
+    // columns 32h .. 32h + 31 of each page, and writes row 16q + j of the peer's receive buffer.
+    // Finishing a page: once both CTAs' rows of P are in place, rescale O (32x32b view, thread =
+    // lane 32q + lane) if a row's running maximum moved, then let PV run.
+    const int q = warp & 3, j = lane & 15, hcol = lane >> 4;
+    const uint32_t lanes_peer = static_cast<uint32_t>(32 * q + 16 * peer) << 16;
+    const uint32_t lanes_all = static_cast<uint32_t>(32 * q) << 16;
+    const int rho = 16 * q + j;
+    const uint32_t x_peer = mapa_shared(smem_u32(smem + kOffX), peer);
+    const uint32_t xfull_peer[2] = {mapa_shared(smem_u32(&bars->x_full[0]), peer),
+                                    mapa_shared(smem_u32(&bars->x_full[1]), peer)};
+    const float* alpha_in = reinterpret_cast<const float*>(smem + kOffAlphaIn);
+    const float* alpha_own = reinterpret_cast<const float*>(smem + kOffAlphaOwn);
+    // send side
+    SegIter its{plan.seq_pages(), plan.seq_prefix(), p.batch, g_begin, g_end, b_begin};
+    int s_seq, s0, s1;
+    bool s_more = its.next(s_seq, s0, s1);
+    int s_i = 0, s_t = 0, s_g = 0, s_state = 0, s_k = 0, s_npg = 0;
+    int s_len = s_more ? min(p.seq_lens[s_seq], p.max_pages * kPage) : 0;
+    uint32_t e[2][16];  // the quantised partials of the current page group
+    float scale[2];
+    // finish side
+    SegIter itf{plan.seq_pages(), plan.seq_prefix(), p.batch, g_begin, g_end, b_begin};
+    int f_seq, f0, f1;
+    bool f_more = itf.next(f_seq, f0, f1);
+    int f_i = 0, f_t = 0;
+    uint64_t idle_since = 0;
+    uint32_t spins = 0;
+    bool ok = true;
+    while (ok && (s_more || f_more)) {
+      bool progress = false;
+      if (f_more && warp_test(&bars->p_own[f_t & 1], (f_t >> 1) & 1) &&
+          warp_test(&bars->p_peer[f_t & 1], (f_t >> 1) & 1)) {
+        const int pb = f_t & 1;
+        if (warp == 8 && lane == 0) mbar_arrive_expect_tx(&bars->p_peer[pb], kPMsgBytes);
+        // O rescale (rare): rows of the quarter whose running maximum moved, ours or the peer's
+        const float a_own = alpha_own[pb * 64 + rho];
+        const float a_peer = alpha_in[pb * 64 + rho];
+        if (f_i > 0 && __any_sync(kFull, a_own != 1.f || a_peer != 1.f)) {
+          if (!(ok = warp_wait(&bars->p_free[pb ^ 1], ((f_t - 1) >> 1) & 1, wc))) break;
           tc_fence_after();
+          const float fa = __shfl_sync(kFull, a_own, j);
+          const float fb = __shfl_sync(kFull, a_peer, j);
+          const float f = (lane >> 4) == static_cast<int>(rank) ? fa : fb;
 #pragma unroll 1
           for (int c = 0; c < 256; c += 32) {
             uint32_t r[32];
-            tmem_ld32(tmem + kTmemO + c + lane_off, r);
+            tmem_ld32(tmem + kTmemO + c + lanes_all, r);
             tmem_wait_ld();
 #pragma unroll
-            for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * alpha);
-            tmem_st32(tmem + kTmemO + c + lane_off, r);
+            for (int u = 0; u < 32; ++u) r[u] = __float_as_uint(__uint_as_float(r[u]) * f);
+            tmem_st32(tmem + kTmemO + c + lanes_all, r);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->p_ready[pb]);
+        ++f_t;
+        if (++f_i == f1 - f0) {
+          f_i = 0;
+          f_more = itf.next(f_seq, f0, f1);
+        }
+        progress = true;
+      }
+      // send side: state 0 waits for a page group's S, drains the peer's rows and quantises
+      // them; state 1 sends each page once the peer has freed that receive buffer
+      if (s_more && s_state == 0 && warp_test(&bars->s_full, s_g & 1)) {
+        s_npg = min(2, (s1 - s0) - s_i);
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          if (k == 1 && s_npg == 1) break;
+          uint32_t a[32];
+          tmem_ld16x2_32(tmem + kTmemS + 64 * k + lanes_peer, a);
+          tmem_wait_ld();
+          float sv[32];
+#pragma unroll
+          for (int u = 0; u < 32; ++u) sv[u] = __uint_as_float(a[u]);
+          // columns past the sequence's end are never used: they travel as zeros
+          const int valid = min(kPage, s_len - (s0 + s_i + k) * kPage) - 32 * hcol;
+          if (valid < 32) {
+#pragma unroll
+            for (int u = 0; u < 32; ++u) sv[u] = u < valid ? sv[u] : 0.f;
+          }
+          float mabs = maxabs32(sv);
+          mabs = fmaxf(mabs, __shfl_xor_sync(kFull, mabs, 16));
+          const float inv = mabs > 0.f ? 32767.f / mabs : 0.f;
+#pragma unroll
+          for (int u = 0; u < 16; ++u) e[k][u] = enc_u16x2(sv[2 * u], sv[2 * u + 1], inv);
+          scale[k] = mabs * (1.f / 32767.f);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->s_free);
+        s_state = 1;
+        s_k = 0;
+        progress = true;
+      }
+      while (s_more && s_state == 1) {
+        const int tt = s_t + s_k, pb = tt & 1;
+        if (tt >= 2 && !warp_test(&bars->x_free[pb], ((tt >> 1) - 1) & 1)) break;
+        const uint32_t xb = x_peer + pb * kXBytes;
+        auto send = [&](const uint32_t (&ek)[16], float sc) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            st_async_u4(xb + xrow_off(rho, 4 * hcol + c), ek[4 * c], ek[4 * c + 1],
+                        ek[4 * c + 2], ek[4 * c + 3], xfull_peer[pb]);
+          if (hcol == 0) st_async_u1(xb + kXPayload + rho * 4, __float_as_uint(sc), xfull_peer[pb]);
+        };
+        if (s_k == 0)
+          send(e[0], scale[0]);
+        else
+          send(e[1], scale[1]);
+        progress = true;
+        if (++s_k == s_npg) {
+          s_t += s_npg;
+          s_i += s_npg;
+          ++s_g;
+          s_state = 0;
+          if (s_i == s1 - s0) {
+            s_i = 0;
+            s_more = its.next(s_seq, s0, s1);
+            if (s_more) s_len = min(p.seq_lens[s_seq], p.max_pages * kPage);
           }
         }
-        // ---- P -> shared memory (canonical K-major, 128B swizzle) once PV of page tt - 1
-        // has read it ----
-        if (tt >= 1 && !(ok = warp_wait(&bars->pv_done, (tt - 1) & 1, wc))) break;
-        {
-          const uint32_t pa = smem_u32(smem + kOffP);
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pa + xrow_off(row, c)),
-                         "r"(pk[4 * c]), "r"(pk[4 * c + 1]), "r"(pk[4 * c + 2]),
-                         "r"(pk[4 * c + 3])
-                         : "memory");
+      }
+      if (progress) {
+        idle_since = 0;
+        spins = 0;
+      } else if ((++spins & 63) == 0) {
+        if (bars->abort_flag) {
+          ok = false;
+        } else {
+          const uint64_t now = globaltimer_ns();
+          if (idle_since == 0) {
+            idle_since = now;
+          } else if (now - idle_since > p.wait_ns) {
+            bars->abort_flag = 1;
+            atomicOr(p.status, MLA_STATUS_TIMEOUT);
+            ok = false;
+          }
         }
-        fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
-        mbar_arrive(&bars->p_full);
+      }
+    }
+    if (ok) {  // the peer's hand-backs for our last two pages land before this CTA exits
+      for (int u = max(0, s_t - 2); u < s_t; ++u)
+        mbar_wait<true>(&bars->x_free[u & 1], (u >> 1) & 1, drain_ctx);
+    }
+  } else {
+    // =================== softmax warps (own rows), query load, epilogue ====================
+    // 16x32bx2 view: warp w owns row 32q + 16 rank + j (q = w & 3) and the 32 columns
+    // 32k .. 32k + 31 of each page (k = w >> 2); thread (j, h) takes 16 of them, 32k + 16h on.
+    // The row maximum is shared by the two warps of a quarter through shared memory; each keeps
+    // its own partial row sum.  Warps 0-3 load the query; all 8 write O out (32x32b view).
+    const int q = warp & 3, kh = warp >> 2, j = lane & 15, hcol = lane >> 4;
+    const int rho = 16 * q + j;
+    const int c0 = 32 * kh + 16 * hcol;  // this thread's first column within a page
+    const int row_own = 32 * q + 16 * static_cast<int>(rank) + j;
+    const int row_lane = 32 * q + lane;
+    const uint32_t lanes_own = static_cast<uint32_t>(32 * q + 16 * rank) << 16;
+    const uint32_t lanes_all = static_cast<uint32_t>(32 * q) << 16;
+    const float NEG_INF = -__int_as_float(0x7f800000);
+    const uint32_t x_loc = smem_u32(smem + kOffX);
+    const uint32_t p_loc = smem_u32(smem + kOffP);
+    const uint32_t stats_rem = mapa_shared(smem_u32(smem + kOffStats), peer);
+    const uint32_t xfree_rem[2] = {mapa_shared(smem_u32(&bars->x_free[0]), peer),
+                                   mapa_shared(smem_u32(&bars->x_free[1]), peer)};
+    const uint32_t stfull_rem = mapa_shared(smem_u32(&bars->st_full), peer);
+    float* alpha_own = reinterpret_cast<float*>(smem + kOffAlphaOwn);
+    float* max_x = reinterpret_cast<float*>(smem + kOffMaxX);  // [page parity][half][row]
+    float* l_part = reinterpret_cast<float*>(smem + kOffLPart);  // [seg parity][half][row]
+    const float2* stats_in = reinterpret_cast<const float2*>(smem + kOffStats);
+    // this CTA's latent half of the query rows of sequence sq -> TMEM (A operand of QK)
+    auto load_q = [&](int sq) {
+      const int hd = rows.head(row_lane);
+      const bool in = hd < p.n_heads;
+      const uint4* src = reinterpret_cast<const uint4*>(
+          (rows.lo(row_lane) ? p.q_lo : p.q_cat) +
+          (static_cast<size_t>(sq) * p.n_heads + (in ? hd : 0)) * kRow);
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint4 v = in ? __ldg(src + (256 * rank + 64 * c) / 8 + k) : make_uint4(0u, 0u, 0u, 0u);
+          r[4 * k] = v.x;
+          r[4 * k + 1] = v.y;
+          r[4 * k + 2] = v.z;
+          r[4 * k + 3] = v.w;
+        }
+        tmem_st32(tmem + kTmemQ + 32 * c + lanes_all, r);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->q_ready);
+    };
+    SegIter it{plan.seq_pages(), plan.seq_prefix(), p.batch, g_begin, g_end, b_begin};
+    int seq, p0, p1, t = 0, g = 0, sg = 0;
+    bool ok = true;
+    bool have = it.next(seq, p0, p1);
+    if (have && kh == 0) load_q(seq);
+    while (ok && have) {
+      const int n = p1 - p0;
+      const int len = min(p.seq_lens[seq], p.max_pages * kPage);
+      float m_ref = NEG_INF, l_sum = 0.f;
+      for (int i = 0; ok && i < n; i += 2, ++g) {
+        const int npg = min(2, n - i);
+        if (!(ok = warp_wait(&bars->s_full, g & 1, wc))) break;
+        tc_fence_after();
+        uint32_t a[16], b[16];
+        tmem_ld16x2_16(tmem + kTmemS + 32 * kh + lanes_own, a);
+        if (npg == 2) tmem_ld16x2_16(tmem + kTmemS + 64 + 32 * kh + lanes_own, b);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->s_free);
+        for (int k = 0; ok && k < npg; ++k) {
+          const int tt = t + i + k, pb = tt & 1;
+          const bool first = i + k == 0;
+          float s[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) s[u] = __uint_as_float(k ? b[u] : a[u]);
+          // ---- plus the peer's partial (16-bit, relative to its row's largest magnitude) ----
+          if (!(ok = warp_wait<true>(&bars->x_full[pb], (tt >> 1) & 1, wc))) break;
+          {
+            const uint32_t xb = x_loc + pb * kXBytes;
+            float dq;
+            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(dq) : "r"(xb + kXPayload + rho * 4));
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              uint32_t v[4];
+              asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                           : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
+                           : "r"(xb + xrow_off(rho, c0 / 8 + c)));
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                s[8 * c + 2 * kk] = fmaf(dec_lo(v[kk]), dq, s[8 * c + 2 * kk]);
+                s[8 * c + 2 * kk + 1] = fmaf(dec_hi(v[kk]), dq, s[8 * c + 2 * kk + 1]);
+              }
+            }
+            // decoded: warp 0 re-arms the buffer for page tt + 2, every warp hands it back
+            __syncwarp();
+            if (lane == 0) {
+              if (warp == 0) mbar_arrive_expect_tx(&bars->x_full[pb], kXBytes);
+              mbar_arrive_remote_relaxed(xfree_rem[pb]);
+            }
+          }
+          // ---- a head's score with the query remainder: the sum of its two rows ----
+          if (rows.hi_lo) {
+#pragma unroll
+            for (int u = 0; u < 16; ++u) s[u] += __shfl_xor_sync(kFull, s[u], 8);
+          }
+          // ---- online softmax: the row maximum over both warps of the quarter ----
+          const int valid = min(kPage, len - (p0 + i + k) * kPage) - c0;
+          if (valid < 16) {
+#pragma unroll
+            for (int u = 0; u < 16; ++u) s[u] = u < valid ? s[u] : NEG_INF;
+          }
+          float mx = max16(s);
+          mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
+          if (hcol == 0) max_x[(pb * 2 + kh) * 64 + rho] = mx;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->mx_bar[q][pb]);
+          if (!(ok = warp_wait(&bars->mx_bar[q][pb], (tt >> 1) & 1, wc))) break;
+          mx = fmaxf(mx, max_x[(pb * 2 + (kh ^ 1)) * 64 + rho]);
+          mx *= p.scale_log2;  // log2 units (scale > 0 keeps the arg max)
+          float alpha = 1.f;
+          if (first) {
+            m_ref = mx;
+          } else if (mx > m_ref + kRescaleThreshold) {
+            alpha = ex2_approx(m_ref - mx);
+            m_ref = mx;
+          }
+          float rs[4] = {0.f, 0.f, 0.f, 0.f};
+          uint32_t pk[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const float e0 = ex2_approx(fmaf(s[2 * u], p.scale_log2, -m_ref));
+            const float e1 = ex2_approx(fmaf(s[2 * u + 1], p.scale_log2, -m_ref));
+            rs[u & 3] += e0 + e1;
+            pk[u] = pack_bf16x2(e0, e1);
+          }
+          float tot = (rs[0] + rs[1]) + (rs[2] + rs[3]);
+          tot += __shfl_xor_sync(kFull, tot, 16);
+          l_sum = l_sum * alpha + tot;  // this warp's 32 columns of the row
+          // ---- our rows of P, once PV(tt - 2) has read buffer pb and its copy is out ----
+          if (tt >= 2 && !(ok = warp_wait(&bars->p_free[pb], ((tt >> 1) - 1) & 1, wc))) break;
+#pragma unroll
+          for (int c = 0; c < 2; ++c)
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                             p_loc + pb * kPBytes + xrow_off(row_own, c0 / 8 + c)),
+                         "r"(pk[4 * c]), "r"(pk[4 * c + 1]), "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
+                         : "memory");
+          if (kh == 0 && hcol == 0) alpha_own[pb * 64 + rho] = alpha;
+          fence_proxy_async_smem();  // -> visible to the tensor core and the bulk copy
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->p_own[pb]);
+        }
       }
       if (!ok) break;
-      // ---- segment epilogue: O / l -> global ----
-      if (!(ok = warp_wait(&bars->seg_done, sg & 1, wc))) break;
-      tc_fence_after();
-      const int nparts = plan.seq_nparts()[seq];
-      const float lse_nat = (m_ref + __log2f(l_sum)) * 0.69314718055994531f;
-      const float inv_l = 1.f / l_sum;
-      float* dst;
-      float* dst_lse;
-      if (nparts == 1) {
-        dst = p.o_lat + (static_cast<size_t>(seq) * p.n_heads + head) * 512 + 256 * rank;
-        dst_lse = p.lse ? p.lse + static_cast<size_t>(seq) * p.n_heads + head : nullptr;
-      } else {
-        const int slot = plan.seq_slot()[seq] + (part - plan.seq_first_part()[seq]);
-        dst = p.part_o + (static_cast<size_t>(slot) * p.n_heads + head) * 512 + 256 * rank;
-        dst_lse = p.part_lse + static_cast<size_t>(slot) * p.n_heads + head;
-      }
-#pragma unroll 1
-      for (int c = 0; c < 256; c += 32) {
-        uint32_t r[32];
-        tmem_ld32(tmem + kTmemO + c + lane_off, r);
-        tmem_wait_ld();
-        if (row_out) {
-          float4* d4 = reinterpret_cast<float4*>(dst + c);
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            d4[k] = make_float4(__uint_as_float(r[4 * k]) * inv_l,
-                                __uint_as_float(r[4 * k + 1]) * inv_l,
-                                __uint_as_float(r[4 * k + 2]) * inv_l,
-                                __uint_as_float(r[4 * k + 3]) * inv_l);
-        }
-      }
-      if (row_out && rank == 0 && dst_lse) *dst_lse = lse_nat;
-      tc_fence_before();
-      mbar_arrive(&bars->o_free);
       t += n;
+      // ---- row sums of both column halves; own rows' (max, sum) to the peer ----
+      float* lp = l_part + (sg & 1) * 128;
+      if (hcol == 0) lp[kh * 64 + rho] = l_sum;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->ls_bar[sg & 1]);
+      if (!(ok = warp_wait(&bars->ls_bar[sg & 1], (sg >> 1) & 1, wc))) break;
+      const float l_row_own = lp[rho] + lp[64 + rho];
+      if (kh == 0 && hcol == 0)
+        st_async_u2(stats_rem + rho * 8, __float_as_uint(m_ref), __float_as_uint(l_row_own),
+                    stfull_rem);
+      // ---- the next segment's query half, as soon as the last QK of this one has run ----
+      int nseq = 0, np0 = 0, np1 = 0;
+      const bool next = it.next(nseq, np0, np1);
+      if (next && kh == 0) {
+        if (!(ok = warp_wait(&bars->q_empty, sg & 1, wc))) break;
+        load_q(nseq);
+      }
+      // ---- segment epilogue: O / l -> global (32x32b view; warp w writes columns 128k ..) ----
+      if (!(ok = warp_wait(&bars->seg_done, sg & 1, wc))) break;
+      if (!(ok = warp_wait<true>(&bars->st_full, sg & 1, wc))) break;
+      tc_fence_after();
+      {
+        const float2 ps = stats_in[rho];
+        const float m_o = __shfl_sync(kFull, m_ref, j);
+        const float l_o = __shfl_sync(kFull, l_row_own, j);
+        const bool own = (lane >> 4) == static_cast<int>(rank);
+        const float m_row = own ? m_o : ps.x;
+        const float l_row = own ? l_o : ps.y;
+        const int hd = rows.head(row_lane);
+        const bool out_row = hd < p.n_heads && !rows.lo(row_lane);
+        const int nparts = plan.seq_nparts()[seq];
+        float* dst;
+        float* dst_lse;
+        if (nparts == 1) {
+          dst = p.o_lat + (static_cast<size_t>(seq) * p.n_heads + hd) * 512 + 256 * rank;
+          dst_lse = p.lse ? p.lse + static_cast<size_t>(seq) * p.n_heads + hd : nullptr;
+        } else {
+          const int slot = plan.seq_slot()[seq] + (part - plan.seq_first_part()[seq]);
+          dst = p.part_o + (static_cast<size_t>(slot) * p.n_heads + hd) * 512 + 256 * rank;
+          dst_lse = p.part_lse + static_cast<size_t>(slot) * p.n_heads + hd;
+        }
+        const float inv_l = 1.f / l_row;
+#pragma unroll 1
+        for (int c = 128 * kh; c < 128 * kh + 128; c += 32) {
+          uint32_t r[32];
+          tmem_ld32(tmem + kTmemO + c + lanes_all, r);
+          tmem_wait_ld();
+          if (out_row) {
+            float4* d4 = reinterpret_cast<float4*>(dst + c);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              d4[k] = make_float4(__uint_as_float(r[4 * k]) * inv_l,
+                                  __uint_as_float(r[4 * k + 1]) * inv_l,
+                                  __uint_as_float(r[4 * k + 2]) * inv_l,
+                                  __uint_as_float(r[4 * k + 3]) * inv_l);
+          }
+        }
+        if (kh == 0 && out_row && own && dst_lse)
+          *dst_lse = (m_row + __log2f(l_row)) * 0.69314718055994531f;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&bars->o_free);
+        if (warp == 0) mbar_arrive_expect_tx(&bars->st_full, 512);  // for the next segment
+      }
       ++sg;
+      seq = nseq;
+      p0 = np0;
+      p1 = np1;
+      have = next;
     }
-    // The peer's remote arrivals for our last two partials must land before this CTA exits.
-    {
-      volatile int never = 0;
-      WaitCtx drain{&never, p.status, p.wait_ns};
+    if (ok && warp == 0) {  // the peer's PV commits for our last two pages land before exit
       for (int u = max(0, t - 2); u < t; ++u)
-        mbar_wait<true>(&bars->peer_done[u & 1], (u >> 1) & 1, ok ? wc : drain);
+        mbar_wait<true>(&bars->pv_done[u & 1], (u >> 1) & 1, drain_ctx);
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  cluster_sync();
+  uint32_t peer_abort;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];"
+               : "=r"(peer_abort)
+               : "r"(mapa_shared(smem_u32(&bars->abort_flag), peer)));
+  const bool aborted = bars->abort_flag != 0 || peer_abort != 0;
+  // After an abort, remote stores and arrivals of the peer that nothing waited for may still be
+  // in flight towards this CTA's shared memory: give them time to land before it is released.
+  if (aborted) spin_ns(200000);
+  if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }

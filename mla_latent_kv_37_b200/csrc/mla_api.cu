@@ -74,57 +74,69 @@ int g_prof_count = 0;
 int g_prof_next = 0;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
+// Description of the last CUDA call of this thread that failed inside the library.
+thread_local char g_err_detail[256] = "";
+
+int cuda_fail(cudaError_t e, const char* where) {
+  std::snprintf(g_err_detail, sizeof(g_err_detail), "%s: %s (%s)", where, cudaGetErrorName(e),
+                cudaGetErrorString(e));
+  return MLA_ERR_CUDA;
+}
+
 int device_ctx(DevCtx** out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MLA_ERR_CUDA;
+  cudaError_t e;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return MLA_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_mu);
   DevCtx& c = g_dev[dev];
   if (!c.init) {
-    if (cudaDeviceGetAttribute(&c.cc_major, cudaDevAttrComputeCapabilityMajor, dev) !=
+    if ((e = cudaDeviceGetAttribute(&c.cc_major, cudaDevAttrComputeCapabilityMajor, dev)) !=
         cudaSuccess)
-      return MLA_ERR_CUDA;
+      return cuda_fail(e, "cudaDeviceGetAttribute");
     if (c.cc_major != 10) return MLA_ERR_DEVICE;
-    if (cudaDeviceGetAttribute(&c.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      return MLA_ERR_CUDA;
+    if ((e = cudaDeviceGetAttribute(&c.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute");
     void* sym = nullptr;
-    if (cudaGetSymbolAddress(&sym, g_status_word) != cudaSuccess) return MLA_ERR_CUDA;
+    if ((e = cudaGetSymbolAddress(&sym, g_status_word)) != cudaSuccess)
+      return cuda_fail(e, "cudaGetSymbolAddress(status word)");
     c.status = static_cast<unsigned int*>(sym);
     if (!g_encode) {
       cudaDriverEntryPointQueryResult q;
       void* fn = nullptr;
-      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
-              cudaSuccess ||
-          q != cudaDriverEntryPointSuccess || !fn)
-        return MLA_ERR_CUDA;
+      if ((e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q)) !=
+          cudaSuccess)
+        return cuda_fail(e, "cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)");
+      if (q != cudaDriverEntryPointSuccess || !fn) return MLA_ERR_CUDA;
       g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     }
     // kernel attributes (once per device)
     const int attn_smem = static_cast<int>(attn::kSmemBytes);
-    if (cudaFuncSetAttribute(attn::split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             attn_smem) != cudaSuccess)
-      return MLA_ERR_CUDA;
+    if ((e = cudaFuncSetAttribute(attn::split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  attn_smem)) != cudaSuccess)
+      return cuda_fail(e, "cudaFuncSetAttribute(split_kernel)");
     const int sk_smem = static_cast<int>(kSmemPerBlockMax);
-    if (cudaFuncSetAttribute(sk::streamk_gemm_kernel<sk::EpiAppend>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, sk_smem) != cudaSuccess ||
-        cudaFuncSetAttribute(sk::streamk_gemm_kernel<sk::EpiWq>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, sk_smem) != cudaSuccess ||
-        cudaFuncSetAttribute(sk::streamk_gemm_kernel<sk::EpiWuk>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, sk_smem) != cudaSuccess ||
-        cudaFuncSetAttribute(sk::streamk_gemm_kernel<sk::EpiWuv>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, sk_smem) != cudaSuccess ||
-        cudaFuncSetAttribute(sk::streamk_gemm_kernel<sk::EpiWo>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, sk_smem) != cudaSuccess ||
-        cudaFuncSetAttribute(sk::streamk_gemm_kernel<sk::EpiAppendWq>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, sk_smem) != cudaSuccess)
-      return MLA_ERR_CUDA;
+    const void* sk_kernels[6] = {
+        reinterpret_cast<const void*>(sk::streamk_gemm_kernel<sk::EpiAppend>),
+        reinterpret_cast<const void*>(sk::streamk_gemm_kernel<sk::EpiWq>),
+        reinterpret_cast<const void*>(sk::streamk_gemm_kernel<sk::EpiWuk>),
+        reinterpret_cast<const void*>(sk::streamk_gemm_kernel<sk::EpiWuv>),
+        reinterpret_cast<const void*>(sk::streamk_gemm_kernel<sk::EpiWo>),
+        reinterpret_cast<const void*>(sk::streamk_gemm_kernel<sk::EpiAppendWq>)};
+    for (const void* k : sk_kernels)
+      if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, sk_smem)) !=
+          cudaSuccess)
+        return cuda_fail(e, "cudaFuncSetAttribute(streamk_gemm_kernel)");
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2, 1, 1);
     cfg.blockDim = dim3(attn::kThreads, 1, 1);
     cfg.dynamicSmemBytes = attn::kSmemBytes;
     int nclusters = 0;
     if (cudaOccupancyMaxActiveClusters(&nclusters, attn::split_kernel, &cfg) != cudaSuccess ||
-        nclusters <= 0)
+        nclusters <= 0) {
+      (void)cudaGetLastError();  // a failed query only means: fall back to one per SM pair
       nclusters = c.sms / 2;
+    }
     c.max_clusters = nclusters;
     c.init = true;
   }
@@ -337,7 +349,8 @@ int map_acts(CUtensorMap* m, const void* base, uint64_t groups, uint64_t n_rows,
 // ------------------------------------------------------------------------------------------
 int last_launch(int kernels = 1) {
   g_launches.fetch_add(static_cast<unsigned long long>(kernels), std::memory_order_relaxed);
-  return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MLA_OK : cuda_fail(e, "kernel launch");
 }
 
 // The kernels of the bf16 decode path are launched with programmatic stream serialisation:
@@ -478,8 +491,8 @@ int enqueue_decode(const DevCtx* c, const mla_dims* dims, const void* q_cat, con
   if (dims->dtype == MLA_BF16) {
     CUtensorMap tc_lat, tc_rope, tq_rope, tql_rope;
     const uint64_t rows = static_cast<uint64_t>(num_pages) * kPageN;
-    // query RoPE halves: one 128-head box, or 16-head boxes from q_cat and q_lo
-    const uint32_t qbox = q_lo ? 16 : 128;
+    // query RoPE halves: one 128-head box, or 8-head boxes from q_cat and q_lo
+    const uint32_t qbox = q_lo ? 8 : 128;
     if ((rc = map3(&tq_rope, q_cat, kRowN, H, B, kRowN * 2ull, kRowN * 2ull * H, 32, qbox, 1,
                    CU_TENSOR_MAP_SWIZZLE_64B)))
       return rc;
@@ -869,6 +882,8 @@ const char* mla_error_string(int code) {
   }
   return "unknown code";
 }
+
+const char* mla_error_detail(void) { return g_err_detail; }
 
 const char* mla_version(void) { return "mla_latent_kv_37_b200 0.1 (sm_100a)"; }
 

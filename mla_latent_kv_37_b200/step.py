@@ -30,7 +30,10 @@ class Layer:
 
 class DecodeStep:
     def __init__(self, layers: list[Layer], batch: int, n_heads: int, d_model: int,
-                 dtype=torch.bfloat16, num_splits: int = 0, device="cuda", graph: bool = False):
+                 dtype=torch.bfloat16, num_splits: int = 0, device="cuda", graph: bool = False,
+                 query_remainder: bool = False):
+        """`query_remainder` carries the absorbed query's bf16 rounding remainder (q_lo) from
+        the projection into the attention, for inputs with large logits."""
         self.layers = layers
         self.B, self.H, self.D, self.dtype = batch, n_heads, d_model, dtype
         self.dims = make_dims(batch, n_heads, d_model, dtype)
@@ -38,6 +41,8 @@ class DecodeStep:
         L = len(layers)
         self.ws = workspace(self.dims, num_splits, device)
         self.q_cat = torch.empty(batch, n_heads, 576, dtype=dtype, device=device)
+        self.q_lo = (torch.empty(batch, n_heads, 576, dtype=torch.bfloat16, device=device)
+                     if query_remainder else None)
         self.o_lat = torch.empty(batch, n_heads, 512, dtype=torch.float32, device=device)
         self.lse = torch.empty(batch, n_heads, dtype=torch.float32, device=device)
         self.o_heads = torch.empty(L, batch, n_heads, 128, dtype=dtype, device=device)
@@ -86,9 +91,9 @@ class DecodeStep:
     def _layer(self, l, h_l, positions, seq_lens, stream=None):
         d, ly = self.dims, self.layers[l]
         mla_append_absorb(d, h_l, ly.w_dkv, ly.w_kr, ly.w_q, ly.w_uk, positions, ly.page_table,
-                          ly.pool, self.q_cat, self.ws, stream=stream)
+                          ly.pool, self.q_cat, self.ws, q_lo=self.q_lo, stream=stream)
         mla_decode_attn(d, self.q_cat, ly.pool, ly.page_table, seq_lens, self.o_lat, self.ws,
-                        lse=self.lse, num_splits=self.num_splits, stream=stream)
+                        lse=self.lse, q_lo=self.q_lo, num_splits=self.num_splits, stream=stream)
         mla_out_proj(d, self.o_lat, ly.w_uv, self.ws, w_o=ly.w_o, o_heads=self.o_heads[l],
                      out=self.out[l] if ly.w_o is not None else None, stream=stream)
 
