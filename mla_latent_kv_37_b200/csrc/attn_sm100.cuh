@@ -65,16 +65,15 @@
 namespace mla {
 namespace attn {
 
-constexpr int kThreads = 480;  // 15 warps: 8 softmax, 4 send + finish, TMA, MMA, P copy
+constexpr int kThreads = 448;  // 14 warps: 8 softmax, 4 send, TMA producer, MMA issuer
 constexpr int kPage = 64;
 constexpr int kRow = 576;
 constexpr int kSlots = 4;  // page slots of the ring
 constexpr uint32_t kBoxBytes = 64 * 128;      // one page's 64 rows x 64 latent columns (bf16)
 constexpr uint32_t kRopeBoxBytes = 64 * 64;   // one page's 64 rows x 32 RoPE columns (bf16)
 constexpr uint32_t kSlotBytes = 4 * kBoxBytes + kRopeBoxBytes;  // this CTA's half of a page
-// The ring is box-major: latent box i of slot s at i * kSlots * kBoxBytes + s * kBoxBytes, so
-// the rows of slots s and s + 1 are contiguous in every box (one N = 128 operand for a page
-// pair); the RoPE boxes of the slots follow, contiguous in slot order.
+// The ring is box-major: latent box i of slot s at i * kSlots * kBoxBytes + s * kBoxBytes; the
+// RoPE boxes of the slots follow.
 constexpr uint32_t kOffRing = 0;
 constexpr uint32_t kBoxStride = kSlots * kBoxBytes;
 constexpr uint32_t kOffRope = kOffRing + 4 * kBoxStride;
@@ -82,28 +81,21 @@ constexpr uint32_t kPBytes = 128 * 128;  // P of one page: 128 rows x 64 bf16
 constexpr uint32_t kOffP = kOffRope + kSlots * kRopeBoxBytes;  // two P buffers (page parity)
 constexpr uint32_t kQRopeBytes = 128 * 64;                    // 128 rows x 32 bf16
 constexpr uint32_t kOffQRope = kOffP + 2 * kPBytes;
-constexpr uint32_t kXPayload = 64 * 128;          // 64 rows x 64 partial scores x 16 bits
-constexpr uint32_t kXBytes = kXPayload + 64 * 4;  // + one fp32 step per row
+constexpr uint32_t kXPayload = 128 * 128;         // 128 rows x 64 partial scores x 16 bits
+constexpr uint32_t kXBytes = kXPayload + 128 * 4;  // + one fp32 step per row
 constexpr uint32_t kOffX = kOffQRope + kQRopeBytes;  // two receive buffers (page parity)
-constexpr uint32_t kOffAlphaIn = kOffX + 2 * kXBytes;     // the peer's rescale factors [2][64]
-constexpr uint32_t kOffAlphaOwn = kOffAlphaIn + 2 * 256;  // our rows' factors [2][64]
-constexpr uint32_t kOffStats = kOffAlphaOwn + 2 * 256;    // the peer's (max, sum) per row [64]
-constexpr uint32_t kOffMaxX = kOffStats + 512;            // row maxima of the column halves [2][2][64]
-constexpr uint32_t kOffLPart = kOffMaxX + 1024;  // row sums of the column halves [2][2][64]
-constexpr uint32_t kOffBar = kOffLPart + 1024;
+constexpr uint32_t kOffBar = kOffX + 2 * kXBytes;
 constexpr uint32_t kSmemBytes = kOffBar + 512 + 1024;  // barriers + alignment slack
-constexpr uint32_t kPMsgBytes = 64 * 128 + 64 * 4;     // P rows sent to the peer + factors
-// TMEM columns
+// TMEM columns: O half | query latent half | S of two pages (page parity)
 constexpr uint32_t kTmemO = 0, kTmemQ = 256, kTmemS = 384, kTmemCols = 512;
 constexpr int kAhead = 4;  // pages prefetched into L2 ahead of the TMA ring
 constexpr uint32_t kPageBytes = kPage * kRow * 2;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 static_assert(kSmemBytes <= 232448, "shared memory budget");
-static_assert(kTmemS + 128 == kTmemCols, "tensor memory budget");
+static_assert(kTmemS + 2 * 64 == kTmemCols, "tensor memory budget");
 static_assert(kXBytes % 16 == 0 && kOffP % 1024 == 0 && kOffQRope % 1024 == 0 &&
-                  kOffRope % 1024 == 0 && kOffX % 16 == 0 && kOffAlphaIn % 16 == 0 &&
-                  kOffAlphaOwn % 16 == 0 && kOffBar % 8 == 0,
+                  kOffRope % 1024 == 0 && kOffX % 16 == 0 && kOffBar % 8 == 0,
               "alignment");
 
 struct Params {
@@ -318,7 +310,7 @@ __device__ __forceinline__ float dec_hi(uint32_t v) {
 // TMEM lanes (MMA rows) and heads.  Without the query remainder, lane L computes head L.  With
 // it, in quarter q of the lanes (one warp's 32) lanes 16h + 8k + j (h, k in {0, 1}, j < 8)
 // compute head 64 group + 16q + 8h + j, from q_cat for k = 0 and from q_lo for k = 1, so that
-// the two rows of a head sit in the same 16-lane half of the quarter.
+// the two rows of a head sit in the same 16-lane half of the quarter (one softmax warp).
 struct RowMap {
   bool hi_lo;
   int group;
@@ -331,29 +323,22 @@ struct RowMap {
 // Every mbarrier below completes one phase per use and is waited phase by phase, never more
 // than one phase behind its current state (buffers that could run two pages ahead of their
 // waiter have one barrier per buffer), so parity waits cannot alias.  Barriers marked "bytes"
-// complete when the stated number of bytes has landed (TMA, bulk copy or st.async from the
-// peer CTA); the ones the peer writes are armed here, one use ahead.
+// complete when the stated number of bytes has landed (TMA, or st.async from the peer CTA);
+// the ones the peer writes are armed here, one use ahead.
 struct Bars {
   uint64_t full[kSlots];   // TMA: the page slot is filled (bytes)
   uint64_t empty[kSlots];  // MMA: the PV that read the slot finished (commit)
   uint64_t q_full;         // TMA: the segment's query RoPE half landed (bytes)
   uint64_t q_empty;        // MMA: the segment's last QK finished (commit)
   uint64_t q_ready;        // softmax warps 0-3: the query latent half is in TMEM (4)
-  uint64_t s_full;         // MMA: S of a page group is written (commit)
-  uint64_t s_free;         // the 8 softmax and 4 send warps drained S (12)
-  uint64_t x_full[2];      // the peer's partial scores for our rows landed (bytes)
+  uint64_t s_full[2];      // MMA: S of a page is written (commit)
+  uint64_t s_free[2];      // the 8 softmax and 4 send warps drained S of the page (12)
+  uint64_t x_full[2];      // the peer's partial scores of a page landed (bytes)
   uint64_t x_free[2];      // the peer's softmax warps decoded our partials of a page (8 remote)
-  uint64_t p_own[2];       // softmax warps: our rows of P and their factors are written (8)
-  uint64_t p_peer[2];      // the peer's rows of P and their factors landed (bytes)
-  uint64_t p_ready[2];     // send warps: P complete, O rescaled, PV may run (4)
-  uint64_t p_free[2];      // our PV of the page finished (commit) and the copy of our rows to
-                           // the peer has read them (1 arrival): the buffer may be rewritten
-  uint64_t pv_done[2];     // PV of the page finished in both CTAs (2 commits)
+  uint64_t p_full[2];      // softmax warps: P of the page written, O rescaled (8)
+  uint64_t pv_done[2];     // MMA: PV of the page finished, its P buffer is free (commit)
   uint64_t seg_done;       // MMA: every PV of the segment finished (commit)
   uint64_t o_free;         // softmax warps: the epilogue drained O (8)
-  uint64_t st_full;        // the peer's row statistics for the segment landed (bytes)
-  uint64_t mx_bar[4][2];   // the two softmax warps of quarter q posted their row maxima (2)
-  uint64_t ls_bar[2];      // the 8 softmax warps posted their row sums of a segment (8)
   uint64_t drain;          // MMA: final drain after an abort
   uint32_t tmem_base;
   int abort_flag;
@@ -363,20 +348,21 @@ static_assert(sizeof(Bars) <= 512, "barrier block");
 constexpr uint64_t kDrainNs = 200000000ull;  // waits for copies and MMAs already in flight
 constexpr uint32_t kFull = 0xffffffffu;
 
-__device__ __forceinline__ float max16(const float* s) {
-  float m[4];
+__device__ __forceinline__ float max32(const float* s) {
+  float m[8];
 #pragma unroll
-  for (int j = 0; j < 4; ++j) m[j] = s[j];
+  for (int j = 0; j < 8; ++j) m[j] = s[j];
 #pragma unroll
-  for (int k = 4; k < 16; ++k) m[k & 3] = fmaxf(m[k & 3], s[k]);
-  return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+  for (int k = 8; k < 32; ++k) m[k & 7] = fmaxf(m[k & 7], s[k]);
+  return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])),
+               fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
 }
-__device__ __forceinline__ float maxabs32(const float* s) {
+__device__ __forceinline__ float maxabs64(const float* s) {
   float m[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) m[j] = fabsf(s[j]);
 #pragma unroll
-  for (int k = 8; k < 32; ++k) m[k & 7] = fmaxf(m[k & 7], fabsf(s[k]));
+  for (int k = 8; k < 64; ++k) m[k & 7] = fmaxf(m[k & 7], fabsf(s[k]));
   return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])),
                fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
 }
@@ -385,13 +371,6 @@ __device__ __forceinline__ void spin_ns(uint64_t ns) {
   const uint64_t t0 = globaltimer_ns();
   while (globaltimer_ns() - t0 < ns) {
   }
-}
-
-// One lane tests, the warp gets the answer (a warp-uniform decision for an event loop).
-__device__ __forceinline__ bool warp_test(uint64_t* bar, uint32_t parity) {
-  bool ok = false;
-  if ((threadIdx.x & 31) == 0) ok = mbar_test(bar, parity);
-  return __shfl_sync(kFull, ok ? 1 : 0, 0) != 0;
 }
 
 // Advance the start-address field (bits 0-13, in 16-byte units) of a shared-memory matrix
@@ -426,32 +405,22 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
     mbar_init(&bars->q_full, 1);
     mbar_init(&bars->q_empty, 1);
     mbar_init(&bars->q_ready, 4);
-    mbar_init(&bars->s_full, 1);
-    mbar_init(&bars->s_free, 12);
     for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->s_full[i], 1);
+      mbar_init(&bars->s_free[i], 12);
       mbar_init(&bars->x_full[i], 1);
       mbar_init(&bars->x_free[i], 8);
-      mbar_init(&bars->p_own[i], 8);
-      mbar_init(&bars->p_peer[i], 1);
-      mbar_init(&bars->p_ready[i], 4);
-      mbar_init(&bars->p_free[i], 2);
-      mbar_init(&bars->pv_done[i], 2);
+      mbar_init(&bars->p_full[i], 8);
+      mbar_init(&bars->pv_done[i], 1);
     }
     mbar_init(&bars->seg_done, 1);
     mbar_init(&bars->o_free, 8);
-    mbar_init(&bars->st_full, 1);
-    for (int i = 0; i < 8; ++i) mbar_init(&bars->mx_bar[i >> 1][i & 1], 2);
-    mbar_init(&bars->ls_bar[0], 8);
-    mbar_init(&bars->ls_bar[1], 8);
     mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
     fence_mbar_init_cluster();
-    // receive-side barriers, armed for their first use
-    for (int i = 0; i < 2; ++i) {
-      mbar_arrive_expect_tx(&bars->x_full[i], kXBytes);
-      mbar_arrive_expect_tx(&bars->p_peer[i], kPMsgBytes);
-    }
-    mbar_arrive_expect_tx(&bars->st_full, 512);
+    // receive buffers armed for their first use
+    mbar_arrive_expect_tx(&bars->x_full[0], kXBytes);
+    mbar_arrive_expect_tx(&bars->x_full[1], kXBytes);
   }
   if (warp == 13) {
     tmem_alloc(&bars->tmem_base, kTmemCols);
@@ -556,10 +525,9 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
       if (sg > 0) mbar_wait(&bars->q_full, (sg - 1) & 1, drain_ctx);
     }
   } else if (warp == 13) {
-    // =================== MMA issuer: QK per page group, PV per page, as each is ready ========
+    // =================== MMA issuer: QK and PV per page, each as soon as it is ready ==========
     if (lane == 0) {
-      const uint32_t idesc_qk128 = idesc_bf16(128, 128, 0, 0);
-      const uint32_t idesc_qk64 = idesc_bf16(128, 64, 0, 0);
+      const uint32_t idesc_qk = idesc_bf16(128, 64, 0, 0);
       const uint32_t idesc_pv = idesc_bf16(128, 256, 0, 1);
       // descriptors at the buffers' starts; every operand below is one of these advanced
       const uint64_t d_ring = smem_desc(smem_u32(smem + kOffRing), 16, 1024, kSwizzle128B);
@@ -567,25 +535,19 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
       const uint64_t d_qrope = smem_desc(smem_u32(sQRope), 16, 512, kSwizzle64B);
       const uint64_t d_p = smem_desc(smem_u32(smem + kOffP), 16, 1024, kSwizzle128B);
       const uint64_t d_pv_b = smem_desc(smem_u32(smem + kOffRing), kBoxStride, 1024, kSwizzle128B);
-      // S = Q_r C_r^T for the npg (1 or 2) pages from global page t on: one N = 128 product
-      // when the two slots are adjacent in the ring, else one N = 64 product per page
-      auto issue_qk = [&](int t, int npg) {
-        const int s0 = t % kSlots;
-        const int runs = (npg == 2 && s0 + 1 < kSlots) ? 1 : npg;
-        const uint32_t idesc = (npg == 2 && runs == 1) ? idesc_qk128 : idesc_qk64;
-        for (int u = 0; u < runs; ++u) {
-          const uint32_t s = static_cast<uint32_t>((s0 + u) % kSlots);
-          const uint32_t d = tmem + kTmemS + 64 * u;
-          const uint64_t b0 = desc_add(d_ring, s * kBoxBytes);
+      // S_t = Q_r C_r^T into S buffer t & 1: latent half A from TMEM, RoPE half A from smem
+      auto issue_qk = [&](int t) {
+        const uint32_t s = static_cast<uint32_t>(t % kSlots);
+        const uint32_t d = tmem + kTmemS + 64 * (t & 1);
+        const uint64_t b0 = desc_add(d_ring, s * kBoxBytes);
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            mma_ts(d, tmem + kTmemQ + 8 * j,
-                   desc_add(b0, (j >> 2) * kBoxStride + (j & 3) * 32), idesc, j > 0 ? 1u : 0u);
-          const uint64_t r0 = desc_add(d_rope, s * kRopeBoxBytes);
-          mma_ss(d, d_qrope, r0, idesc, 1u);
-          mma_ss(d, desc_add(d_qrope, 32), desc_add(r0, 32), idesc, 1u);
-        }
-        mma_commit(&bars->s_full);
+        for (int j = 0; j < 16; ++j)
+          mma_ts(d, tmem + kTmemQ + 8 * j, desc_add(b0, (j >> 2) * kBoxStride + (j & 3) * 32),
+                 idesc_qk, j > 0 ? 1u : 0u);
+        const uint64_t r0 = desc_add(d_rope, s * kRopeBoxBytes);
+        mma_ss(d, d_qrope, r0, idesc_qk, 1u);
+        mma_ss(d, desc_add(d_qrope, 32), desc_add(r0, 32), idesc_qk, 1u);
+        mma_commit(&bars->s_full[t & 1]);
       };
       // O += P_t C_lat,t: A = P (bf16, shared memory), B = the page's latent half (MN-major)
       auto issue_pv = [&](int t, bool first) {
@@ -596,29 +558,27 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
         for (int kk = 0; kk < 4; ++kk)
           mma_ss(tmem + kTmemO, desc_add(a0, kk * 32), desc_add(b0, kk * 2048), idesc_pv,
                  (first && kk == 0) ? 0u : 1u);
-        mma_commit(&bars->p_free[t & 1]);
-        mma_commit_cluster(&bars->pv_done[t & 1], 0x3);  // both CTAs learn that P_t is read
+        mma_commit(&bars->pv_done[t & 1]);
         mma_commit(&bars->empty[s]);
       };
       SegIter itq{plan.seq_pages(), plan.seq_prefix(), p.batch, g_begin, g_end, b_begin};
       SegIter itv = itq;
       int qs, q0, q1, vs, v0, v1;
       bool q_more = itq.next(qs, q0, q1), v_more = itv.next(vs, v0, v1);
-      int q_i = 0, q_t = 0, q_g = 0, q_sg = 0;  // QK: page in segment, global page, group, seg
-      int v_i = 0, v_t = 0, v_sg = 0;           // PV: page in segment, global page, segment
+      int q_i = 0, q_t = 0, q_sg = 0;  // QK: page in segment, global page, segment
+      int v_i = 0, v_t = 0, v_sg = 0;  // PV: page in segment, global page, segment
       uint64_t idle_since = 0;
       uint32_t spins = 0;
       bool ok = true;
       while (ok && (q_more || v_more)) {
         bool progress = false;
-        // PV first: it frees the ring slots and the P buffers the rest of the pipe waits for
-        if (v_more && mbar_test(&bars->p_ready[v_t & 1], (v_t >> 1) & 1) &&
+        // PV first: it frees the ring slot and the P buffer the rest of the pipe waits for
+        if (v_more && mbar_test(&bars->p_full[v_t & 1], (v_t >> 1) & 1) &&
             (v_i > 0 || v_sg == 0 || mbar_test(&bars->o_free, (v_sg - 1) & 1))) {
           tc_fence_after();
           issue_pv(v_t, v_i == 0);
-          ++v_i;
           ++v_t;
-          if (v_i == v1 - v0) {
+          if (++v_i == v1 - v0) {
             mma_commit(&bars->seg_done);
             ++v_sg;
             v_i = 0;
@@ -626,27 +586,21 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
           }
           progress = true;
         }
-        if (q_more) {
-          const int n = q1 - q0, npg = min(2, n - q_i);
-          if ((q_i > 0 ||
-               (mbar_test(&bars->q_ready, q_sg & 1) && mbar_test(&bars->q_full, q_sg & 1))) &&
-              (q_g == 0 || mbar_test(&bars->s_free, (q_g - 1) & 1)) &&
-              mbar_test(&bars->full[q_t % kSlots], (q_t / kSlots) & 1) &&
-              (npg == 1 ||
-               mbar_test(&bars->full[(q_t + 1) % kSlots], ((q_t + 1) / kSlots) & 1))) {
-            tc_fence_after();
-            issue_qk(q_t, npg);
-            q_i += npg;
-            q_t += npg;
-            ++q_g;
-            if (q_i == n) {
-              mma_commit(&bars->q_empty);
-              ++q_sg;
-              q_i = 0;
-              q_more = itq.next(qs, q0, q1);
-            }
-            progress = true;
+        if (q_more &&
+            (q_i > 0 ||
+             (mbar_test(&bars->q_ready, q_sg & 1) && mbar_test(&bars->q_full, q_sg & 1))) &&
+            (q_t < 2 || mbar_test(&bars->s_free[q_t & 1], ((q_t >> 1) - 1) & 1)) &&
+            mbar_test(&bars->full[q_t % kSlots], (q_t / kSlots) & 1)) {
+          tc_fence_after();
+          issue_qk(q_t);
+          ++q_t;
+          if (++q_i == q1 - q0) {
+            mma_commit(&bars->q_empty);
+            ++q_sg;
+            q_i = 0;
+            q_more = itq.next(qs, q0, q1);
           }
+          progress = true;
         }
         if (progress) {
           idle_since = 0;
@@ -671,231 +625,108 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
         mbar_wait(&bars->drain, 0, drain_ctx);
       }
     }
-  } else if (warp == 14) {
-    // =================== P copy: our rows of P and their factors into the peer ================
-    if (lane == 0) {
-      const uint32_t p_loc = smem_u32(smem + kOffP);
-      const uint32_t p_rem = mapa_shared(p_loc, peer);
-      const uint32_t a_loc = smem_u32(smem + kOffAlphaOwn);
-      const uint32_t a_rem = mapa_shared(smem_u32(smem + kOffAlphaIn), peer);
-      const uint32_t ppeer_rem[2] = {mapa_shared(smem_u32(&bars->p_peer[0]), peer),
-                                     mapa_shared(smem_u32(&bars->p_peer[1]), peer)};
-      int total = 0;
-      SegIter it{plan.seq_pages(), plan.seq_prefix(), p.batch, g_begin, g_end, b_begin};
-      int seq, p0, p1;
-      while (it.next(seq, p0, p1)) total += p1 - p0;
-      bool ok = true;
-      for (int t = 0; ok && t < total; ++t) {
-        const int pb = t & 1;
-        if (!(ok = mbar_wait(&bars->p_own[pb], (t >> 1) & 1, wc))) break;
-        // the peer's buffer pb is free once PV(t - 2) has run in both CTAs
-        if (t >= 2 && !(ok = mbar_wait<true>(&bars->pv_done[pb], ((t >> 1) - 1) & 1, wc))) break;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint32_t off = pb * kPBytes + (32 * q + 16 * rank) * 128;
-          bulk_copy_s2cluster(p_rem + off, p_loc + off, 16 * 128, ppeer_rem[pb]);
-        }
-        bulk_copy_s2cluster(a_rem + pb * 256, a_loc + pb * 256, 256, ppeer_rem[pb]);
-        bulk_commit_group();
-        bulk_wait_read_all();
-        mbar_arrive(&bars->p_free[pb]);
-      }
-      if (!ok) bulk_wait_read_all();
-    }
   } else if (warp >= 8) {
-    // =================== send warps: partials out; P completion and O rescale ================
-    // Sending: 16x32bx2 view, thread (j, h) = (lane & 15, lane >> 4) reads row 32q + 16 peer + j,
-    // columns 32h .. 32h + 31 of each page, and writes row 16q + j of the peer's receive buffer.
-    // Finishing a page: once both CTAs' rows of P are in place, rescale O (32x32b view, thread =
-    // lane 32q + lane) if a row's running maximum moved, then let PV run.
-    const int q = warp & 3, j = lane & 15, hcol = lane >> 4;
-    const uint32_t lanes_peer = static_cast<uint32_t>(32 * q + 16 * peer) << 16;
-    const uint32_t lanes_all = static_cast<uint32_t>(32 * q) << 16;
-    const int rho = 16 * q + j;
+    // =================== send warps: this CTA's partial scores, quantised, into the peer ======
+    // Thread = TMEM lane 32q + lane = row; all 64 columns of the page; row 32q + lane of the
+    // peer's receive buffer.
+    const int q = warp & 3;
+    const int row = 32 * q + lane;
+    const uint32_t lanes = static_cast<uint32_t>(32 * q) << 16;
     const uint32_t x_peer = mapa_shared(smem_u32(smem + kOffX), peer);
     const uint32_t xfull_peer[2] = {mapa_shared(smem_u32(&bars->x_full[0]), peer),
                                     mapa_shared(smem_u32(&bars->x_full[1]), peer)};
-    const float* alpha_in = reinterpret_cast<const float*>(smem + kOffAlphaIn);
-    const float* alpha_own = reinterpret_cast<const float*>(smem + kOffAlphaOwn);
-    // send side
-    SegIter its{plan.seq_pages(), plan.seq_prefix(), p.batch, g_begin, g_end, b_begin};
-    int s_seq, s0, s1;
-    bool s_more = its.next(s_seq, s0, s1);
-    int s_i = 0, s_t = 0, s_g = 0, s_state = 0, s_k = 0, s_npg = 0;
-    int s_len = s_more ? min(p.seq_lens[s_seq], p.max_pages * kPage) : 0;
-    uint32_t e[2][16];  // the quantised partials of the current page group
-    float scale[2];
-    // finish side
-    SegIter itf{plan.seq_pages(), plan.seq_prefix(), p.batch, g_begin, g_end, b_begin};
-    int f_seq, f0, f1;
-    bool f_more = itf.next(f_seq, f0, f1);
-    int f_i = 0, f_t = 0;
-    uint64_t idle_since = 0;
-    uint32_t spins = 0;
+    SegIter it{plan.seq_pages(), plan.seq_prefix(), p.batch, g_begin, g_end, b_begin};
+    int seq, p0, p1, t = 0;
     bool ok = true;
-    while (ok && (s_more || f_more)) {
-      bool progress = false;
-      if (f_more && warp_test(&bars->p_own[f_t & 1], (f_t >> 1) & 1) &&
-          warp_test(&bars->p_peer[f_t & 1], (f_t >> 1) & 1)) {
-        const int pb = f_t & 1;
-        if (warp == 8 && lane == 0) mbar_arrive_expect_tx(&bars->p_peer[pb], kPMsgBytes);
-        // O rescale (rare): rows of the quarter whose running maximum moved, ours or the peer's
-        const float a_own = alpha_own[pb * 64 + rho];
-        const float a_peer = alpha_in[pb * 64 + rho];
-        if (f_i > 0 && __any_sync(kFull, a_own != 1.f || a_peer != 1.f)) {
-          if (!(ok = warp_wait(&bars->p_free[pb ^ 1], ((f_t - 1) >> 1) & 1, wc))) break;
-          tc_fence_after();
-          const float fa = __shfl_sync(kFull, a_own, j);
-          const float fb = __shfl_sync(kFull, a_peer, j);
-          const float f = (lane >> 4) == static_cast<int>(rank) ? fa : fb;
-#pragma unroll 1
-          for (int c = 0; c < 256; c += 32) {
-            uint32_t r[32];
-            tmem_ld32(tmem + kTmemO + c + lanes_all, r);
-            tmem_wait_ld();
-#pragma unroll
-            for (int u = 0; u < 32; ++u) r[u] = __float_as_uint(__uint_as_float(r[u]) * f);
-            tmem_st32(tmem + kTmemO + c + lanes_all, r);
-          }
-          tmem_wait_st();
-          tc_fence_before();
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->p_ready[pb]);
-        ++f_t;
-        if (++f_i == f1 - f0) {
-          f_i = 0;
-          f_more = itf.next(f_seq, f0, f1);
-        }
-        progress = true;
-      }
-      // send side: state 0 waits for a page group's S, drains the peer's rows and quantises
-      // them; state 1 sends each page once the peer has freed that receive buffer
-      if (s_more && s_state == 0 && warp_test(&bars->s_full, s_g & 1)) {
-        s_npg = min(2, (s1 - s0) - s_i);
+    while (ok && it.next(seq, p0, p1)) {
+      const int len = min(p.seq_lens[seq], p.max_pages * kPage);
+      for (int i = 0; i < p1 - p0; ++i, ++t) {
+        const int pb = t & 1;
+        if (!(ok = warp_wait(&bars->s_full[pb], (t >> 1) & 1, wc))) break;
         tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          if (k == 1 && s_npg == 1) break;
-          uint32_t a[32];
-          tmem_ld16x2_32(tmem + kTmemS + 64 * k + lanes_peer, a);
+        float s[64];
+        {
+          uint32_t r[32];
+          tmem_ld32(tmem + kTmemS + 64 * pb + lanes, r);
           tmem_wait_ld();
-          float sv[32];
 #pragma unroll
-          for (int u = 0; u < 32; ++u) sv[u] = __uint_as_float(a[u]);
-          // columns past the sequence's end are never used: they travel as zeros
-          const int valid = min(kPage, s_len - (s0 + s_i + k) * kPage) - 32 * hcol;
-          if (valid < 32) {
+          for (int k = 0; k < 32; ++k) s[k] = __uint_as_float(r[k]);
+          tmem_ld32(tmem + kTmemS + 64 * pb + 32 + lanes, r);
+          tmem_wait_ld();
 #pragma unroll
-            for (int u = 0; u < 32; ++u) sv[u] = u < valid ? sv[u] : 0.f;
-          }
-          float mabs = maxabs32(sv);
-          mabs = fmaxf(mabs, __shfl_xor_sync(kFull, mabs, 16));
-          const float inv = mabs > 0.f ? 32767.f / mabs : 0.f;
-#pragma unroll
-          for (int u = 0; u < 16; ++u) e[k][u] = enc_u16x2(sv[2 * u], sv[2 * u + 1], inv);
-          scale[k] = mabs * (1.f / 32767.f);
+          for (int k = 0; k < 32; ++k) s[32 + k] = __uint_as_float(r[k]);
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->s_free);
-        s_state = 1;
-        s_k = 0;
-        progress = true;
-      }
-      while (s_more && s_state == 1) {
-        const int tt = s_t + s_k, pb = tt & 1;
-        if (tt >= 2 && !warp_test(&bars->x_free[pb], ((tt >> 1) - 1) & 1)) break;
-        const uint32_t xb = x_peer + pb * kXBytes;
-        auto send = [&](const uint32_t (&ek)[16], float sc) {
+        if (lane == 0) mbar_arrive(&bars->s_free[pb]);
+        // columns past the sequence's end are never used: they travel as zeros
+        const int valid = min(kPage, len - (p0 + i) * kPage);
+        if (valid < kPage) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
-            st_async_u4(xb + xrow_off(rho, 4 * hcol + c), ek[4 * c], ek[4 * c + 1],
-                        ek[4 * c + 2], ek[4 * c + 3], xfull_peer[pb]);
-          if (hcol == 0) st_async_u1(xb + kXPayload + rho * 4, __float_as_uint(sc), xfull_peer[pb]);
-        };
-        if (s_k == 0)
-          send(e[0], scale[0]);
-        else
-          send(e[1], scale[1]);
-        progress = true;
-        if (++s_k == s_npg) {
-          s_t += s_npg;
-          s_i += s_npg;
-          ++s_g;
-          s_state = 0;
-          if (s_i == s1 - s0) {
-            s_i = 0;
-            s_more = its.next(s_seq, s0, s1);
-            if (s_more) s_len = min(p.seq_lens[s_seq], p.max_pages * kPage);
-          }
+          for (int k = 0; k < 64; ++k) s[k] = k < valid ? s[k] : 0.f;
         }
-      }
-      if (progress) {
-        idle_since = 0;
-        spins = 0;
-      } else if ((++spins & 63) == 0) {
-        if (bars->abort_flag) {
-          ok = false;
-        } else {
-          const uint64_t now = globaltimer_ns();
-          if (idle_since == 0) {
-            idle_since = now;
-          } else if (now - idle_since > p.wait_ns) {
-            bars->abort_flag = 1;
-            atomicOr(p.status, MLA_STATUS_TIMEOUT);
-            ok = false;
-          }
-        }
+        const float mabs = maxabs64(s);
+        const float inv = mabs > 0.f ? 32767.f / mabs : 0.f;
+        if (t >= 2 && !(ok = warp_wait<true>(&bars->x_free[pb], ((t >> 1) - 1) & 1, wc))) break;
+        const uint32_t xb = x_peer + pb * kXBytes;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          st_async_u4(xb + xrow_off(row, c), enc_u16x2(s[8 * c], s[8 * c + 1], inv),
+                      enc_u16x2(s[8 * c + 2], s[8 * c + 3], inv),
+                      enc_u16x2(s[8 * c + 4], s[8 * c + 5], inv),
+                      enc_u16x2(s[8 * c + 6], s[8 * c + 7], inv), xfull_peer[pb]);
+        st_async_u1(xb + kXPayload + row * 4, __float_as_uint(mabs * (1.f / 32767.f)),
+                    xfull_peer[pb]);
       }
     }
     if (ok) {  // the peer's hand-backs for our last two pages land before this CTA exits
-      for (int u = max(0, s_t - 2); u < s_t; ++u)
+      for (int u = max(0, t - 2); u < t; ++u)
         mbar_wait<true>(&bars->x_free[u & 1], (u >> 1) & 1, drain_ctx);
     }
   } else {
-    // =================== softmax warps (own rows), query load, epilogue ====================
-    // 16x32bx2 view: warp w owns row 32q + 16 rank + j (q = w & 3) and the 32 columns
-    // 32k .. 32k + 31 of each page (k = w >> 2); thread (j, h) takes 16 of them, 32k + 16h on.
-    // The row maximum is shared by the two warps of a quarter through shared memory; each keeps
-    // its own partial row sum.  Warps 0-3 load the query; all 8 write O out (32x32b view).
+    // =================== softmax warps, query load, epilogue ===================
+    // 16x32bx2 view: warp w owns the 16 rows 32q + 16k .. 32q + 16k + 15 (q = w & 3, k = w >> 2),
+    // two threads per row: thread (j, h) = (lane & 15, lane >> 4) takes columns 32h .. 32h + 31
+    // of each page and O columns 128h .. 128h + 127.  A row lives in one warp, so its maximum
+    // and sum take one shuffle.  Warps 0-3 load the query (32x32b view, thread = lane 32q + lane).
     const int q = warp & 3, kh = warp >> 2, j = lane & 15, hcol = lane >> 4;
-    const int rho = 16 * q + j;
-    const int c0 = 32 * kh + 16 * hcol;  // this thread's first column within a page
-    const int row_own = 32 * q + 16 * static_cast<int>(rank) + j;
-    const int row_lane = 32 * q + lane;
-    const uint32_t lanes_own = static_cast<uint32_t>(32 * q + 16 * rank) << 16;
+    const int row = 32 * q + 16 * kh + j;
+    const uint32_t lanes_own = static_cast<uint32_t>(32 * q + 16 * kh) << 16;
     const uint32_t lanes_all = static_cast<uint32_t>(32 * q) << 16;
     const float NEG_INF = -__int_as_float(0x7f800000);
     const uint32_t x_loc = smem_u32(smem + kOffX);
     const uint32_t p_loc = smem_u32(smem + kOffP);
-    const uint32_t stats_rem = mapa_shared(smem_u32(smem + kOffStats), peer);
     const uint32_t xfree_rem[2] = {mapa_shared(smem_u32(&bars->x_free[0]), peer),
                                    mapa_shared(smem_u32(&bars->x_free[1]), peer)};
-    const uint32_t stfull_rem = mapa_shared(smem_u32(&bars->st_full), peer);
-    float* alpha_own = reinterpret_cast<float*>(smem + kOffAlphaOwn);
-    float* max_x = reinterpret_cast<float*>(smem + kOffMaxX);  // [page parity][half][row]
-    float* l_part = reinterpret_cast<float*>(smem + kOffLPart);  // [seg parity][half][row]
-    const float2* stats_in = reinterpret_cast<const float2*>(smem + kOffStats);
-    // this CTA's latent half of the query rows of sequence sq -> TMEM (A operand of QK)
+    const int hd = rows.head(row);
+    const bool out_row = hd < p.n_heads && !rows.lo(row);
+    // this CTA's latent half of the query rows of sequence sq -> TMEM (A operand of QK), in two
+    // batches of 16 loads issued before their first use
     auto load_q = [&](int sq) {
-      const int hd = rows.head(row_lane);
-      const bool in = hd < p.n_heads;
+      const int qrow = 32 * q + lane;
+      const int qhd = rows.head(qrow);
+      const bool in = qhd < p.n_heads;
       const uint4* src = reinterpret_cast<const uint4*>(
-          (rows.lo(row_lane) ? p.q_lo : p.q_cat) +
-          (static_cast<size_t>(sq) * p.n_heads + (in ? hd : 0)) * kRow);
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
+          (rows.lo(qrow) ? p.q_lo : p.q_cat) +
+          (static_cast<size_t>(sq) * p.n_heads + (in ? qhd : 0)) * kRow) + 32 * rank;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint4 v = in ? __ldg(src + (256 * rank + 64 * c) / 8 + k) : make_uint4(0u, 0u, 0u, 0u);
-          r[4 * k] = v.x;
-          r[4 * k + 1] = v.y;
-          r[4 * k + 2] = v.z;
-          r[4 * k + 3] = v.w;
+      for (int half = 0; half < 2; ++half) {
+        uint4 v[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+          v[k] = in ? __ldg(src + 16 * half + k) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t r[32];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            r[4 * k] = v[8 * c + k].x;
+            r[4 * k + 1] = v[8 * c + k].y;
+            r[4 * k + 2] = v[8 * c + k].z;
+            r[4 * k + 3] = v[8 * c + k].w;
+          }
+          tmem_st32(tmem + kTmemQ + 32 * (2 * half + c) + lanes_all, r);
         }
-        tmem_st32(tmem + kTmemQ + 32 * c + lanes_all, r);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -903,7 +734,7 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
       if (lane == 0) mbar_arrive(&bars->q_ready);
     };
     SegIter it{plan.seq_pages(), plan.seq_prefix(), p.batch, g_begin, g_end, b_begin};
-    int seq, p0, p1, t = 0, g = 0, sg = 0;
+    int seq, p0, p1, t = 0, sg = 0;
     bool ok = true;
     bool have = it.next(seq, p0, p1);
     if (have && kh == 0) load_q(seq);
@@ -911,112 +742,112 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
       const int n = p1 - p0;
       const int len = min(p.seq_lens[seq], p.max_pages * kPage);
       float m_ref = NEG_INF, l_sum = 0.f;
-      for (int i = 0; ok && i < n; i += 2, ++g) {
-        const int npg = min(2, n - i);
-        if (!(ok = warp_wait(&bars->s_full, g & 1, wc))) break;
+      for (int i = 0; ok && i < n; ++i, ++t) {
+        const int pb = t & 1;
+        const bool first = i == 0;
+        // ---- own exact partial: this thread's 32 columns of its row ----
+        if (!(ok = warp_wait(&bars->s_full[pb], (t >> 1) & 1, wc))) break;
         tc_fence_after();
-        uint32_t a[16], b[16];
-        tmem_ld16x2_16(tmem + kTmemS + 32 * kh + lanes_own, a);
-        if (npg == 2) tmem_ld16x2_16(tmem + kTmemS + 64 + 32 * kh + lanes_own, b);
-        tmem_wait_ld();
+        float s[32];
+        {
+          uint32_t r[32];
+          tmem_ld16x2_32(tmem + kTmemS + 64 * pb + lanes_own, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) s[k] = __uint_as_float(r[k]);
+        }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->s_free);
-        for (int k = 0; ok && k < npg; ++k) {
-          const int tt = t + i + k, pb = tt & 1;
-          const bool first = i + k == 0;
-          float s[16];
+        if (lane == 0) mbar_arrive(&bars->s_free[pb]);
+        // ---- plus the peer's partial (16-bit, relative to its row's largest magnitude) ----
+        if (!(ok = warp_wait(&bars->x_full[pb], (t >> 1) & 1, wc))) break;
+        {
+          const uint32_t xb = x_loc + pb * kXBytes;
+          float dq;
+          asm volatile("ld.shared.f32 %0, [%1];" : "=f"(dq) : "r"(xb + kXPayload + row * 4));
 #pragma unroll
-          for (int u = 0; u < 16; ++u) s[u] = __uint_as_float(k ? b[u] : a[u]);
-          // ---- plus the peer's partial (16-bit, relative to its row's largest magnitude) ----
-          if (!(ok = warp_wait<true>(&bars->x_full[pb], (tt >> 1) & 1, wc))) break;
-          {
-            const uint32_t xb = x_loc + pb * kXBytes;
-            float dq;
-            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(dq) : "r"(xb + kXPayload + rho * 4));
+          for (int c = 0; c < 4; ++c) {
+            uint32_t v[4];
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
+                         : "r"(xb + xrow_off(row, 4 * hcol + c)));
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-              uint32_t v[4];
-              asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                           : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
-                           : "r"(xb + xrow_off(rho, c0 / 8 + c)));
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk) {
-                s[8 * c + 2 * kk] = fmaf(dec_lo(v[kk]), dq, s[8 * c + 2 * kk]);
-                s[8 * c + 2 * kk + 1] = fmaf(dec_hi(v[kk]), dq, s[8 * c + 2 * kk + 1]);
-              }
-            }
-            // decoded: warp 0 re-arms the buffer for page tt + 2, every warp hands it back
-            __syncwarp();
-            if (lane == 0) {
-              if (warp == 0) mbar_arrive_expect_tx(&bars->x_full[pb], kXBytes);
-              mbar_arrive_remote_relaxed(xfree_rem[pb]);
+            for (int k = 0; k < 4; ++k) {
+              s[8 * c + 2 * k] = fmaf(dec_lo(v[k]), dq, s[8 * c + 2 * k]);
+              s[8 * c + 2 * k + 1] = fmaf(dec_hi(v[k]), dq, s[8 * c + 2 * k + 1]);
             }
           }
-          // ---- a head's score with the query remainder: the sum of its two rows ----
-          if (rows.hi_lo) {
-#pragma unroll
-            for (int u = 0; u < 16; ++u) s[u] += __shfl_xor_sync(kFull, s[u], 8);
-          }
-          // ---- online softmax: the row maximum over both warps of the quarter ----
-          const int valid = min(kPage, len - (p0 + i + k) * kPage) - c0;
-          if (valid < 16) {
-#pragma unroll
-            for (int u = 0; u < 16; ++u) s[u] = u < valid ? s[u] : NEG_INF;
-          }
-          float mx = max16(s);
-          mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
-          if (hcol == 0) max_x[(pb * 2 + kh) * 64 + rho] = mx;
+          // decoded: warp 0 re-arms the buffer for page t + 2, every warp hands it back
           __syncwarp();
-          if (lane == 0) mbar_arrive(&bars->mx_bar[q][pb]);
-          if (!(ok = warp_wait(&bars->mx_bar[q][pb], (tt >> 1) & 1, wc))) break;
-          mx = fmaxf(mx, max_x[(pb * 2 + (kh ^ 1)) * 64 + rho]);
-          mx *= p.scale_log2;  // log2 units (scale > 0 keeps the arg max)
-          float alpha = 1.f;
-          if (first) {
-            m_ref = mx;
-          } else if (mx > m_ref + kRescaleThreshold) {
-            alpha = ex2_approx(m_ref - mx);
-            m_ref = mx;
+          if (lane == 0) {
+            if (warp == 0) mbar_arrive_expect_tx(&bars->x_full[pb], kXBytes);
+            mbar_arrive_remote_relaxed(xfree_rem[pb]);
           }
-          float rs[4] = {0.f, 0.f, 0.f, 0.f};
-          uint32_t pk[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const float e0 = ex2_approx(fmaf(s[2 * u], p.scale_log2, -m_ref));
-            const float e1 = ex2_approx(fmaf(s[2 * u + 1], p.scale_log2, -m_ref));
-            rs[u & 3] += e0 + e1;
-            pk[u] = pack_bf16x2(e0, e1);
-          }
-          float tot = (rs[0] + rs[1]) + (rs[2] + rs[3]);
-          tot += __shfl_xor_sync(kFull, tot, 16);
-          l_sum = l_sum * alpha + tot;  // this warp's 32 columns of the row
-          // ---- our rows of P, once PV(tt - 2) has read buffer pb and its copy is out ----
-          if (tt >= 2 && !(ok = warp_wait(&bars->p_free[pb], ((tt >> 1) - 1) & 1, wc))) break;
-#pragma unroll
-          for (int c = 0; c < 2; ++c)
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
-                             p_loc + pb * kPBytes + xrow_off(row_own, c0 / 8 + c)),
-                         "r"(pk[4 * c]), "r"(pk[4 * c + 1]), "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
-                         : "memory");
-          if (kh == 0 && hcol == 0) alpha_own[pb * 64 + rho] = alpha;
-          fence_proxy_async_smem();  // -> visible to the tensor core and the bulk copy
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bars->p_own[pb]);
         }
+        // ---- a head's score with the query remainder: the sum of its two rows ----
+        if (rows.hi_lo) {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) s[k] += __shfl_xor_sync(kFull, s[k], 8);
+        }
+        // ---- online softmax over the row (two threads) ----
+        const int valid = min(kPage, len - (p0 + i) * kPage) - 32 * hcol;
+        if (valid < 32) {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) s[k] = k < valid ? s[k] : NEG_INF;
+        }
+        float mx = max32(s);
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
+        mx *= p.scale_log2;  // log2 units (scale > 0 keeps the arg max)
+        float alpha = 1.f;
+        bool resc = false;
+        if (first) {
+          m_ref = mx;
+        } else if (mx > m_ref + kRescaleThreshold) {
+          alpha = ex2_approx(m_ref - mx);
+          m_ref = mx;
+          resc = true;
+        }
+        float rs[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        uint32_t pk[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const float e0 = ex2_approx(fmaf(s[2 * k], p.scale_log2, -m_ref));
+          const float e1 = ex2_approx(fmaf(s[2 * k + 1], p.scale_log2, -m_ref));
+          rs[k & 7] += e0 + e1;
+          pk[k] = pack_bf16x2(e0, e1);
+        }
+        float tot = ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
+        tot += __shfl_xor_sync(kFull, tot, 16);
+        l_sum = l_sum * alpha + tot;
+        // ---- O rescale (rare): O must hold PV of the previous page first ----
+        if (!first && __any_sync(kFull, resc)) {
+          if (!(ok = warp_wait(&bars->pv_done[pb ^ 1], ((t - 1) >> 1) & 1, wc))) break;
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < 256; c += 64) {
+            uint32_t r[32];
+            tmem_ld16x2_32(tmem + kTmemO + c + lanes_own, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * alpha);
+            tmem_st16x2_32(tmem + kTmemO + c + lanes_own, r);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+        }
+        // ---- P -> shared memory (K-major, 128B swizzle) once PV(t - 2) has read buffer pb ----
+        if (t >= 2 && !(ok = warp_wait(&bars->pv_done[pb], ((t >> 1) - 1) & 1, wc))) break;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                           p_loc + pb * kPBytes + xrow_off(row, 4 * hcol + c)),
+                       "r"(pk[4 * c]), "r"(pk[4 * c + 1]), "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
+                       : "memory");
+        fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->p_full[pb]);
       }
       if (!ok) break;
-      t += n;
-      // ---- row sums of both column halves; own rows' (max, sum) to the peer ----
-      float* lp = l_part + (sg & 1) * 128;
-      if (hcol == 0) lp[kh * 64 + rho] = l_sum;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->ls_bar[sg & 1]);
-      if (!(ok = warp_wait(&bars->ls_bar[sg & 1], (sg >> 1) & 1, wc))) break;
-      const float l_row_own = lp[rho] + lp[64 + rho];
-      if (kh == 0 && hcol == 0)
-        st_async_u2(stats_rem + rho * 8, __float_as_uint(m_ref), __float_as_uint(l_row_own),
-                    stfull_rem);
       // ---- the next segment's query half, as soon as the last QK of this one has run ----
       int nseq = 0, np0 = 0, np1 = 0;
       const bool next = it.next(nseq, np0, np1);
@@ -1024,19 +855,10 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
         if (!(ok = warp_wait(&bars->q_empty, sg & 1, wc))) break;
         load_q(nseq);
       }
-      // ---- segment epilogue: O / l -> global (32x32b view; warp w writes columns 128k ..) ----
+      // ---- segment epilogue: O / l -> global ----
       if (!(ok = warp_wait(&bars->seg_done, sg & 1, wc))) break;
-      if (!(ok = warp_wait<true>(&bars->st_full, sg & 1, wc))) break;
       tc_fence_after();
       {
-        const float2 ps = stats_in[rho];
-        const float m_o = __shfl_sync(kFull, m_ref, j);
-        const float l_o = __shfl_sync(kFull, l_row_own, j);
-        const bool own = (lane >> 4) == static_cast<int>(rank);
-        const float m_row = own ? m_o : ps.x;
-        const float l_row = own ? l_o : ps.y;
-        const int hd = rows.head(row_lane);
-        const bool out_row = hd < p.n_heads && !rows.lo(row_lane);
         const int nparts = plan.seq_nparts()[seq];
         float* dst;
         float* dst_lse;
@@ -1048,14 +870,15 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
           dst = p.part_o + (static_cast<size_t>(slot) * p.n_heads + hd) * 512 + 256 * rank;
           dst_lse = p.part_lse + static_cast<size_t>(slot) * p.n_heads + hd;
         }
-        const float inv_l = 1.f / l_row;
+        const float inv_l = 1.f / l_sum;
 #pragma unroll 1
-        for (int c = 128 * kh; c < 128 * kh + 128; c += 32) {
+        for (int c = 0; c < 256; c += 64) {
           uint32_t r[32];
-          tmem_ld32(tmem + kTmemO + c + lanes_all, r);
+          // thread (j, h) gets O columns c + 32h .. c + 32h + 31 of its row
+          tmem_ld16x2_32(tmem + kTmemO + c + lanes_own, r);
           tmem_wait_ld();
           if (out_row) {
-            float4* d4 = reinterpret_cast<float4*>(dst + c);
+            float4* d4 = reinterpret_cast<float4*>(dst + c + 32 * hcol);
 #pragma unroll
             for (int k = 0; k < 8; ++k)
               d4[k] = make_float4(__uint_as_float(r[4 * k]) * inv_l,
@@ -1064,24 +887,17 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
                                   __uint_as_float(r[4 * k + 3]) * inv_l);
           }
         }
-        if (kh == 0 && out_row && own && dst_lse)
-          *dst_lse = (m_row + __log2f(l_row)) * 0.69314718055994531f;
+        if (hcol == 0 && rank == 0 && out_row && dst_lse)
+          *dst_lse = (m_ref + __log2f(l_sum)) * 0.69314718055994531f;
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&bars->o_free);
-        if (warp == 0) mbar_arrive_expect_tx(&bars->st_full, 512);  // for the next segment
-      }
+      if (lane == 0) mbar_arrive(&bars->o_free);
       ++sg;
       seq = nseq;
       p0 = np0;
       p1 = np1;
       have = next;
-    }
-    if (ok && warp == 0) {  // the peer's PV commits for our last two pages land before exit
-      for (int u = max(0, t - 2); u < t; ++u)
-        mbar_wait<true>(&bars->pv_done[u & 1], (u >> 1) & 1, drain_ctx);
     }
   }
 
