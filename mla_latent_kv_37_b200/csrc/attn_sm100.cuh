@@ -605,7 +605,10 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
         if (progress) {
           idle_since = 0;
           spins = 0;
-        } else if ((++spins & 63) == 0) {
+        } else {
+          // back off briefly: this warp shares its SM sub-partition with softmax and send warps
+          __nanosleep(32);
+          if ((++spins & 63) != 0) continue;
           if (bars->abort_flag) {
             ok = false;
           } else {
@@ -760,11 +763,15 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->s_free[pb]);
         // ---- plus the peer's partial (16-bit, relative to its row's largest magnitude) ----
+        // The bits 0x4B000000 | u are the float 2^23 + u exactly; subtracting 2^23 + 32768 is
+        // exact too, and one FMA per value scales and adds the result (pairs at a time).
         if (!(ok = warp_wait(&bars->x_full[pb], (t >> 1) & 1, wc))) break;
         {
           const uint32_t xb = x_loc + pb * kXBytes;
           float dq;
           asm volatile("ld.shared.f32 %0, [%1];" : "=f"(dq) : "r"(xb + kXPayload + row * 4));
+          const uint64_t dq2 = f2_pack(dq, dq);
+          const uint64_t nbias2 = f2_pack(-kDecBias, -kDecBias);
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             uint32_t v[4];
@@ -773,15 +780,13 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
                          : "r"(xb + xrow_off(row, 4 * hcol + c)));
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              s[8 * c + 2 * k] = fmaf(dec_lo(v[k]), dq, s[8 * c + 2 * k]);
-              s[8 * c + 2 * k + 1] = fmaf(dec_hi(v[k]), dq, s[8 * c + 2 * k + 1]);
+              const uint64_t d2 = f2_add(
+                  f2_pack(__uint_as_float(__byte_perm(v[k], kDecBits, 0x7610)),
+                          __uint_as_float(__byte_perm(v[k], kDecBits, 0x7632))),
+                  nbias2);
+              const uint64_t r2 = f2_fma(d2, dq2, f2_pack(s[8 * c + 2 * k], s[8 * c + 2 * k + 1]));
+              f2_unpack(r2, s[8 * c + 2 * k], s[8 * c + 2 * k + 1]);
             }
-          }
-          // decoded: warp 0 re-arms the buffer for page t + 2, every warp hands it back
-          __syncwarp();
-          if (lane == 0) {
-            if (warp == 0) mbar_arrive_expect_tx(&bars->x_full[pb], kXBytes);
-            mbar_arrive_remote_relaxed(xfree_rem[pb]);
           }
         }
         // ---- a head's score with the query remainder: the sum of its two rows ----
@@ -795,7 +800,17 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
 #pragma unroll
           for (int k = 0; k < 32; ++k) s[k] = k < valid ? s[k] : NEG_INF;
         }
-        float mx = max32(s);
+        float mx;
+        {
+          float m[5];
+#pragma unroll
+          for (int k = 0; k < 5; ++k) m[k] = max3f(s[6 * k], s[6 * k + 1], s[6 * k + 2]);
+#pragma unroll
+          for (int k = 0; k < 5; ++k) m[k] = max3f(m[k], s[6 * k + 3], s[6 * k + 4]);
+#pragma unroll
+          for (int k = 0; k < 5; ++k) m[k] = fmaxf(m[k], s[6 * k + 5]);
+          mx = max3f(max3f(m[0], m[1], m[2]), max3f(m[3], m[4], s[30]), s[31]);
+        }
         mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
         mx *= p.scale_log2;  // log2 units (scale > 0 keeps the arg max)
         float alpha = 1.f;
@@ -807,16 +822,25 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
           m_ref = mx;
           resc = true;
         }
-        float rs[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         uint32_t pk[16];
+        float tot;
+        {
+          const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
+          const uint64_t nb2 = f2_pack(-m_ref, -m_ref);
+          uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const float e0 = ex2_approx(fmaf(s[2 * k], p.scale_log2, -m_ref));
-          const float e1 = ex2_approx(fmaf(s[2 * k + 1], p.scale_log2, -m_ref));
-          rs[k & 7] += e0 + e1;
-          pk[k] = pack_bf16x2(e0, e1);
+          for (int k = 0; k < 16; ++k) {
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(s[2 * k], s[2 * k + 1]), sc2, nb2), x0, x1);
+            const float e0 = ex2_approx(x0);
+            const float e1 = ex2_approx(x1);
+            acc[k & 3] = f2_add(acc[k & 3], f2_pack(e0, e1));
+            pk[k] = pack_bf16x2(e0, e1);
+          }
+          float a0, a1;
+          f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a0, a1);
+          tot = a0 + a1;
         }
-        float tot = ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
         tot += __shfl_xor_sync(kFull, tot, 16);
         l_sum = l_sum * alpha + tot;
         // ---- O rescale (rare): O must hold PV of the previous page first ----
@@ -845,7 +869,13 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
                        : "memory");
         fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->p_full[pb]);
+        if (lane == 0) {
+          mbar_arrive(&bars->p_full[pb]);
+          // the receive buffer was decoded long ago: warp 0 re-arms it for page t + 2 and every
+          // warp hands it back (off the page's critical path)
+          if (warp == 0) mbar_arrive_expect_tx(&bars->x_full[pb], kXBytes);
+          mbar_arrive_remote_relaxed(xfree_rem[pb]);
+        }
       }
       if (!ok) break;
       // ---- the next segment's query half, as soon as the last QK of this one has run ----
