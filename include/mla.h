@@ -24,6 +24,12 @@
  *     scheduled while the work before it on the stream drains, but it reads and writes nothing
  *     until that work has completed, so stream order holds exactly as for ordinary launches.
  *     Setting MLA_NO_PDL=1 in the environment before the first call turns this off.
+ *   - Every wait inside a kernel is bounded (2 s; MLA_WAIT_NS in the environment, in
+ *     nanoseconds, read at each call, overrides it).  A wait that runs out raises
+ *     MLA_STATUS_TIMEOUT; the kernel then waits (on its own, longer limit) for the copies and
+ *     tensor-core operations it has in flight, releases its resources and returns, and the
+ *     CUDA context stays usable.  MLA_TEST_STALL=1 (read at each call) makes one warp of the
+ *     decode kernel wait on a barrier nothing arrives on, to exercise that path in tests.
  *   - Weights are row-major [out_features, in_features] (column-vector form, [TN]):
  *       w_dkv [d_c, D], w_kr [d_rope, D], w_q [H*(d_nope+d_rope), D] (per head d_nope rows then
  *       d_rope rows), w_uk [H*d_nope, d_c], w_uv [H*d_v, d_c], w_o [D, H*d_v].

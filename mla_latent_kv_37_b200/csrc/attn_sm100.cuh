@@ -118,6 +118,7 @@ struct Params {
   float* part_lse;   // [slots][H]
   unsigned int* status;
   uint64_t wait_ns;
+  int stall_test;  // 1: warp 0 first waits on a barrier nothing arrives on (timeout-path test)
 };
 
 // Plan layout (int32 words in the workspace), written by plan_kernel.
@@ -340,6 +341,7 @@ struct Bars {
   uint64_t seg_done;       // MMA: every PV of the segment finished (commit)
   uint64_t o_free;         // softmax warps: the epilogue drained O (8)
   uint64_t drain;          // MMA: final drain after an abort
+  uint64_t stall;          // nothing ever arrives here (timeout-path test)
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -416,6 +418,7 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
     mbar_init(&bars->seg_done, 1);
     mbar_init(&bars->o_free, 8);
     mbar_init(&bars->drain, 1);
+    mbar_init(&bars->stall, 1);
     bars->abort_flag = 0;
     fence_mbar_init_cluster();
     // receive buffers armed for their first use
@@ -519,7 +522,10 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
       }
       ++sg;
     }
-    if (lane == 0 && bars->abort_flag) {  // no copy may still be landing when the CTA exits
+    // No copy may still be landing when the CTA exits.  Normally every load has been consumed
+    // by now and these return at once; after an abort (raised by any role, at any time) they
+    // wait for the copies still in flight.
+    if (lane == 0) {
       for (int i = max(0, issued - kSlots); i < issued; ++i)
         mbar_wait(&bars->full[i % kSlots], (i / kSlots) & 1, drain_ctx);
       if (sg > 0) mbar_wait(&bars->q_full, (sg - 1) & 1, drain_ctx);
@@ -623,10 +629,10 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
           }
         }
       }
-      if (!ok) {  // no MMA may be in flight when TMEM is released
-        mma_commit(&bars->drain);
-        mbar_wait(&bars->drain, 0, drain_ctx);
-      }
+      // No MMA may be in flight when TMEM is released: normally they have all completed, after
+      // an abort (by any role) the commit waits for the last ones.
+      mma_commit(&bars->drain);
+      mbar_wait(&bars->drain, 0, drain_ctx);
     }
   } else if (warp >= 8) {
     // =================== send warps: this CTA's partial scores, quantised, into the peer ======
@@ -740,6 +746,8 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
     int seq, p0, p1, t = 0, sg = 0;
     bool ok = true;
     bool have = it.next(seq, p0, p1);
+    // timeout-path test: a wait that can only run out, raising the status and the abort
+    if (p.stall_test && warp == 0) ok = warp_wait(&bars->stall, 0, wc);
     if (have && kh == 0) load_q(seq);
     while (ok && have) {
       const int n = p1 - p0;

@@ -4,6 +4,7 @@
 // bf16 rows (hi = bf16(x), lo = bf16(x - hi)); the product's two halves are summed here.
 #pragma once
 #include "ptx_sm100.cuh"
+#include "rope.cuh"
 
 namespace mla {
 
@@ -15,15 +16,11 @@ template <> __device__ __forceinline__ __nv_bfloat16 to_elem<__nv_bfloat16>(floa
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
 
-// cos/sin of pos * theta^(-2 pair / d_rope), evaluated in double precision (angles reach
-// ~1.3e5 rad at 128K positions, where a float angle would be off by ~1e-2 rad).
-__device__ __forceinline__ void rope_cos_sin(int pos, int pair, int d_rope, float theta,
-                                             float& c, float& s) {
-  const double inv_freq = pow(static_cast<double>(theta), -2.0 * pair / d_rope);
-  double sn, cs;
-  sincos(static_cast<double>(pos) * inv_freq, &sn, &cs);
-  c = static_cast<float>(cs);
-  s = static_cast<float>(sn);
+// cos/sin of the RoPE angle of rotary pair `pair` at position `pos` (see rope_cs).
+__device__ __forceinline__ void rope_cos_sin(int pos, int pair, float theta, float& c, float& s) {
+  const float2 cs = rope_cs(theta, pair, pos);
+  c = cs.x;
+  s = cs.y;
 }
 
 __device__ __forceinline__ float sum_splits(const float* part, int k_splits, size_t split_stride,
@@ -70,7 +67,7 @@ __global__ void append_epilogue_kernel(const float* __restrict__ part, int k_spl
   float v1 = sum_splits(part, k_splits, split_stride, static_cast<size_t>(2 * q + 1) * n_pad + b);
   if (2 * q >= kDc) {
     float c, s;
-    rope_cos_sin(pos, (2 * q - kDc) / 2, kDr, theta, c, s);
+    rope_cos_sin(pos, (2 * q - kDc) / 2, theta, c, s);
     const float r0 = v0 * c - v1 * s, r1 = v0 * s + v1 * c;
     v0 = r0;
     v1 = r1;
@@ -116,7 +113,7 @@ __global__ void wq_epilogue_kernel(const float* __restrict__ part, int k_splits,
   }
   const int pos = positions[b];
   float c, s;
-  rope_cos_sin(pos, (d - kDn) / 2, kDr, theta, c, s);
+  rope_cos_sin(pos, (d - kDn) / 2, theta, c, s);
   const float r0 = v0 * c - v1 * s, r1 = v0 * s + v1 * c;
   const size_t o = (static_cast<size_t>(b) * H + h) * kRow + kDc + (d - kDn);
   const T e0 = to_elem<T>(r0), e1 = to_elem<T>(r1);

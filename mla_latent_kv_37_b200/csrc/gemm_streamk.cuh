@@ -35,11 +35,13 @@
 //   X         : box (64 k, 1, n_pad) -> [n_pad rows][128 B], SBO = 1024 B
 #pragma once
 #include "ptx_sm100.cuh"
+#include "rope.cuh"
 
 namespace mla {
 namespace sk {
 
 constexpr int kThreads = 192;
+constexpr uint64_t kDrainNs = 200000000ull;  // waits for copies and MMAs already in flight
 constexpr uint32_t kATileBytes = 128 * 64 * 2;
 constexpr int kRopePairs = 32;  // d_rope / 2
 
@@ -104,24 +106,6 @@ __device__ __forceinline__ uint32_t count_in(unsigned long long* ctr, uint32_t e
 // RoPE rows exchange their pair partner with the neighbouring lane (pairs are (even, odd)
 // rows, and a warp's 32 rows never straddle a RoPE boundary).
 // ---------------------------------------------------------------------------------------------
-// cos and sin of the RoPE angle pos * theta^(-2 pair / 64).  The angle (up to ~1.3e5 rad at
-// 128K positions) is formed in double precision and reduced modulo 2 pi with 2 pi split into
-// a double head and a tail (Cody and Waite's two-constant reduction); what is left,
-// |r| <= pi, goes to the float sincos.  Absolute error ~2e-7, far below the bf16 rounding
-// that follows.
-__device__ __forceinline__ float2 rope_cs(float theta, int pair, int pos) {
-  constexpr double kTwoPiHi = 6.283185307179586;       // nearest double to 2 pi
-  constexpr double kTwoPiLo = 2.4492935982947064e-16;  // 2 pi - kTwoPiHi
-  constexpr double kInvTwoPi = 0.15915494309189535;
-  const double inv_freq = pow(static_cast<double>(theta), -2.0 * pair / (2 * kRopePairs));
-  const double a = static_cast<double>(pos) * inv_freq;
-  const double k = rint(a * kInvTwoPi);
-  const double r = fma(-k, kTwoPiLo, fma(-k, kTwoPiHi, a));
-  float sn, cs;
-  sincosf(static_cast<float>(r), &sn, &cs);
-  return make_float2(cs, sn);
-}
-
 // Fill the [n][32] (cos, sin) table for the n RoPE positions (epilogue warps, once per CTA).
 __device__ __forceinline__ void rope_table(float2* tab, const int32_t* positions, int n,
                                            float theta, int tid, int nthreads) {
@@ -504,10 +488,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         load_a(i, s);
         load_x(i, s);
       }
-      if (*abort_flag) {
-        // wait (bounded, ignoring the abort flag) for every copy still landing in the ring
+      // No copy may still be landing when the CTA exits: normally the MMA warp has consumed
+      // every stage and these return at once; after an abort (raised by any role, at any
+      // time) they wait, on their own limit, for the copies still in flight.
+      {
         volatile int never = 0;
-        WaitCtx drain{&never, p.status, p.wait_ns};
+        WaitCtx drain{&never, p.status, kDrainNs};
         for (long long j = (issued > p.stages ? issued - p.stages : 0); j < issued; ++j)
           mbar_wait(&full_bar[j % p.stages], static_cast<uint32_t>((j / p.stages) & 1), drain);
       }
@@ -663,7 +649,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Never release TMEM while issued MMAs may still write it.
   if (warp == 1 && lane == 0) {
     volatile int never = 0;
-    WaitCtx drain{&never, p.status, p.wait_ns};
+    WaitCtx drain{&never, p.status, kDrainNs};
     mbar_wait(mma_done, 0, drain);
   }
   tc_fence_before();

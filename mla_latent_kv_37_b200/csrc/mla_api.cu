@@ -26,6 +26,25 @@ namespace {
 
 constexpr int kDc = 512, kDr = 64, kDn = 128, kDv = 128, kRowN = 576, kPageN = 64;
 constexpr uint64_t kDefaultWaitNs = 2000000000ull;  // 2 s per bounded wait
+
+// Time limit of one bounded wait inside a kernel: 2 s, or MLA_WAIT_NS (nanoseconds, >= 1) from
+// the environment, read at every call.  A small value makes the waits give up early, which is
+// how the timeout path (status bit, abort and drain, usable context afterwards) is exercised.
+uint64_t wait_limit_ns() {
+  const char* e = std::getenv("MLA_WAIT_NS");
+  if (!e || !*e) return kDefaultWaitNs;
+  char* end = nullptr;
+  const unsigned long long v = std::strtoull(e, &end, 10);
+  return (end && *end == '\0' && v >= 1) ? static_cast<uint64_t>(v) : kDefaultWaitNs;
+}
+
+// MLA_TEST_STALL=1 in the environment (read at each call): one warp of every split-KV CTA
+// first waits on a barrier nothing arrives on, so that the wait runs out and the timeout path
+// is taken.  A test hook; results of such a call are meaningless and the status says so.
+int stall_test_requested() {
+  const char* e = std::getenv("MLA_TEST_STALL");
+  return (e && e[0] == '1' && e[1] == '\0') ? 1 : 0;
+}
 constexpr int kMinPagesPerPart = 4;
 constexpr int kMaxParts = 1 << 16;  // upper bound on num_splits (host check before any arithmetic)
 constexpr int kSkMinUnits = 2;    // fewest stages' worth of weights a stream-K CTA streams
@@ -419,7 +438,7 @@ int run_streamk(const DevCtx* c, const GemmShape& s, const SkPlan& q, int n_out,
   p.positions = positions;
   p.rope_theta = theta;
   p.status = c->status;
-  p.wait_ns = kDefaultWaitNs;
+  p.wait_ns = wait_limit_ns();
   launch_pdl(sk::streamk_gemm_kernel<Epi>, dim3(q.ctas), dim3(sk::kThreads), q.smem, st, a0, a1,
              a2 ? *a2 : a1, xmap, p, epi);
   return last_launch();
@@ -528,7 +547,8 @@ int enqueue_decode(const DevCtx* c, const mla_dims* dims, const void* q_cat, con
     p.part_o = part_o;
     p.part_lse = part_lse;
     p.status = c->status;
-    p.wait_ns = kDefaultWaitNs;
+    p.wait_ns = wait_limit_ns();
+    p.stall_test = stall_test_requested();
     const bool prof = g_prof_next < g_prof_count;
     if (prof && record_profile_event(g_prof_begin[g_prof_next], st) != cudaSuccess)
       return MLA_ERR_CUDA;

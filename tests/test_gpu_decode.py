@@ -201,3 +201,22 @@ def test_query_remainder_zero_matches_plain_call():
     rel, _ = errors(o2.numpy(), o1.numpy())
     assert rel < 1e-3
     np.testing.assert_allclose(l2.numpy(), l1.numpy(), rtol=1e-4, atol=1e-4)
+
+
+def test_timeout_path_reports_and_recovers(monkeypatch):
+    """A wait that can only run out (MLA_TEST_STALL: one warp of every CTA waits on a barrier
+    nothing arrives on, with a 20 ms limit): the call reports MLA_STATUS_TIMEOUT instead of
+    hanging, the other roles unwind, and the next ordinary call, in the same context, is
+    correct."""
+    import mla_latent_kv_37_b200 as M
+    lens = [4096, 1000, 64]
+    q, cache = _case(15, lens, 128)
+    monkeypatch.setenv("MLA_TEST_STALL", "1")
+    monkeypatch.setenv("MLA_WAIT_NS", "20000000")
+    _, _, st = _run(q, cache, lens, 128)
+    assert st & M.STATUS_TIMEOUT
+    monkeypatch.delenv("MLA_TEST_STALL")
+    monkeypatch.delenv("MLA_WAIT_NS")
+    o, l, st = _run(q, cache, lens, 128)
+    assert st == 0
+    _check(q, cache, lens, o, l)

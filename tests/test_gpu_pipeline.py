@@ -175,3 +175,32 @@ def test_max_and_ragged_batch(B):
     got = wl.run_gpu()
     assert got["status"] == 0
     _check_step(wl, got, [0, B // 2, B - 1])
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_append_rope_at_position_131071(dtype):
+    """The appended row at the largest position of the long-context workload (angles up to
+    ~1.3e5 rad): the rotary part is checked against the oracle's fp64 RoPE on both arithmetic
+    paths (fp32 at 1e-5, bf16 within the row's rounding).  Only the addressed page exists: the
+    page table maps page index 2047 to pool page 0."""
+    import mla_latent_kv_37_b200 as M
+    B, D, pos = 1, 1024, 131071
+    w = I.weights(50, 16, D, dtype, with_w_o=False)
+    h = I.hidden(51, B, D, 1.0, dtype)
+    table = torch.full((B, 2048), -1, dtype=torch.int32)
+    table[0, pos // 64] = 0
+    pool = torch.zeros(1, 64, 576, dtype=dtype)
+    d = M.dims(B, 16, D, dtype)
+    ws = M.workspace(d)
+    pool_d = dev(pool)
+    M.mla_cache_append(d, dev(h), dev(w.w_dkv), dev(w.w_kr), dev(torch.tensor([pos], dtype=torch.int32)),
+                       dev(table), pool_d, ws)
+    assert M.mla_get_status() == 0
+    got = to_np(pool_d.cpu()[0, pos % 64])
+    c_kv, k_r = O.latent_row(h[0], w.w_dkv, w.w_kr, pos)
+    exp = np.concatenate([c_kv, k_r])
+    if dtype == torch.float32:
+        np.testing.assert_allclose(got, exp, rtol=1e-5, atol=1e-5 * np.abs(exp).max())
+    else:
+        # bf16 storage: within one rounding (2^-8 relative) of the exact value
+        assert np.all(np.abs(got - exp) <= 2.0 ** -8 * np.abs(exp) + 1e-5)

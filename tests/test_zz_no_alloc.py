@@ -70,3 +70,34 @@ def test_static_scratch_rejects_oversize():
     # The rejected call launched nothing; a following call that fits still works.
     o_ref, l_ref, o_new, l_new = _both(31, [300, 129], H, torch.bfloat16, 3)
     assert_close(to_np(o_new), to_np(o_ref), torch.bfloat16, "after rejection")
+
+
+def test_static_scratch_matches_oracle():
+    # The static-scratch call on its own, against the oracle's latent-space attention (not
+    # only against the workspace path, which runs the same kernels).
+    import mla_latent_kv_37_b200 as M
+    from tests.gpu_common import latent_reference
+    history = [700, 64, 129, 1]
+    B, H = len(history), 128
+    q = I.query_cat(41, B, H)
+    cache = I.paged_cache(42, history, history)
+    d = M.dims(B, H)
+    o = torch.full((B, H, 512), float("nan"), dtype=torch.float32, device="cuda")
+    M.mla_decode_attn_static_scratch(d, dev(q), dev(cache.pool), dev(cache.page_table),
+                                     dev(torch.tensor(history, dtype=torch.int32)), o,
+                                     num_splits=5)
+    assert M.mla_get_status() == 0
+    ref, _ = latent_reference(q, cache, history)
+    for b in range(B):
+        assert_close(to_np(o[b]), ref[b], torch.bfloat16, f"o_lat b={b}")
+
+
+def test_static_scratch_near_capacity():
+    # 128 sequences x 128 heads split into 127 parts: the plan and partials fill the fixed
+    # array to within a fraction of a percent of MLA_STATIC_SCRATCH_BYTES, so its far end is
+    # written and read; the result must match the workspace path and leave no NaN behind.
+    history = [256] * 128
+    o_ref, l_ref, o_new, l_new = _both(61, history, 128, torch.bfloat16, 127)
+    assert not torch.isnan(o_new).any() and not torch.isnan(l_new).any()
+    assert_close(to_np(o_new), to_np(o_ref), torch.bfloat16, "near capacity")
+    assert_close(to_np(l_new), to_np(l_ref), torch.bfloat16, "near capacity lse")
