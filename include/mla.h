@@ -189,6 +189,22 @@ int mla_out_proj(const mla_dims* dims, const float* o_lat, const void* w_uv, con
                  mla_stream_t stream);
 
 /*
+ * mla_merge_partials -- merge attention results computed apart over disjoint parts of the
+ * cached rows, e.g. one per GPU when a long sequence's pages are spread over several GPUs
+ * (split-KV across devices; each GPU runs mla_decode_attn over its own pages and the results
+ * are gathered).  For every (b, h):
+ *   lse = log sum_r exp(lse_r),   o_lat = sum_r exp(lse_r - lse) o_lat_r
+ * ([LP] "Classic attention ...": softmax over the union of the parts equals this weighting of
+ * the parts' softmaxes; the same merge the decode call applies to its own split-KV parts).
+ *   part_o   [n_parts, B, H, d_c] fp32, each normalised (mla_decode_attn's o_lat).
+ *   part_lse [n_parts, B, H] fp32 (mla_decode_attn's lse); -inf marks a part without rows.
+ *   o_lat    [B, H, d_c] fp32;  lse [B, H] fp32, nullable.  Rows whose parts are all empty
+ *            get o_lat = 0, lse = -inf.
+ */
+int mla_merge_partials(const mla_dims* dims, int32_t n_parts, const float* part_o,
+                       const float* part_lse, float* o_lat, float* lse, mla_stream_t stream);
+
+/*
  * mla_decode_attn_static_scratch -- mla_decode_attn for callers that cannot allocate device
  * memory.  (The MLA pages have no counterpart to this: it is a deployment convenience.)
  * A process whose memory manager already owns all of the GPU's memory, or a code path where a

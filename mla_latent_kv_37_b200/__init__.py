@@ -70,6 +70,7 @@ _SIGS = {
     "mla_decode_attn_static_scratch": (ctypes.c_int, [ctypes.POINTER(mla_dims), _P, _P, _P, _I,
                                                       _P, _I, _P, ctypes.c_float, _I, _P, _P,
                                                       _P]),
+    "mla_merge_partials": (ctypes.c_int, [ctypes.POINTER(mla_dims), _I, _P, _P, _P, _P, _P]),
     "mla_get_status": (ctypes.c_int, [_P]),
     "mla_error_string": (ctypes.c_char_p, [ctypes.c_int]),
     "mla_error_detail": (ctypes.c_char_p, []),
@@ -266,6 +267,18 @@ def mla_out_proj(d: mla_dims, o_lat, w_uv, ws, w_o=None, o_heads=None, out=None,
     rc = lib().mla_out_proj(ctypes.byref(d), _ptr(o_lat), _ptr(w_uv), _ptr(w_o), _ptr(o_heads),
                             _ptr(out), _ptr(ws), ws.numel(), _stream(stream))
     _check(rc, "mla_out_proj")
+
+
+def mla_merge_partials(d: mla_dims, part_o, part_lse, o_lat, lse=None, stream=None):
+    """Merge partial attention results [n, B, H, 512] / [n, B, H] into o_lat / lse."""
+    n = part_o.shape[0]
+    _need(part_o, "part_o", torch.float32, (n, d.batch, d.n_heads, d.d_c))
+    _need(part_lse, "part_lse", torch.float32, (n, d.batch, d.n_heads))
+    _need(o_lat, "o_lat", torch.float32, (d.batch, d.n_heads, d.d_c))
+    _need(lse, "lse", torch.float32, (d.batch, d.n_heads))
+    rc = lib().mla_merge_partials(ctypes.byref(d), n, _ptr(part_o), _ptr(part_lse), _ptr(o_lat),
+                                  _ptr(lse), _stream(stream))
+    _check(rc, "mla_merge_partials")
 
 
 def mla_get_status(stream=None) -> int:

@@ -1022,5 +1022,60 @@ __global__ void __launch_bounds__(32 * kCombineWarps)
   if (lane == 0 && lse) lse[static_cast<size_t>(b) * H + h] = m + __logf(tot);
 }
 
+// ------------------------------------------------------------------------------------------
+// Merge of partial results that were computed apart (e.g. one per GPU, each over a range of a
+// sequence's pages): part_o [n][rows][512] normalised, part_lse [n][rows]; for every row
+//     lse = log sum_r exp(lse_r),   o = sum_r exp(lse_r - lse) o_r,
+// the same log-sum-exp weights as the combine kernel.  A part with lse = -inf (no tokens)
+// weighs nothing; a row whose parts are all empty gets o = 0, lse = -inf.
+// ------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(32 * kCombineWarps)
+    merge_kernel(int n, int rows, const float* __restrict__ part_o,
+                 const float* __restrict__ part_lse, float* __restrict__ o_lat,
+                 float* __restrict__ lse) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const int row = blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const float NEG_INF = -__int_as_float(0x7f800000);
+  float m = NEG_INF;
+  for (int r = lane; r < n; r += 32) m = fmaxf(m, part_lse[static_cast<size_t>(r) * rows + row]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float4* out = reinterpret_cast<float4*>(o_lat + static_cast<size_t>(row) * 512);
+  if (m == NEG_INF) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) out[lane + 32 * k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (lane == 0 && lse) lse[row] = NEG_INF;
+    return;
+  }
+  float tot = 0.f;
+  float4 acc[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int r = 0; r < n; ++r) {
+    const float l = part_lse[static_cast<size_t>(r) * rows + row];
+    if (l == NEG_INF) continue;  // warp-uniform
+    const float w = __expf(l - m);
+    tot += w;
+    const float4* src = reinterpret_cast<const float4*>(
+        part_o + (static_cast<size_t>(r) * rows + row) * 512);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float4 v = src[lane + 32 * k];
+      acc[k].x += w * v.x;
+      acc[k].y += w * v.y;
+      acc[k].z += w * v.z;
+      acc[k].w += w * v.w;
+    }
+  }
+  const float inv = 1.f / tot;
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    out[lane + 32 * k] = make_float4(acc[k].x * inv, acc[k].y * inv, acc[k].z * inv, acc[k].w * inv);
+  if (lane == 0 && lse) lse[row] = m + __logf(tot);
+}
+
 }  // namespace attn
 }  // namespace mla

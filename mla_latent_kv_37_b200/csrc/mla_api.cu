@@ -869,6 +869,25 @@ int mla_out_proj(const mla_dims* dims, const float* o_lat, const void* w_uv, con
   return MLA_OK;
 }
 
+int mla_merge_partials(const mla_dims* dims, int32_t n_parts, const float* part_o,
+                       const float* part_lse, float* o_lat, float* lse, mla_stream_t stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (!part_o || !part_lse || !o_lat) return MLA_ERR_NULL_ARG;
+  if (n_parts < 1 || n_parts > kMaxParts) return MLA_ERR_ARG;
+  if (!aligned(part_o, 16) || !aligned(o_lat, 16) || !aligned(part_lse, 4) ||
+      (lse && !aligned(lse, 4)))
+    return MLA_ERR_ALIGN;
+  DevCtx* c = nullptr;
+  if ((rc = device_ctx(&c))) return rc;
+  const int rows = dims->batch * dims->n_heads;
+  launch_pdl(attn::merge_kernel,
+             dim3(static_cast<unsigned>((rows + attn::kCombineWarps - 1) / attn::kCombineWarps)),
+             dim3(32 * attn::kCombineWarps), 0, reinterpret_cast<cudaStream_t>(stream), n_parts,
+             rows, part_o, part_lse, o_lat, lse);
+  return last_launch();
+}
+
 int mla_get_status(mla_stream_t stream) {
   DevCtx* c = nullptr;
   int rc = device_ctx(&c);

@@ -114,3 +114,15 @@ class Workload:
         hist = O.gather_rows(self.cache.pool, self.cache.page_table[b].numpy(), self.history[b])
         return O.decode_step(self.h[b], self.w, hist, self.history[b], self.H,
                              round_row=round_to(self.dtype), heads=heads, with_out=with_out)
+
+
+def _check_all(q_exact, cache, lens, o_lat, lse, dtype=torch.bfloat16):
+    """o_lat / lse of every sequence against the oracle's latent-space attention."""
+    ref_o, ref_l = latent_reference(q_exact, cache, lens)
+    for b, n in enumerate(lens):
+        if n == 0:
+            assert torch.all(o_lat[b] == 0)
+            assert torch.all(torch.isneginf(lse[b]))
+            continue
+        assert_close(o_lat[b].double().numpy(), ref_o[b], dtype, f"o_lat b={b} n={n}")
+        np.testing.assert_allclose(lse[b].double().numpy(), ref_l[b], rtol=2e-4, atol=2e-4)

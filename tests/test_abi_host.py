@@ -153,3 +153,14 @@ def test_error_strings(M):
     for code in (0, -1, -2, -3, -4, -5, -6, -7, 1, 4):
         assert L.mla_error_string(code)
     assert b"sm_100a" in L.mla_version()
+
+
+def test_merge_partials_arguments(M):
+    d = _d(M)
+    L = M.lib()
+    f = ctypes.c_void_p(0x10000)
+    odd = ctypes.c_void_p(0x10008)
+    assert L.mla_merge_partials(ctypes.byref(d), 0, f, f, f, None, None) == -5
+    assert L.mla_merge_partials(ctypes.byref(d), 2, None, f, f, None, None) == -1
+    assert L.mla_merge_partials(ctypes.byref(d), 2, odd, f, f, None, None) == -3
+    assert L.mla_merge_partials(ctypes.byref(_d(M, d_c=256)), 2, f, f, f, None, None) == -2
