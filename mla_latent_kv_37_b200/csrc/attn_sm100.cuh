@@ -11,30 +11,28 @@
 // ([128 x 64] x [64 x 512]).  O (128 x 512 fp32) alone would fill a whole SM's tensor memory,
 // so each work unit runs on a CLUSTER OF TWO CTAs that split the 576 columns of every row:
 // CTA r owns latent columns [256r, 256r+256) and RoPE columns [512+32r, 512+32r+32).
-//   * TMEM (512 columns): O half 256 | query latent half 128 (A operand of QK) | S 128, the
-//     scores of a pair of pages.  QK runs once per page pair (N = 128; the tensor core needs
-//     N >= 128 for its full rate), PV once per page (N = 256).
-//   * Pages arrive by TMA into a 4-slot ring laid out box-major, so the rows of two adjacent
-//     slots form one N = 128 operand.  Four pages ahead of the ring each CTA issues a bulk L2
-//     prefetch of half of the page's rows, so the ring's loads find their lines in L2.
-//   * S_r = Q_r C_r^T is a partial score, and the softmax of a row needs both CTAs' partials.
-//     CTA r runs the softmax for half of the rows only (in every warp's 32 TMEM lanes, the 16
-//     lanes 16r .. 16r+15), two threads per row, 32 columns each (the 16x32bx2 TMEM load), so
-//     each SM does half the exponentials.  Per page:
-//       - the send warps read the PEER's rows of S, quantise them to 16-bit fixed point
-//         relative to the row's largest magnitude (error <= 2^-16 of it, ~1e-4 in a logit) and
-//         store them straight from registers into the peer's receive buffer (st.async,
-//         completion counted in bytes on the peer's mbarrier; double-buffered by page);
-//       - the softmax warps add the peer's partial to their own rows, run the online softmax,
-//         and write their rows of P both into their own P buffer and into the peer's, with each
-//         row's rescale factor;
-//       - once the peer's rows of P have landed, PV runs; its completion is committed to both
-//         CTAs' barriers (multicast commit), which frees the P buffers on both sides.
-//     A row's running maximum and sum live with the CTA that owns the row; the other CTA gets
-//     the factor whenever the maximum moves (to rescale its half of O) and the final (max, sum)
-//     at the end of a segment (to normalise its half of O).
-//   * The MMA warp issues from an event loop: each page group's QK as soon as its pages have
-//     landed and S is free, each page's PV as soon as P is complete, whichever comes first.
+//   * TMEM (512 columns): O half 256 | query latent half 128 (A operand of QK) | S of two
+//     pages, 2 x 64 (page parity), so the QK of page t+1 never waits for the softmax of page t.
+//   * Pages arrive by TMA into a 4-slot ring laid out box-major.  Four pages ahead of the ring
+//     each CTA issues a bulk L2 prefetch of its half of the page's rows, so the ring's loads
+//     find their lines in L2.
+//   * S_r = Q_r C_r^T is a partial score; every row's softmax needs both CTAs' partials.  Both
+//     CTAs run the same softmax over all 128 rows (symmetric), so each holds the full P of the
+//     page for its own PV and no P or rescale factor crosses the pair.  Per page:
+//       - four send warps (one per TMEM quarter, one thread per row) read this CTA's partial,
+//         quantise it to 16-bit fixed point relative to the row's largest magnitude (error
+//         <= 2^-16 of it, ~1e-4 in a logit) and store it straight from registers into the
+//         peer's receive buffer (st.async, completion counted in bytes on the peer's
+//         mbarrier; two receive buffers, by page parity);
+//       - eight softmax warps, two per TMEM quarter, each own 16 whole rows (two threads per
+//         row, 32 columns each: the 16x32bx2 TMEM load), so a row's maximum and sum take one
+//         shuffle.  They add the peer's decoded partial to their own, run the online softmax
+//         on packed f32x2 arithmetic, write P (bf16) into the page's P buffer, rescale their
+//         rows of O when needed, and hand the receive buffer back to the peer;
+//       - PV runs as soon as P is complete; its completion frees the P buffer and the slot.
+//   * The MMA warp issues from an event loop with precomputed descriptors: each page's QK as
+//     soon as the page has landed and its S buffer is free, each PV as soon as its P is
+//     written, whichever comes first; it backs off with nanosleep while idle.
 //   * The next segment's query half goes into TMEM as soon as the last QK of the previous one
 //     has run, before that segment's epilogue, so a sequence boundary costs no pipeline drain.
 //
@@ -55,10 +53,10 @@
 // doubles; the page bytes are read by the part's clusters at about the same time and mostly
 // come from L2 the second time.
 //
-// Roles (320 threads): warps 0-3 softmax (own rows), query load, O rescale and epilogue;
-// warps 4-7 send; warp 8 TMA producer; warp 9 MMA issuer and TMEM owner.  The online softmax
-// keeps a per-row reference maximum and rescales O only when the running maximum grows by
-// more than 2^8.
+// Roles (448 threads, 128 registers each): warps 0-7 softmax, query load (warps 0-3), O
+// rescale and epilogue; warps 8-11 send; warp 12 TMA producer; warp 13 MMA issuer and TMEM
+// owner.  The online softmax keeps a per-row reference maximum and rescales O only when the
+// running maximum grows by more than 2^8.
 #pragma once
 #include "ptx_sm100.cuh"
 
