@@ -669,10 +669,10 @@ def main():
                 "hbm_gbs": r["gbs"], "hbm_frac": r["hbm_frac"],
                 "tflops": r["tflops"],
                 "tensor_frac": r["tensor_frac_sustained"],
-                "tensor_frac_label": "achieved TFLOP/s / measured sustained bf16 GEMM rate",
+                "tensor_frac_label": f"achieved TFLOP/s / sustained bf16 GEMM rate, {peak_src}",
                 "tensor_frac_burst": r["tensor_frac_burst"],
-                "tensor_frac_burst_label": "achieved TFLOP/s / measured burst bf16 dense GEMM "
-                                           "rate (the dense peak a kernel timed alone reaches)",
+                "tensor_frac_burst_label": f"achieved TFLOP/s / burst bf16 dense GEMM rate (the "
+                                           f"dense peak a kernel timed alone reaches), {peak_src}",
                 "bytes_per_launch": r["bytes"], "flops_per_launch": r["flops"],
                 "roofline_us": r["roofline_us"],
                 "frac_of_roofline_time": r["frac"]}
