@@ -640,8 +640,8 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
     const int row = 32 * q + lane;
     const uint32_t lanes = static_cast<uint32_t>(32 * q) << 16;
     const uint32_t x_peer = mapa_shared(smem_u32(smem + kOffX), peer);
-    const uint32_t xfull_peer[2] = {mapa_shared(smem_u32(&bars->x_full[0]), peer),
-                                    mapa_shared(smem_u32(&bars->x_full[1]), peer)};
+    // the peer's x_full[0]; x_full[1] is the next 8 bytes
+    const uint32_t xfull_peer = mapa_shared(smem_u32(&bars->x_full[0]), peer);
     SegIter it{plan.seq_pages(), plan.seq_prefix(), p.batch, g_begin, g_end, b_begin};
     int seq, p0, p1, t = 0;
     bool ok = true;
@@ -681,9 +681,9 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
           st_async_u4(xb + xrow_off(row, c), enc_u16x2(s[8 * c], s[8 * c + 1], inv),
                       enc_u16x2(s[8 * c + 2], s[8 * c + 3], inv),
                       enc_u16x2(s[8 * c + 4], s[8 * c + 5], inv),
-                      enc_u16x2(s[8 * c + 6], s[8 * c + 7], inv), xfull_peer[pb]);
+                      enc_u16x2(s[8 * c + 6], s[8 * c + 7], inv), xfull_peer + 8 * pb);
         st_async_u1(xb + kXPayload + row * 4, __float_as_uint(mabs * (1.f / 32767.f)),
-                    xfull_peer[pb]);
+                    xfull_peer + 8 * pb);
       }
     }
     if (ok) {  // the peer's hand-backs for our last two pages land before this CTA exits
@@ -703,8 +703,8 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
     const float NEG_INF = -__int_as_float(0x7f800000);
     const uint32_t x_loc = smem_u32(smem + kOffX);
     const uint32_t p_loc = smem_u32(smem + kOffP);
-    const uint32_t xfree_rem[2] = {mapa_shared(smem_u32(&bars->x_free[0]), peer),
-                                   mapa_shared(smem_u32(&bars->x_free[1]), peer)};
+    // the peer's x_free[0]; x_free[1] is the next 8 bytes
+    const uint32_t xfree_rem = mapa_shared(smem_u32(&bars->x_free[0]), peer);
     const int hd = rows.head(row);
     const bool out_row = hd < p.n_heads && !rows.lo(row);
     // this CTA's latent half of the query rows of sequence sq -> TMEM (A operand of QK), in two
@@ -880,7 +880,7 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
           // the receive buffer was decoded long ago: warp 0 re-arms it for page t + 2 and every
           // warp hands it back (off the page's critical path)
           if (warp == 0) mbar_arrive_expect_tx(&bars->x_full[pb], kXBytes);
-          mbar_arrive_remote_relaxed(xfree_rem[pb]);
+          mbar_arrive_remote_relaxed(xfree_rem + 8 * pb);
         }
       }
       if (!ok) break;
