@@ -490,6 +490,70 @@ def run_extra_configs(dev, peaks, steps=10):
     return out
 
 
+def run_execution_modes(dev, peaks, reps=10, B=32, H=128, D=7168):
+    """The projections of one layer (cache append + query, then the output product) in the
+    absorbed form the step uses and in the folded form (W_UK multiplied into W_Q and W_UV into
+    W_O ahead of time): time per layer and weight bytes streamed.  Attention is the same in
+    both and is not timed here."""
+    import mla_latent_kv_37_b200 as M
+    import mla_inputs as I
+    d = M.dims(B, H, D)
+    w = I.weights(11, H, D, device=dev)
+    h = I.hidden(12, B, D, device=dev)
+    pos = torch.zeros(B, dtype=torch.int32, device=dev)
+    table = torch.arange(B, dtype=torch.int32, device=dev).view(B, 1)
+    pool = torch.zeros(B, 64, 576, dtype=torch.bfloat16, device=dev)
+    sq, so = M.fold_shapes(d)
+    w_qf = torch.empty(sq, dtype=torch.bfloat16, device=dev)
+    w_of = torch.empty(so, dtype=torch.bfloat16, device=dev)
+    M.mla_fold_weights(d, w_q=w.w_q, w_uk=w.w_uk, w_uv=w.w_uv, w_o=w.w_o, w_qf=w_qf, w_of=w_of)
+    ws = M.workspace(d, 0, dev)
+    q_cat = torch.empty(B, H, 576, dtype=torch.bfloat16, device=dev)
+    o_lat = torch.randn(B, H, 512, dtype=torch.float32, device=dev)
+    o_heads = torch.empty(B, H, 128, dtype=torch.bfloat16, device=dev)
+    out = torch.empty(B, D, dtype=torch.bfloat16, device=dev)
+
+    def absorbed():
+        M.mla_append_absorb(d, h, w.w_dkv, w.w_kr, w.w_q, w.w_uk, pos, table, pool, q_cat, ws)
+        M.mla_out_proj(d, o_lat, w.w_uv, ws, w_o=w.w_o, o_heads=o_heads, out=out)
+
+    def folded():
+        M.mla_append_absorb_folded(d, h, w.w_dkv, w.w_kr, w_qf, pos, table, pool, q_cat, ws)
+        M.mla_out_proj_folded(d, o_lat, w_of, out, ws)
+
+    def nbytes(*ts):
+        return sum(t.numel() * t.element_size() for t in ts)
+
+    res = {}
+    for name, fn, wbytes in (
+            ("absorbed", absorbed, nbytes(w.w_dkv, w.w_kr, w.w_q, w.w_uk, w.w_uv, w.w_o)),
+            ("folded", folded, nbytes(w.w_dkv, w.w_kr, w_qf, w_of))):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e3)
+        us = sorted(ts)[len(ts) // 2]
+        gbs = wbytes / (us * 1e-6) / 1e9
+        res[name] = {"us_per_layer": us, "weight_bytes_per_layer": wbytes, "gbs": gbs,
+                     "hbm_frac": gbs / peaks.get("hbm_gbs", 6650.0)}
+    st = M.mla_get_status()
+    if st:
+        raise RuntimeError(f"device status {st:#x} in the execution-mode measurement")
+    res["what"] = ("projections of one layer (cache append + query, output product) at "
+                   f"B={B}, H={H}, D={D}, median of {reps}; attention is identical in both")
+    res["folded_over_absorbed_time"] = res["folded"]["us_per_layer"] / res["absorbed"]["us_per_layer"]
+    del w, w_qf, w_of, ws
+    torch.cuda.empty_cache()
+    return res
+
+
 def config_block(cfg, lens, world):
     """The workload description both arms print (identical for the same configuration)."""
     B, L = cfg["batch"], cfg["layers"]
@@ -713,13 +777,14 @@ def main():
         cpu = cpu_baseline_from(sec, cfg, heads_timed, wall)
 
     # ---------------- the other configurations and the attention sweep (one GPU) ----------
-    configs = sweep = None
+    configs = sweep = modes = None
     if rank == 0 and world == 1 and not args.no_extras:
         del layers, h, step
         torch.cuda.synchronize()
         torch.cuda.empty_cache()
         configs = run_extra_configs(dev, peaks)
         sweep = compact_sweep(dev, peaks)
+        modes = run_execution_modes(dev, peaks)
 
     if rank == 0:
         line = {
@@ -734,7 +799,7 @@ def main():
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": int(launches), "clocks": clocks, "parity": parity,
             "attention_us_per_layer": roofline["us_per_launch"],
-            "configs": configs, "attention_sweep": sweep,
+            "configs": configs, "attention_sweep": sweep, "execution_modes": modes,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

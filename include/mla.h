@@ -205,6 +205,43 @@ int mla_merge_partials(const mla_dims* dims, int32_t n_parts, const float* part_
                        const float* part_lse, float* o_lat, float* lse, mla_stream_t stream);
 
 /*
+ * Folded execution mode (bf16 only).  The absorbed form multiplies by W_UK_h and W_UV_h at
+ * every step; the associativity that allows it ([LP] "MLA: compress the pair, not the heads":
+ * Q K^T = (Q W_UK^T) c^T) also allows multiplying the weights together once, ahead of time
+ * ([IA] "O preço da economia: mais contas": the mode that reuses pre-multiplied matrices).  For
+ * decode the folded matrices are larger (576 x D per head instead of 192 x D plus 128 x 512,
+ * and D x 512 per head instead of D x 128 plus 128 x 512), so every step streams more weight
+ * bytes; the mode exists to measure that trade.
+ *
+ * mla_fold_weights -- the one-time folding, fp32 accumulation, bf16 (round to nearest even):
+ *   w_qf [H, d_c + d_R, D]: rows m < d_c of head h = sum_k W_UK[h*d_nope + k][m] W_Q[h*192 + k]
+ *                           (W_UK_h^T W_Q,nope,h); rows d_c + i = W_Q[h*192 + d_nope + i].
+ *   w_of [D, H*d_c]:        column h*d_c + m = sum_k W_O[:, h*d_v + k] W_UV[h*d_v + k][m].
+ *   Either output may be NULL (then its two inputs may be NULL too).  Caller-owned buffers.
+ */
+int mla_fold_weights(const mla_dims* dims, const void* w_q, const void* w_uk, const void* w_uv,
+                     const void* w_o, void* w_qf, void* w_of, mla_stream_t stream);
+
+/*
+ * mla_append_absorb_folded -- mla_append_absorb with the folded query weights: one product
+ * [W_DKV; W_KR; W_QF] h writes the cache row (as mla_cache_append) and
+ *   q_cat[b][h][m] = (W_QF h)[h*576 + m],  m < d_c;   q_cat[b][h][d_c..] = RoPE(rows d_c..).
+ *   q_lo optional, as in mla_absorb_q.  Same arguments otherwise; bf16 only (MLA_ERR_ARG).
+ */
+int mla_append_absorb_folded(const mla_dims* dims, const void* h, const void* w_dkv,
+                             const void* w_kr, const void* w_qf, const int32_t* positions,
+                             const int32_t* page_table, int32_t max_pages, void* cache_pool,
+                             int32_t num_pages, void* q_cat, void* q_lo, void* workspace,
+                             size_t workspace_bytes, mla_stream_t stream);
+
+/*
+ * mla_out_proj_folded -- out[b] = W_OF o_lat[b] (o_lat flattened to H*d_c), the output of
+ * mla_out_proj without the per-head o_heads.  o_lat fp32 [B, H, d_c]; out [B, D] bf16.
+ */
+int mla_out_proj_folded(const mla_dims* dims, const float* o_lat, const void* w_of, void* out,
+                        void* workspace, size_t workspace_bytes, mla_stream_t stream);
+
+/*
  * mla_decode_attn_static_scratch -- mla_decode_attn for callers that cannot allocate device
  * memory.  (The MLA pages have no counterpart to this: it is a deployment convenience.)
  * A process whose memory manager already owns all of the GPU's memory, or a code path where a

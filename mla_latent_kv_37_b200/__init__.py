@@ -71,6 +71,10 @@ _SIGS = {
                                                       _P, _I, _P, ctypes.c_float, _I, _P, _P,
                                                       _P]),
     "mla_merge_partials": (ctypes.c_int, [ctypes.POINTER(mla_dims), _I, _P, _P, _P, _P, _P]),
+    "mla_fold_weights": (ctypes.c_int, [ctypes.POINTER(mla_dims), _P, _P, _P, _P, _P, _P, _P]),
+    "mla_append_absorb_folded": (ctypes.c_int, [ctypes.POINTER(mla_dims), _P, _P, _P, _P, _P,
+                                                _P, _I, _P, _I, _P, _P, _P, _SZ, _P]),
+    "mla_out_proj_folded": (ctypes.c_int, [ctypes.POINTER(mla_dims), _P, _P, _P, _P, _SZ, _P]),
     "mla_get_status": (ctypes.c_int, [_P]),
     "mla_error_string": (ctypes.c_char_p, [ctypes.c_int]),
     "mla_error_detail": (ctypes.c_char_p, []),
@@ -267,6 +271,64 @@ def mla_out_proj(d: mla_dims, o_lat, w_uv, ws, w_o=None, o_heads=None, out=None,
     rc = lib().mla_out_proj(ctypes.byref(d), _ptr(o_lat), _ptr(w_uv), _ptr(w_o), _ptr(o_heads),
                             _ptr(out), _ptr(ws), ws.numel(), _stream(stream))
     _check(rc, "mla_out_proj")
+
+
+def fold_shapes(d: mla_dims):
+    """Shapes of the folded weights: (w_qf [H, d_c + d_R, D], w_of [D, H * d_c])."""
+    H = d.n_heads
+    return (H, d.d_c + d.d_rope, d.d_model), (d.d_model, H * d.d_c)
+
+
+def mla_fold_weights(d: mla_dims, w_q=None, w_uk=None, w_uv=None, w_o=None, w_qf=None,
+                     w_of=None, stream=None):
+    """The one-time folding of the folded execution mode (bf16): W_UK into W_Q, W_UV into W_O."""
+    e = _elem(d)
+    H = d.n_heads
+    sq, so = fold_shapes(d)
+    _need(w_q, "w_q", e, (H * (d.d_nope + d.d_rope), d.d_model))
+    _need(w_uk, "w_uk", e, (H * d.d_nope, d.d_c))
+    _need(w_uv, "w_uv", e, (H * d.d_v, d.d_c))
+    _need(w_o, "w_o", e, (d.d_model, H * d.d_v))
+    _need(w_qf, "w_qf", e, sq)
+    _need(w_of, "w_of", e, so)
+    rc = lib().mla_fold_weights(ctypes.byref(d), _ptr(w_q), _ptr(w_uk), _ptr(w_uv), _ptr(w_o),
+                                _ptr(w_qf), _ptr(w_of), _stream(stream))
+    _check(rc, "mla_fold_weights")
+
+
+def mla_append_absorb_folded(d: mla_dims, h, w_dkv, w_kr, w_qf, positions, page_table,
+                             cache_pool, q_cat, ws, q_lo=None, stream=None):
+    """Cache append and the folded query in one projection launch (bf16)."""
+    e = _elem(d)
+    H = d.n_heads
+    _need(h, "h", e, (d.batch, d.d_model))
+    _need(w_dkv, "w_dkv", e, (d.d_c, d.d_model))
+    _need(w_kr, "w_kr", e, (d.d_rope, d.d_model))
+    _need(w_qf, "w_qf", e, fold_shapes(d)[0])
+    _need(positions, "positions", torch.int32, (d.batch,))
+    _need(page_table, "page_table", torch.int32)
+    _need(cache_pool, "cache_pool", e)
+    _need(q_cat, "q_cat", e, (d.batch, H, d.d_c + d.d_rope))
+    _need(q_lo, "q_lo", torch.bfloat16, (d.batch, H, d.d_c + d.d_rope))
+    _need(ws, "workspace", torch.uint8)
+    rc = lib().mla_append_absorb_folded(ctypes.byref(d), _ptr(h), _ptr(w_dkv), _ptr(w_kr),
+                                        _ptr(w_qf), _ptr(positions), _ptr(page_table),
+                                        page_table.shape[1], _ptr(cache_pool),
+                                        cache_pool.shape[0], _ptr(q_cat), _ptr(q_lo), _ptr(ws),
+                                        ws.numel(), _stream(stream))
+    _check(rc, "mla_append_absorb_folded")
+
+
+def mla_out_proj_folded(d: mla_dims, o_lat, w_of, out, ws, stream=None):
+    """out = W_OF o_lat with the folded output weights (bf16)."""
+    e = _elem(d)
+    _need(o_lat, "o_lat", torch.float32, (d.batch, d.n_heads, d.d_c))
+    _need(w_of, "w_of", e, fold_shapes(d)[1])
+    _need(out, "out", e, (d.batch, d.d_model))
+    _need(ws, "workspace", torch.uint8)
+    rc = lib().mla_out_proj_folded(ctypes.byref(d), _ptr(o_lat), _ptr(w_of), _ptr(out), _ptr(ws),
+                                   ws.numel(), _stream(stream))
+    _check(rc, "mla_out_proj_folded")
 
 
 def mla_merge_partials(d: mla_dims, part_o, part_lse, o_lat, lse=None, stream=None):

@@ -229,15 +229,57 @@ struct EpiWq {
   }
 };
 
+// Folded query: with W_UK absorbed into W_Q offline, the folded matrix has 576 rows per head
+// (512 latent rows W_UK_h^T W_Q,nope,h, then W_Q's 64 RoPE rows) and its product with h maps
+// row for row onto q_cat[b][h][0..575]; the last 64 rows of a head are rotated at the token's
+// position.  Head boundaries and the 512 split fall on 32-row (warp) boundaries.
+struct EpiWqFold {
+  static constexpr bool kRope = true;
+  int H;
+  __nv_bfloat16* q_cat;
+  __nv_bfloat16* q_lo;
+  const int32_t* positions;
+  float theta;
+  __host__ __device__ static size_t smem_bytes(int n) {
+    return static_cast<size_t>(n) * kRopePairs * 8;
+  }
+  __device__ void prepare(uint8_t* sm, int n, int tid, int nthreads) const {
+    rope_table(reinterpret_cast<float2*>(sm), positions, n, theta, tid, nthreads);
+  }
+  __device__ void apply(const uint8_t* sm, int, int r, bool valid, int c0, int n_out,
+                        float (&v)[16]) const {
+    constexpr int kRow = 576, kDc = 512;
+    const float2* tab = reinterpret_cast<const float2*>(sm);
+    const int h = r / kRow, d = r - h * kRow;
+    const bool rope = d >= kDc;  // warp-uniform
+    float p[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) p[j] = __shfl_xor_sync(0xffffffffu, v[j], 1);
+    if (!valid) return;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int b = c0 + j;
+      if (b >= n_out) break;
+      float x = v[j];
+      if (rope) rope_rotate(tab, b, (d - kDc) >> 1, d & 1, v[j], p[j], x);
+      const size_t o = (static_cast<size_t>(b) * H + h) * kRow + d;
+      const __nv_bfloat16 e = __float2bfloat16_rn(x);
+      q_cat[o] = e;
+      if (q_lo) q_lo[o] = __float2bfloat16_rn(x - __bfloat162float(e));
+    }
+  }
+};
+
 // q_lat_h = W_UK_h^T q_nope_h (hi + lo already summed) -> q_cat[b][h][0..511] (+ q_lo).
-// Cache append and q = W_Q h in one launch (both multiply the same hidden states): rows
+// Cache append and a query product in one launch (both multiply the same hidden states): rows
 // [0, 640) are the append tiles (W_DKV then W_KR; rows 576..639 padding), rows from 640 on are
-// W_Q's.  Both use the RoPE table that EpiAppend::prepare builds at the start of the area.
-struct EpiAppendWq {
+// the query's.  Both use the RoPE table that EpiAppend::prepare builds at the start of the area.
+template <class Q>
+struct EpiAppendQ {
   static constexpr bool kRope = true;
   static constexpr int kSplitRow = 640;
   EpiAppend a;
-  EpiWq q;
+  Q q;
   __host__ __device__ static size_t smem_bytes(int n) { return EpiAppend::smem_bytes(n); }
   __device__ void prepare(uint8_t* sm, int n, int tid, int nthreads) const {
     a.prepare(sm, n, tid, nthreads);
@@ -250,6 +292,8 @@ struct EpiAppendWq {
       q.apply(sm, g, r - kSplitRow, valid, c0, n_out, v);
   }
 };
+using EpiAppendWq = EpiAppendQ<EpiWq>;
+using EpiAppendWqFold = EpiAppendQ<EpiWqFold>;
 
 struct EpiWuk {
   static constexpr bool kRope = false;

@@ -16,6 +16,7 @@
 #include "attn_f32.cuh"
 #include "attn_sm100.cuh"
 #include "epilogue.cuh"
+#include "fold.cuh"
 #include "gemm_streamk.cuh"
 
 namespace mla {
@@ -135,13 +136,14 @@ int device_ctx(DevCtx** out) {
                                   attn_smem)) != cudaSuccess)
       return cuda_fail(e, "cudaFuncSetAttribute(split_kernel)");
     const int sk_smem = static_cast<int>(kSmemPerBlockMax);
-    const void* sk_kernels[6] = {
+    const void* sk_kernels[7] = {
         reinterpret_cast<const void*>(sk::streamk_gemm_kernel<sk::EpiAppend>),
         reinterpret_cast<const void*>(sk::streamk_gemm_kernel<sk::EpiWq>),
         reinterpret_cast<const void*>(sk::streamk_gemm_kernel<sk::EpiWuk>),
         reinterpret_cast<const void*>(sk::streamk_gemm_kernel<sk::EpiWuv>),
         reinterpret_cast<const void*>(sk::streamk_gemm_kernel<sk::EpiWo>),
-        reinterpret_cast<const void*>(sk::streamk_gemm_kernel<sk::EpiAppendWq>)};
+        reinterpret_cast<const void*>(sk::streamk_gemm_kernel<sk::EpiAppendWq>),
+        reinterpret_cast<const void*>(sk::streamk_gemm_kernel<sk::EpiAppendWqFold>)};
     for (const void* k : sk_kernels)
       if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, sk_smem)) !=
           cudaSuccess)
@@ -199,6 +201,16 @@ GemmShape shape_wuv(const mla_dims* d) {
 }
 GemmShape shape_wo(const mla_dims* d) {
   return {d->d_model, (d->d_model + 127) / 128, d->n_heads * kDv, 1, 2 * round16(d->batch),
+          round16(d->batch)};
+}
+// the folded execution mode: cache append + the folded query (576 rows per head) in one
+// product, and the folded output product over all heads' latent columns (K = H * 512)
+GemmShape shape_append_wq_fold(const mla_dims* d) {
+  const int m = d->n_heads * kRowN;
+  return {sk::EpiAppendWqFold::kSplitRow + m, 5 + m / 128, d->d_model, 1, round16(d->batch), 0};
+}
+GemmShape shape_wo_fold(const mla_dims* d) {
+  return {d->d_model, (d->d_model + 127) / 128, d->n_heads * kDc, 1, 2 * round16(d->batch),
           round16(d->batch)};
 }
 
@@ -260,11 +272,13 @@ Workspace layout(const mla_dims* d, int num_parts, int sms) {
   size_t part = 0, ctr = 0;
   if (d->dtype == MLA_BF16) {
     // the same (shape, epilogue table size) pairs the launches use
-    const GemmShape shapes[6] = {shape_append(d), shape_wq(d), shape_wuk(d), shape_wuv(d),
-                                 shape_wo(d), shape_append_wq(d)};
-    const size_t epi[6] = {sk::EpiAppend::smem_bytes(d->batch), sk::EpiWq::smem_bytes(d->batch),
-                           0, 0, 0, sk::EpiAppendWq::smem_bytes(d->batch)};
-    for (int i = 0; i < 6; ++i) {
+    const GemmShape shapes[8] = {shape_append(d), shape_wq(d), shape_wuk(d),
+                                 shape_wuv(d), shape_wo(d), shape_append_wq(d),
+                                 shape_append_wq_fold(d), shape_wo_fold(d)};
+    const size_t epi[8] = {sk::EpiAppend::smem_bytes(d->batch), sk::EpiWq::smem_bytes(d->batch),
+                           0, 0, 0, sk::EpiAppendWq::smem_bytes(d->batch),
+                           sk::EpiAppendWqFold::smem_bytes(d->batch), 0};
+    for (int i = 0; i < 8; ++i) {
       const SkPlan q = sk_plan(shapes[i], epi[i], sms);
       part = std::max(part, q.partial_bytes);
       ctr = std::max(ctr, static_cast<size_t>(q.tiles) * 8);
@@ -867,6 +881,131 @@ int mla_out_proj(const mla_dims* dims, const float* o_lat, const void* w_uv, con
     }
   }
   return MLA_OK;
+}
+
+// ------------------------------------------------------------------------------------------
+// folded execution mode
+// ------------------------------------------------------------------------------------------
+int mla_fold_weights(const mla_dims* dims, const void* w_q, const void* w_uk, const void* w_uv,
+                     const void* w_o, void* w_qf, void* w_of, mla_stream_t stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (dims->dtype != MLA_BF16) return MLA_ERR_ARG;
+  if (!w_qf && !w_of) return MLA_ERR_NULL_ARG;
+  if (w_qf && (!w_q || !w_uk)) return MLA_ERR_NULL_ARG;
+  if (w_of && (!w_uv || !w_o)) return MLA_ERR_NULL_ARG;
+  if ((w_q && !aligned(w_q, 16)) || (w_uk && !aligned(w_uk, 16)) || (w_uv && !aligned(w_uv, 16)) ||
+      (w_o && !aligned(w_o, 16)) || (w_qf && !aligned(w_qf, 16)) || (w_of && !aligned(w_of, 16)))
+    return MLA_ERR_ALIGN;
+  DevCtx* c = nullptr;
+  if ((rc = device_ctx(&c))) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int D = dims->d_model, H = dims->n_heads;
+  using fold::kTile;
+  const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(w_q);
+  const __nv_bfloat16* uk = static_cast<const __nv_bfloat16*>(w_uk);
+  const __nv_bfloat16* uv = static_cast<const __nv_bfloat16*>(w_uv);
+  const __nv_bfloat16* o = static_cast<const __nv_bfloat16*>(w_o);
+  if (w_qf) {
+    __nv_bfloat16* qf = static_cast<__nv_bfloat16*>(w_qf);
+    // rows m < 512 of head h: sum_k W_UK[h*128 + k][m] W_Q[h*192 + k][:]
+    fold::batched_gemm_kernel<<<dim3((D + kTile - 1) / kTile, kDc / kTile, H), fold::kThreads, 0,
+                                st>>>(uk, static_cast<long long>(kDn) * kDc, 1, kDc, q,
+                                      static_cast<long long>(kDn + kDr) * D, D, 1, qf,
+                                      static_cast<long long>(kRowN) * D, D, 1, kDc, D, kDn);
+    if ((rc = last_launch())) return rc;
+    // rows 512..575 of head h: W_Q's RoPE rows as they are
+    fold::copy_rows_kernel<<<1024, 256, 0, st>>>(q + static_cast<size_t>(kDn) * D,
+                                                 static_cast<long long>(kDn + kDr) * D,
+                                                 qf + static_cast<size_t>(kDc) * D,
+                                                 static_cast<long long>(kRowN) * D, H, kDr, D);
+    if ((rc = last_launch())) return rc;
+  }
+  if (w_of) {
+    // column h*512 + m of row n: sum_k W_O[n][h*128 + k] W_UV[h*128 + k][m]
+    fold::batched_gemm_kernel<<<dim3(kDc / kTile, (D + kTile - 1) / kTile, H), fold::kThreads, 0,
+                                st>>>(o, kDv, static_cast<long long>(H) * kDv, 1, uv,
+                                      static_cast<long long>(kDv) * kDc, kDc, 1,
+                                      static_cast<__nv_bfloat16*>(w_of), kDc,
+                                      static_cast<long long>(H) * kDc, 1, D, kDc, kDv);
+    if ((rc = last_launch())) return rc;
+  }
+  return MLA_OK;
+}
+
+int mla_append_absorb_folded(const mla_dims* dims, const void* h, const void* w_dkv,
+                             const void* w_kr, const void* w_qf, const int32_t* positions,
+                             const int32_t* page_table, int32_t max_pages, void* cache_pool,
+                             int32_t num_pages, void* q_cat, void* q_lo, void* workspace,
+                             size_t workspace_bytes, mla_stream_t stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (dims->dtype != MLA_BF16) return MLA_ERR_ARG;
+  if (!h || !w_dkv || !w_kr || !w_qf || !positions || !page_table || !cache_pool || !q_cat)
+    return MLA_ERR_NULL_ARG;
+  if (!workspace) return MLA_ERR_WORKSPACE;
+  if (max_pages < 1 || num_pages < 1) return MLA_ERR_ARG;
+  if (!aligned(h, 16) || !aligned(w_dkv, 16) || !aligned(w_kr, 16) || !aligned(w_qf, 16) ||
+      !aligned(cache_pool, 16) || !aligned(q_cat, 16) || (q_lo && !aligned(q_lo, 16)) ||
+      !aligned(positions, 4) || !aligned(page_table, 4))
+    return MLA_ERR_ALIGN;
+  if (!aligned(workspace, 256)) return MLA_ERR_ALIGN;
+  DevCtx* c = nullptr;
+  if ((rc = device_ctx(&c))) return rc;
+  const Workspace w = layout(dims, resolve_parts(0, c), c->sms);
+  if (workspace_bytes < w.total) return MLA_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int B = dims->batch, D = dims->d_model, H = dims->n_heads;
+  char* ws = static_cast<char*>(workspace);
+  // [W_DKV; W_KR; W_QF] h in one stream-K product: cache rows + q_cat rows
+  const GemmShape s = shape_append_wq_fold(dims);
+  const SkPlan q = sk_plan(s, sk::EpiAppendWqFold::smem_bytes(B), c->sms);
+  CUtensorMap a0, a1, a2, bm;
+  if ((rc = map_weights(&a0, w_dkv, kDc, 1, D, q.kbs))) return rc;
+  if ((rc = map_weights(&a1, w_kr, kDr, 1, D, q.kbs))) return rc;
+  if ((rc = map_weights(&a2, w_qf, static_cast<uint64_t>(H) * kRowN, 1, D, q.kbs))) return rc;
+  if ((rc = map_acts(&bm, h, 1, B, D, D * 2ull, D * 2ull, s.n_pad, q.kbs))) return rc;
+  sk::EpiAppendWqFold e{
+      sk::EpiAppend{positions, page_table, max_pages, static_cast<__nv_bfloat16*>(cache_pool),
+                    num_pages, c->status, dims->rope_theta},
+      sk::EpiWqFold{H, static_cast<__nv_bfloat16*>(q_cat), static_cast<__nv_bfloat16*>(q_lo),
+                    positions, dims->rope_theta}};
+  return run_streamk(c, s, q, B, positions, dims->rope_theta, a0, a1, kDc / 128, 0, bm, ws, w, e,
+                     st, &a2, sk::EpiAppendWqFold::kSplitRow / 128);
+}
+
+int mla_out_proj_folded(const mla_dims* dims, const float* o_lat, const void* w_of, void* out,
+                        void* workspace, size_t workspace_bytes, mla_stream_t stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (dims->dtype != MLA_BF16) return MLA_ERR_ARG;
+  if (!o_lat || !w_of || !out) return MLA_ERR_NULL_ARG;
+  if (!workspace) return MLA_ERR_WORKSPACE;
+  if (!aligned(o_lat, 16) || !aligned(w_of, 16) || !aligned(out, 16)) return MLA_ERR_ALIGN;
+  if (!aligned(workspace, 256)) return MLA_ERR_ALIGN;
+  DevCtx* c = nullptr;
+  if ((rc = device_ctx(&c))) return rc;
+  const Workspace w = layout(dims, resolve_parts(0, c), c->sms);
+  if (workspace_bytes < w.total) return MLA_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int B = dims->batch, D = dims->d_model, H = dims->n_heads;
+  char* ws = static_cast<char*>(workspace);
+  __nv_bfloat16* os = reinterpret_cast<__nv_bfloat16*>(ws + w.o_split);
+  const GemmShape s = shape_wo_fold(dims);
+  const int Bp = s.n_lo;
+  const size_t n = static_cast<size_t>(B) * H * kDc;
+  // o_lat -> bf16 hi/lo planes [2][Bp][H * 512], the K layout of the folded product
+  launch_pdl(split_hi_lo_kernel,
+             dim3(static_cast<unsigned>(std::min<size_t>((n / 8 + 255) / 256, 4096))), dim3(256),
+             0, st, o_lat, n, static_cast<size_t>(Bp) * H * kDc, os);
+  if ((rc = last_launch())) return rc;
+  const uint64_t K = static_cast<uint64_t>(H) * kDc;
+  const SkPlan q = sk_plan(s, 0, c->sms);
+  CUtensorMap a, bm;
+  if ((rc = map_weights(&a, w_of, D, 1, K, q.kbs))) return rc;
+  if ((rc = map_acts(&bm, os, 1, 2 * Bp, K, K * 2, K * 2, s.n_pad, q.kbs))) return rc;
+  sk::EpiWo e{D, static_cast<__nv_bfloat16*>(out)};
+  return run_streamk(c, s, q, B, nullptr, 0.f, a, a, 1 << 30, 0, bm, ws, w, e, st);
 }
 
 int mla_merge_partials(const mla_dims* dims, int32_t n_parts, const float* part_o,

@@ -164,3 +164,42 @@ def test_merge_partials_arguments(M):
     assert L.mla_merge_partials(ctypes.byref(d), 2, None, f, f, None, None) == -1
     assert L.mla_merge_partials(ctypes.byref(d), 2, odd, f, f, None, None) == -3
     assert L.mla_merge_partials(ctypes.byref(_d(M, d_c=256)), 2, f, f, f, None, None) == -2
+
+
+def test_folded_mode_arguments(M):
+    """The folded execution mode is bf16 only and checks its pointers on the host."""
+    import torch
+    d = _d(M)
+    d32 = M.dims(4, 16, 1024, dtype=torch.float32)
+    L = M.lib()
+    f = ctypes.c_void_p(0x10000)
+    odd = ctypes.c_void_p(0x10008)
+    ws = ctypes.c_void_p(0x100000)
+    big = ctypes.c_size_t(1 << 40)
+    # folding: fp32 rejected; nothing to fold; an output without its inputs; misaligned
+    assert L.mla_fold_weights(ctypes.byref(d32), f, f, f, f, f, f, None) == -5
+    assert L.mla_fold_weights(ctypes.byref(d), f, f, f, f, None, None, None) == -1
+    assert L.mla_fold_weights(ctypes.byref(d), None, f, None, None, f, None, None) == -1
+    assert L.mla_fold_weights(ctypes.byref(d), None, None, f, None, None, f, None) == -1
+    assert L.mla_fold_weights(ctypes.byref(d), odd, f, None, None, f, None, None) == -3
+    assert L.mla_fold_weights(ctypes.byref(_d(M, d_c=256)), f, f, f, f, f, f, None) == -2
+    # folded append + query
+    args = [f, f, f, f, f, f, 4, f, 8, f, None, ws, big, None]
+    assert L.mla_append_absorb_folded(ctypes.byref(d32), *args) == -5
+    bad = list(args)
+    bad[3] = None  # w_qf
+    assert L.mla_append_absorb_folded(ctypes.byref(d), *bad) == -1
+    bad = list(args)
+    bad[3] = odd
+    assert L.mla_append_absorb_folded(ctypes.byref(d), *bad) == -3
+    bad = list(args)
+    bad[6] = 0  # max_pages
+    assert L.mla_append_absorb_folded(ctypes.byref(d), *bad) == -5
+    bad = list(args)
+    bad[11] = None  # workspace
+    assert L.mla_append_absorb_folded(ctypes.byref(d), *bad) == -4
+    # folded output product
+    assert L.mla_out_proj_folded(ctypes.byref(d32), f, f, f, ws, big, None) == -5
+    assert L.mla_out_proj_folded(ctypes.byref(d), f, None, f, ws, big, None) == -1
+    assert L.mla_out_proj_folded(ctypes.byref(d), f, f, odd, ws, big, None) == -3
+    assert L.mla_out_proj_folded(ctypes.byref(d), f, f, f, None, big, None) == -4
