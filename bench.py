@@ -742,29 +742,45 @@ def main():
                 "frac_of_roofline_time": r["frac"]}
 
     # ---------------- end-to-end through the API with host buffers ----------------
+    # The headline: the library's native step executor (mla_decode_step_host, one C-ABI call
+    # per step: page-locked host inputs in, every copy and launch made in C++, `out` back in
+    # host memory).  Beside it, the same step through the Python runner's host path replayed
+    # as one CUDA graph.
     e2e = None
     if not args.no_e2e:
         h_host = h.cpu().pin_memory()
         pos_host = pos.cpu().pin_memory()
         lens_host = lens_dev.cpu().pin_memory()
         out_host = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
-        h_dev = torch.empty_like(h)
-        p_dev, l_dev = torch.empty_like(pos), torch.empty_like(lens_dev)
-        for _ in range(2):
-            step.run_host(h_host, pos_host, lens_host, out_host, h_dev, p_dev, l_dev)
-        torch.cuda.synchronize()
-        barrier(world)
-        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        f0.record(stream)
-        for _ in range(args.steps):
-            step.run_host(h_host, pos_host, lens_host, out_host, h_dev, p_dev, l_dev)
-        f1.record(stream)
-        torch.cuda.synchronize()
-        e2e_ms = max_over_ranks(f0.elapsed_time(f1) / args.steps, world)
         bi = h_host.numel() * h_host.element_size() + 2 * B * 4
         bo = out_host.numel() * out_host.element_size()
-        e2e = {"value": tokens_per_step / (e2e_ms / 1e3), "unit": "tokens/s",
-               "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": e2e_ms}
+
+        def timed(run):
+            for _ in range(2):
+                run()
+            torch.cuda.synchronize()
+            barrier(world)
+            f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            f0.record(stream)
+            for _ in range(args.steps):
+                run()
+            f1.record(stream)
+            torch.cuda.synchronize()
+            return max_over_ranks(f0.elapsed_time(f1) / args.steps, world)
+
+        native_ms = timed(lambda: step.run_native(h_host, pos_host, lens_host, out_host))
+        h_dev = torch.empty_like(h)
+        p_dev, l_dev = torch.empty_like(pos), torch.empty_like(lens_dev)
+        graph_ms = timed(lambda: step.run_host(h_host, pos_host, lens_host, out_host, h_dev,
+                                               p_dev, l_dev))
+        st = M.mla_get_status()
+        if st:
+            raise RuntimeError(f"device status {st:#x} in the end-to-end steps")
+        e2e = {"value": tokens_per_step / (native_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": native_ms,
+               "path": "mla_decode_step_host (C ABI, page-locked host buffers, eager launches)",
+               "python_graph_host_path": {"value": tokens_per_step / (graph_ms / 1e3),
+                                          "ms_per_step": graph_ms}}
 
     # ---------------- CPU oracle baseline and parity sample (rank 0) ----------------
     cpu = None

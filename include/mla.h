@@ -242,6 +242,49 @@ int mla_out_proj_folded(const mla_dims* dims, const float* o_lat, const void* w_
                         void* workspace, size_t workspace_bytes, mla_stream_t stream);
 
 /*
+ * Native decode step over a stack of layers, end to end from host memory.
+ *
+ * mla_layer -- one layer's device-resident weights and paged cache (layouts as in the calls
+ * above; w_o must be given: the step's result is `out`).
+ *
+ * mla_step_workspace_size -- bytes of device workspace mla_decode_step_host needs: device
+ *   copies of every layer's h and out, positions, lengths, q_cat, o_lat, lse, o_heads, and the
+ *   workspace of the per-layer calls.  0 for unsupported dims or n_layers < 1.
+ *
+ * mla_decode_step_host -- for every layer l in order ([TN] MLA equations; [LP] "MLA: compress
+ * the pair, not the heads"):  mla_append_absorb -> mla_decode_attn -> mla_out_proj, with
+ *   h_host        [n_layers, B, D] (dims.dtype) host memory: layer l's hidden states,
+ *   positions_host, seq_lens_host [B] int32 host memory (the same for every layer),
+ *   out_host      [n_layers, B, D] (dims.dtype) host memory: layer l's output W_O concat_h o_h.
+ * The inputs are copied up on a copy stream ahead of the layers, each layer's output is copied
+ * back on another as soon as it is written (page-locked host memory lets the copies overlap the
+ * kernels; pageable memory works but copies synchronously), and `stream` waits for the last
+ * copy: the host buffers may be read (out) or reused (inputs) once `stream` has reached that
+ * point.  Host-detected errors return before anything is enqueued; a failure of a layer's call
+ * returns its code, with the earlier layers' work already enqueued.  Calls from several host
+ * threads on one device are serialised.
+ */
+typedef struct mla_layer {
+  const void* w_dkv;
+  const void* w_kr;
+  const void* w_q;
+  const void* w_uk;
+  const void* w_uv;
+  const void* w_o;
+  void* cache_pool;
+  int32_t num_pages;
+  const int32_t* page_table;
+  int32_t max_pages;
+} mla_layer;
+
+size_t mla_step_workspace_size(const mla_dims* dims, int32_t n_layers, int32_t num_splits);
+
+int mla_decode_step_host(const mla_dims* dims, int32_t n_layers, const mla_layer* layers,
+                         const void* h_host, const int32_t* positions_host,
+                         const int32_t* seq_lens_host, void* out_host, int32_t num_splits,
+                         void* workspace, size_t workspace_bytes, mla_stream_t stream);
+
+/*
  * mla_decode_attn_static_scratch -- mla_decode_attn for callers that cannot allocate device
  * memory.  (The MLA pages have no counterpart to this: it is a deployment convenience.)
  * A process whose memory manager already owns all of the GPU's memory, or a code path where a

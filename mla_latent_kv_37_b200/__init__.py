@@ -51,6 +51,13 @@ def dims(batch: int, n_heads: int = 128, d_model: int = 7168, dtype=torch.bfloat
                     MLA_BF16 if dtype == torch.bfloat16 else MLA_FP32, rope_theta)
 
 
+class mla_layer(ctypes.Structure):
+    _fields_ = [("w_dkv", ctypes.c_void_p), ("w_kr", ctypes.c_void_p), ("w_q", ctypes.c_void_p),
+                ("w_uk", ctypes.c_void_p), ("w_uv", ctypes.c_void_p), ("w_o", ctypes.c_void_p),
+                ("cache_pool", ctypes.c_void_p), ("num_pages", ctypes.c_int32),
+                ("page_table", ctypes.c_void_p), ("max_pages", ctypes.c_int32)]
+
+
 _lib = None
 _P = ctypes.c_void_p
 _I = ctypes.c_int32
@@ -72,6 +79,9 @@ _SIGS = {
                                                       _P]),
     "mla_merge_partials": (ctypes.c_int, [ctypes.POINTER(mla_dims), _I, _P, _P, _P, _P, _P]),
     "mla_fold_weights": (ctypes.c_int, [ctypes.POINTER(mla_dims), _P, _P, _P, _P, _P, _P, _P]),
+    "mla_step_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(mla_dims), _I, _I]),
+    "mla_decode_step_host": (ctypes.c_int, [ctypes.POINTER(mla_dims), _I, ctypes.POINTER(mla_layer),
+                                            _P, _P, _P, _P, _I, _P, _SZ, _P]),
     "mla_append_absorb_folded": (ctypes.c_int, [ctypes.POINTER(mla_dims), _P, _P, _P, _P, _P,
                                                 _P, _I, _P, _I, _P, _P, _P, _SZ, _P]),
     "mla_out_proj_folded": (ctypes.c_int, [ctypes.POINTER(mla_dims), _P, _P, _P, _P, _SZ, _P]),
@@ -271,6 +281,54 @@ def mla_out_proj(d: mla_dims, o_lat, w_uv, ws, w_o=None, o_heads=None, out=None,
     rc = lib().mla_out_proj(ctypes.byref(d), _ptr(o_lat), _ptr(w_uv), _ptr(w_o), _ptr(o_heads),
                             _ptr(out), _ptr(ws), ws.numel(), _stream(stream))
     _check(rc, "mla_out_proj")
+
+
+def layer_structs(d: mla_dims, layers):
+    """ctypes array of mla_layer for step layers (objects with the Layer fields)."""
+    e = _elem(d)
+    arr = (mla_layer * len(layers))()
+    for i, ly in enumerate(layers):
+        H = d.n_heads
+        _need(ly.w_dkv, "w_dkv", e, (d.d_c, d.d_model))
+        _need(ly.w_kr, "w_kr", e, (d.d_rope, d.d_model))
+        _need(ly.w_q, "w_q", e, (H * (d.d_nope + d.d_rope), d.d_model))
+        _need(ly.w_uk, "w_uk", e, (H * d.d_nope, d.d_c))
+        _need(ly.w_uv, "w_uv", e, (H * d.d_v, d.d_c))
+        if ly.w_o is None:
+            raise ValueError("w_o is required: the step's result is out")
+        _need(ly.w_o, "w_o", e, (d.d_model, H * d.d_v))
+        _need(ly.pool, "cache_pool", e)
+        _need(ly.page_table, "page_table", torch.int32)
+        arr[i] = mla_layer(_ptr(ly.w_dkv), _ptr(ly.w_kr), _ptr(ly.w_q), _ptr(ly.w_uk),
+                           _ptr(ly.w_uv), _ptr(ly.w_o), _ptr(ly.pool), ly.pool.shape[0],
+                           _ptr(ly.page_table), ly.page_table.shape[1])
+    return arr
+
+
+def step_workspace(d: mla_dims, n_layers: int, num_splits: int = 0, device="cuda"):
+    n = lib().mla_step_workspace_size(ctypes.byref(d), n_layers, num_splits)
+    if n == 0:
+        raise MlaError(-2, "mla_step_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def mla_decode_step_host(d: mla_dims, layer_array, h_host, positions_host, seq_lens_host,
+                         out_host, ws, num_splits: int = 0, stream=None):
+    """One decode step over len(layer_array) layers from host buffers (the native executor)."""
+    L = len(layer_array)
+    e = _elem(d)
+    for t, name, dt, shape in ((h_host, "h_host", e, (L, d.batch, d.d_model)),
+                               (positions_host, "positions_host", torch.int32, (d.batch,)),
+                               (seq_lens_host, "seq_lens_host", torch.int32, (d.batch,)),
+                               (out_host, "out_host", e, (L, d.batch, d.d_model))):
+        if t.is_cuda or not t.is_contiguous() or t.dtype != dt or tuple(t.shape) != shape:
+            raise ValueError(f"{name} must be a contiguous host tensor {dt} {shape}")
+    _need(ws, "workspace", torch.uint8)
+    rc = lib().mla_decode_step_host(ctypes.byref(d), L, layer_array, h_host.data_ptr(),
+                                    positions_host.data_ptr(), seq_lens_host.data_ptr(),
+                                    out_host.data_ptr(), num_splits, _ptr(ws), ws.numel(),
+                                    _stream(stream))
+    _check(rc, "mla_decode_step_host")
 
 
 def fold_shapes(d: mla_dims):

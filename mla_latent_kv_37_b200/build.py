@@ -9,7 +9,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libmla_b200.so")
-SOURCES = [os.path.join(HERE, "csrc", "mla_api.cu")]
+SOURCES = [os.path.join(HERE, "csrc", "mla_api.cu"), os.path.join(HERE, "csrc", "step_host.cu")]
 DEPS = [os.path.join(HERE, "csrc", f) for f in sorted(os.listdir(os.path.join(HERE, "csrc")))] + [
     os.path.join(ROOT, "include", "mla.h")]
 

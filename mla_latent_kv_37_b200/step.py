@@ -127,6 +127,18 @@ class DecodeStep:
                 out_host[l].copy_(self.out[l], non_blocking=True)
         s.wait_stream(cout)
 
+    def run_native(self, h_host, pos_host, lens_host, out_host, stream=None):
+        """End-to-end through the library's native step executor (mla_decode_step_host): the
+        host buffers go in and `out` comes back with every copy and launch made in C++."""
+        from . import layer_structs, mla_decode_step_host, step_workspace
+        if getattr(self, "_native", None) is None:
+            self._native = (layer_structs(self.dims, self.layers),
+                            step_workspace(self.dims, len(self.layers), self.num_splits,
+                                           self.ws.device))
+        arr, ws = self._native
+        mla_decode_step_host(self.dims, arr, h_host, pos_host, lens_host, out_host, ws,
+                             self.num_splits, stream)
+
     def run_host(self, h_host, pos_host, lens_host, out_host, h_dev, pos_dev, lens_dev,
                  stream=None):
         """End-to-end: the step's inputs come from pinned host memory and `out` goes back to

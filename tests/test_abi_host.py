@@ -203,3 +203,30 @@ def test_folded_mode_arguments(M):
     assert L.mla_out_proj_folded(ctypes.byref(d), f, None, f, ws, big, None) == -1
     assert L.mla_out_proj_folded(ctypes.byref(d), f, f, odd, ws, big, None) == -3
     assert L.mla_out_proj_folded(ctypes.byref(d), f, f, f, None, big, None) == -4
+
+
+def test_step_executor_arguments(M):
+    """The native step executor's host checks, before it touches CUDA."""
+    d = _d(M)
+    L = M.lib()
+    f = ctypes.c_void_p(0x10000)
+    ws = ctypes.c_void_p(0x100000)
+    big = ctypes.c_size_t(1 << 40)
+    assert L.mla_step_workspace_size(ctypes.byref(d), 0, 0) == 0
+    assert L.mla_step_workspace_size(ctypes.byref(d), 2, 0) > L.mla_step_workspace_size(
+        ctypes.byref(d), 1, 0) > L.mla_workspace_size(ctypes.byref(d), 0)
+    lay = (M.mla_layer * 2)()
+    for i in range(2):
+        lay[i] = M.mla_layer(0x10000, 0x10000, 0x10000, 0x10000, 0x10000, 0x10000, 0x10000, 8,
+                             0x10000, 4)
+    assert L.mla_decode_step_host(ctypes.byref(d), 0, lay, f, f, f, f, 0, ws, big, None) == -5
+    assert L.mla_decode_step_host(ctypes.byref(d), 2, None, f, f, f, f, 0, ws, big, None) == -1
+    assert L.mla_decode_step_host(ctypes.byref(d), 2, lay, None, f, f, f, 0, ws, big, None) == -1
+    assert L.mla_decode_step_host(ctypes.byref(d), 2, lay, f, f, f, f, 0, None, big, None) == -4
+    assert L.mla_decode_step_host(ctypes.byref(d), 2, lay, f, f, f, f, 0,
+                                  ctypes.c_void_p(0x100010), big, None) == -3
+    assert L.mla_decode_step_host(ctypes.byref(d), 2, lay, f, f, f, f, 0, ws,
+                                  ctypes.c_size_t(1024), None) == -4
+    lay[1] = M.mla_layer(0x10000, 0x10000, 0x10000, 0x10000, 0x10000, None, 0x10000, 8,
+                         0x10000, 4)
+    assert L.mla_decode_step_host(ctypes.byref(d), 2, lay, f, f, f, f, 0, ws, big, None) == -1

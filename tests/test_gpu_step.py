@@ -104,3 +104,41 @@ def test_every_layer_matches_the_oracle():
             ref = wl.oracle(b)
             assert_close(to_np(step.o_heads[l, b]), ref["o_heads"], wl.dtype, f"o_heads l={l} b={b}")
             assert_close(to_np(step.out[l, b]), ref["out"], wl.dtype, f"out l={l} b={b}")
+
+
+def test_native_step_executor_matches_device_step():
+    """mla_decode_step_host (the C++ executor: host buffers in, copies and launches in the
+    library, `out` back in host memory) gives the device-resident step's bytes, from page-locked
+    and from pageable host memory, and twice in a row on the same buffers."""
+    import mla_latent_kv_37_b200 as M
+    out_e, _ = eager_outputs()
+    wls = _workloads()
+    step, h, pos, lens = _step(wls, graph=False)
+    for pinned in (True, False):
+        h_host = h.cpu()
+        pos_host, lens_host = pos.cpu(), lens.cpu()
+        out_host = torch.full((L, B, D), float("nan"), dtype=torch.bfloat16)
+        if pinned:
+            h_host, pos_host, lens_host = (t.pin_memory() for t in (h_host, pos_host, lens_host))
+            out_host = out_host.pin_memory()
+        for _ in range(2):
+            step.run_native(h_host, pos_host, lens_host, out_host)
+            torch.cuda.synchronize()
+            assert M.mla_get_status() == 0
+            assert torch.equal(out_host, out_e)
+
+
+def test_native_step_rejects_bad_host_arguments():
+    import mla_latent_kv_37_b200 as M
+    wls = _workloads()
+    step, h, pos, lens = _step(wls, graph=False)
+    with pytest.raises(ValueError):
+        step.run_native(h, pos.cpu(), lens.cpu(), torch.empty(L, B, D, dtype=torch.bfloat16))
+    d = M.dims(B, H, D)
+    arr = M.layer_structs(d, step.layers)
+    ws = M.step_workspace(d, L)
+    small = ws[: ws.numel() // 2]
+    with pytest.raises(M.MlaError) as e:
+        M.mla_decode_step_host(d, arr, h.cpu(), pos.cpu(), lens.cpu(),
+                               torch.empty(L, B, D, dtype=torch.bfloat16), small)
+    assert e.value.code == -4
