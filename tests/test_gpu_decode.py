@@ -118,6 +118,33 @@ def test_headline_shape():
     _check(q, cache, lens, o, l)
 
 
+def test_max_batch_long_context_sampled():
+    """The largest shape of the attention sweep: batch 128 (the bf16 path's maximum) x 32768
+    tokens, 128 heads, the automatic split; inputs made on the device; four sequences (the
+    first, the last and two inside) checked on every head against the oracle."""
+    import mla_latent_kv_37_b200 as M
+    from oracle import mla_oracle as O
+    B, N, H = 128, 32768, 128
+    lens = [N] * B
+    q = I.query_cat(17, B, H, device="cuda")
+    cache = I.paged_cache(18, lens, lens, device="cuda")
+    d = M.dims(B, H)
+    ws = M.workspace(d)
+    o = torch.full((B, H, 512), float("nan"), dtype=torch.float32, device="cuda")
+    lse = torch.full((B, H), float("nan"), dtype=torch.float32, device="cuda")
+    M.mla_decode_attn(d, q, cache.pool, cache.page_table, cache.seq_lens, o, ws, lse=lse)
+    torch.cuda.synchronize()
+    assert M.mla_get_status() == 0
+    assert not torch.isnan(o).any() and not torch.isnan(lse).any()
+    for b in (0, 41, 97, 127):
+        rows = O.f64(cache.pool[cache.page_table[b].long()].reshape(-1, 576)[:N].cpu())
+        qb = O.f64(q[b].cpu())
+        o_ref, l_ref = O.latent_attention(qb[:, :512], qb[:, 512:], rows[:, :512],
+                                          rows[:, 512:])
+        assert_close(o[b].double().cpu().numpy(), o_ref, torch.bfloat16, f"o_lat b={b}")
+        np.testing.assert_allclose(lse[b].double().cpu().numpy(), l_ref, rtol=2e-4, atol=2e-4)
+
+
 def test_fp32_path():
     lens = [256, 100, 1]
     q, cache = _case(11, lens, 16, dtype=torch.float32)
