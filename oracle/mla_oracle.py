@@ -226,6 +226,58 @@ def output_projection(o_heads, w_o) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------------------------
+# FP8 (E4M3) storage of weights
+# ---------------------------------------------------------------------------------------------
+# [IA] "De onde vem o 93%": the pages' one throughput figure was measured with the weights
+# converted to FP8.  The pages do not define the 8-bit format; this reads it as the common
+# "E4M3" float: 1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits, subnormals at
+# exponent field 0, no infinities, S.1111.111 = NaN, largest finite magnitude 448.  A weight
+# row is stored as codes of w / s with one fp32 scale s per row (so the row's largest
+# magnitude maps to 448).
+
+def e4m3_decode(codes) -> np.ndarray:
+    """The value of each E4M3 byte, in float64 (NaN for the two NaN codes)."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    return np.where((c & 0x7F) == 0x7F, np.nan, sign * mag)
+
+
+def e4m3_quantize(x) -> np.ndarray:
+    """The E4M3 byte of each value: the nearest finite E4M3 value, a tie going to the code whose
+    last mantissa bit is 0, magnitudes above 448 saturating to 448; the sign is kept (also on
+    zero)."""
+    x = np.asarray(x, dtype=np.float64)
+    grid = e4m3_decode(np.arange(0x7F))  # codes 0x00 .. 0x7E: 0 .. 448, increasing
+    a = np.minimum(np.abs(x), 448.0)
+    hi = np.clip(np.searchsorted(grid, a), 0, 0x7E)
+    lo = np.clip(hi - 1, 0, 0x7E)
+    d_lo, d_hi = a - grid[lo], grid[hi] - a
+    code = np.where((d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0)), hi, lo)
+    code = np.where(grid[hi] == a, hi, code)
+    return (code | (np.signbit(x).astype(np.int64) << 7)).astype(np.uint8)
+
+
+def quantize_rows_e4m3(w):
+    """Per-row E4M3 storage of a weight matrix [rows, cols]: s_r = max_j |w_rj| / 448 in fp32
+    (1 for a zero row) and the codes of w_rj / s_r, the division in fp32 -- the precision in
+    which the GPU takes the same decision.  Returns (codes uint8 [rows, cols], s float32
+    [rows])."""
+    w32 = np.asarray(w, dtype=np.float32)
+    amax = np.abs(w32).max(axis=1)
+    s = np.where(amax > 0, amax / np.float32(448.0), np.float32(1.0)).astype(np.float32)
+    y = (w32 / s[:, None]).astype(np.float32)
+    return e4m3_quantize(y.astype(np.float64)), s
+
+
+def dequantize_rows_e4m3(codes, s) -> np.ndarray:
+    """The weights an E4M3-stored matrix stands for: decode(code) * s_r, in float64."""
+    return e4m3_decode(codes) * np.asarray(s, dtype=np.float64)[:, None]
+
+
+# ---------------------------------------------------------------------------------------------
 # One whole decode step for one sequence of one layer
 # ---------------------------------------------------------------------------------------------
 

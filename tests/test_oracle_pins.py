@@ -405,3 +405,65 @@ def test_decode_step_appends_at_position_and_attends_to_itself():
     # position 0: the rotary part is unrotated
     np.testing.assert_allclose(step["row"][512:], w.w_kr @ h, rtol=1e-14)
     np.testing.assert_allclose(step["out"], w.w_o @ step["o_heads"].reshape(-1), rtol=1e-13)
+
+
+# ---------------------------------------------------------------------------------------------
+# FP8 (E4M3) weight storage: values the format definition fixes, invariants, brute force
+# ---------------------------------------------------------------------------------------------
+E4M3_KNOWN = {  # code: value, from the E4M3 definition (bias 7, 3 mantissa bits, max 448)
+    0x00: 0.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6, 0x30: 0.5, 0x38: 1.0,
+    0x39: 1.125, 0x3F: 1.875, 0x40: 2.0, 0x77: 240.0, 0x78: 256.0, 0x7E: 448.0,
+    0x81: -(2.0 ** -9), 0xB8: -1.0, 0xFE: -448.0,
+}
+
+
+def test_e4m3_decode_known_codes():
+    for code, value in E4M3_KNOWN.items():
+        assert O.e4m3_decode([code])[0] == value, hex(code)
+    assert np.signbit(O.e4m3_decode([0x80])[0]) and O.e4m3_decode([0x80])[0] == 0.0
+    assert np.isnan(O.e4m3_decode([0x7F, 0xFF])).all()
+
+
+def test_e4m3_decode_is_monotone_and_symmetric():
+    pos = O.e4m3_decode(np.arange(0x7F))
+    assert np.all(np.diff(pos) > 0)                       # 0 .. 448, strictly increasing
+    neg = O.e4m3_decode(np.arange(0x7F) | 0x80)
+    assert np.array_equal(neg, -pos)
+    # spacing doubles with each exponent step: 8 values per binade above the subnormals
+    assert np.allclose(np.diff(pos[8:16]), 2.0 ** -9) and np.allclose(np.diff(pos[16:24]), 2.0 ** -8)
+
+
+def test_e4m3_quantize_round_trip_ties_and_saturation():
+    codes = np.arange(256)
+    finite = codes[(codes & 0x7F) != 0x7F]
+    assert np.array_equal(O.e4m3_quantize(O.e4m3_decode(finite)), finite.astype(np.uint8))
+    # ties go to the code with an even last mantissa bit
+    assert O.e4m3_quantize([1.0625])[0] == 0x38 and O.e4m3_quantize([1.1875])[0] == 0x3A
+    assert O.e4m3_quantize([-1.0625])[0] == 0xB8
+    assert O.e4m3_quantize([2.0 ** -10])[0] == 0x00   # halfway to the smallest subnormal
+    assert O.e4m3_quantize([500.0, -1e9])[0] == 0x7E and O.e4m3_quantize([-1e9])[0] == 0xFE
+
+
+def test_e4m3_quantize_is_nearest_by_brute_force():
+    rng = np.random.default_rng(7)
+    x = np.concatenate([rng.normal(0, 3, 2000), rng.uniform(-450, 450, 2000),
+                        rng.uniform(-0.02, 0.02, 2000)])
+    grid = O.e4m3_decode(np.arange(256))
+    grid = grid[~np.isnan(grid)]
+    got = O.e4m3_decode(O.e4m3_quantize(x))
+    best = np.abs(x[:, None] - grid[None, :]).min(axis=1)
+    assert np.allclose(np.abs(x - np.clip(got, -448, 448)), best, rtol=0, atol=0)
+
+
+def test_quantize_rows_maps_each_row_max_to_448():
+    rng = np.random.default_rng(3)
+    w = rng.normal(0, 0.02, (5, 300)).astype(np.float32)
+    w[3] = 0.0
+    codes, s = O.quantize_rows_e4m3(w)
+    deq = O.dequantize_rows_e4m3(codes, s)
+    for r in (0, 1, 2, 4):
+        j = np.argmax(np.abs(w[r]))
+        assert abs(O.e4m3_decode([codes[r, j]])[0]) == 448.0
+        # every element within half a spacing of its binade (3 mantissa bits: 2^-4 relative)
+        assert np.all(np.abs(deq[r] - w[r]) <= 2.0 ** -4 * np.abs(w[r]) + 2.0 ** -10 * s[r])
+    assert s[3] == 1.0 and np.all(codes[3] == 0)
