@@ -554,6 +554,56 @@ def run_execution_modes(dev, peaks, reps=10, B=32, H=128, D=7168):
     return res
 
 
+def run_fp8_weights(dev, peaks, reps=10, B=32, H=128, D=7168):
+    """The output projection of one layer (W_UV then W_O) with W_O in bf16 and with W_O stored
+    as E4M3 codes + row scales (one byte per weight streamed from HBM): time per call and the
+    weight bytes it streams."""
+    import mla_latent_kv_37_b200 as M
+    import mla_inputs as I
+    d = M.dims(B, H, D)
+    w = I.weights(13, H, D, device=dev)
+    codes = torch.empty(D, H * 128, dtype=torch.uint8, device=dev)
+    scale = torch.empty(D, dtype=torch.float32, device=dev)
+    M.mla_quantize_weights_fp8(w.w_o, codes, scale)
+    ws = M.workspace(d, 0, dev)
+    o_lat = torch.randn(B, H, 512, dtype=torch.float32, device=dev)
+    out = torch.empty(B, D, dtype=torch.bfloat16, device=dev)
+
+    def nbytes(*ts):
+        return sum(t.numel() * t.element_size() for t in ts)
+
+    res = {}
+    for name, fn, wbytes in (
+            ("bf16", lambda: M.mla_out_proj(d, o_lat, w.w_uv, ws, w_o=w.w_o, out=out),
+             nbytes(w.w_uv, w.w_o)),
+            ("e4m3", lambda: M.mla_out_proj_fp8(d, o_lat, w.w_uv, codes, scale, out, ws),
+             nbytes(w.w_uv, codes, scale))):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e3)
+        us = sorted(ts)[len(ts) // 2]
+        gbs = wbytes / (us * 1e-6) / 1e9
+        res[name] = {"us_per_layer": us, "weight_bytes_per_layer": wbytes, "gbs": gbs,
+                     "hbm_frac": gbs / peaks.get("hbm_gbs", 6650.0)}
+    st = M.mla_get_status()
+    if st:
+        raise RuntimeError(f"device status {st:#x} in the E4M3 measurement")
+    res["what"] = (f"output projection of one layer (W_UV bf16, then W_O) at B={B}, H={H}, "
+                   f"D={D}, median of {reps}")
+    res["e4m3_over_bf16_time"] = res["e4m3"]["us_per_layer"] / res["bf16"]["us_per_layer"]
+    del w, codes, scale, ws
+    torch.cuda.empty_cache()
+    return res
+
+
 def config_block(cfg, lens, world):
     """The workload description both arms print (identical for the same configuration)."""
     B, L = cfg["batch"], cfg["layers"]
@@ -793,7 +843,7 @@ def main():
         cpu = cpu_baseline_from(sec, cfg, heads_timed, wall)
 
     # ---------------- the other configurations and the attention sweep (one GPU) ----------
-    configs = sweep = modes = None
+    configs = sweep = modes = fp8w = None
     if rank == 0 and world == 1 and not args.no_extras:
         del layers, h, step
         torch.cuda.synchronize()
@@ -801,6 +851,7 @@ def main():
         configs = run_extra_configs(dev, peaks)
         sweep = compact_sweep(dev, peaks)
         modes = run_execution_modes(dev, peaks)
+        fp8w = run_fp8_weights(dev, peaks)
 
     if rank == 0:
         line = {
@@ -816,6 +867,7 @@ def main():
             "gpu_launches": int(launches), "clocks": clocks, "parity": parity,
             "attention_us_per_layer": roofline["us_per_launch"],
             "configs": configs, "attention_sweep": sweep, "execution_modes": modes,
+            "fp8_weights": fp8w,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

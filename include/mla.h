@@ -242,6 +242,31 @@ int mla_out_proj_folded(const mla_dims* dims, const float* o_lat, const void* w_
                         void* workspace, size_t workspace_bytes, mla_stream_t stream);
 
 /*
+ * E4M3 (FP8) weights ([IA] "De onde vem o 93%": the pages' throughput figure was measured with
+ * the weights converted to FP8).  A weight matrix is stored as one byte per element, E4M3
+ * (sign, 4 exponent bits with bias 7, 3 mantissa bits, subnormals, largest finite 448), and
+ * one fp32 scale per row: weight = decode(code) * scale[row].
+ *
+ * mla_quantize_weights_fp8 -- w [rows, cols] bf16 -> codes [rows, cols] bytes, scale [rows]:
+ *   scale[r] = max_j |w[r][j]| / 448 (fp32, round to nearest; 1 for a zero row),
+ *   codes[r][j] = w[r][j] / scale[r] (fp32) rounded to the nearest E4M3 value, ties to even,
+ *   saturating at +-448.  cols a positive multiple of 64.  No dims: any bf16 matrix.
+ *
+ * mla_out_proj_fp8 -- mla_out_proj with W_O stored as E4M3 codes + row scales (w_o_codes
+ *   [D, H*d_v], w_o_scale [D]); W_UV stays bf16.  out is required, o_heads optional.  bf16
+ *   path only, batch <= 64 (MLA_ERR_DIMS above: the widened weight tiles share tensor memory
+ *   with the accumulators).  The codes stream from HBM at one byte per weight and are widened
+ *   to f16 on chip, exactly (every E4M3 value is an f16 value); o_heads enters that product as
+ *   f16 hi + lo halves; the scale is applied to the fp32 sums.
+ */
+int mla_quantize_weights_fp8(const void* w, int64_t rows, int64_t cols, void* codes,
+                             float* scale, mla_stream_t stream);
+
+int mla_out_proj_fp8(const mla_dims* dims, const float* o_lat, const void* w_uv,
+                     const void* w_o_codes, const float* w_o_scale, void* o_heads, void* out,
+                     void* workspace, size_t workspace_bytes, mla_stream_t stream);
+
+/*
  * Native decode step over a stack of layers, end to end from host memory.
  *
  * mla_layer -- one layer's device-resident weights and paged cache (layouts as in the calls

@@ -80,6 +80,9 @@ _SIGS = {
     "mla_merge_partials": (ctypes.c_int, [ctypes.POINTER(mla_dims), _I, _P, _P, _P, _P, _P]),
     "mla_fold_weights": (ctypes.c_int, [ctypes.POINTER(mla_dims), _P, _P, _P, _P, _P, _P, _P]),
     "mla_step_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(mla_dims), _I, _I]),
+    "mla_quantize_weights_fp8": (ctypes.c_int, [_P, ctypes.c_int64, ctypes.c_int64, _P, _P, _P]),
+    "mla_out_proj_fp8": (ctypes.c_int, [ctypes.POINTER(mla_dims), _P, _P, _P, _P, _P, _P, _P, _SZ,
+                                        _P]),
     "mla_decode_step_host": (ctypes.c_int, [ctypes.POINTER(mla_dims), _I, ctypes.POINTER(mla_layer),
                                             _P, _P, _P, _P, _I, _P, _SZ, _P]),
     "mla_append_absorb_folded": (ctypes.c_int, [ctypes.POINTER(mla_dims), _P, _P, _P, _P, _P,
@@ -329,6 +332,36 @@ def mla_decode_step_host(d: mla_dims, layer_array, h_host, positions_host, seq_l
                                     out_host.data_ptr(), num_splits, _ptr(ws), ws.numel(),
                                     _stream(stream))
     _check(rc, "mla_decode_step_host")
+
+
+def mla_quantize_weights_fp8(w, codes, scale, stream=None):
+    """E4M3 storage of a bf16 matrix w [rows, cols]: codes [rows, cols] uint8, scale [rows] fp32."""
+    _need(w, "w", torch.bfloat16)
+    if w.dim() != 2:
+        raise ValueError("w must be a matrix")
+    rows, cols = w.shape
+    _need(codes, "codes", torch.uint8, (rows, cols))
+    _need(scale, "scale", torch.float32, (rows,))
+    rc = lib().mla_quantize_weights_fp8(_ptr(w), rows, cols, _ptr(codes), _ptr(scale),
+                                        _stream(stream))
+    _check(rc, "mla_quantize_weights_fp8")
+
+
+def mla_out_proj_fp8(d: mla_dims, o_lat, w_uv, w_o_codes, w_o_scale, out, ws, o_heads=None,
+                     stream=None):
+    """mla_out_proj with W_O stored as E4M3 codes and row scales (bf16 path, batch <= 64)."""
+    H = d.n_heads
+    _need(o_lat, "o_lat", torch.float32, (d.batch, H, d.d_c))
+    _need(w_uv, "w_uv", torch.bfloat16, (H * d.d_v, d.d_c))
+    _need(w_o_codes, "w_o_codes", torch.uint8, (d.d_model, H * d.d_v))
+    _need(w_o_scale, "w_o_scale", torch.float32, (d.d_model,))
+    _need(o_heads, "o_heads", torch.bfloat16, (d.batch, H, d.d_v))
+    _need(out, "out", torch.bfloat16, (d.batch, d.d_model))
+    _need(ws, "workspace", torch.uint8)
+    rc = lib().mla_out_proj_fp8(ctypes.byref(d), _ptr(o_lat), _ptr(w_uv), _ptr(w_o_codes),
+                                _ptr(w_o_scale), _ptr(o_heads), _ptr(out), _ptr(ws), ws.numel(),
+                                _stream(stream))
+    _check(rc, "mla_out_proj_fp8")
 
 
 def fold_shapes(d: mla_dims):

@@ -36,6 +36,7 @@
 #pragma once
 #include "ptx_sm100.cuh"
 #include "rope.cuh"
+#include <cuda_fp16.h>
 
 namespace mla {
 namespace sk {
@@ -68,12 +69,34 @@ struct Params {
   float rope_theta;
   unsigned int* status;
   uint64_t wait_ns;
+  const float* a_scale;  // E4M3 weights: one scale per weight row (the product's rows)
 };
 
 // A stage holds kbs K blocks: A [kbs][128 rows][128 B] (K-major) or [2][64 kbs][128 B]
 // (MN-major), then X [kbs][n_pad][128 B].
 __host__ __device__ inline uint32_t stage_bytes(int n_pad, int kbs) {
   return static_cast<uint32_t>(kbs) * (kATileBytes + static_cast<uint32_t>(n_pad) * 128u);
+}
+
+// Two E4M3 codes (low byte first) -> their values as an f16 pair (low half first), exactly
+// (every E4M3 value, 2^-9 .. 448 with 3 mantissa bits, is an f16 value): one instruction.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t codes) {
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(codes));
+  return h2;
+}
+
+// f16 x f16 -> fp32, shape M x N, both operands K-major (operand formats 0 = f16).
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N) {
+  return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// E4M3 weights: A [kbs][128 rows][64 B] (64-byte swizzle), then X as above (f16 here).  The
+// converter warps widen each block to f16 in tensor memory, where the MMAs read it.
+constexpr uint32_t kA8TileBytes = 128 * 64;
+constexpr int kThreadsFp8 = 320;
+__host__ __device__ inline uint32_t stage_bytes_fp8(int n_pad, int kbs) {
+  return static_cast<uint32_t>(kbs) * (kA8TileBytes + static_cast<uint32_t>(n_pad) * 128u);
 }
 
 // First iteration of CTA c's range, and the CTA whose range holds iteration i.
@@ -325,6 +348,7 @@ struct EpiWuv {
   int b_pad;
   __nv_bfloat16* o_heads;
   __nv_bfloat16* oh;
+  __half* oh16 = nullptr;  // or f16 hi/lo planes (the operand of an f16 product)
   __host__ __device__ static size_t smem_bytes(int) { return 0; }
   __device__ void prepare(uint8_t*, int, int, int) const {}
   __device__ void apply(const uint8_t*, int g, int r, bool valid, int c0, int n_out,
@@ -342,6 +366,11 @@ struct EpiWuv {
       if (oh) {
         oh[o] = hi;
         oh[plane + o] = __float2bfloat16_rn(v[j] - __bfloat162float(hi));
+      }
+      if (oh16) {
+        const __half h16 = __float2half_rn(v[j]);
+        oh16[o] = h16;
+        oh16[plane + o] = __float2half_rn(v[j] - __half2float(h16));
       }
     }
   }
@@ -412,8 +441,8 @@ __device__ __forceinline__ void sum_slots(const float4* src, size_t slot_stride,
 }
 
 // ---------------------------------------------------------------------------------------------
-template <class Epi>
-__global__ void __launch_bounds__(kThreads, 1)
+template <class Epi, bool kFp8 = false>
+__global__ void __launch_bounds__(kFp8 ? kThreadsFp8 : kThreads, 1)
     streamk_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,
                         const __grid_constant__ CUtensorMap tmA1,
                         const __grid_constant__ CUtensorMap tmA2,
@@ -421,8 +450,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  const uint32_t sbytes = stage_bytes(p.n_pad, p.kbs);
-  const uint32_t a_bytes = static_cast<uint32_t>(p.kbs) * kATileBytes;
+  const uint32_t sbytes = kFp8 ? stage_bytes_fp8(p.n_pad, p.kbs) : stage_bytes(p.n_pad, p.kbs);
+  const uint32_t a_bytes = static_cast<uint32_t>(p.kbs) * (kFp8 ? kA8TileBytes : kATileBytes);
   uint8_t* epi_smem = smem + p.stages * sbytes;
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(
       epi_smem + ((Epi::smem_bytes(p.n_out) + 15) & ~static_cast<size_t>(15)));
@@ -432,7 +461,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* epi_sync = acc_empty + 2;          // 4 arrivals
   uint64_t* fin_ready = epi_sync + 1;          // 1 arrival
   uint64_t* mma_done = fin_ready + 1;          // final drain of the MMA pipe
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* a_full = mma_done + 1;             // [stages] (E4M3): widened A in TMEM, 4 arrivals
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(a_full + (kFp8 ? p.stages : 0));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* fin_flag = abort_flag + 1;
 
@@ -443,8 +473,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const long long i_begin = range_start(c, p.iters, P);
   const long long i_end = range_start(c + 1, p.iters, P);
   const long long kb = p.units;  // work units per tile
+  // TMEM: two accumulator buffers [0, 2 n_pad); E4M3: the widened A of each stage after them
   uint32_t tmem_cols = 32;
   while (tmem_cols < 2u * static_cast<uint32_t>(p.n_pad)) tmem_cols <<= 1;
+  const uint32_t a_col0 = 2u * static_cast<uint32_t>(p.n_pad);
+  if (kFp8) tmem_cols = 512;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.stages; ++s) {
@@ -458,6 +491,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(epi_sync, 4);
     mbar_init(fin_ready, 1);
     mbar_init(mma_done, 1);
+    if (kFp8)
+      for (int s = 0; s < p.stages; ++s) mbar_init(&a_full[s], 4);
     *abort_flag = 0;
     *fin_flag = 0;
     fence_mbar_init_cluster();
@@ -545,7 +580,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16(128, p.n_pad, p.a_mn_major, 0);
+      const uint32_t idesc =
+          kFp8 ? idesc_f16(128, p.n_pad) : idesc_bf16(128, p.n_pad, p.a_mn_major, 0);
       long long it = 0;  // iteration counter (ring position)
       int seg = 0;
       bool ok = true;
@@ -565,26 +601,74 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
+          if (kFp8 && !mbar_wait(&a_full[s], static_cast<uint32_t>((it / p.stages) & 1), wc)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
           const uint32_t a_base = smem_u32(smem + s * sbytes);
           const uint32_t x_base = a_base + a_bytes;
           const bool first = (i == t * kb) || (i == i_begin);
           for (int kk = 0; kk < 4 * p.kbs; ++kk) {
             const uint32_t kq = static_cast<uint32_t>(kk >> 2), kr = static_cast<uint32_t>(kk & 3);
-            const uint64_t adesc =
-                p.a_mn_major
-                    ? smem_desc(a_base + kk * 2048, a_bytes / 2, 1024, kSwizzle128B)
-                    : smem_desc(a_base + kq * kATileBytes + kr * 32, 16, 1024, kSwizzle128B);
             const uint64_t xdesc =
                 smem_desc(x_base + kq * static_cast<uint32_t>(p.n_pad) * 128u + kr * 32, 16, 1024,
                           kSwizzle128B);
-            mma_ss(d_tmem, adesc, xdesc, idesc, (first && kk == 0) ? 0u : 1u);
+            if (kFp8) {
+              // A: K step kk of the stage's widened block, 8 TMEM columns of bf16 pairs
+              const uint32_t a_tmem = tmem_base + a_col0 +
+                                      static_cast<uint32_t>(s * p.kbs) * 32u + kq * 32u + kr * 8u;
+              mma_ts(d_tmem, a_tmem, xdesc, idesc, (first && kk == 0) ? 0u : 1u);
+            } else {
+              const uint64_t adesc =
+                  p.a_mn_major
+                      ? smem_desc(a_base + kk * 2048, a_bytes / 2, 1024, kSwizzle128B)
+                      : smem_desc(a_base + kq * kATileBytes + kr * 32, 16, 1024, kSwizzle128B);
+              mma_ss(d_tmem, adesc, xdesc, idesc, (first && kk == 0) ? 0u : 1u);
+            }
           }
           mma_commit(&empty_bar[s]);
         }
         if (ok) mma_commit(&acc_full[buf]);
       }
       mma_commit(mma_done);  // fires once every issued MMA has completed
+    }
+  } else if (kFp8 && warp >= 6) {
+    // ---------------- converters (E4M3 weights) ----------------
+    // Thread = tile row 32 q + lane (TMEM lane): its 64 codes of a K block (four 16-byte
+    // pieces, 64-byte swizzle: piece c of row r sits at piece c ^ ((r >> 1) & 3)) widened
+    // exactly to f16 and stored as 32 columns of f16 pairs, the layout of an MMA A operand in
+    // tensor memory.
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lanes = static_cast<uint32_t>(quarter * 32) << 16;
+    long long it = 0;
+    bool ok = true;
+    for (long long i = i_begin; i < i_end && ok; ++i, ++it) {
+      const int s = static_cast<int>(it % p.stages);
+      if (!(ok = warp_wait(&full_bar[s], static_cast<uint32_t>((it / p.stages) & 1), wc))) break;
+      const uint32_t a_base = smem_u32(smem + s * sbytes);
+      for (int j = 0; j < p.kbs; ++j) {
+        const uint32_t rb = a_base + static_cast<uint32_t>(j) * kA8TileBytes +
+                            static_cast<uint32_t>(row) * 64u;
+        uint32_t w[16];
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(w[4 * c]), "=r"(w[4 * c + 1]), "=r"(w[4 * c + 2]), "=r"(w[4 * c + 3])
+                       : "r"(rb + static_cast<uint32_t>((c ^ ((row >> 1) & 3)) * 16)));
+        uint32_t r[32];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          r[2 * k] = e4m3x2_to_f16x2(static_cast<uint16_t>(w[k] & 0xffffu));
+          r[2 * k + 1] = e4m3x2_to_f16x2(static_cast<uint16_t>(w[k] >> 16));
+        }
+        tmem_st32(tmem_base + lanes + a_col0 + static_cast<uint32_t>(s * p.kbs + j) * 32u, r);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&a_full[s]);
     }
   } else {
     // ---------------- epilogue ----------------
@@ -626,6 +710,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_wait_ld();
 #pragma unroll
             for (int j = 0; j < 16; ++j) v[j] += __uint_as_float(a[j]);
+          }
+          if (kFp8) {
+            const float sc = valid ? p.a_scale[r] : 0.f;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] *= sc;
           }
           epi.apply(epi_smem, g, r, valid, c0, p.n_out, v);
         }
@@ -684,6 +773,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           sum_slots(part_tile + ((p.n_lo + c0) / 4) * 128, slot_stride, n_contrib, w);
 #pragma unroll
           for (int j = 0; j < 16; ++j) v[j] += w[j];
+        }
+        if (kFp8) {
+          const float sc = valid ? p.a_scale[r] : 0.f;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[j] *= sc;
         }
         epi.apply(epi_smem, g, r, valid, c0, p.n_out, v);
       }

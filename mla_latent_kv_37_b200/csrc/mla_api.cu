@@ -17,6 +17,7 @@
 #include "attn_sm100.cuh"
 #include "epilogue.cuh"
 #include "fold.cuh"
+#include "fp8.cuh"
 #include "gemm_streamk.cuh"
 
 namespace mla {
@@ -51,6 +52,7 @@ constexpr int kMaxParts = 1 << 16;  // upper bound on num_splits (host check bef
 constexpr int kSkMinUnits = 2;    // fewest stages' worth of weights a stream-K CTA streams
 constexpr int kSkMaxContrib = 4;  // aim for at most this many CTAs sharing one tile
 constexpr int kSkMaxStages = 12;
+constexpr int kFp8MaxBatch = 64;  // E4M3 products: 2 * 2B accumulator columns leave room for A
 constexpr size_t kSmemPerBlockMax = 232448;  // 227 KiB opt-in limit per CTA
 
 // ------------------------------------------------------------------------------------------
@@ -136,14 +138,15 @@ int device_ctx(DevCtx** out) {
                                   attn_smem)) != cudaSuccess)
       return cuda_fail(e, "cudaFuncSetAttribute(split_kernel)");
     const int sk_smem = static_cast<int>(kSmemPerBlockMax);
-    const void* sk_kernels[7] = {
+    const void* sk_kernels[8] = {
         reinterpret_cast<const void*>(sk::streamk_gemm_kernel<sk::EpiAppend>),
         reinterpret_cast<const void*>(sk::streamk_gemm_kernel<sk::EpiWq>),
         reinterpret_cast<const void*>(sk::streamk_gemm_kernel<sk::EpiWuk>),
         reinterpret_cast<const void*>(sk::streamk_gemm_kernel<sk::EpiWuv>),
         reinterpret_cast<const void*>(sk::streamk_gemm_kernel<sk::EpiWo>),
         reinterpret_cast<const void*>(sk::streamk_gemm_kernel<sk::EpiAppendWq>),
-        reinterpret_cast<const void*>(sk::streamk_gemm_kernel<sk::EpiAppendWqFold>)};
+        reinterpret_cast<const void*>(sk::streamk_gemm_kernel<sk::EpiAppendWqFold>),
+        reinterpret_cast<const void*>(sk::streamk_gemm_kernel<sk::EpiWo, true>)};
     for (const void* k : sk_kernels)
       if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, sk_smem)) !=
           cudaSuccess)
@@ -251,6 +254,39 @@ SkPlan sk_plan(const GemmShape& s, size_t epi_bytes, int sms) {
   return q;
 }
 
+// The same plan for E4M3 weights: smaller stages (64-byte A rows), and the widened A of every
+// stage in tensor memory next to the two accumulator buffers: stages * kbs * 32 + 2 n_pad <= 512.
+SkPlan sk_plan_fp8(const GemmShape& s, size_t epi_bytes, int sms) {
+  SkPlan q;
+  q.tiles = s.m_tiles * s.groups;
+  // alignment, tables, barriers (three per stage here)
+  const size_t fixed = 1024 + (epi_bytes + 15) / 16 * 16 + 512;
+  const size_t budget = kSmemPerBlockMax - fixed;
+  const int tmem_a = 512 - 2 * s.n_pad;
+  q.kbs = 1;
+  for (int kbs = 2; kbs <= 4 && kbs <= s.k_blocks(); kbs *= 2)
+    if (budget / sk::stage_bytes_fp8(s.n_pad, kbs) >= 2 && tmem_a / (kbs * 32) >= 2) q.kbs = kbs;
+  q.units = (s.k_blocks() + q.kbs - 1) / q.kbs;
+  q.iters = static_cast<long long>(q.tiles) * q.units;
+  long long P = std::min<long long>(sms, (q.iters + kSkMinUnits - 1) / kSkMinUnits);
+  P = std::min<long long>(P, static_cast<long long>(q.tiles) * kSkMaxContrib);
+  P = std::max<long long>(1, std::min(P, q.iters));
+  q.ctas = static_cast<int>(P);
+  for (long long t = 0; t < q.tiles; ++t) {
+    const int cf = sk::cta_of(t * q.units, q.iters, P);
+    const int cl = sk::cta_of((t + 1) * q.units - 1, q.iters, P);
+    q.max_slots = std::max(q.max_slots, cl - cf + 1);
+  }
+  const size_t sb = sk::stage_bytes_fp8(s.n_pad, q.kbs);
+  q.stages = static_cast<int>(std::min<size_t>({static_cast<size_t>(kSkMaxStages), budget / sb,
+                                                 static_cast<size_t>(tmem_a / (q.kbs * 32))}));
+  q.smem = fixed + static_cast<size_t>(q.stages) * sb;
+  q.partial_bytes = q.max_slots > 1 ? static_cast<size_t>(q.tiles) * q.max_slots * s.n_pad *
+                                          128 * sizeof(float)
+                                    : 0;
+  return q;
+}
+
 std::atomic<uint32_t> g_sk_epoch{0x5EED0000u};
 uint32_t next_epoch() {
   uint32_t e = g_sk_epoch.fetch_add(1, std::memory_order_relaxed) + 1;
@@ -280,6 +316,11 @@ Workspace layout(const mla_dims* d, int num_parts, int sms) {
                            sk::EpiAppendWqFold::smem_bytes(d->batch), 0};
     for (int i = 0; i < 8; ++i) {
       const SkPlan q = sk_plan(shapes[i], epi[i], sms);
+      part = std::max(part, q.partial_bytes);
+      ctr = std::max(ctr, static_cast<size_t>(q.tiles) * 8);
+    }
+    if (d->batch <= kFp8MaxBatch) {
+      const SkPlan q = sk_plan_fp8(shape_wo(d), 0, sms);
       part = std::max(part, q.partial_bytes);
       ctr = std::max(ctr, static_cast<size_t>(q.tiles) * 8);
     }
@@ -366,6 +407,17 @@ int map_weights(CUtensorMap* m, const void* base, uint64_t rows, uint64_t groups
                 CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
+// E4M3 weights [groups][rows][K] bytes as the view (64 k, rows, groups, K / 64), box
+// (64, 128, 1, kbs), 64-byte swizzle (the converters read it back row by row).
+int map_weights_fp8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t groups, uint64_t K,
+                    int kbs) {
+  const uint64_t dims[4] = {64, rows, groups, K / 64};
+  const uint64_t str[3] = {K, rows * K, 64};
+  const uint32_t box[4] = {64, 128, 1, static_cast<uint32_t>(kbs)};
+  return encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, 4, dims, str, box,
+                CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
 // Activations X: element (k, g, n) at n * n_stride + g * g_stride + 2 k (bytes), as the view
 // (64 k, groups, n, K / 64) with box (64, 1, n_pad, kbs); rows n >= n_rows read as zero.
 int map_acts(CUtensorMap* m, const void* base, uint64_t groups, uint64_t n_rows, uint64_t K,
@@ -424,12 +476,13 @@ cudaError_t record_profile_event(cudaEvent_t ev, cudaStream_t st) {
 }
 
 // One weight product on the tensor cores, its epilogue fused (stream-K, see gemm_streamk.cuh).
-template <class Epi>
+template <class Epi, bool kFp8 = false>
 int run_streamk(const DevCtx* c, const GemmShape& s, const SkPlan& q, int n_out,
                 const int32_t* positions, float theta, const CUtensorMap& a0,
                 const CUtensorMap& a1, int a1_tile_start, int a_mn_major,
                 const CUtensorMap& xmap, char* ws, const Workspace& w, const Epi& epi,
-                cudaStream_t st, const CUtensorMap* a2 = nullptr, int a2_tile_start = 1 << 30) {
+                cudaStream_t st, const CUtensorMap* a2 = nullptr, int a2_tile_start = 1 << 30,
+                const float* a_scale = nullptr) {
   sk::Params p{};
   p.m_total = s.m_total;
   p.m_tiles = s.m_tiles;
@@ -453,8 +506,10 @@ int run_streamk(const DevCtx* c, const GemmShape& s, const SkPlan& q, int n_out,
   p.rope_theta = theta;
   p.status = c->status;
   p.wait_ns = wait_limit_ns();
-  launch_pdl(sk::streamk_gemm_kernel<Epi>, dim3(q.ctas), dim3(sk::kThreads), q.smem, st, a0, a1,
-             a2 ? *a2 : a1, xmap, p, epi);
+  p.a_scale = a_scale;
+  launch_pdl(sk::streamk_gemm_kernel<Epi, kFp8>, dim3(q.ctas),
+             dim3(kFp8 ? sk::kThreadsFp8 : sk::kThreads), q.smem, st, a0, a1, a2 ? *a2 : a1, xmap,
+             p, epi);
   return last_launch();
 }
 
@@ -1006,6 +1061,76 @@ int mla_out_proj_folded(const mla_dims* dims, const float* o_lat, const void* w_
   if ((rc = map_acts(&bm, os, 1, 2 * Bp, K, K * 2, K * 2, s.n_pad, q.kbs))) return rc;
   sk::EpiWo e{D, static_cast<__nv_bfloat16*>(out)};
   return run_streamk(c, s, q, B, nullptr, 0.f, a, a, 1 << 30, 0, bm, ws, w, e, st);
+}
+
+// ------------------------------------------------------------------------------------------
+// E4M3 weights
+// ------------------------------------------------------------------------------------------
+int mla_quantize_weights_fp8(const void* w, int64_t rows, int64_t cols, void* codes,
+                             float* scale, mla_stream_t stream) {
+  if (!w || !codes || !scale) return MLA_ERR_NULL_ARG;
+  if (rows < 1 || rows > INT32_MAX || cols < 64 || cols % 64) return MLA_ERR_ARG;
+  if (!aligned(w, 16) || !aligned(codes, 16) || !aligned(scale, 4)) return MLA_ERR_ALIGN;
+  DevCtx* c = nullptr;
+  int rc = device_ctx(&c);
+  if (rc) return rc;
+  fp8::quantize_rows_kernel<<<static_cast<unsigned>(rows), 256, 0,
+                              reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(w), cols, static_cast<uint8_t*>(codes), scale);
+  return last_launch();
+}
+
+int mla_out_proj_fp8(const mla_dims* dims, const float* o_lat, const void* w_uv,
+                     const void* w_o_codes, const float* w_o_scale, void* o_heads, void* out,
+                     void* workspace, size_t workspace_bytes, mla_stream_t stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (dims->dtype != MLA_BF16) return MLA_ERR_ARG;
+  if (dims->batch > kFp8MaxBatch) return MLA_ERR_DIMS;
+  if (!o_lat || !w_uv || !w_o_codes || !w_o_scale || !out) return MLA_ERR_NULL_ARG;
+  if (!workspace) return MLA_ERR_WORKSPACE;
+  if (!aligned(o_lat, 16) || !aligned(w_uv, 16) || !aligned(w_o_codes, 16) ||
+      !aligned(w_o_scale, 4) || (o_heads && !aligned(o_heads, 16)) || !aligned(out, 16))
+    return MLA_ERR_ALIGN;
+  if (!aligned(workspace, 256)) return MLA_ERR_ALIGN;
+  DevCtx* c = nullptr;
+  if ((rc = device_ctx(&c))) return rc;
+  const Workspace w = layout(dims, resolve_parts(0, c), c->sms);
+  if (workspace_bytes < w.total) return MLA_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int B = dims->batch, D = dims->d_model, H = dims->n_heads;
+  char* ws = static_cast<char*>(workspace);
+  __nv_bfloat16* os = reinterpret_cast<__nv_bfloat16*>(ws + w.o_split);
+  void* oh_split = ws + w.oh_split;
+  // o_h = W_UV_h [o_lat_hi | o_lat_lo] (bf16 weights, as in mla_out_proj)
+  const GemmShape s1 = shape_wuv(dims);
+  const int Bp = s1.n_lo;
+  const size_t n = static_cast<size_t>(B) * H * kDc;
+  launch_pdl(split_hi_lo_kernel,
+             dim3(static_cast<unsigned>(std::min<size_t>((n / 8 + 255) / 256, 4096))), dim3(256),
+             0, st, o_lat, n, static_cast<size_t>(Bp) * H * kDc, os);
+  if ((rc = last_launch())) return rc;
+  const SkPlan q1 = sk_plan(s1, 0, c->sms);
+  CUtensorMap a, bm;
+  if ((rc = map_weights(&a, w_uv, kDv, H, kDc, q1.kbs))) return rc;
+  if ((rc = map_acts(&bm, os, H, 2 * Bp, kDc, kDc * 2ull, kDc * 2ull * H, s1.n_pad, q1.kbs)))
+    return rc;
+  // o_heads as f16 hi/lo planes: the E4M3 codes widen exactly to f16, so the W_O product runs
+  // on f16 operands (22 bits of o_heads instead of the bf16 planes' 16)
+  sk::EpiWuv e1{H, Bp, static_cast<__nv_bfloat16*>(o_heads), nullptr,
+                static_cast<__half*>(oh_split)};
+  if ((rc = run_streamk(c, s1, q1, B, nullptr, 0.f, a, a, 1 << 30, 0, bm, ws, w, e1, st)))
+    return rc;
+  // out = (decode(W_O codes) * s) [o_heads_hi | o_heads_lo]  (f16 x f16 -> fp32)
+  const GemmShape s2 = shape_wo(dims);
+  const uint64_t K = static_cast<uint64_t>(H) * kDv;
+  const SkPlan q2 = sk_plan_fp8(s2, 0, c->sms);
+  CUtensorMap a2, b2;
+  if ((rc = map_weights_fp8(&a2, w_o_codes, D, 1, K, q2.kbs))) return rc;
+  if ((rc = map_acts(&b2, oh_split, 1, 2 * Bp, K, K * 2, K * 2, s2.n_pad, q2.kbs))) return rc;
+  sk::EpiWo e2{D, static_cast<__nv_bfloat16*>(out)};
+  return run_streamk<sk::EpiWo, true>(c, s2, q2, B, nullptr, 0.f, a2, a2, 1 << 30, 0, b2, ws, w,
+                                      e2, st, nullptr, 1 << 30, w_o_scale);
 }
 
 int mla_merge_partials(const mla_dims* dims, int32_t n_parts, const float* part_o,

@@ -1,0 +1,70 @@
+"""E4M3 (FP8) weights: the GPU quantization against the oracle's (codes and scales bit for
+bit), and the output projection with W_O stored as E4M3 against the oracle's fp64 step computed
+with the weights the codes stand for."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import mla_oracle as O
+from tests.gpu_common import Workload, assert_close, dev, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("rows,cols,std", [(300, 1024, 0.02), (7, 16384, 1.0), (129, 64, 3e-3)])
+def test_quantize_matches_oracle_bit_for_bit(rows, cols, std):
+    import mla_latent_kv_37_b200 as M
+    g = torch.Generator().manual_seed(rows + cols)
+    w = (torch.randn(rows, cols, generator=g) * std).to(torch.bfloat16)
+    w[1, :] = 0.0                      # a zero row: scale 1, all codes 0
+    w[0, 5] = 1e-30                    # far below the smallest step of its row: a zero code
+    codes = torch.empty(rows, cols, dtype=torch.uint8, device="cuda")
+    scale = torch.empty(rows, dtype=torch.float32, device="cuda")
+    M.mla_quantize_weights_fp8(dev(w), codes, scale)
+    torch.cuda.synchronize()
+    exp_codes, exp_scale = O.quantize_rows_e4m3(w.float().numpy())
+    assert np.array_equal(scale.cpu().numpy(), exp_scale)
+    assert np.array_equal(codes.cpu().numpy(), exp_codes)
+
+
+@pytest.mark.parametrize("B,H,D", [(3, 16, 1024), (32, 128, 7168), (64, 32, 512)])
+def test_out_proj_fp8_matches_oracle(B, H, D):
+    import mla_latent_kv_37_b200 as M
+    hist = [(41 * i + 3) % 200 for i in range(B)]
+    wl = Workload(80 + B, B, H, D, hist)
+    d = M.dims(B, H, D)
+    codes = torch.empty(D, H * 128, dtype=torch.uint8, device="cuda")
+    scale = torch.empty(D, dtype=torch.float32, device="cuda")
+    M.mla_quantize_weights_fp8(dev(wl.w.w_o), codes, scale)
+    ws = M.workspace(d)
+    q_cat = torch.empty(B, H, 576, dtype=torch.bfloat16, device="cuda")
+    pool, table = dev(wl.cache.pool), dev(wl.cache.page_table)
+    o_lat = torch.empty(B, H, 512, dtype=torch.float32, device="cuda")
+    w = wl.w
+    M.mla_append_absorb(d, dev(wl.h), dev(w.w_dkv), dev(w.w_kr), dev(w.w_q), dev(w.w_uk),
+                        dev(wl.pos), table, pool, q_cat, ws)
+    M.mla_decode_attn(d, q_cat, pool, table, dev(wl.lens), o_lat, ws)
+    out = torch.full((B, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    o_heads = torch.empty(B, H, 128, dtype=torch.bfloat16, device="cuda")
+    M.mla_out_proj_fp8(d, o_lat, dev(w.w_uv), codes, scale, out, ws, o_heads=o_heads)
+    torch.cuda.synchronize()
+    assert M.mla_get_status() == 0
+    w_o_deq = O.dequantize_rows_e4m3(codes.cpu().numpy(), scale.cpu().numpy())
+    for b in sorted({0, B // 2, B - 1}):
+        ref = wl.oracle(b)  # o_heads from the bf16 W_UV; out recomputed with the E4M3 W_O
+        assert_close(to_np(o_heads[b].cpu()), ref["o_heads"], torch.bfloat16, f"o_heads b={b}")
+        exp = O.output_projection(ref["o_heads"], w_o_deq)
+        assert_close(to_np(out[b].cpu()), exp, torch.bfloat16, f"out b={b}")
+
+
+def test_out_proj_fp8_rejects_large_batch():
+    import mla_latent_kv_37_b200 as M
+    d = M.dims(65, 16, 1024)
+    with pytest.raises(M.MlaError) as e:
+        M.mla_out_proj_fp8(d, torch.empty(65, 16, 512, device="cuda"),
+                           torch.empty(16 * 128, 512, dtype=torch.bfloat16, device="cuda"),
+                           torch.empty(1024, 16 * 128, dtype=torch.uint8, device="cuda"),
+                           torch.empty(1024, device="cuda"),
+                           torch.empty(65, 1024, dtype=torch.bfloat16, device="cuda"),
+                           M.workspace(d))
+    assert e.value.code == -2
