@@ -142,3 +142,29 @@ def test_native_step_rejects_bad_host_arguments():
         M.mla_decode_step_host(d, arr, h.cpu(), pos.cpu(), lens.cpu(),
                                torch.empty(L, B, D, dtype=torch.bfloat16), small)
     assert e.value.code == -4
+
+
+def test_native_step_executor_fp32_and_fixed_split():
+    """The native executor on the fp32 path (16 heads) and with a fixed split count: the same
+    bytes as the device-resident step."""
+    import mla_latent_kv_37_b200 as M
+    from mla_latent_kv_37_b200.step import DecodeStep, Layer
+    for dtype, splits in ((torch.float32, 0), (torch.bfloat16, 3)):
+        Lf, Bf, Hf, Df = 2, 3, 16, 1024
+        wls = [Workload(90 + l, Bf, Hf, Df, [70, 1, 130], dtype=dtype) for l in range(Lf)]
+        layers = [Layer(w_dkv=dev(wl.w.w_dkv), w_kr=dev(wl.w.w_kr), w_q=dev(wl.w.w_q),
+                        w_uk=dev(wl.w.w_uk), w_uv=dev(wl.w.w_uv), w_o=dev(wl.w.w_o),
+                        pool=dev(wl.cache.pool), page_table=dev(wl.cache.page_table))
+                  for wl in wls]
+        step = DecodeStep(layers, Bf, Hf, Df, dtype=dtype, num_splits=splits)
+        h = torch.stack([dev(wl.h) for wl in wls])
+        pos, lens = dev(wls[0].pos), dev(wls[0].lens)
+        step.run(h, pos, lens)
+        torch.cuda.synchronize()
+        ref = step.out.cpu()
+        out_host = torch.full((Lf, Bf, Df), float("nan"), dtype=dtype).pin_memory()
+        step.run_native(h.cpu().pin_memory(), pos.cpu().pin_memory(), lens.cpu().pin_memory(),
+                        out_host)
+        torch.cuda.synchronize()
+        assert M.mla_get_status() == 0
+        assert torch.equal(out_host, ref), (dtype, splits)

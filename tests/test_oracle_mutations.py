@@ -99,7 +99,47 @@ def _mla_bytes_with_heads(d_c, d_rope, n_layers, bytes_per_elem):
     return (d_c + 2 * d_rope) * n_layers * bytes_per_elem
 
 
+_real_e4m3_decode = O.e4m3_decode
+_real_e4m3_quantize = O.e4m3_quantize
+
+
+def _e4m3_bias_8(codes):
+    # exponent bias 8 instead of 7: every normal value halved
+    v = _real_e4m3_decode(codes)
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    return np.where((c >> 3) & 0xF, v / 2.0, v)
+
+
+def _e4m3_no_subnormals(codes):
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    return np.where(((c >> 3) & 0xF) == 0, 0.0, _real_e4m3_decode(codes))
+
+
+def _e4m3_ties_up(x):
+    # ties resolved away from zero instead of to the even code
+    x = np.asarray(x, dtype=np.float64)
+    grid = _real_e4m3_decode(np.arange(0x7F))
+    a = np.minimum(np.abs(x), 448.0)
+    hi = np.clip(np.searchsorted(grid, a), 0, 0x7E)
+    lo = np.clip(hi - 1, 0, 0x7E)
+    code = np.where(grid[hi] - a <= a - grid[lo], hi, lo)
+    return (code | (np.signbit(x).astype(np.int64) << 7)).astype(np.uint8)
+
+
+def _e4m3_truncate(x):
+    # rounding toward zero instead of to nearest
+    x = np.asarray(x, dtype=np.float64)
+    grid = _real_e4m3_decode(np.arange(0x7F))
+    a = np.minimum(np.abs(x), 448.0)
+    code = np.clip(np.searchsorted(grid, a, side="right") - 1, 0, 0x7E)
+    return (code | (np.signbit(x).astype(np.int64) << 7)).astype(np.uint8)
+
+
 MUTATIONS = {
+    "E4M3 exponent bias 8": ("e4m3_decode", _e4m3_bias_8),
+    "E4M3 subnormals read as zero": ("e4m3_decode", _e4m3_no_subnormals),
+    "E4M3 ties away from zero": ("e4m3_quantize", _e4m3_ties_up),
+    "E4M3 rounding toward zero": ("e4m3_quantize", _e4m3_truncate),
     "rope sign flipped": ("rope", _rope_sign_flip),
     "rope half-split pairs": ("rope", _rope_half_split),
     "rope wrong frequencies": ("rope", _rope_wrong_freq),
