@@ -95,7 +95,9 @@ typedef struct mla_dims {
 #define MLA_STATUS_BAD_POSITION 0x8u /* an append position outside the sequence's pages */
 
 /* Scratch bytes needed by every compute call for these dims when the decode call is split
- * into at most `num_splits` parts (0 = the library's automatic choice).  Never fails. */
+ * into at most `num_splits` parts (0 = the library's automatic choice).  Never fails.  The
+ * projection calls use only the part that does not depend on the split count, so a workspace
+ * sized for any num_splits serves them; mla_decode_attn needs the size for its own count. */
 size_t mla_workspace_size(const mla_dims* dims, int32_t num_splits);
 
 /* Bytes one cached token occupies in one layer's pool: (d_c + d_rope) * element size.

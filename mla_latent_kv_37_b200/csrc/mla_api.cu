@@ -297,6 +297,9 @@ uint32_t next_epoch() {
 // ------------------------------------------------------------------------------------------
 // workspace layout
 // ------------------------------------------------------------------------------------------
+// [partial, counters, qn, o_split, oh_split) serve the projection products and are the same for
+// every split count; [plan, part_o, part_lse) serve the decode call and grow with its parts.  A
+// projection call therefore needs only `plan` bytes, the decode call all `total`.
 struct Workspace {
   size_t partial, counters, qn, o_split, oh_split, plan, part_o, part_lse, total;
 };
@@ -698,7 +701,7 @@ int mla_cache_append(const mla_dims* dims, const void* h, const void* w_dkv, con
     return last_launch();
   }
   const Workspace w = layout(dims, resolve_parts(0, c), c->sms);
-  if (workspace_bytes < w.total) return MLA_ERR_WORKSPACE;
+  if (workspace_bytes < w.plan) return MLA_ERR_WORKSPACE;  // projection scratch only
   char* ws = static_cast<char*>(workspace);
   float* part = reinterpret_cast<float*>(ws + w.partial);
   if (dims->dtype == MLA_BF16) {
@@ -744,7 +747,7 @@ int mla_absorb_q(const mla_dims* dims, const void* h, const void* w_q, const voi
   DevCtx* c = nullptr;
   if ((rc = device_ctx(&c))) return rc;
   const Workspace w = layout(dims, resolve_parts(0, c), c->sms);
-  if (workspace_bytes < w.total) return MLA_ERR_WORKSPACE;
+  if (workspace_bytes < w.plan) return MLA_ERR_WORKSPACE;  // projection scratch only
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int B = dims->batch, D = dims->d_model, H = dims->n_heads;
   char* ws = static_cast<char*>(workspace);
@@ -815,7 +818,7 @@ int mla_append_absorb(const mla_dims* dims, const void* h, const void* w_dkv, co
   DevCtx* c = nullptr;
   if ((rc = device_ctx(&c))) return rc;
   const Workspace w = layout(dims, resolve_parts(0, c), c->sms);
-  if (workspace_bytes < w.total) return MLA_ERR_WORKSPACE;
+  if (workspace_bytes < w.plan) return MLA_ERR_WORKSPACE;  // projection scratch only
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int B = dims->batch, D = dims->d_model, H = dims->n_heads;
   char* ws = static_cast<char*>(workspace);
@@ -880,7 +883,7 @@ int mla_out_proj(const mla_dims* dims, const float* o_lat, const void* w_uv, con
   DevCtx* c = nullptr;
   if ((rc = device_ctx(&c))) return rc;
   const Workspace w = layout(dims, resolve_parts(0, c), c->sms);
-  if (workspace_bytes < w.total) return MLA_ERR_WORKSPACE;
+  if (workspace_bytes < w.plan) return MLA_ERR_WORKSPACE;  // projection scratch only
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int B = dims->batch, D = dims->d_model, H = dims->n_heads;
   char* ws = static_cast<char*>(workspace);
@@ -1008,7 +1011,7 @@ int mla_append_absorb_folded(const mla_dims* dims, const void* h, const void* w_
   DevCtx* c = nullptr;
   if ((rc = device_ctx(&c))) return rc;
   const Workspace w = layout(dims, resolve_parts(0, c), c->sms);
-  if (workspace_bytes < w.total) return MLA_ERR_WORKSPACE;
+  if (workspace_bytes < w.plan) return MLA_ERR_WORKSPACE;  // projection scratch only
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int B = dims->batch, D = dims->d_model, H = dims->n_heads;
   char* ws = static_cast<char*>(workspace);
@@ -1041,7 +1044,7 @@ int mla_out_proj_folded(const mla_dims* dims, const float* o_lat, const void* w_
   DevCtx* c = nullptr;
   if ((rc = device_ctx(&c))) return rc;
   const Workspace w = layout(dims, resolve_parts(0, c), c->sms);
-  if (workspace_bytes < w.total) return MLA_ERR_WORKSPACE;
+  if (workspace_bytes < w.plan) return MLA_ERR_WORKSPACE;  // projection scratch only
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int B = dims->batch, D = dims->d_model, H = dims->n_heads;
   char* ws = static_cast<char*>(workspace);
@@ -1096,7 +1099,7 @@ int mla_out_proj_fp8(const mla_dims* dims, const float* o_lat, const void* w_uv,
   DevCtx* c = nullptr;
   if ((rc = device_ctx(&c))) return rc;
   const Workspace w = layout(dims, resolve_parts(0, c), c->sms);
-  if (workspace_bytes < w.total) return MLA_ERR_WORKSPACE;
+  if (workspace_bytes < w.plan) return MLA_ERR_WORKSPACE;  // projection scratch only
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int B = dims->batch, D = dims->d_model, H = dims->n_heads;
   char* ws = static_cast<char*>(workspace);

@@ -230,3 +230,4 @@ def test_step_executor_arguments(M):
     lay[1] = M.mla_layer(0x10000, 0x10000, 0x10000, 0x10000, 0x10000, None, 0x10000, 8,
                          0x10000, 4)
     assert L.mla_decode_step_host(ctypes.byref(d), 2, lay, f, f, f, f, 0, ws, big, None) == -1
+
