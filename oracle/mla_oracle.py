@@ -28,6 +28,8 @@ Readings where the pages are silent (each is also listed in the design notes):
     theta^(-2i/d_R) for pair i, rotation angle = position * frequency.  The same rotation is
     applied to k_R (shared by all heads) and to each head's q_rope at the new token's position.
   * The new token attends to itself: with a cache of n rows the query sits at position n-1.
+  * FP8 weights ([IA] "De onde vem o 93%" names FP8 without a format): E4M3 (bias 7, 3
+    mantissa bits, subnormals, max 448), one fp32 scale per row, round to nearest even.
 
 All arithmetic here is float64; inputs are upcast from whatever dtype the caller holds.
 """
