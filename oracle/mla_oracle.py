@@ -21,7 +21,7 @@ Sources (web pages on MLA; cited by title and section):
   [IA]  ia.com.br, "Como a MLA da DeepSeek cortou 93% da memoria ...", sections
         "Um resumo no lugar de 128 copias" and "A conta feita fora da DeepSeek".
 
-Readings where the pages are silent (each is also listed in the design notes):
+Readings where the pages are silent:
   * Query path: plain q = W_Q h_t, per head 128 non-rotary then 64 rotary rows.
   * Score scale 1/sqrt(d_k) with d_k = d_nope + d_R = 192.
   * RoPE: original interleaved-pair form, base theta (10000), frequencies
