@@ -249,17 +249,24 @@ int mla_out_proj_folded(const mla_dims* dims, const float* o_lat, const void* w_
  * (sign, 4 exponent bits with bias 7, 3 mantissa bits, subnormals, largest finite 448), and
  * one fp32 scale per row: weight = decode(code) * scale[row].
  *
- * mla_quantize_weights_fp8 -- w [rows, cols] bf16 -> codes [rows, cols] bytes, scale [rows]:
+ * mla_quantize_weights_fp8 -- w [rows, cols] bf16 -> codes, scale [rows]:
  *   scale[r] = max_j |w[r][j]| / 448 (fp32, round to nearest; 1 for a zero row),
- *   codes[r][j] = w[r][j] / scale[r] (fp32) rounded to the nearest E4M3 value, ties to even,
- *   saturating at +-448.  cols a positive multiple of 64.  No dims: any bf16 matrix.
+ *   code(r, j) = w[r][j] / scale[r] (fp32) rounded to the nearest E4M3 value, ties to even,
+ *   saturating at +-448.  cols a positive multiple of 128.  No dims: any bf16 matrix.
+ *   Layout of codes (round_up(rows, 128) * cols bytes): tiles of 128 rows x 128 columns, each
+ *   contiguous and row-major inside, ordered by row tile, then column tile, so that code(r, j)
+ *   is at byte ((r / 128) * (cols / 128) + j / 128) * 16384 + (r % 128) * 128 + j % 128.  A
+ *   product then streams whole 16 KB tiles from HBM.  The padding rows of the last row tile
+ *   are not written and never reach a result.
  *
- * mla_out_proj_fp8 -- mla_out_proj with W_O stored as E4M3 codes + row scales (w_o_codes
- *   [D, H*d_v], w_o_scale [D]); W_UV stays bf16.  out is required, o_heads optional.  bf16
- *   path only, batch <= 64 (MLA_ERR_DIMS above: the widened weight tiles share tensor memory
- *   with the accumulators).  The codes stream from HBM at one byte per weight and are widened
- *   to f16 on chip, exactly (every E4M3 value is an f16 value); o_heads enters that product as
- *   f16 hi + lo halves; the scale is applied to the fp32 sums.
+ * mla_out_proj_fp8 -- mla_out_proj with W_O stored as E4M3 codes + row scales (w_o_codes:
+ *   W_O [D, H*d_v] as mla_quantize_weights_fp8 writes it, w_o_scale [D]); W_UV stays bf16.  out is required, o_heads optional.  bf16
+ *   path only, batch <= 80 (MLA_ERR_DIMS above: the three activation planes below take
+ *   3 * round16(batch) of the 256 columns of one MMA).  The codes stream from HBM at one byte
+ *   per weight into E4M3 x E4M3 tensor-core products (fp32 sums).  Each o_heads row b enters
+ *   as a scale s_b = max|o_b| / 448 and three E4M3 planes whose sum keeps about 12 significant
+ *   bits of o_b / s_b; out[b][r] = w_o_scale[r] * s_b * (sum over planes), rounded to bf16.
+ *   The workspace of mla_workspace_size serves it (projection part only, as mla_out_proj).
  */
 int mla_quantize_weights_fp8(const void* w, int64_t rows, int64_t cols, void* codes,
                              float* scale, mla_stream_t stream);

@@ -335,12 +335,13 @@ def mla_decode_step_host(d: mla_dims, layer_array, h_host, positions_host, seq_l
 
 
 def mla_quantize_weights_fp8(w, codes, scale, stream=None):
-    """E4M3 storage of a bf16 matrix w [rows, cols]: codes [rows, cols] uint8, scale [rows] fp32."""
+    """E4M3 storage of a bf16 matrix w [rows, cols]: scale [rows] fp32 and codes uint8 in
+    128 x 128 tiles, [round_up(rows, 128), cols] bytes (see mla_quantize_weights_fp8 in mla.h)."""
     _need(w, "w", torch.bfloat16)
     if w.dim() != 2:
         raise ValueError("w must be a matrix")
     rows, cols = w.shape
-    _need(codes, "codes", torch.uint8, (rows, cols))
+    _need(codes, "codes", torch.uint8, ((rows + 127) // 128 * 128, cols))
     _need(scale, "scale", torch.float32, (rows,))
     rc = lib().mla_quantize_weights_fp8(_ptr(w), rows, cols, _ptr(codes), _ptr(scale),
                                         _stream(stream))
@@ -349,11 +350,12 @@ def mla_quantize_weights_fp8(w, codes, scale, stream=None):
 
 def mla_out_proj_fp8(d: mla_dims, o_lat, w_uv, w_o_codes, w_o_scale, out, ws, o_heads=None,
                      stream=None):
-    """mla_out_proj with W_O stored as E4M3 codes and row scales (bf16 path, batch <= 64)."""
+    """mla_out_proj with W_O stored as E4M3 codes (tiled, as mla_quantize_weights_fp8 writes
+    them) and row scales (bf16 path, batch <= 80)."""
     H = d.n_heads
     _need(o_lat, "o_lat", torch.float32, (d.batch, H, d.d_c))
     _need(w_uv, "w_uv", torch.bfloat16, (H * d.d_v, d.d_c))
-    _need(w_o_codes, "w_o_codes", torch.uint8, (d.d_model, H * d.d_v))
+    _need(w_o_codes, "w_o_codes", torch.uint8, ((d.d_model + 127) // 128 * 128, H * d.d_v))
     _need(w_o_scale, "w_o_scale", torch.float32, (d.d_model,))
     _need(o_heads, "o_heads", torch.bfloat16, (d.batch, H, d.d_v))
     _need(out, "out", torch.bfloat16, (d.batch, d.d_model))

@@ -4,13 +4,20 @@
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cfloat>
+
+#include "ptx_sm100.cuh"
 
 namespace mla {
 namespace fp8 {
 
 // Row r of w [rows][cols] (bf16): s_r = max_j |w_rj| / 448 (fp32, round to nearest; 1 for a zero
 // row), code_rj = w_rj / s_r (fp32) rounded to the nearest E4M3 value, ties to even,
-// saturating at +-448.  One block per row; cols is even.
+// saturating at +-448.  The codes are stored in tiles of 128 rows x 128 columns, each tile
+// contiguous and row-major inside, tiles ordered by row tile then column tile:
+// code_rj at ((r / 128) * (cols / 128) + j / 128) * 16384 + (r % 128) * 128 + j % 128.  One block
+// per row; cols a multiple of 128.
 __global__ void __launch_bounds__(256)
     quantize_rows_kernel(const __nv_bfloat16* __restrict__ w, long long cols,
                          uint8_t* __restrict__ q, float* __restrict__ scale) {
@@ -28,13 +35,84 @@ __global__ void __launch_bounds__(256)
   for (int k = 1; k < static_cast<int>(blockDim.x >> 5); ++k) m = fmaxf(m, part[k]);
   const float s = m > 0.f ? __fdiv_rn(m, 448.f) : 1.f;
   if (threadIdx.x == 0) scale[row] = s;
-  uint16_t* qr = reinterpret_cast<uint16_t*>(q + row * cols);
+  uint8_t* qt = q + (row / 128) * cols * 128 + (row % 128) * 128;
   for (long long j = threadIdx.x; j < cols / 2; j += blockDim.x) {
     const float y0 = __fdiv_rn(__bfloat162float(wr[2 * j]), s);
     const float y1 = __fdiv_rn(__bfloat162float(wr[2 * j + 1]), s);
     uint16_t c;
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(c) : "f"(y1), "f"(y0));
-    qr[j] = c;  // low byte: element 2j
+    // low byte: element 2j; a pair never straddles a tile
+    *reinterpret_cast<uint16_t*>(qt + (2 * j / 128) * 16384 + (2 * j) % 128) = c;
+  }
+}
+
+// Two fp32 values -> two E4M3 codes (round to nearest even, saturating), low byte from `lo`.
+__device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
+  uint16_t c;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(c) : "f"(hi), "f"(lo));
+  return c;
+}
+// Two E4M3 codes -> their exact values (every E4M3 value is an f16 value).
+__device__ __forceinline__ float2 e4m3x2_value(uint16_t c) {
+  uint32_t h;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(c));
+  return __half22float2(*reinterpret_cast<const __half2*>(&h));
+}
+
+// An fp32 activation row x_b (K values) as a scale and three E4M3 planes: s_b = max_k |x_bk| / 448
+// (at least FLT_MIN), y = x / s_b; p1 = E4M3(y), p2 = E4M3(y - p1), p3 = E4M3(y - p1 - p2), each
+// difference exact in fp32.  p1 + p2 + p3 keeps about 12 significant bits of y, so
+// s_b (p1 + p2 + p3) stands in for x_b in a product with E4M3 weights.  planes: [3][rows_pad][K];
+// rows in [rows, rows_pad) are written as zeros.  One block per row; K a multiple of 8; x and
+// planes 16- and 8-byte aligned.
+__global__ void __launch_bounds__(256)
+    split_planes_kernel(const float* __restrict__ x, int rows, long long K, int rows_pad,
+                        uint8_t* __restrict__ planes, float* __restrict__ scale) {
+  __shared__ float part[8];
+  griddep_launch_dependents();
+  griddep_wait();
+  const int b = blockIdx.x;
+  const size_t plane = static_cast<size_t>(rows_pad) * K;
+  uint2* out = reinterpret_cast<uint2*>(planes + static_cast<size_t>(b) * K);
+  const long long n8 = K / 8;
+  if (b >= rows) {
+    for (long long j = threadIdx.x; j < n8; j += blockDim.x)
+      for (int pl = 0; pl < 3; ++pl) out[pl * (plane / 8) + j] = make_uint2(0u, 0u);
+    if (threadIdx.x == 0) scale[b] = 0.f;
+    return;
+  }
+  const float4* xr = reinterpret_cast<const float4*>(x + static_cast<size_t>(b) * K);
+  float m = 0.f;
+  for (long long j = threadIdx.x; j < K / 4; j += blockDim.x) {
+    const float4 v = xr[j];
+    m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = m;
+  __syncthreads();
+  m = part[0];
+  for (int k = 1; k < static_cast<int>(blockDim.x >> 5); ++k) m = fmaxf(m, part[k]);
+  const float s = fmaxf(__fdiv_rn(m, 448.f), FLT_MIN);
+  if (threadIdx.x == 0) scale[b] = s;
+  for (long long j = threadIdx.x; j < n8; j += blockDim.x) {
+    const float4 u = xr[2 * j], w = xr[2 * j + 1];
+    float y[8] = {u.x, u.y, u.z, u.w, w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) y[i] = __fdiv_rn(y[i], s);
+#pragma unroll
+    for (int pl = 0; pl < 3; ++pl) {
+      uint32_t c[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint16_t q = e4m3x2(y[2 * i], y[2 * i + 1]);
+        const float2 d = e4m3x2_value(q);
+        y[2 * i] -= d.x;
+        y[2 * i + 1] -= d.y;
+        c[i] = q;
+      }
+      out[pl * (plane / 8) + j] = make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+    }
   }
 }
 

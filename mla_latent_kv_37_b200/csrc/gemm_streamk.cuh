@@ -36,7 +36,6 @@
 #pragma once
 #include "ptx_sm100.cuh"
 #include "rope.cuh"
-#include <cuda_fp16.h>
 
 namespace mla {
 namespace sk {
@@ -59,17 +58,21 @@ struct Params {
   int n_lo;           // > 0: columns [n_lo, 2 n_lo) hold the low halves of columns [0, n_lo)
   int n_out;          // valid output columns (the batch)
   int a_mn_major;     // 0: A K-major, 1: A MN-major
+  int a_tiled;        // 1: A (map A0 only) stored as contiguous tiles of 128 rows x 128 bytes,
+                      //    [groups * m_tiles][K / 128 bytes][128][128 B]
   int stages;         // shared-memory ring depth
   int max_slots;      // partial slots per tile
   long long iters;    // m_tiles * groups * units
   uint32_t epoch;     // launch tag for the tile counters (never 0)
-  float* partial;     // [tiles][max_slots][n_pad / 4][128][4]
+  float* partial;     // [tiles][max_slots][n_cols / 4][128][4], n_cols = n_lo or n_pad
   unsigned long long* counters;  // [tiles]
   const int32_t* positions;      // RoPE positions [n_out] (products with RoPE rows)
   float rope_theta;
   unsigned int* status;
   uint64_t wait_ns;
-  const float* a_scale;  // E4M3 weights: one scale per weight row (the product's rows)
+  int n_planes;          // X column planes summed into each output: 1, 2 (hi/lo) or 3
+  const float* a_scale;  // E4M3: one scale per weight row (the product's rows)
+  const float* x_scale;  // E4M3: one scale per output column (an activation row)
 };
 
 // A stage holds kbs K blocks: A [kbs][128 rows][128 B] (K-major) or [2][64 kbs][128 B]
@@ -78,25 +81,20 @@ __host__ __device__ inline uint32_t stage_bytes(int n_pad, int kbs) {
   return static_cast<uint32_t>(kbs) * (kATileBytes + static_cast<uint32_t>(n_pad) * 128u);
 }
 
-// Two E4M3 codes (low byte first) -> their values as an f16 pair (low half first), exactly
-// (every E4M3 value, 2^-9 .. 448 with 3 mantissa bits, is an f16 value): one instruction.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t codes) {
-  uint32_t h2;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(codes));
-  return h2;
-}
-
-// f16 x f16 -> fp32, shape M x N, both operands K-major (operand formats 0 = f16).
-__host__ __device__ constexpr uint32_t idesc_f16(int M, int N) {
+// E4M3 operands (tcgen05 kind::f8f6f4): a 128-byte row of a K block holds 128 elements, so the
+// shared-memory tiles, their descriptors and the 32-byte K step of one MMA are those of the
+// bf16 path byte for byte.  Instruction descriptor: D f32, both operand formats 0 (E4M3).
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N) {
   return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
-
-// E4M3 weights: A [kbs][128 rows][64 B] (64-byte swizzle), then X as above (f16 here).  The
-// converter warps widen each block to f16 in tensor memory, where the MMAs read it.
-constexpr uint32_t kA8TileBytes = 128 * 64;
-constexpr int kThreadsFp8 = 320;
-__host__ __device__ inline uint32_t stage_bytes_fp8(int n_pad, int kbs) {
-  return static_cast<uint32_t>(kbs) * (kA8TileBytes + static_cast<uint32_t>(n_pad) * 128u);
+__device__ __forceinline__ void mma_ss_e4m3(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
 }
 
 // First iteration of CTA c's range, and the CTA whose range holds iteration i.
@@ -348,7 +346,7 @@ struct EpiWuv {
   int b_pad;
   __nv_bfloat16* o_heads;
   __nv_bfloat16* oh;
-  __half* oh16 = nullptr;  // or f16 hi/lo planes (the operand of an f16 product)
+  float* oh32 = nullptr;  // or o_heads in fp32 [b][h][128] (split into E4M3 planes next)
   __host__ __device__ static size_t smem_bytes(int) { return 0; }
   __device__ void prepare(uint8_t*, int, int, int) const {}
   __device__ void apply(const uint8_t*, int g, int r, bool valid, int c0, int n_out,
@@ -367,11 +365,7 @@ struct EpiWuv {
         oh[o] = hi;
         oh[plane + o] = __float2bfloat16_rn(v[j] - __bfloat162float(hi));
       }
-      if (oh16) {
-        const __half h16 = __float2half_rn(v[j]);
-        oh16[o] = h16;
-        oh16[plane + o] = __float2half_rn(v[j] - __half2float(h16));
-      }
+      if (oh32) oh32[o] = v[j];
     }
   }
 };
@@ -396,53 +390,69 @@ struct EpiWo {
 };
 
 // Sum of 16 columns of one row over slots 0 .. n-1, added in slot order.  src points at the
-// row's first float4 of the 16 columns in slot 0; four slots' loads are in flight at a time.
+// row's first float4 of the 16 columns in slot 0; the loads of four slots are in flight at once.
 __device__ __forceinline__ void sum_slots(const float4* src, size_t slot_stride, int n,
                                           float (&v)[16]) {
-  float4 x[4];
-#pragma unroll
-  for (int q = 0; q < 4; ++q) x[q] = __ldcg(src + q * 128);
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    v[4 * q] = x[q].x;
-    v[4 * q + 1] = x[q].y;
-    v[4 * q + 2] = x[q].z;
-    v[4 * q + 3] = x[q].w;
-  }
-  int s = 1;
-  for (; s + 3 < n; s += 4) {
+  for (int s0 = 0; s0 < n; s0 += 4) {
     float4 y[4][4];
 #pragma unroll
     for (int u = 0; u < 4; ++u)
+      if (s0 + u < n)
 #pragma unroll
-      for (int q = 0; q < 4; ++q) y[u][q] = __ldcg(src + (s + u) * slot_stride + q * 128);
+        for (int q = 0; q < 4; ++q) y[u][q] = __ldcg(src + (s0 + u) * slot_stride + q * 128);
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
+    for (int u = 0; u < 4; ++u) {
+      if (s0 + u >= n) break;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        v[4 * q] += y[u][q].x;
-        v[4 * q + 1] += y[u][q].y;
-        v[4 * q + 2] += y[u][q].z;
-        v[4 * q + 3] += y[u][q].w;
+        if (s0 + u == 0) {
+          v[4 * q] = y[u][q].x;
+          v[4 * q + 1] = y[u][q].y;
+          v[4 * q + 2] = y[u][q].z;
+          v[4 * q + 3] = y[u][q].w;
+        } else {
+          v[4 * q] += y[u][q].x;
+          v[4 * q + 1] += y[u][q].y;
+          v[4 * q + 2] += y[u][q].z;
+          v[4 * q + 3] += y[u][q].w;
+        }
       }
-  }
-  for (; s < n; ++s) {
-    float4 y[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) y[q] = __ldcg(src + s * slot_stride + q * 128);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      v[4 * q] += y[q].x;
-      v[4 * q + 1] += y[q].y;
-      v[4 * q + 2] += y[q].z;
-      v[4 * q + 3] += y[q].w;
     }
+  }
+}
+
+// 16 accumulator columns c0 .. c0+15 of this warp's TMEM lanes, summed over the n_planes column
+// planes (plane pl at columns pl * n_lo + c): all planes' loads are issued before one wait.
+__device__ __forceinline__ void tmem_sum_planes(uint32_t tacc, int c0, int n_planes, int n_lo,
+                                                float (&v)[16]) {
+  uint32_t a[3][16];
+  tmem_ld16(tacc + c0, a[0]);
+  if (n_planes > 1) tmem_ld16(tacc + n_lo + c0, a[1]);
+  if (n_planes > 2) tmem_ld16(tacc + 2 * n_lo + c0, a[2]);
+  tmem_wait_ld();
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    float x = __uint_as_float(a[0][j]);
+    if (n_planes > 1) x += __uint_as_float(a[1][j]);
+    if (n_planes > 2) x += __uint_as_float(a[2][j]);
+    v[j] = x;
+  }
+}
+
+// E4M3 products: the fp32 sum of a row times its weight row's scale and the column's scale.
+__device__ __forceinline__ void scale_e4m3(const Params& p, int r, bool valid, int c0,
+                                           float (&v)[16]) {
+  const float sr = valid ? p.a_scale[r] : 0.f;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const int b = c0 + j;
+    v[j] *= b < p.n_out ? sr * p.x_scale[b] : 0.f;
   }
 }
 
 // ---------------------------------------------------------------------------------------------
 template <class Epi, bool kFp8 = false>
-__global__ void __launch_bounds__(kFp8 ? kThreadsFp8 : kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     streamk_gemm_kernel(const __grid_constant__ CUtensorMap tmA0,
                         const __grid_constant__ CUtensorMap tmA1,
                         const __grid_constant__ CUtensorMap tmA2,
@@ -450,8 +460,8 @@ __global__ void __launch_bounds__(kFp8 ? kThreadsFp8 : kThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  const uint32_t sbytes = kFp8 ? stage_bytes_fp8(p.n_pad, p.kbs) : stage_bytes(p.n_pad, p.kbs);
-  const uint32_t a_bytes = static_cast<uint32_t>(p.kbs) * (kFp8 ? kA8TileBytes : kATileBytes);
+  const uint32_t sbytes = stage_bytes(p.n_pad, p.kbs);
+  const uint32_t a_bytes = static_cast<uint32_t>(p.kbs) * kATileBytes;
   uint8_t* epi_smem = smem + p.stages * sbytes;
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(
       epi_smem + ((Epi::smem_bytes(p.n_out) + 15) & ~static_cast<size_t>(15)));
@@ -461,8 +471,7 @@ __global__ void __launch_bounds__(kFp8 ? kThreadsFp8 : kThreads, 1)
   uint64_t* epi_sync = acc_empty + 2;          // 4 arrivals
   uint64_t* fin_ready = epi_sync + 1;          // 1 arrival
   uint64_t* mma_done = fin_ready + 1;          // final drain of the MMA pipe
-  uint64_t* a_full = mma_done + 1;             // [stages] (E4M3): widened A in TMEM, 4 arrivals
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(a_full + (kFp8 ? p.stages : 0));
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* fin_flag = abort_flag + 1;
 
@@ -473,11 +482,8 @@ __global__ void __launch_bounds__(kFp8 ? kThreadsFp8 : kThreads, 1)
   const long long i_begin = range_start(c, p.iters, P);
   const long long i_end = range_start(c + 1, p.iters, P);
   const long long kb = p.units;  // work units per tile
-  // TMEM: two accumulator buffers [0, 2 n_pad); E4M3: the widened A of each stage after them
   uint32_t tmem_cols = 32;
   while (tmem_cols < 2u * static_cast<uint32_t>(p.n_pad)) tmem_cols <<= 1;
-  const uint32_t a_col0 = 2u * static_cast<uint32_t>(p.n_pad);
-  if (kFp8) tmem_cols = 512;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.stages; ++s) {
@@ -491,8 +497,6 @@ __global__ void __launch_bounds__(kFp8 ? kThreadsFp8 : kThreads, 1)
     mbar_init(epi_sync, 4);
     mbar_init(fin_ready, 1);
     mbar_init(mma_done, 1);
-    if (kFp8)
-      for (int s = 0; s < p.stages; ++s) mbar_init(&a_full[s], 4);
     *abort_flag = 0;
     *fin_flag = 0;
     fence_mbar_init_cluster();
@@ -532,7 +536,11 @@ __global__ void __launch_bounds__(kFp8 ? kThreadsFp8 : kThreads, 1)
           m_row0 = (mt - p.a1_tile_start) * 128;
         }
         uint8_t* a_dst = smem + s * sbytes;
-        if (p.a_mn_major) {
+        if (p.a_tiled) {
+          // view (128 B, 128 rows, K blocks, row tiles): box (128 B, 128, kbs, 1) is one
+          // contiguous run of kbs tiles in HBM
+          tma_load_4d_hint(a_dst, tmA, &full_bar[s], 0, 0, kb0, g * p.m_tiles + mt, pol_w);
+        } else if (p.a_mn_major) {
           // [g][k][m] with m contiguous: box (64 m, 64 kbs k) per 64-row half of the tile
           tma_load_3d_hint(a_dst, tmA, &full_bar[s], m_row0, kb0 * 64, g, pol_w);
           tma_load_3d_hint(a_dst + a_bytes / 2, tmA, &full_bar[s], m_row0 + 64, kb0 * 64, g,
@@ -581,7 +589,7 @@ __global__ void __launch_bounds__(kFp8 ? kThreadsFp8 : kThreads, 1)
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       const uint32_t idesc =
-          kFp8 ? idesc_f16(128, p.n_pad) : idesc_bf16(128, p.n_pad, p.a_mn_major, 0);
+          kFp8 ? idesc_e4m3(128, p.n_pad) : idesc_bf16(128, p.n_pad, p.a_mn_major, 0);
       long long it = 0;  // iteration counter (ring position)
       int seg = 0;
       bool ok = true;
@@ -601,10 +609,6 @@ __global__ void __launch_bounds__(kFp8 ? kThreadsFp8 : kThreads, 1)
             ok = false;
             break;
           }
-          if (kFp8 && !mbar_wait(&a_full[s], static_cast<uint32_t>((it / p.stages) & 1), wc)) {
-            ok = false;
-            break;
-          }
           tc_fence_after();
           const uint32_t a_base = smem_u32(smem + s * sbytes);
           const uint32_t x_base = a_base + a_bytes;
@@ -614,61 +618,20 @@ __global__ void __launch_bounds__(kFp8 ? kThreadsFp8 : kThreads, 1)
             const uint64_t xdesc =
                 smem_desc(x_base + kq * static_cast<uint32_t>(p.n_pad) * 128u + kr * 32, 16, 1024,
                           kSwizzle128B);
-            if (kFp8) {
-              // A: K step kk of the stage's widened block, 8 TMEM columns of bf16 pairs
-              const uint32_t a_tmem = tmem_base + a_col0 +
-                                      static_cast<uint32_t>(s * p.kbs) * 32u + kq * 32u + kr * 8u;
-              mma_ts(d_tmem, a_tmem, xdesc, idesc, (first && kk == 0) ? 0u : 1u);
-            } else {
-              const uint64_t adesc =
-                  p.a_mn_major
-                      ? smem_desc(a_base + kk * 2048, a_bytes / 2, 1024, kSwizzle128B)
-                      : smem_desc(a_base + kq * kATileBytes + kr * 32, 16, 1024, kSwizzle128B);
+            const uint64_t adesc =
+                p.a_mn_major
+                    ? smem_desc(a_base + kk * 2048, a_bytes / 2, 1024, kSwizzle128B)
+                    : smem_desc(a_base + kq * kATileBytes + kr * 32, 16, 1024, kSwizzle128B);
+            if (kFp8)
+              mma_ss_e4m3(d_tmem, adesc, xdesc, idesc, (first && kk == 0) ? 0u : 1u);
+            else
               mma_ss(d_tmem, adesc, xdesc, idesc, (first && kk == 0) ? 0u : 1u);
-            }
           }
           mma_commit(&empty_bar[s]);
         }
         if (ok) mma_commit(&acc_full[buf]);
       }
       mma_commit(mma_done);  // fires once every issued MMA has completed
-    }
-  } else if (kFp8 && warp >= 6) {
-    // ---------------- converters (E4M3 weights) ----------------
-    // Thread = tile row 32 q + lane (TMEM lane): its 64 codes of a K block (four 16-byte
-    // pieces, 64-byte swizzle: piece c of row r sits at piece c ^ ((r >> 1) & 3)) widened
-    // exactly to f16 and stored as 32 columns of f16 pairs, the layout of an MMA A operand in
-    // tensor memory.
-    const int quarter = warp & 3;
-    const int row = quarter * 32 + lane;
-    const uint32_t lanes = static_cast<uint32_t>(quarter * 32) << 16;
-    long long it = 0;
-    bool ok = true;
-    for (long long i = i_begin; i < i_end && ok; ++i, ++it) {
-      const int s = static_cast<int>(it % p.stages);
-      if (!(ok = warp_wait(&full_bar[s], static_cast<uint32_t>((it / p.stages) & 1), wc))) break;
-      const uint32_t a_base = smem_u32(smem + s * sbytes);
-      for (int j = 0; j < p.kbs; ++j) {
-        const uint32_t rb = a_base + static_cast<uint32_t>(j) * kA8TileBytes +
-                            static_cast<uint32_t>(row) * 64u;
-        uint32_t w[16];
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                       : "=r"(w[4 * c]), "=r"(w[4 * c + 1]), "=r"(w[4 * c + 2]), "=r"(w[4 * c + 3])
-                       : "r"(rb + static_cast<uint32_t>((c ^ ((row >> 1) & 3)) * 16)));
-        uint32_t r[32];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          r[2 * k] = e4m3x2_to_f16x2(static_cast<uint16_t>(w[k] & 0xffffu));
-          r[2 * k + 1] = e4m3x2_to_f16x2(static_cast<uint16_t>(w[k] >> 16));
-        }
-        tmem_st32(tmem_base + lanes + a_col0 + static_cast<uint32_t>(s * p.kbs + j) * 32u, r);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&a_full[s]);
     }
   } else {
     // ---------------- epilogue ----------------
@@ -699,23 +662,9 @@ __global__ void __launch_bounds__(kFp8 ? kThreadsFp8 : kThreads, 1)
       if (c_first == c_last) {
         // whole tile in this CTA: finish from TMEM
         for (int c0 = 0; c0 < n_cols; c0 += 16) {
-          uint32_t a[16];
           float v[16];
-          tmem_ld16(tacc + c0, a);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(a[j]);
-          if (p.n_lo > 0) {
-            tmem_ld16(tacc + p.n_lo + c0, a);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 16; ++j) v[j] += __uint_as_float(a[j]);
-          }
-          if (kFp8) {
-            const float sc = valid ? p.a_scale[r] : 0.f;
-#pragma unroll
-            for (int j = 0; j < 16; ++j) v[j] *= sc;
-          }
+          tmem_sum_planes(tacc, c0, p.n_planes, p.n_lo, v);
+          if (kFp8) scale_e4m3(p, r, valid, c0, v);
           epi.apply(epi_smem, g, r, valid, c0, p.n_out, v);
         }
         tc_fence_before();
@@ -723,24 +672,23 @@ __global__ void __launch_bounds__(kFp8 ? kThreadsFp8 : kThreads, 1)
         if (lane == 0) mbar_arrive(&acc_empty[buf]);
         continue;
       }
-      // shared tile: publish this CTA's partial, count in, finish if last
+      // shared tile: publish this CTA's partial (its column planes already summed), count in,
+      // finish if last
       const int slot = static_cast<int>(c - c_first);
       const int n_contrib = c_last - c_first + 1;
-      // slot layout [n_pad / 4][128 rows][4 columns]: a warp moves 512 contiguous bytes
+      // slot layout [n_cols / 4][128 rows][4 columns]: a warp moves 512 contiguous bytes
       float4* part_tile = reinterpret_cast<float4*>(p.partial) +
-                          static_cast<size_t>(t) * p.max_slots * (p.n_pad / 4) * 128 + m_local;
-      const size_t slot_stride = static_cast<size_t>(p.n_pad / 4) * 128;  // in float4
+                          static_cast<size_t>(t) * p.max_slots * (n_cols / 4) * 128 + m_local;
+      const size_t slot_stride = static_cast<size_t>(n_cols / 4) * 128;  // in float4
       {
         float4* dst = part_tile + slot * slot_stride;
-        for (int c0 = 0; c0 < p.n_pad; c0 += 16) {
-          uint32_t a[16];
-          tmem_ld16(tacc + c0, a);
-          tmem_wait_ld();
+        for (int c0 = 0; c0 < n_cols; c0 += 16) {
+          float v[16];
+          tmem_sum_planes(tacc, c0, p.n_planes, p.n_lo, v);
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4)
             __stcg(dst + (c0 / 4 + q4) * 128,
-                   make_float4(__uint_as_float(a[4 * q4]), __uint_as_float(a[4 * q4 + 1]),
-                               __uint_as_float(a[4 * q4 + 2]), __uint_as_float(a[4 * q4 + 3])));
+                   make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]));
         }
       }
       tc_fence_before();
@@ -768,17 +716,7 @@ __global__ void __launch_bounds__(kFp8 ? kThreadsFp8 : kThreads, 1)
       for (int c0 = 0; c0 < n_cols; c0 += 16) {
         float v[16];
         sum_slots(part_tile + (c0 / 4) * 128, slot_stride, n_contrib, v);
-        if (p.n_lo > 0) {
-          float w[16];
-          sum_slots(part_tile + ((p.n_lo + c0) / 4) * 128, slot_stride, n_contrib, w);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) v[j] += w[j];
-        }
-        if (kFp8) {
-          const float sc = valid ? p.a_scale[r] : 0.f;
-#pragma unroll
-          for (int j = 0; j < 16; ++j) v[j] *= sc;
-        }
+        if (kFp8) scale_e4m3(p, r, valid, c0, v);
         epi.apply(epi_smem, g, r, valid, c0, p.n_out, v);
       }
     }

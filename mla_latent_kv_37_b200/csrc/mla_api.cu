@@ -52,7 +52,7 @@ constexpr int kMaxParts = 1 << 16;  // upper bound on num_splits (host check bef
 constexpr int kSkMinUnits = 2;    // fewest stages' worth of weights a stream-K CTA streams
 constexpr int kSkMaxContrib = 4;  // aim for at most this many CTAs sharing one tile
 constexpr int kSkMaxStages = 12;
-constexpr int kFp8MaxBatch = 64;  // E4M3 products: 2 * 2B accumulator columns leave room for A
+constexpr int kFp8MaxBatch = 80;  // E4M3 W_O product: 3 planes x round16(B) <= 256 MMA columns
 constexpr size_t kSmemPerBlockMax = 232448;  // 227 KiB opt-in limit per CTA
 
 // ------------------------------------------------------------------------------------------
@@ -176,11 +176,15 @@ int default_parts(int sms, int max_clusters) { return max_clusters > 0 ? max_clu
 int round16(int x) { return (x + 15) / 16 * 16; }
 
 // One weight product of a layer: rows per group, 128-row tiles per group, K, groups, and the
-// activation columns (n_pad on the MMA's N side; n_lo > 0 when columns [n_lo, 2 n_lo) carry the
-// bf16 low halves of an fp32 input).
+// activation columns (n_pad on the MMA's N side; n_lo > 0 when the columns are n_pad / n_lo
+// planes of n_lo columns each, summed by the epilogue: the bf16 high and low halves of an fp32
+// input, or three E4M3 pieces); elem = bytes per element (2 bf16, 1 E4M3).  A K block is one
+// 128-byte row piece.
 struct GemmShape {
   int m_total, m_tiles, k, groups, n_pad, n_lo;
-  int k_blocks() const { return (k + 63) / 64; }
+  int elem = 2;
+  int k_blocks() const { return (k * elem + 127) / 128; }
+  int planes() const { return n_lo > 0 ? n_pad / n_lo : 1; }
 };
 
 // the five products of a layer on the bf16 path
@@ -216,6 +220,11 @@ GemmShape shape_wo_fold(const mla_dims* d) {
   return {d->d_model, (d->d_model + 127) / 128, d->n_heads * kDc, 1, 2 * round16(d->batch),
           round16(d->batch)};
 }
+// W_O in E4M3 against o_heads as three E4M3 planes (tcgen05 kind::f8f6f4)
+GemmShape shape_wo_e4m3(const mla_dims* d) {
+  return {d->d_model, (d->d_model + 127) / 128, d->n_heads * kDv, 1, 3 * round16(d->batch),
+          round16(d->batch), 1};
+}
 
 // Stream-K launch plan: K blocks per stage, CTAs, partial slots per tile, ring depth, smem.
 struct SkPlan {
@@ -248,41 +257,10 @@ SkPlan sk_plan(const GemmShape& s, size_t epi_bytes, int sms) {
   const size_t sb = sk::stage_bytes(s.n_pad, q.kbs);
   q.stages = static_cast<int>(std::min<size_t>(kSkMaxStages, budget / sb));
   q.smem = fixed + static_cast<size_t>(q.stages) * sb;
-  q.partial_bytes = q.max_slots > 1 ? static_cast<size_t>(q.tiles) * q.max_slots * s.n_pad *
-                                          128 * sizeof(float)
-                                    : 0;
-  return q;
-}
-
-// The same plan for E4M3 weights: smaller stages (64-byte A rows), and the widened A of every
-// stage in tensor memory next to the two accumulator buffers: stages * kbs * 32 + 2 n_pad <= 512.
-SkPlan sk_plan_fp8(const GemmShape& s, size_t epi_bytes, int sms) {
-  SkPlan q;
-  q.tiles = s.m_tiles * s.groups;
-  // alignment, tables, barriers (three per stage here)
-  const size_t fixed = 1024 + (epi_bytes + 15) / 16 * 16 + 512;
-  const size_t budget = kSmemPerBlockMax - fixed;
-  const int tmem_a = 512 - 2 * s.n_pad;
-  q.kbs = 1;
-  for (int kbs = 2; kbs <= 4 && kbs <= s.k_blocks(); kbs *= 2)
-    if (budget / sk::stage_bytes_fp8(s.n_pad, kbs) >= 2 && tmem_a / (kbs * 32) >= 2) q.kbs = kbs;
-  q.units = (s.k_blocks() + q.kbs - 1) / q.kbs;
-  q.iters = static_cast<long long>(q.tiles) * q.units;
-  long long P = std::min<long long>(sms, (q.iters + kSkMinUnits - 1) / kSkMinUnits);
-  P = std::min<long long>(P, static_cast<long long>(q.tiles) * kSkMaxContrib);
-  P = std::max<long long>(1, std::min(P, q.iters));
-  q.ctas = static_cast<int>(P);
-  for (long long t = 0; t < q.tiles; ++t) {
-    const int cf = sk::cta_of(t * q.units, q.iters, P);
-    const int cl = sk::cta_of((t + 1) * q.units - 1, q.iters, P);
-    q.max_slots = std::max(q.max_slots, cl - cf + 1);
-  }
-  const size_t sb = sk::stage_bytes_fp8(s.n_pad, q.kbs);
-  q.stages = static_cast<int>(std::min<size_t>({static_cast<size_t>(kSkMaxStages), budget / sb,
-                                                 static_cast<size_t>(tmem_a / (q.kbs * 32))}));
-  q.smem = fixed + static_cast<size_t>(q.stages) * sb;
-  q.partial_bytes = q.max_slots > 1 ? static_cast<size_t>(q.tiles) * q.max_slots * s.n_pad *
-                                          128 * sizeof(float)
+  // a partial slot holds the output columns only (the column planes are summed before it)
+  const int n_cols = s.n_lo > 0 ? s.n_lo : s.n_pad;
+  q.partial_bytes = q.max_slots > 1 ? static_cast<size_t>(q.tiles) * q.max_slots * n_cols * 128 *
+                                          sizeof(float)
                                     : 0;
   return q;
 }
@@ -323,7 +301,7 @@ Workspace layout(const mla_dims* d, int num_parts, int sms) {
       ctr = std::max(ctr, static_cast<size_t>(q.tiles) * 8);
     }
     if (d->batch <= kFp8MaxBatch) {
-      const SkPlan q = sk_plan_fp8(shape_wo(d), 0, sms);
+      const SkPlan q = sk_plan(shape_wo_e4m3(d), 0, sms);
       part = std::max(part, q.partial_bytes);
       ctr = std::max(ctr, static_cast<size_t>(q.tiles) * 8);
     }
@@ -342,7 +320,9 @@ Workspace layout(const mla_dims* d, int num_parts, int sms) {
   w.partial = take(part);
   w.counters = take(ctr);
   w.qn = take(std::max(2 * Bp * H * kDn * 2, B * H * kDn * 4));      // bf16 hi/lo, or fp32
-  w.o_split = take(2 * Bp * H * kDc * 2);                             // bf16 hi/lo of o_lat
+  // bf16 hi/lo of o_lat; once the W_UV product has read them, the E4M3 W_O call puts o_heads'
+  // three E4M3 planes [3][Bp][H*128] and their Bp scales here
+  w.o_split = take(2 * Bp * H * kDc * 2);
   w.oh_split = take(std::max(2 * Bp * H * kDv * 2, B * H * kDv * 4)); // bf16 hi/lo, or fp32
   w.plan = take(attn::PlanView::words(static_cast<int>(B), num_parts) * 4);
   w.part_o = take((B + num_parts) * H * kDc * 4);
@@ -410,15 +390,26 @@ int map_weights(CUtensorMap* m, const void* base, uint64_t rows, uint64_t groups
                 CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-// E4M3 weights [groups][rows][K] bytes as the view (64 k, rows, groups, K / 64), box
-// (64, 128, 1, kbs), 64-byte swizzle (the converters read it back row by row).
-int map_weights_fp8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t groups, uint64_t K,
-                    int kbs) {
-  const uint64_t dims[4] = {64, rows, groups, K / 64};
-  const uint64_t str[3] = {K, rows * K, 64};
-  const uint32_t box[4] = {64, 128, 1, static_cast<uint32_t>(kbs)};
+// E4M3 weights in 128 x 128 tiles (the layout mla_quantize_weights_fp8 writes) as the view
+// (128 k, 128 rows, K / 128, row tiles), box (128, 128, kbs, 1): kbs tiles in one contiguous run,
+// landing as the same 128-byte swizzled row pieces as map_weights.
+int map_weights_e4m3(CUtensorMap* m, const void* base, uint64_t rows, uint64_t K, int kbs) {
+  const uint64_t dims[4] = {128, 128, K / 128, (rows + 127) / 128};
+  const uint64_t str[3] = {128, 128 * 128, K * 128};
+  const uint32_t box[4] = {128, 128, static_cast<uint32_t>(kbs), 1};
   return encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, 4, dims, str, box,
-                CU_TENSOR_MAP_SWIZZLE_64B);
+                CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// E4M3 activation planes [n_rows][K] bytes as the view (128 k, 1, n_rows, K / 128), box
+// (128, 1, n_pad, kbs).
+int map_acts_e4m3(CUtensorMap* m, const void* base, uint64_t n_rows, uint64_t K, int n_pad,
+                  int kbs) {
+  const uint64_t dims[4] = {128, 1, n_rows, K / 128};
+  const uint64_t str[3] = {K, K, 128};
+  const uint32_t box[4] = {128, 1, static_cast<uint32_t>(n_pad), static_cast<uint32_t>(kbs)};
+  return encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, 4, dims, str, box,
+                CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 // Activations X: element (k, g, n) at n * n_stride + g * g_stride + 2 k (bytes), as the view
@@ -485,7 +476,8 @@ int run_streamk(const DevCtx* c, const GemmShape& s, const SkPlan& q, int n_out,
                 const CUtensorMap& a1, int a1_tile_start, int a_mn_major,
                 const CUtensorMap& xmap, char* ws, const Workspace& w, const Epi& epi,
                 cudaStream_t st, const CUtensorMap* a2 = nullptr, int a2_tile_start = 1 << 30,
-                const float* a_scale = nullptr) {
+                const float* a_scale = nullptr, const float* x_scale = nullptr,
+                int a_tiled = 0) {
   sk::Params p{};
   p.m_total = s.m_total;
   p.m_tiles = s.m_tiles;
@@ -497,8 +489,10 @@ int run_streamk(const DevCtx* c, const GemmShape& s, const SkPlan& q, int n_out,
   p.units = q.units;
   p.n_pad = s.n_pad;
   p.n_lo = s.n_lo;
+  p.n_planes = s.planes();
   p.n_out = n_out;
   p.a_mn_major = a_mn_major;
+  p.a_tiled = a_tiled;
   p.stages = q.stages;
   p.max_slots = q.max_slots;
   p.iters = q.iters;
@@ -510,9 +504,9 @@ int run_streamk(const DevCtx* c, const GemmShape& s, const SkPlan& q, int n_out,
   p.status = c->status;
   p.wait_ns = wait_limit_ns();
   p.a_scale = a_scale;
-  launch_pdl(sk::streamk_gemm_kernel<Epi, kFp8>, dim3(q.ctas),
-             dim3(kFp8 ? sk::kThreadsFp8 : sk::kThreads), q.smem, st, a0, a1, a2 ? *a2 : a1, xmap,
-             p, epi);
+  p.x_scale = x_scale;
+  launch_pdl(sk::streamk_gemm_kernel<Epi, kFp8>, dim3(q.ctas), dim3(sk::kThreads), q.smem, st, a0,
+             a1, a2 ? *a2 : a1, xmap, p, epi);
   return last_launch();
 }
 
@@ -1072,7 +1066,7 @@ int mla_out_proj_folded(const mla_dims* dims, const float* o_lat, const void* w_
 int mla_quantize_weights_fp8(const void* w, int64_t rows, int64_t cols, void* codes,
                              float* scale, mla_stream_t stream) {
   if (!w || !codes || !scale) return MLA_ERR_NULL_ARG;
-  if (rows < 1 || rows > INT32_MAX || cols < 64 || cols % 64) return MLA_ERR_ARG;
+  if (rows < 1 || rows > INT32_MAX || cols < 128 || cols % 128) return MLA_ERR_ARG;
   if (!aligned(w, 16) || !aligned(codes, 16) || !aligned(scale, 4)) return MLA_ERR_ALIGN;
   DevCtx* c = nullptr;
   int rc = device_ctx(&c);
@@ -1104,8 +1098,8 @@ int mla_out_proj_fp8(const mla_dims* dims, const float* o_lat, const void* w_uv,
   const int B = dims->batch, D = dims->d_model, H = dims->n_heads;
   char* ws = static_cast<char*>(workspace);
   __nv_bfloat16* os = reinterpret_cast<__nv_bfloat16*>(ws + w.o_split);
-  void* oh_split = ws + w.oh_split;
-  // o_h = W_UV_h [o_lat_hi | o_lat_lo] (bf16 weights, as in mla_out_proj)
+  float* oh32 = reinterpret_cast<float*>(ws + w.oh_split);
+  // o_h = W_UV_h [o_lat_hi | o_lat_lo] (bf16 weights, as in mla_out_proj); o_heads kept in fp32
   const GemmShape s1 = shape_wuv(dims);
   const int Bp = s1.n_lo;
   const size_t n = static_cast<size_t>(B) * H * kDc;
@@ -1118,22 +1112,25 @@ int mla_out_proj_fp8(const mla_dims* dims, const float* o_lat, const void* w_uv,
   if ((rc = map_weights(&a, w_uv, kDv, H, kDc, q1.kbs))) return rc;
   if ((rc = map_acts(&bm, os, H, 2 * Bp, kDc, kDc * 2ull, kDc * 2ull * H, s1.n_pad, q1.kbs)))
     return rc;
-  // o_heads as f16 hi/lo planes: the E4M3 codes widen exactly to f16, so the W_O product runs
-  // on f16 operands (22 bits of o_heads instead of the bf16 planes' 16)
-  sk::EpiWuv e1{H, Bp, static_cast<__nv_bfloat16*>(o_heads), nullptr,
-                static_cast<__half*>(oh_split)};
+  sk::EpiWuv e1{H, Bp, static_cast<__nv_bfloat16*>(o_heads), nullptr, oh32};
   if ((rc = run_streamk(c, s1, q1, B, nullptr, 0.f, a, a, 1 << 30, 0, bm, ws, w, e1, st)))
     return rc;
-  // out = (decode(W_O codes) * s) [o_heads_hi | o_heads_lo]  (f16 x f16 -> fp32)
-  const GemmShape s2 = shape_wo(dims);
+  // o_heads row b -> three E4M3 planes and a scale (the W_UV input is consumed by now)
+  const GemmShape s2 = shape_wo_e4m3(dims);
   const uint64_t K = static_cast<uint64_t>(H) * kDv;
-  const SkPlan q2 = sk_plan_fp8(s2, 0, c->sms);
+  uint8_t* planes = reinterpret_cast<uint8_t*>(ws + w.o_split);
+  float* x_scale = reinterpret_cast<float*>(ws + w.o_split + align_up(3 * Bp * K, 256));
+  launch_pdl(fp8::split_planes_kernel, dim3(static_cast<unsigned>(Bp)), dim3(256), 0, st,
+             static_cast<const float*>(oh32), B, static_cast<long long>(K), Bp, planes, x_scale);
+  if ((rc = last_launch())) return rc;
+  // out = s_W,r * s_x,b * sum over planes of (W_O codes) x (plane codes), kind::f8f6f4
+  const SkPlan q2 = sk_plan(s2, 0, c->sms);
   CUtensorMap a2, b2;
-  if ((rc = map_weights_fp8(&a2, w_o_codes, D, 1, K, q2.kbs))) return rc;
-  if ((rc = map_acts(&b2, oh_split, 1, 2 * Bp, K, K * 2, K * 2, s2.n_pad, q2.kbs))) return rc;
+  if ((rc = map_weights_e4m3(&a2, w_o_codes, D, K, q2.kbs))) return rc;
+  if ((rc = map_acts_e4m3(&b2, planes, 3 * Bp, K, s2.n_pad, q2.kbs))) return rc;
   sk::EpiWo e2{D, static_cast<__nv_bfloat16*>(out)};
   return run_streamk<sk::EpiWo, true>(c, s2, q2, B, nullptr, 0.f, a2, a2, 1 << 30, 0, b2, ws, w,
-                                      e2, st, nullptr, 1 << 30, w_o_scale);
+                                      e2, st, nullptr, 1 << 30, w_o_scale, x_scale, 1);
 }
 
 int mla_merge_partials(const mla_dims* dims, int32_t n_parts, const float* part_o,

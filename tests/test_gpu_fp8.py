@@ -1,6 +1,7 @@
 """E4M3 (FP8) weights: the GPU quantization against the oracle's (codes and scales bit for
-bit), and the output projection with W_O stored as E4M3 against the oracle's fp64 step computed
-with the weights the codes stand for."""
+bit), and the output projection with W_O stored as E4M3 (tcgen05 kind::f8f6f4, o_heads as three
+scaled E4M3 planes) against the oracle's fp64 step computed with the weights the codes stand
+for."""
 import numpy as np
 import pytest
 import torch
@@ -11,23 +12,35 @@ from tests.gpu_common import Workload, assert_close, dev, to_np
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("rows,cols,std", [(300, 1024, 0.02), (7, 16384, 1.0), (129, 64, 3e-3)])
+def untile(codes, rows, cols):
+    """Codes in 128 x 128 tiles (row tile, then column tile; row-major inside) -> [rows][cols]."""
+    rt = codes.numel() // (128 * cols)
+    t = codes.reshape(rt, cols // 128, 128, 128).permute(0, 2, 1, 3).reshape(rt * 128, cols)
+    return t[:rows].numpy()
+
+
+def tiled_rows(rows):
+    return (rows + 127) // 128 * 128
+
+
+@pytest.mark.parametrize("rows,cols,std", [(300, 1024, 0.02), (7, 16384, 1.0), (129, 128, 3e-3)])
 def test_quantize_matches_oracle_bit_for_bit(rows, cols, std):
     import mla_latent_kv_37_b200 as M
     g = torch.Generator().manual_seed(rows + cols)
     w = (torch.randn(rows, cols, generator=g) * std).to(torch.bfloat16)
     w[1, :] = 0.0                      # a zero row: scale 1, all codes 0
     w[0, 5] = 1e-30                    # far below the smallest step of its row: a zero code
-    codes = torch.empty(rows, cols, dtype=torch.uint8, device="cuda")
+    codes = torch.empty(tiled_rows(rows), cols, dtype=torch.uint8, device="cuda")
     scale = torch.empty(rows, dtype=torch.float32, device="cuda")
     M.mla_quantize_weights_fp8(dev(w), codes, scale)
     torch.cuda.synchronize()
     exp_codes, exp_scale = O.quantize_rows_e4m3(w.float().numpy())
     assert np.array_equal(scale.cpu().numpy(), exp_scale)
-    assert np.array_equal(codes.cpu().numpy(), exp_codes)
+    assert np.array_equal(untile(codes.cpu(), rows, cols), exp_codes)
 
 
-@pytest.mark.parametrize("B,H,D", [(3, 16, 1024), (32, 128, 7168), (64, 32, 512)])
+@pytest.mark.parametrize("B,H,D", [(3, 16, 1024), (32, 128, 7168), (64, 32, 512),
+                                   (80, 16, 1024)])
 def test_out_proj_fp8_matches_oracle(B, H, D):
     import mla_latent_kv_37_b200 as M
     hist = [(41 * i + 3) % 200 for i in range(B)]
@@ -49,7 +62,7 @@ def test_out_proj_fp8_matches_oracle(B, H, D):
     M.mla_out_proj_fp8(d, o_lat, dev(w.w_uv), codes, scale, out, ws, o_heads=o_heads)
     torch.cuda.synchronize()
     assert M.mla_get_status() == 0
-    w_o_deq = O.dequantize_rows_e4m3(codes.cpu().numpy(), scale.cpu().numpy())
+    w_o_deq = O.dequantize_rows_e4m3(untile(codes.cpu(), D, H * 128), scale.cpu().numpy())
     for b in sorted({0, B // 2, B - 1}):
         ref = wl.oracle(b)  # o_heads from the bf16 W_UV; out recomputed with the E4M3 W_O
         assert_close(to_np(o_heads[b].cpu()), ref["o_heads"], torch.bfloat16, f"o_heads b={b}")
@@ -58,13 +71,14 @@ def test_out_proj_fp8_matches_oracle(B, H, D):
 
 
 def test_out_proj_fp8_rejects_large_batch():
+    """Batch 81: three E4M3 planes of round16(81) = 96 columns exceed the MMA's 256."""
     import mla_latent_kv_37_b200 as M
-    d = M.dims(65, 16, 1024)
+    d = M.dims(81, 16, 1024)
     with pytest.raises(M.MlaError) as e:
-        M.mla_out_proj_fp8(d, torch.empty(65, 16, 512, device="cuda"),
+        M.mla_out_proj_fp8(d, torch.empty(81, 16, 512, device="cuda"),
                            torch.empty(16 * 128, 512, dtype=torch.bfloat16, device="cuda"),
                            torch.empty(1024, 16 * 128, dtype=torch.uint8, device="cuda"),
                            torch.empty(1024, device="cuda"),
-                           torch.empty(65, 1024, dtype=torch.bfloat16, device="cuda"),
+                           torch.empty(81, 1024, dtype=torch.bfloat16, device="cuda"),
                            M.workspace(d))
     assert e.value.code == -2
