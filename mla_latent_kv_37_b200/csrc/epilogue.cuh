@@ -147,11 +147,15 @@ __global__ void wuk_epilogue_kernel(const float* __restrict__ part, int n_pad, i
 
 // o_lat fp32 [n] -> bf16 hi/lo planes: out[i] = hi, out[plane + i] = lo (plane >= n).  n and
 // plane are multiples of 8 and x, out 16-byte aligned: each thread converts 8 values with one
-// 32-byte load and two 16-byte stores.
+// 32-byte load and two 16-byte stores.  Also zeroes zero[0 .. n_zero) (block 0), a buffer the
+// next kernel accumulates into.
 __global__ void split_hi_lo_kernel(const float* __restrict__ x, size_t n, size_t plane,
-                                   __nv_bfloat16* __restrict__ out) {
+                                   __nv_bfloat16* __restrict__ out, unsigned int* zero,
+                                   int n_zero) {
   griddep_launch_dependents();
   griddep_wait();
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero[i] = 0u;
   const size_t n8 = n / 8;
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n8;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {

@@ -59,59 +59,48 @@ __device__ __forceinline__ float2 e4m3x2_value(uint16_t c) {
   return __half22float2(*reinterpret_cast<const __half2*>(&h));
 }
 
-// An fp32 activation row x_b (K values) as a scale and three E4M3 planes: s_b = max_k |x_bk| / 448
-// (at least FLT_MIN), y = x / s_b; p1 = E4M3(y), p2 = E4M3(y - p1), p3 = E4M3(y - p1 - p2), each
-// difference exact in fp32.  p1 + p2 + p3 keeps about 12 significant bits of y, so
-// s_b (p1 + p2 + p3) stands in for x_b in a product with E4M3 weights.  planes: [3][rows_pad][K];
-// rows in [rows, rows_pad) are written as zeros.  One block per row; K a multiple of 8; x and
+// fp32 activation rows x_b (K values each) as a scale and three E4M3 planes: s_b = m_b / 448
+// (at least FLT_MIN) with m_b = max_k |x_bk| given as fp32 bits in rowmax[b]; y = x / s_b;
+// p1 = E4M3(y), p2 = E4M3(y - p1), p3 = E4M3(y - p1 - p2), each difference exact in fp32.
+// p1 + p2 + p3 keeps about 12 significant bits of y, so s_b (p1 + p2 + p3) stands in for x_b in a
+// product with E4M3 weights.  planes: [3][rows_pad][K]; rows in [rows, rows_pad) are written as
+// zeros.  Each thread converts 8 consecutive values (grid-stride); K a multiple of 8; x and
 // planes 16- and 8-byte aligned.
 __global__ void __launch_bounds__(256)
-    split_planes_kernel(const float* __restrict__ x, int rows, long long K, int rows_pad,
-                        uint8_t* __restrict__ planes, float* __restrict__ scale) {
-  __shared__ float part[8];
+    split_planes_kernel(const float* __restrict__ x, const unsigned int* __restrict__ rowmax,
+                        int rows, long long K, int rows_pad, uint8_t* __restrict__ planes,
+                        float* __restrict__ scale) {
   griddep_launch_dependents();
   griddep_wait();
-  const int b = blockIdx.x;
-  const size_t plane = static_cast<size_t>(rows_pad) * K;
-  uint2* out = reinterpret_cast<uint2*>(planes + static_cast<size_t>(b) * K);
   const long long n8 = K / 8;
-  if (b >= rows) {
-    for (long long j = threadIdx.x; j < n8; j += blockDim.x)
-      for (int pl = 0; pl < 3; ++pl) out[pl * (plane / 8) + j] = make_uint2(0u, 0u);
-    if (threadIdx.x == 0) scale[b] = 0.f;
-    return;
-  }
-  const float4* xr = reinterpret_cast<const float4*>(x + static_cast<size_t>(b) * K);
-  float m = 0.f;
-  for (long long j = threadIdx.x; j < K / 4; j += blockDim.x) {
-    const float4 v = xr[j];
-    m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = m;
-  __syncthreads();
-  m = part[0];
-  for (int k = 1; k < static_cast<int>(blockDim.x >> 5); ++k) m = fmaxf(m, part[k]);
-  const float s = fmaxf(__fdiv_rn(m, 448.f), FLT_MIN);
-  if (threadIdx.x == 0) scale[b] = s;
-  for (long long j = threadIdx.x; j < n8; j += blockDim.x) {
-    const float4 u = xr[2 * j], w = xr[2 * j + 1];
+  const size_t plane8 = static_cast<size_t>(rows_pad) * n8;  // one plane, in 8-byte groups
+  uint2* out = reinterpret_cast<uint2*>(planes);
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
+       i < static_cast<long long>(plane8); i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int b = static_cast<int>(i / n8);
+    if (b >= rows) {
+      for (int pl = 0; pl < 3; ++pl) out[pl * plane8 + i] = make_uint2(0u, 0u);
+      continue;
+    }
+    const float s = fmaxf(__fdiv_rn(__uint_as_float(rowmax[b]), 448.f), FLT_MIN);
+    if (i - static_cast<long long>(b) * n8 == 0) scale[b] = s;
+    const float4 u = reinterpret_cast<const float4*>(x)[2 * i];
+    const float4 w = reinterpret_cast<const float4*>(x)[2 * i + 1];
     float y[8] = {u.x, u.y, u.z, u.w, w.x, w.y, w.z, w.w};
 #pragma unroll
-    for (int i = 0; i < 8; ++i) y[i] = __fdiv_rn(y[i], s);
+    for (int k = 0; k < 8; ++k) y[k] = __fdiv_rn(y[k], s);
 #pragma unroll
     for (int pl = 0; pl < 3; ++pl) {
       uint32_t c[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint16_t q = e4m3x2(y[2 * i], y[2 * i + 1]);
+      for (int k = 0; k < 4; ++k) {
+        const uint16_t q = e4m3x2(y[2 * k], y[2 * k + 1]);
         const float2 d = e4m3x2_value(q);
-        y[2 * i] -= d.x;
-        y[2 * i + 1] -= d.y;
-        c[i] = q;
+        y[2 * k] -= d.x;
+        y[2 * k + 1] -= d.y;
+        c[k] = q;
       }
-      out[pl * (plane / 8) + j] = make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+      out[pl * plane8 + i] = make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
     }
   }
 }

@@ -12,12 +12,16 @@
 // the next).
 //
 // A tile covered by one CTA is finished straight from TMEM.  A tile shared by several CTAs is
-// finished by whichever contributor arrives last: each contributor writes its partial sum to
-// slot (its CTA index - the tile's first CTA index) of the tile's partial area and counts
-// itself on the tile's counter; the one that completes the count adds the slots in slot order
-// (so the result does not depend on arrival order) and runs the epilogue.  Nobody waits for
-// another CTA.  Counters are tagged with a per-launch epoch in their upper 32 bits, so stale
-// counts from earlier launches read as zero and the workspace never needs clearing; the
+// finished by its first contributor, the CTA that accumulates the tile's first K blocks: that
+// segment is the last of the CTA's range, while the other contributors cover the tile at the
+// start (or all) of theirs, so by the time it gets there their partial sums are long written.
+// Each other contributor writes its partial sum (column planes already added) to slot (its CTA
+// index - the tile's first CTA index) of the tile's partial area, and each of its epilogue
+// warps counts itself on the tile's counter; the finisher waits (bounded) for the full count,
+// adds slots 1, 2, ... in slot order to its own sum from TMEM (so the result does not depend on
+// arrival order) and runs the epilogue.  Only the finisher ever waits, and only for CTAs that
+// wait for nobody.  Counters are tagged with a per-launch epoch in their upper 32 bits, so
+// stale counts from earlier launches read as zero and the workspace never needs clearing; the
 // finisher also clears its tile's counter, so a launch replayed with the same epoch (from a
 // CUDA graph) starts from zero too.
 //
@@ -346,12 +350,27 @@ struct EpiWuv {
   int b_pad;
   __nv_bfloat16* o_heads;
   __nv_bfloat16* oh;
-  float* oh32 = nullptr;  // or o_heads in fp32 [b][h][128] (split into E4M3 planes next)
+  float* oh32 = nullptr;  // or o_heads in fp32 [b][h][128] (split into E4M3 planes next),
+  unsigned int* rowmax = nullptr;  // with max_{h,i} |o_heads[b][h][i]| per b (fp32 bits,
+                                   // zeroed before the launch) raised by atomicMax
   __host__ __device__ static size_t smem_bytes(int) { return 0; }
   __device__ void prepare(uint8_t*, int, int, int) const {}
   __device__ void apply(const uint8_t*, int g, int r, bool valid, int c0, int n_out,
                         float (&v)[16]) const {
     constexpr int kDv = 128;
+    if (rowmax) {
+      // |v| over the warp's 32 rows for each of the 16 columns; lane j raises column c0 + j
+      float mine = 0.f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        float m = valid ? fabsf(v[j]) : 0.f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if ((threadIdx.x & 31) == j) mine = m;
+      }
+      const int lane = threadIdx.x & 31;
+      if (lane < 16 && c0 + lane < n_out) atomicMax(rowmax + c0 + lane, __float_as_uint(mine));
+    }
     if (!valid) return;
     const size_t plane = static_cast<size_t>(b_pad) * H * kDv;
 #pragma unroll
@@ -389,11 +408,11 @@ struct EpiWo {
   }
 };
 
-// Sum of 16 columns of one row over slots 0 .. n-1, added in slot order.  src points at the
-// row's first float4 of the 16 columns in slot 0; the loads of four slots are in flight at once.
-__device__ __forceinline__ void sum_slots(const float4* src, size_t slot_stride, int n,
+// Adds 16 columns of one row from slots 1 .. n-1, in slot order, to v.  src points at the row's
+// first float4 of the 16 columns in slot 0; the loads of four slots are in flight at once.
+__device__ __forceinline__ void add_slots(const float4* src, size_t slot_stride, int n,
                                           float (&v)[16]) {
-  for (int s0 = 0; s0 < n; s0 += 4) {
+  for (int s0 = 1; s0 < n; s0 += 4) {
     float4 y[4][4];
 #pragma unroll
     for (int u = 0; u < 4; ++u)
@@ -405,17 +424,30 @@ __device__ __forceinline__ void sum_slots(const float4* src, size_t slot_stride,
       if (s0 + u >= n) break;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        if (s0 + u == 0) {
-          v[4 * q] = y[u][q].x;
-          v[4 * q + 1] = y[u][q].y;
-          v[4 * q + 2] = y[u][q].z;
-          v[4 * q + 3] = y[u][q].w;
-        } else {
-          v[4 * q] += y[u][q].x;
-          v[4 * q + 1] += y[u][q].y;
-          v[4 * q + 2] += y[u][q].z;
-          v[4 * q + 3] += y[u][q].w;
-        }
+        v[4 * q] += y[u][q].x;
+        v[4 * q + 1] += y[u][q].y;
+        v[4 * q + 2] += y[u][q].z;
+        v[4 * q + 3] += y[u][q].w;
+      }
+    }
+  }
+}
+
+// The finishing CTA of a shared tile waits until the other contributors' warps (4 each) have
+// counted in under this launch's epoch.  Bounded like every wait: false on abort or timeout.
+__device__ __forceinline__ bool wait_count(const unsigned long long* ctr, uint32_t epoch,
+                                           uint32_t target, const WaitCtx& w) {
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 1;; ++i) {
+    const unsigned long long v = *reinterpret_cast<const volatile unsigned long long*>(ctr);
+    if (static_cast<uint32_t>(v >> 32) == epoch && static_cast<uint32_t>(v) >= target)
+      return true;
+    if ((i & 15) == 0) {
+      if (*w.abort_flag) return false;
+      if (globaltimer_ns() - t0 > w.limit_ns) {
+        *w.abort_flag = 1;
+        atomicOr(w.status, MLA_STATUS_TIMEOUT);
+        return false;
       }
     }
   }
@@ -468,8 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty_bar = full_bar + p.stages;
   uint64_t* acc_full = empty_bar + p.stages;   // [2]
   uint64_t* acc_empty = acc_full + 2;          // [2], 4 arrivals (one per epilogue warp)
-  uint64_t* epi_sync = acc_empty + 2;          // 4 arrivals
-  uint64_t* fin_ready = epi_sync + 1;          // 1 arrival
+  uint64_t* fin_ready = acc_empty + 2;         // 1 arrival: a shared tile's count is complete
   uint64_t* mma_done = fin_ready + 1;          // final drain of the MMA pipe
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -494,7 +525,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], 4);
     }
-    mbar_init(epi_sync, 4);
     mbar_init(fin_ready, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -672,16 +702,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(&acc_empty[buf]);
         continue;
       }
-      // shared tile: publish this CTA's partial (its column planes already summed), count in,
-      // finish if last
-      const int slot = static_cast<int>(c - c_first);
       const int n_contrib = c_last - c_first + 1;
       // slot layout [n_cols / 4][128 rows][4 columns]: a warp moves 512 contiguous bytes
       float4* part_tile = reinterpret_cast<float4*>(p.partial) +
                           static_cast<size_t>(t) * p.max_slots * (n_cols / 4) * 128 + m_local;
       const size_t slot_stride = static_cast<size_t>(n_cols / 4) * 128;  // in float4
-      {
-        float4* dst = part_tile + slot * slot_stride;
+      if (c != c_first) {
+        // shared tile, not ours to finish: publish the partial sum, count this warp in
+        float4* dst = part_tile + static_cast<size_t>(c - c_first) * slot_stride;
         for (int c0 = 0; c0 < n_cols; c0 += 16) {
           float v[16];
           tmem_sum_planes(tacc, c0, p.n_planes, p.n_lo, v);
@@ -690,35 +718,39 @@ __global__ void __launch_bounds__(kThreads, 1)
             __stcg(dst + (c0 / 4 + q4) * 128,
                    make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]));
         }
+        tc_fence_before();
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&acc_empty[buf]);
+          count_in(&p.counters[t], p.epoch, p.status);
+        }
+        continue;
       }
-      tc_fence_before();
-      __threadfence();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&acc_empty[buf]);
-        mbar_arrive(epi_sync);
-      }
+      // shared tile to finish: wait for the other contributors' 4 (n_contrib - 1) warps
       const uint32_t ph = static_cast<uint32_t>(multi & 1);
       ++multi;
       if (warp == 2 && lane == 0) {
-        int fin = 0;
-        if (mbar_wait(epi_sync, ph, wc)) {
-          const uint32_t n = count_in(&p.counters[t], p.epoch, p.status);
-          fin = (n == static_cast<uint32_t>(n_contrib)) ? 1 : 0;
-          if (fin) atomicExch(&p.counters[t], 0ull);  // last user of this counter in the launch
-          __threadfence();
-        }
-        *fin_flag = fin;
+        const bool ok = wait_count(&p.counters[t], p.epoch,
+                                   4u * static_cast<uint32_t>(n_contrib - 1), wc);
+        if (ok) atomicExch(&p.counters[t], 0ull);  // last user of this counter in the launch
+        __threadfence();
+        *fin_flag = ok ? 1 : 0;
         mbar_arrive(fin_ready);
       }
       if (!warp_wait(fin_ready, ph, wc)) break;
-      if (!*fin_flag) continue;
-      for (int c0 = 0; c0 < n_cols; c0 += 16) {
-        float v[16];
-        sum_slots(part_tile + (c0 / 4) * 128, slot_stride, n_contrib, v);
-        if (kFp8) scale_e4m3(p, r, valid, c0, v);
-        epi.apply(epi_smem, g, r, valid, c0, p.n_out, v);
+      if (*fin_flag) {
+        for (int c0 = 0; c0 < n_cols; c0 += 16) {
+          float v[16];
+          tmem_sum_planes(tacc, c0, p.n_planes, p.n_lo, v);
+          add_slots(part_tile + (c0 / 4) * 128, slot_stride, n_contrib, v);
+          if (kFp8) scale_e4m3(p, r, valid, c0, v);
+          epi.apply(epi_smem, g, r, valid, c0, p.n_out, v);
+        }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
     }
   }
 

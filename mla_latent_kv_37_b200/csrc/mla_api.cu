@@ -275,11 +275,11 @@ uint32_t next_epoch() {
 // ------------------------------------------------------------------------------------------
 // workspace layout
 // ------------------------------------------------------------------------------------------
-// [partial, counters, qn, o_split, oh_split) serve the projection products and are the same for
-// every split count; [plan, part_o, part_lse) serve the decode call and grow with its parts.  A
-// projection call therefore needs only `plan` bytes, the decode call all `total`.
+// [partial, counters, qn, o_split, oh_split, xmax) serve the projection products and are the
+// same for every split count; [plan, part_o, part_lse) serve the decode call and grow with its
+// parts.  A projection call therefore needs only `plan` bytes, the decode call all `total`.
 struct Workspace {
-  size_t partial, counters, qn, o_split, oh_split, plan, part_o, part_lse, total;
+  size_t partial, counters, qn, o_split, oh_split, xmax, plan, part_o, part_lse, total;
 };
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -324,6 +324,7 @@ Workspace layout(const mla_dims* d, int num_parts, int sms) {
   // three E4M3 planes [3][Bp][H*128] and their Bp scales here
   w.o_split = take(2 * Bp * H * kDc * 2);
   w.oh_split = take(std::max(2 * Bp * H * kDv * 2, B * H * kDv * 4)); // bf16 hi/lo, or fp32
+  w.xmax = take(Bp * 4);  // E4M3 W_O call: max |o_heads[b]| per batch row (fp32 bits)
   w.plan = take(attn::PlanView::words(static_cast<int>(B), num_parts) * 4);
   w.part_o = take((B + num_parts) * H * kDc * 4);
   w.part_lse = take((B + num_parts) * H * 4);
@@ -890,7 +891,8 @@ int mla_out_proj(const mla_dims* dims, const float* o_lat, const void* w_uv, con
     const size_t n = static_cast<size_t>(B) * H * kDc;
     launch_pdl(split_hi_lo_kernel,
                dim3(static_cast<unsigned>(std::min<size_t>((n / 8 + 255) / 256, 4096))), dim3(256),
-               0, st, o_lat, n, static_cast<size_t>(Bp) * H * kDc, os);
+               0, st, o_lat, n, static_cast<size_t>(Bp) * H * kDc, os,
+               static_cast<unsigned int*>(nullptr), 0);
     if ((rc = last_launch())) return rc;
     // o_h = W_UV_h [o_lat_hi | o_lat_lo]
     const SkPlan q1 = sk_plan(s1, 0, c->sms);
@@ -1049,7 +1051,8 @@ int mla_out_proj_folded(const mla_dims* dims, const float* o_lat, const void* w_
   // o_lat -> bf16 hi/lo planes [2][Bp][H * 512], the K layout of the folded product
   launch_pdl(split_hi_lo_kernel,
              dim3(static_cast<unsigned>(std::min<size_t>((n / 8 + 255) / 256, 4096))), dim3(256),
-             0, st, o_lat, n, static_cast<size_t>(Bp) * H * kDc, os);
+             0, st, o_lat, n, static_cast<size_t>(Bp) * H * kDc, os,
+             static_cast<unsigned int*>(nullptr), 0);
   if ((rc = last_launch())) return rc;
   const uint64_t K = static_cast<uint64_t>(H) * kDc;
   const SkPlan q = sk_plan(s, 0, c->sms);
@@ -1099,20 +1102,21 @@ int mla_out_proj_fp8(const mla_dims* dims, const float* o_lat, const void* w_uv,
   char* ws = static_cast<char*>(workspace);
   __nv_bfloat16* os = reinterpret_cast<__nv_bfloat16*>(ws + w.o_split);
   float* oh32 = reinterpret_cast<float*>(ws + w.oh_split);
+  unsigned int* xmax = reinterpret_cast<unsigned int*>(ws + w.xmax);
   // o_h = W_UV_h [o_lat_hi | o_lat_lo] (bf16 weights, as in mla_out_proj); o_heads kept in fp32
   const GemmShape s1 = shape_wuv(dims);
   const int Bp = s1.n_lo;
   const size_t n = static_cast<size_t>(B) * H * kDc;
   launch_pdl(split_hi_lo_kernel,
              dim3(static_cast<unsigned>(std::min<size_t>((n / 8 + 255) / 256, 4096))), dim3(256),
-             0, st, o_lat, n, static_cast<size_t>(Bp) * H * kDc, os);
+             0, st, o_lat, n, static_cast<size_t>(Bp) * H * kDc, os, xmax, Bp);
   if ((rc = last_launch())) return rc;
   const SkPlan q1 = sk_plan(s1, 0, c->sms);
   CUtensorMap a, bm;
   if ((rc = map_weights(&a, w_uv, kDv, H, kDc, q1.kbs))) return rc;
   if ((rc = map_acts(&bm, os, H, 2 * Bp, kDc, kDc * 2ull, kDc * 2ull * H, s1.n_pad, q1.kbs)))
     return rc;
-  sk::EpiWuv e1{H, Bp, static_cast<__nv_bfloat16*>(o_heads), nullptr, oh32};
+  sk::EpiWuv e1{H, Bp, static_cast<__nv_bfloat16*>(o_heads), nullptr, oh32, xmax};
   if ((rc = run_streamk(c, s1, q1, B, nullptr, 0.f, a, a, 1 << 30, 0, bm, ws, w, e1, st)))
     return rc;
   // o_heads row b -> three E4M3 planes and a scale (the W_UV input is consumed by now)
@@ -1120,8 +1124,12 @@ int mla_out_proj_fp8(const mla_dims* dims, const float* o_lat, const void* w_uv,
   const uint64_t K = static_cast<uint64_t>(H) * kDv;
   uint8_t* planes = reinterpret_cast<uint8_t*>(ws + w.o_split);
   float* x_scale = reinterpret_cast<float*>(ws + w.o_split + align_up(3 * Bp * K, 256));
-  launch_pdl(fp8::split_planes_kernel, dim3(static_cast<unsigned>(Bp)), dim3(256), 0, st,
-             static_cast<const float*>(oh32), B, static_cast<long long>(K), Bp, planes, x_scale);
+  const size_t groups8 = static_cast<size_t>(Bp) * K / 8;
+  launch_pdl(fp8::split_planes_kernel,
+             dim3(static_cast<unsigned>(std::min<size_t>((groups8 + 255) / 256, 4 * c->sms))),
+             dim3(256), 0, st, static_cast<const float*>(oh32),
+             static_cast<const unsigned int*>(xmax), B, static_cast<long long>(K), Bp, planes,
+             x_scale);
   if ((rc = last_launch())) return rc;
   // out = s_W,r * s_x,b * sum over planes of (W_O codes) x (plane codes), kind::f8f6f4
   const SkPlan q2 = sk_plan(s2, 0, c->sms);
