@@ -259,9 +259,19 @@ int mla_out_proj_folded(const mla_dims* dims, const float* o_lat, const void* w_
  *   product then streams whole 16 KB tiles from HBM.  The padding rows of the last row tile
  *   are not written and never reach a result.
  *
+ * mla_append_absorb_fp8 -- mla_append_absorb with W_DKV, W_KR and W_Q stored as E4M3 (each
+ *   as mla_quantize_weights_fp8 writes it, with its row scales); W_UK stays bf16.  bf16 path
+ *   only, batch <= 80 and d_model a multiple of 128 (else MLA_ERR_DIMS).  Each hidden-state
+ *   row h_b enters the E4M3 x E4M3 product as a power-of-two scale s_b (the smallest power of
+ *   two >= max|h_b| / 448) and two E4M3 planes whose sum is h_b / s_b exactly (a bf16 value has
+ *   8 significant bits; only parts below E4M3's smallest subnormal, under about 2^-8 of the
+ *   row's largest element, are dropped).  Each product row is w_scale[row] * s_b * (sum over
+ *   planes) in fp32; the epilogue (cache rows, RoPE, q_nope planes, W_UK absorption, q_lo) is
+ *   that of mla_append_absorb.  Workspace as mla_append_absorb.
+ *
  * mla_out_proj_fp8 -- mla_out_proj with W_O stored as E4M3 codes + row scales (w_o_codes:
- *   W_O [D, H*d_v] as mla_quantize_weights_fp8 writes it, w_o_scale [D]); W_UV stays bf16.  out is required, o_heads optional.  bf16
- *   path only, batch <= 80 (MLA_ERR_DIMS above: the three activation planes below take
+ *   W_O [D, H*d_v] as mla_quantize_weights_fp8 writes it, w_o_scale [D]); W_UV stays bf16.
+ *   out is required, o_heads optional.  bf16 path only, batch <= 80 (MLA_ERR_DIMS above: the three activation planes below take
  *   3 * round16(batch) of the 256 columns of one MMA).  The codes stream from HBM at one byte
  *   per weight into E4M3 x E4M3 tensor-core products (fp32 sums).  Each o_heads row b enters
  *   as a scale s_b = max|o_b| / 448 and three E4M3 planes whose sum keeps about 12 significant
@@ -270,6 +280,14 @@ int mla_out_proj_folded(const mla_dims* dims, const float* o_lat, const void* w_
  */
 int mla_quantize_weights_fp8(const void* w, int64_t rows, int64_t cols, void* codes,
                              float* scale, mla_stream_t stream);
+
+int mla_append_absorb_fp8(const mla_dims* dims, const void* h, const void* w_dkv_codes,
+                          const float* w_dkv_scale, const void* w_kr_codes,
+                          const float* w_kr_scale, const void* w_q_codes, const float* w_q_scale,
+                          const void* w_uk, const int32_t* positions, const int32_t* page_table,
+                          int32_t max_pages, void* cache_pool, int32_t num_pages, void* q_cat,
+                          void* q_lo, void* workspace, size_t workspace_bytes,
+                          mla_stream_t stream);
 
 int mla_out_proj_fp8(const mla_dims* dims, const float* o_lat, const void* w_uv,
                      const void* w_o_codes, const float* w_o_scale, void* o_heads, void* out,

@@ -83,6 +83,8 @@ _SIGS = {
     "mla_quantize_weights_fp8": (ctypes.c_int, [_P, ctypes.c_int64, ctypes.c_int64, _P, _P, _P]),
     "mla_out_proj_fp8": (ctypes.c_int, [ctypes.POINTER(mla_dims), _P, _P, _P, _P, _P, _P, _P, _SZ,
                                         _P]),
+    "mla_append_absorb_fp8": (ctypes.c_int, [ctypes.POINTER(mla_dims), _P, _P, _P, _P, _P, _P, _P,
+                                             _P, _P, _P, _I, _P, _I, _P, _P, _P, _SZ, _P]),
     "mla_decode_step_host": (ctypes.c_int, [ctypes.POINTER(mla_dims), _I, ctypes.POINTER(mla_layer),
                                             _P, _P, _P, _P, _I, _P, _SZ, _P]),
     "mla_append_absorb_folded": (ctypes.c_int, [ctypes.POINTER(mla_dims), _P, _P, _P, _P, _P,
@@ -341,11 +343,42 @@ def mla_quantize_weights_fp8(w, codes, scale, stream=None):
     if w.dim() != 2:
         raise ValueError("w must be a matrix")
     rows, cols = w.shape
-    _need(codes, "codes", torch.uint8, ((rows + 127) // 128 * 128, cols))
+    _need(codes, "codes", torch.uint8, fp8_codes_shape(rows, cols))
     _need(scale, "scale", torch.float32, (rows,))
     rc = lib().mla_quantize_weights_fp8(_ptr(w), rows, cols, _ptr(codes), _ptr(scale),
                                         _stream(stream))
     _check(rc, "mla_quantize_weights_fp8")
+
+
+def fp8_codes_shape(rows, cols):
+    """Shape of the E4M3 code buffer of a [rows, cols] matrix (128 x 128 tiles)."""
+    return ((rows + 127) // 128 * 128, cols)
+
+
+def mla_append_absorb_fp8(d: mla_dims, h, w_dkv, w_kr, w_q, w_uk, positions, page_table,
+                          cache_pool, q_cat, ws, q_lo=None, stream=None):
+    """mla_append_absorb with W_DKV, W_KR, W_Q given as (codes, scale) pairs from
+    mla_quantize_weights_fp8 (bf16 path, batch <= 80); W_UK stays bf16."""
+    H = d.n_heads
+    m_q = H * (d.d_nope + d.d_rope)
+    pairs = (("w_dkv", w_dkv, d.d_c), ("w_kr", w_kr, d.d_rope), ("w_q", w_q, m_q))
+    for name, (codes, scale), rows in pairs:
+        _need(codes, name + " codes", torch.uint8, fp8_codes_shape(rows, d.d_model))
+        _need(scale, name + " scale", torch.float32, (rows,))
+    _need(h, "h", torch.bfloat16, (d.batch, d.d_model))
+    _need(w_uk, "w_uk", torch.bfloat16, (H * d.d_nope, d.d_c))
+    _need(positions, "positions", torch.int32, (d.batch,))
+    _need(page_table, "page_table", torch.int32)
+    _need(cache_pool, "cache_pool", torch.bfloat16)
+    _need(q_cat, "q_cat", torch.bfloat16, (d.batch, H, d.d_c + d.d_rope))
+    _need(q_lo, "q_lo", torch.bfloat16, (d.batch, H, d.d_c + d.d_rope))
+    _need(ws, "workspace", torch.uint8)
+    rc = lib().mla_append_absorb_fp8(
+        ctypes.byref(d), _ptr(h), _ptr(w_dkv[0]), _ptr(w_dkv[1]), _ptr(w_kr[0]), _ptr(w_kr[1]),
+        _ptr(w_q[0]), _ptr(w_q[1]), _ptr(w_uk), _ptr(positions), _ptr(page_table),
+        page_table.shape[1], _ptr(cache_pool), cache_pool.shape[0], _ptr(q_cat), _ptr(q_lo),
+        _ptr(ws), ws.numel(), _stream(stream))
+    _check(rc, "mla_append_absorb_fp8")
 
 
 def mla_out_proj_fp8(d: mla_dims, o_lat, w_uv, w_o_codes, w_o_scale, out, ws, o_heads=None,
@@ -355,7 +388,7 @@ def mla_out_proj_fp8(d: mla_dims, o_lat, w_uv, w_o_codes, w_o_scale, out, ws, o_
     H = d.n_heads
     _need(o_lat, "o_lat", torch.float32, (d.batch, H, d.d_c))
     _need(w_uv, "w_uv", torch.bfloat16, (H * d.d_v, d.d_c))
-    _need(w_o_codes, "w_o_codes", torch.uint8, ((d.d_model + 127) // 128 * 128, H * d.d_v))
+    _need(w_o_codes, "w_o_codes", torch.uint8, fp8_codes_shape(d.d_model, H * d.d_v))
     _need(w_o_scale, "w_o_scale", torch.float32, (d.d_model,))
     _need(o_heads, "o_heads", torch.bfloat16, (d.batch, H, d.d_v))
     _need(out, "out", torch.bfloat16, (d.batch, d.d_model))

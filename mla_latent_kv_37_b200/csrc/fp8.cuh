@@ -105,5 +105,82 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// bf16 activation rows x_b (K values each) as a power-of-two scale and two E4M3 planes:
+// s_b = the smallest power of two >= max_k |x_bk| / 448 (fp32; 1 for a zero row), y = x / s_b
+// (exact), p1 = E4M3(y), p2 = E4M3(y - p1).  A bf16 value has 8 significant bits and y - p1 at
+// most the low 4 of them, so p1 + p2 = y exactly unless that remainder falls below E4M3's
+// smallest subnormal (elements under about 2^-8 of the row's largest).  planes: [2][rows_pad][K];
+// rows in [rows, rows_pad) are zeros.  Grid (rows_pad, slices): every block of row b finds the
+// row's maximum itself (K bf16 values, from L2), then converts its slice of K / slices values,
+// 8 per thread.  K a multiple of 8 * slices; x 16-byte and planes 8-byte aligned.
+__global__ void __launch_bounds__(256)
+    split_planes_bf16_kernel(const __nv_bfloat16* __restrict__ x, int rows, long long K,
+                             int rows_pad, uint8_t* __restrict__ planes,
+                             float* __restrict__ scale) {
+  __shared__ float part[8];
+  griddep_launch_dependents();
+  griddep_wait();
+  const int b = blockIdx.x;
+  const long long n8 = K / 8, slice8 = n8 / gridDim.y, j0 = slice8 * blockIdx.y;
+  const size_t plane8 = static_cast<size_t>(rows_pad) * n8;
+  uint2* out = reinterpret_cast<uint2*>(planes) + static_cast<size_t>(b) * n8;
+  if (b >= rows) {
+    for (long long j = j0 + threadIdx.x; j < j0 + slice8; j += blockDim.x) {
+      out[j] = make_uint2(0u, 0u);
+      out[plane8 + j] = make_uint2(0u, 0u);
+    }
+    if (blockIdx.y == 0 && threadIdx.x == 0) scale[b] = 0.f;
+    return;
+  }
+  const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(b) * K);
+  float m = 0.f;
+  for (long long j = threadIdx.x; j < n8; j += blockDim.x) {
+    const uint4 u = xr[j];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      m = fmaxf(m, fmaxf(fabsf(__uint_as_float(w[k] << 16)),
+                         fabsf(__uint_as_float(w[k] & 0xffff0000u))));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = m;
+  __syncthreads();
+  m = part[0];
+  for (int k = 1; k < static_cast<int>(blockDim.x >> 5); ++k) m = fmaxf(m, part[k]);
+  // the smallest power of two >= m / 448 (round the quotient's exponent up unless it is exact)
+  float s = 1.f;
+  if (m > 0.f) {
+    const uint32_t t = __float_as_uint(__fdiv_ru(m, 448.f));
+    const uint32_t e = t >> 23;  // biased exponent (t > 0, so the sign bit is clear)
+    s = (t & 0x7fffffu) == 0u ? __uint_as_float(t) : __uint_as_float(min(e + 1u, 254u) << 23);
+    if (e == 0u) s = 1.17549435e-38f;  // a subnormal quotient: FLT_MIN
+  }
+  if (blockIdx.y == 0 && threadIdx.x == 0) scale[b] = s;
+  for (long long j = j0 + threadIdx.x; j < j0 + slice8; j += blockDim.x) {
+    const uint4 u = xr[j];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    float y[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      y[2 * k] = __fdiv_rn(__uint_as_float(w[k] << 16), s);
+      y[2 * k + 1] = __fdiv_rn(__uint_as_float(w[k] & 0xffff0000u), s);
+    }
+#pragma unroll
+    for (int pl = 0; pl < 2; ++pl) {
+      uint32_t c[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint16_t q = e4m3x2(y[2 * k], y[2 * k + 1]);
+        const float2 d = e4m3x2_value(q);
+        y[2 * k] -= d.x;
+        y[2 * k + 1] -= d.y;
+        c[k] = q;
+      }
+      out[pl * plane8 + j] = make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+    }
+  }
+}
+
 }  // namespace fp8
 }  // namespace mla

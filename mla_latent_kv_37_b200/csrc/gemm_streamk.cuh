@@ -62,8 +62,9 @@ struct Params {
   int n_lo;           // > 0: columns [n_lo, 2 n_lo) hold the low halves of columns [0, n_lo)
   int n_out;          // valid output columns (the batch)
   int a_mn_major;     // 0: A K-major, 1: A MN-major
-  int a_tiled;        // 1: A (map A0 only) stored as contiguous tiles of 128 rows x 128 bytes,
-                      //    [groups * m_tiles][K / 128 bytes][128][128 B]
+  int a_tiled;        // 1: the weights behind each map stored as contiguous tiles of 128 rows x
+                      //    128 bytes, [row tiles][K / 128 bytes][128][128 B] (groups == 1 when
+                      //    several maps are used)
   int stages;         // shared-memory ring depth
   int max_slots;      // partial slots per tile
   long long iters;    // m_tiles * groups * units
@@ -75,8 +76,9 @@ struct Params {
   unsigned int* status;
   uint64_t wait_ns;
   int n_planes;          // X column planes summed into each output: 1, 2 (hi/lo) or 3
-  const float* a_scale;  // E4M3: one scale per weight row (the product's rows)
-  const float* x_scale;  // E4M3: one scale per output column (an activation row)
+  const float* a_scale[3];  // E4M3: one scale per row of the weights behind map A0, A1, A2
+  int a_rows[3];            //        and those weights' row counts
+  const float* x_scale;     // E4M3: one scale per output column (an activation row)
 };
 
 // A stage holds kbs K blocks: A [kbs][128 rows][128 B] (K-major) or [2][64 kbs][128 B]
@@ -472,9 +474,14 @@ __device__ __forceinline__ void tmem_sum_planes(uint32_t tacc, int c0, int n_pla
 }
 
 // E4M3 products: the fp32 sum of a row times its weight row's scale and the column's scale.
+// Row r (within a group) lies in tile r / 128, which selects the weights (map A0, A1 or A2)
+// exactly as the producer does; rows past those weights' end get scale 0.
 __device__ __forceinline__ void scale_e4m3(const Params& p, int r, bool valid, int c0,
                                            float (&v)[16]) {
-  const float sr = valid ? p.a_scale[r] : 0.f;
+  const int mt = r >> 7;
+  const int m = mt >= p.a2_tile_start ? 2 : mt >= p.a1_tile_start ? 1 : 0;
+  const int rr = r - (m == 2 ? p.a2_tile_start * 128 : m == 1 ? p.a1_tile_start * 128 : 0);
+  const float sr = valid && rr < p.a_rows[m] ? p.a_scale[m][rr] : 0.f;
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
     const int b = c0 + j;
@@ -569,7 +576,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (p.a_tiled) {
           // view (128 B, 128 rows, K blocks, row tiles): box (128 B, 128, kbs, 1) is one
           // contiguous run of kbs tiles in HBM
-          tma_load_4d_hint(a_dst, tmA, &full_bar[s], 0, 0, kb0, g * p.m_tiles + mt, pol_w);
+          tma_load_4d_hint(a_dst, tmA, &full_bar[s], 0, 0, kb0, g * p.m_tiles + m_row0 / 128,
+                           pol_w);
         } else if (p.a_mn_major) {
           // [g][k][m] with m contiguous: box (64 m, 64 kbs k) per 64-row half of the tile
           tma_load_3d_hint(a_dst, tmA, &full_bar[s], m_row0, kb0 * 64, g, pol_w);

@@ -138,7 +138,7 @@ int device_ctx(DevCtx** out) {
                                   attn_smem)) != cudaSuccess)
       return cuda_fail(e, "cudaFuncSetAttribute(split_kernel)");
     const int sk_smem = static_cast<int>(kSmemPerBlockMax);
-    const void* sk_kernels[8] = {
+    const void* sk_kernels[9] = {
         reinterpret_cast<const void*>(sk::streamk_gemm_kernel<sk::EpiAppend>),
         reinterpret_cast<const void*>(sk::streamk_gemm_kernel<sk::EpiWq>),
         reinterpret_cast<const void*>(sk::streamk_gemm_kernel<sk::EpiWuk>),
@@ -146,7 +146,8 @@ int device_ctx(DevCtx** out) {
         reinterpret_cast<const void*>(sk::streamk_gemm_kernel<sk::EpiWo>),
         reinterpret_cast<const void*>(sk::streamk_gemm_kernel<sk::EpiAppendWq>),
         reinterpret_cast<const void*>(sk::streamk_gemm_kernel<sk::EpiAppendWqFold>),
-        reinterpret_cast<const void*>(sk::streamk_gemm_kernel<sk::EpiWo, true>)};
+        reinterpret_cast<const void*>(sk::streamk_gemm_kernel<sk::EpiWo, true>),
+        reinterpret_cast<const void*>(sk::streamk_gemm_kernel<sk::EpiAppendWq, true>)};
     for (const void* k : sk_kernels)
       if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, sk_smem)) !=
           cudaSuccess)
@@ -219,6 +220,12 @@ GemmShape shape_append_wq_fold(const mla_dims* d) {
 GemmShape shape_wo_fold(const mla_dims* d) {
   return {d->d_model, (d->d_model + 127) / 128, d->n_heads * kDc, 1, 2 * round16(d->batch),
           round16(d->batch)};
+}
+// cache append and W_Q in E4M3 against h as two E4M3 planes
+GemmShape shape_append_wq_e4m3(const mla_dims* d) {
+  const int m = d->n_heads * (kDn + kDr);
+  return {sk::EpiAppendWq::kSplitRow + m, 5 + m / 128, d->d_model, 1, 2 * round16(d->batch),
+          round16(d->batch), 1};
 }
 // W_O in E4M3 against o_heads as three E4M3 planes (tcgen05 kind::f8f6f4)
 GemmShape shape_wo_e4m3(const mla_dims* d) {
@@ -301,9 +308,13 @@ Workspace layout(const mla_dims* d, int num_parts, int sms) {
       ctr = std::max(ctr, static_cast<size_t>(q.tiles) * 8);
     }
     if (d->batch <= kFp8MaxBatch) {
-      const SkPlan q = sk_plan(shape_wo_e4m3(d), 0, sms);
-      part = std::max(part, q.partial_bytes);
-      ctr = std::max(ctr, static_cast<size_t>(q.tiles) * 8);
+      const SkPlan qs[2] = {sk_plan(shape_wo_e4m3(d), 0, sms),
+                            sk_plan(shape_append_wq_e4m3(d), sk::EpiAppendWq::smem_bytes(d->batch),
+                                    sms)};
+      for (const SkPlan& q : qs) {
+        part = std::max(part, q.partial_bytes);
+        ctr = std::max(ctr, static_cast<size_t>(q.tiles) * 8);
+      }
     }
   } else {
     part = std::max({static_cast<size_t>(kRowN) * B, H * (kDn + kDr) * B, H * kDc * B,
@@ -470,6 +481,14 @@ cudaError_t record_profile_event(cudaEvent_t ev, cudaStream_t st) {
       ev, st, cs == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : cudaEventRecordDefault);
 }
 
+// Scales of an E4M3 product: per weight row of the weights behind maps A0, A1, A2 (with their row
+// counts), per activation row.
+struct E4m3Scales {
+  const float* a[3] = {nullptr, nullptr, nullptr};
+  int rows[3] = {0, 0, 0};
+  const float* x = nullptr;
+};
+
 // One weight product on the tensor cores, its epilogue fused (stream-K, see gemm_streamk.cuh).
 template <class Epi, bool kFp8 = false>
 int run_streamk(const DevCtx* c, const GemmShape& s, const SkPlan& q, int n_out,
@@ -477,8 +496,7 @@ int run_streamk(const DevCtx* c, const GemmShape& s, const SkPlan& q, int n_out,
                 const CUtensorMap& a1, int a1_tile_start, int a_mn_major,
                 const CUtensorMap& xmap, char* ws, const Workspace& w, const Epi& epi,
                 cudaStream_t st, const CUtensorMap* a2 = nullptr, int a2_tile_start = 1 << 30,
-                const float* a_scale = nullptr, const float* x_scale = nullptr,
-                int a_tiled = 0) {
+                const E4m3Scales& scales = E4m3Scales{}, int a_tiled = 0) {
   sk::Params p{};
   p.m_total = s.m_total;
   p.m_tiles = s.m_tiles;
@@ -504,8 +522,11 @@ int run_streamk(const DevCtx* c, const GemmShape& s, const SkPlan& q, int n_out,
   p.rope_theta = theta;
   p.status = c->status;
   p.wait_ns = wait_limit_ns();
-  p.a_scale = a_scale;
-  p.x_scale = x_scale;
+  for (int m = 0; m < 3; ++m) {
+    p.a_scale[m] = scales.a[m];
+    p.a_rows[m] = scales.rows[m];
+  }
+  p.x_scale = scales.x;
   launch_pdl(sk::streamk_gemm_kernel<Epi, kFp8>, dim3(q.ctas), dim3(sk::kThreads), q.smem, st, a0,
              a1, a2 ? *a2 : a1, xmap, p, epi);
   return last_launch();
@@ -1080,6 +1101,79 @@ int mla_quantize_weights_fp8(const void* w, int64_t rows, int64_t cols, void* co
   return last_launch();
 }
 
+int mla_append_absorb_fp8(const mla_dims* dims, const void* h, const void* w_dkv_codes,
+                          const float* w_dkv_scale, const void* w_kr_codes,
+                          const float* w_kr_scale, const void* w_q_codes, const float* w_q_scale,
+                          const void* w_uk, const int32_t* positions, const int32_t* page_table,
+                          int32_t max_pages, void* cache_pool, int32_t num_pages, void* q_cat,
+                          void* q_lo, void* workspace, size_t workspace_bytes,
+                          mla_stream_t stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (dims->dtype != MLA_BF16) return MLA_ERR_ARG;
+  if (dims->batch > kFp8MaxBatch || dims->d_model % 128) return MLA_ERR_DIMS;
+  if (!h || !w_dkv_codes || !w_dkv_scale || !w_kr_codes || !w_kr_scale || !w_q_codes ||
+      !w_q_scale || !w_uk || !positions || !page_table || !cache_pool || !q_cat)
+    return MLA_ERR_NULL_ARG;
+  if (!workspace) return MLA_ERR_WORKSPACE;
+  if (max_pages < 1 || num_pages < 1) return MLA_ERR_ARG;
+  if (!aligned(h, 16) || !aligned(w_dkv_codes, 16) || !aligned(w_kr_codes, 16) ||
+      !aligned(w_q_codes, 16) || !aligned(w_uk, 16) || !aligned(cache_pool, 16) ||
+      !aligned(q_cat, 16) || (q_lo && !aligned(q_lo, 16)) || !aligned(positions, 4) ||
+      !aligned(page_table, 4) || !aligned(w_dkv_scale, 4) || !aligned(w_kr_scale, 4) ||
+      !aligned(w_q_scale, 4))
+    return MLA_ERR_ALIGN;
+  if (!aligned(workspace, 256)) return MLA_ERR_ALIGN;
+  DevCtx* c = nullptr;
+  if ((rc = device_ctx(&c))) return rc;
+  const Workspace w = layout(dims, resolve_parts(0, c), c->sms);
+  if (workspace_bytes < w.plan) return MLA_ERR_WORKSPACE;  // projection scratch only
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int B = dims->batch, D = dims->d_model, H = dims->n_heads;
+  char* ws = static_cast<char*>(workspace);
+  __nv_bfloat16* qc = static_cast<__nv_bfloat16*>(q_cat);
+  __nv_bfloat16* ql = static_cast<__nv_bfloat16*>(q_lo);
+  const GemmShape s = shape_append_wq_e4m3(dims);
+  const int Bp = s.n_lo;
+  // h -> a power-of-two scale and two E4M3 planes per row, in the out-projection's o_split area
+  // (unused until mla_out_proj runs)
+  if (align_up(2ull * Bp * D, 256) + 4ull * Bp > w.oh_split - w.o_split) return MLA_ERR_DIMS;
+  uint8_t* planes = reinterpret_cast<uint8_t*>(ws + w.o_split);
+  float* x_scale = reinterpret_cast<float*>(ws + w.o_split + align_up(2ull * Bp * D, 256));
+  const int slices = (D / 8) % 8 == 0 ? 8 : 1;
+  launch_pdl(fp8::split_planes_bf16_kernel, dim3(static_cast<unsigned>(Bp), slices), dim3(256),
+             0, st, static_cast<const __nv_bfloat16*>(h), B, static_cast<long long>(D), Bp,
+             planes, x_scale);
+  if ((rc = last_launch())) return rc;
+  // [W_DKV; W_KR; W_Q] (E4M3) x [h planes] in one stream-K product, epilogue as in
+  // mla_append_absorb: cache rows + q_nope planes + RoPE(q_rope)
+  const SkPlan q = sk_plan(s, sk::EpiAppendWq::smem_bytes(B), c->sms);
+  const int m_q = H * (kDn + kDr);
+  CUtensorMap a0, a1, a2, bm;
+  if ((rc = map_weights_e4m3(&a0, w_dkv_codes, kDc, D, q.kbs))) return rc;
+  if ((rc = map_weights_e4m3(&a1, w_kr_codes, kDr, D, q.kbs))) return rc;
+  if ((rc = map_weights_e4m3(&a2, w_q_codes, m_q, D, q.kbs))) return rc;
+  if ((rc = map_acts_e4m3(&bm, planes, 2 * Bp, D, s.n_pad, q.kbs))) return rc;
+  sk::EpiAppendWq e{
+      sk::EpiAppend{positions, page_table, max_pages, static_cast<__nv_bfloat16*>(cache_pool),
+                    num_pages, c->status, dims->rope_theta},
+      sk::EpiWq{H, Bp, qc, ql, reinterpret_cast<__nv_bfloat16*>(ws + w.qn), positions,
+                dims->rope_theta}};
+  E4m3Scales sc;
+  sc.a[0] = w_dkv_scale;
+  sc.rows[0] = kDc;
+  sc.a[1] = w_kr_scale;
+  sc.rows[1] = kDr;
+  sc.a[2] = w_q_scale;
+  sc.rows[2] = m_q;
+  sc.x = x_scale;
+  if ((rc = run_streamk<sk::EpiAppendWq, true>(c, s, q, B, positions, dims->rope_theta, a0, a1,
+                                               kDc / 128, 0, bm, ws, w, e, st, &a2,
+                                               sk::EpiAppendWq::kSplitRow / 128, sc, 1)))
+    return rc;
+  return run_wuk(c, dims, w_uk, ws, w, qc, ql, st);
+}
+
 int mla_out_proj_fp8(const mla_dims* dims, const float* o_lat, const void* w_uv,
                      const void* w_o_codes, const float* w_o_scale, void* o_heads, void* out,
                      void* workspace, size_t workspace_bytes, mla_stream_t stream) {
@@ -1137,8 +1231,12 @@ int mla_out_proj_fp8(const mla_dims* dims, const float* o_lat, const void* w_uv,
   if ((rc = map_weights_e4m3(&a2, w_o_codes, D, K, q2.kbs))) return rc;
   if ((rc = map_acts_e4m3(&b2, planes, 3 * Bp, K, s2.n_pad, q2.kbs))) return rc;
   sk::EpiWo e2{D, static_cast<__nv_bfloat16*>(out)};
+  E4m3Scales sc;
+  sc.a[0] = w_o_scale;
+  sc.rows[0] = D;
+  sc.x = x_scale;
   return run_streamk<sk::EpiWo, true>(c, s2, q2, B, nullptr, 0.f, a2, a2, 1 << 30, 0, b2, ws, w,
-                                      e2, st, nullptr, 1 << 30, w_o_scale, x_scale, 1);
+                                      e2, st, nullptr, 1 << 30, sc, 1);
 }
 
 int mla_merge_partials(const mla_dims* dims, int32_t n_parts, const float* part_o,

@@ -7,6 +7,7 @@ import pytest
 import torch
 
 from oracle import mla_oracle as O
+import mla_inputs as I
 from tests.gpu_common import Workload, assert_close, dev, to_np
 
 pytestmark = pytest.mark.gpu
@@ -81,4 +82,73 @@ def test_out_proj_fp8_rejects_large_batch():
                            torch.empty(1024, device="cuda"),
                            torch.empty(81, 1024, dtype=torch.bfloat16, device="cuda"),
                            M.workspace(d))
+    assert e.value.code == -2
+
+
+def _quantize(M, w):
+    """E4M3 codes and scales of a bf16 matrix on the GPU, and the weights they stand for."""
+    rows, cols = w.shape
+    codes = torch.empty(tiled_rows(rows), cols, dtype=torch.uint8, device="cuda")
+    scale = torch.empty(rows, dtype=torch.float32, device="cuda")
+    M.mla_quantize_weights_fp8(dev(w), codes, scale)
+    torch.cuda.synchronize()
+    deq = O.dequantize_rows_e4m3(untile(codes.cpu(), rows, cols), scale.cpu().numpy())
+    return (codes, scale), deq
+
+
+@pytest.mark.parametrize("B,H,D,scale", [(4, 128, 7168, 1.0), (5, 16, 1024, 4.0),
+                                         (33, 32, 512, 1.0), (80, 16, 1024, 1.0)])
+def test_append_absorb_fp8_matches_oracle(B, H, D, scale):
+    """Cache append + absorbed query with W_DKV, W_KR and W_Q stored as E4M3: the appended cache
+    rows and q_cat against the oracle's fp64 projections with the weights the codes stand for
+    (the hidden states enter exactly as two E4M3 planes); every other pool byte untouched."""
+    import mla_latent_kv_37_b200 as M
+    hist = [(53 * i + 7) % 300 for i in range(B)]
+    wl = Workload(90 + B, B, H, D, hist, scale=scale)
+    w = wl.w
+    dkv, dkv_deq = _quantize(M, w.w_dkv)
+    kr, kr_deq = _quantize(M, w.w_kr)
+    wq, wq_deq = _quantize(M, w.w_q)
+    d = M.dims(B, H, D)
+    pool = dev(wl.cache.pool)
+    before = wl.cache.pool.clone()
+    q_cat = torch.full((B, H, 576), float("nan"), dtype=torch.bfloat16, device="cuda")
+    M.mla_append_absorb_fp8(d, dev(wl.h), dkv, kr, wq, dev(w.w_uk), dev(wl.pos),
+                            dev(wl.cache.page_table), pool, q_cat, M.workspace(d))
+    torch.cuda.synchronize()
+    assert M.mla_get_status() == 0
+    pool, q_cat = pool.cpu(), q_cat.cpu()
+    changed = (pool.view(pool.shape[0], 64, -1) != before.view(pool.shape[0], 64, -1)).any(-1)
+    w_uk = O.f64(w.w_uk)
+    for b, pos in enumerate(wl.history):
+        page = int(wl.cache.page_table[b, pos // 64])
+        c, k = O.latent_row(wl.h[b], dkv_deq, kr_deq, pos)
+        assert_close(to_np(pool[page, pos % 64]), np.concatenate([c, k]), torch.bfloat16,
+                     f"cache row b={b}")
+        changed[page, pos % 64] = False
+        if b in (0, B // 2, B - 1):
+            qn, qr = O.query_heads(wl.h[b], wq_deq, H, 128, 64, pos)
+            q_lat = np.stack([w_uk[i * 128:(i + 1) * 128].T @ qn[i] for i in range(H)])
+            assert_close(to_np(q_cat[b, :, :512]), q_lat, torch.bfloat16, f"q_lat b={b}")
+            assert_close(to_np(q_cat[b, :, 512:]), qr, torch.bfloat16, f"q_rope b={b}")
+    assert not changed.any(), "append wrote outside the addressed slots"
+
+
+def test_append_absorb_fp8_rejects_large_batch():
+    import mla_latent_kv_37_b200 as M
+    B, H, D = 81, 16, 1024
+    d = M.dims(B, H, D)
+
+    def pair(rows):
+        return (torch.empty(*M.fp8_codes_shape(rows, D), dtype=torch.uint8, device="cuda"),
+                torch.empty(rows, device="cuda"))
+    cache = I.paged_cache(3, [8] * B, [0] * B)
+    with pytest.raises(M.MlaError) as e:
+        M.mla_append_absorb_fp8(d, torch.empty(B, D, dtype=torch.bfloat16, device="cuda"),
+                                pair(512), pair(64), pair(H * 192),
+                                torch.empty(H * 128, 512, dtype=torch.bfloat16, device="cuda"),
+                                torch.zeros(B, dtype=torch.int32, device="cuda"),
+                                dev(cache.page_table), dev(cache.pool),
+                                torch.empty(B, H, 576, dtype=torch.bfloat16, device="cuda"),
+                                M.workspace(d))
     assert e.value.code == -2
