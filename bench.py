@@ -490,7 +490,47 @@ def run_extra_configs(dev, peaks, steps=10):
     return out
 
 
-def run_execution_modes(dev, peaks, reps=10, B=32, H=128, D=7168):
+def graph_us_per_call(call, n_layers, reps=10):
+    """Median device time of one call, from replays of a CUDA graph holding call(0) ..
+    call(n_layers - 1) back to back (each layer its own weights, together larger than L2): no
+    host launch cost in the timed region, and every call streams its weights from HBM."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for l in range(n_layers):  # eager once: the library's one-time set-up stays outside
+            call(l)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for l in range(n_layers):
+            call(l)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1) * 1e3 / n_layers)
+    del g
+    return sorted(ts)[len(ts) // 2]
+
+
+def _nbytes(*ts):
+    return sum(t.numel() * t.element_size() for t in ts)
+
+
+def _weight_rate(us, wbytes, peaks):
+    gbs = wbytes / (us * 1e-6) / 1e9
+    return {"us_per_layer": us, "weight_bytes_per_layer": wbytes, "gbs": gbs,
+            "hbm_frac": gbs / peaks.get("hbm_gbs", 6650.0)}
+
+
+def run_execution_modes(dev, peaks, n_layers=3, B=32, H=128, D=7168):
     """The projections of one layer (cache append + query, then the output product) in the
     absorbed form the step uses and in the folded form (W_UK multiplied into W_Q and W_UV into
     W_O ahead of time): time per layer and weight bytes streamed.  Attention is the same in
@@ -498,108 +538,159 @@ def run_execution_modes(dev, peaks, reps=10, B=32, H=128, D=7168):
     import mla_latent_kv_37_b200 as M
     import mla_inputs as I
     d = M.dims(B, H, D)
-    w = I.weights(11, H, D, device=dev)
+    ws_ = [I.weights(11 + l, H, D, device=dev) for l in range(n_layers)]
     h = I.hidden(12, B, D, device=dev)
     pos = torch.zeros(B, dtype=torch.int32, device=dev)
     table = torch.arange(B, dtype=torch.int32, device=dev).view(B, 1)
     pool = torch.zeros(B, 64, 576, dtype=torch.bfloat16, device=dev)
     sq, so = M.fold_shapes(d)
-    w_qf = torch.empty(sq, dtype=torch.bfloat16, device=dev)
-    w_of = torch.empty(so, dtype=torch.bfloat16, device=dev)
-    M.mla_fold_weights(d, w_q=w.w_q, w_uk=w.w_uk, w_uv=w.w_uv, w_o=w.w_o, w_qf=w_qf, w_of=w_of)
+    folded_w = []
+    for w in ws_:
+        w_qf = torch.empty(sq, dtype=torch.bfloat16, device=dev)
+        w_of = torch.empty(so, dtype=torch.bfloat16, device=dev)
+        M.mla_fold_weights(d, w_q=w.w_q, w_uk=w.w_uk, w_uv=w.w_uv, w_o=w.w_o, w_qf=w_qf,
+                           w_of=w_of)
+        folded_w.append((w_qf, w_of))
     ws = M.workspace(d, 0, dev)
     q_cat = torch.empty(B, H, 576, dtype=torch.bfloat16, device=dev)
     o_lat = torch.randn(B, H, 512, dtype=torch.float32, device=dev)
     o_heads = torch.empty(B, H, 128, dtype=torch.bfloat16, device=dev)
     out = torch.empty(B, D, dtype=torch.bfloat16, device=dev)
 
-    def absorbed():
+    def absorbed(l):
+        w = ws_[l]
         M.mla_append_absorb(d, h, w.w_dkv, w.w_kr, w.w_q, w.w_uk, pos, table, pool, q_cat, ws)
         M.mla_out_proj(d, o_lat, w.w_uv, ws, w_o=w.w_o, o_heads=o_heads, out=out)
 
-    def folded():
+    def folded(l):
+        w, (w_qf, w_of) = ws_[l], folded_w[l]
         M.mla_append_absorb_folded(d, h, w.w_dkv, w.w_kr, w_qf, pos, table, pool, q_cat, ws)
         M.mla_out_proj_folded(d, o_lat, w_of, out, ws)
 
-    def nbytes(*ts):
-        return sum(t.numel() * t.element_size() for t in ts)
-
-    res = {}
-    for name, fn, wbytes in (
-            ("absorbed", absorbed, nbytes(w.w_dkv, w.w_kr, w.w_q, w.w_uk, w.w_uv, w.w_o)),
-            ("folded", folded, nbytes(w.w_dkv, w.w_kr, w_qf, w_of))):
-        for _ in range(3):
-            fn()
-        torch.cuda.synchronize()
-        ts = []
-        for _ in range(reps):
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            fn()
-            e1.record()
-            torch.cuda.synchronize()
-            ts.append(e0.elapsed_time(e1) * 1e3)
-        us = sorted(ts)[len(ts) // 2]
-        gbs = wbytes / (us * 1e-6) / 1e9
-        res[name] = {"us_per_layer": us, "weight_bytes_per_layer": wbytes, "gbs": gbs,
-                     "hbm_frac": gbs / peaks.get("hbm_gbs", 6650.0)}
+    w0, (qf0, of0) = ws_[0], folded_w[0]
+    res = {"absorbed": _weight_rate(graph_us_per_call(absorbed, n_layers),
+                                    _nbytes(w0.w_dkv, w0.w_kr, w0.w_q, w0.w_uk, w0.w_uv, w0.w_o),
+                                    peaks),
+           "folded": _weight_rate(graph_us_per_call(folded, n_layers),
+                                  _nbytes(w0.w_dkv, w0.w_kr, qf0, of0), peaks)}
     st = M.mla_get_status()
     if st:
         raise RuntimeError(f"device status {st:#x} in the execution-mode measurement")
     res["what"] = ("projections of one layer (cache append + query, output product) at "
-                   f"B={B}, H={H}, D={D}, median of {reps}; attention is identical in both")
+                   f"B={B}, H={H}, D={D}: CUDA-graph replay of {n_layers} layers with their own "
+                   "weights, median of 10; attention is identical in both")
     res["folded_over_absorbed_time"] = res["folded"]["us_per_layer"] / res["absorbed"]["us_per_layer"]
-    del w, w_qf, w_of, ws
+    del ws_, folded_w, ws
     torch.cuda.empty_cache()
     return res
 
 
-def run_fp8_weights(dev, peaks, reps=10, B=32, H=128, D=7168):
-    """The output projection of one layer (W_UV then W_O) with W_O in bf16 and with W_O stored
-    as E4M3 codes + row scales (one byte per weight streamed from HBM): time per call and the
-    weight bytes it streams."""
+def run_fp8_weights(dev, peaks, n_layers=4, B=32, H=128, D=7168):
+    """The two projection calls of one layer with bf16 weights and with W_DKV, W_KR, W_Q and W_O
+    stored as E4M3 codes + row scales (one byte per weight streamed from HBM): time per call
+    and the weight bytes it streams."""
     import mla_latent_kv_37_b200 as M
     import mla_inputs as I
+    from mla_latent_kv_37_b200.step import Layer, quantize_layer
     d = M.dims(B, H, D)
-    w = I.weights(13, H, D, device=dev)
-    codes = torch.empty(D, H * 128, dtype=torch.uint8, device=dev)
-    scale = torch.empty(D, dtype=torch.float32, device=dev)
-    M.mla_quantize_weights_fp8(w.w_o, codes, scale)
+    h = I.hidden(14, B, D, device=dev)
+    pos = torch.zeros(B, dtype=torch.int32, device=dev)
+    table = torch.arange(B, dtype=torch.int32, device=dev).view(B, 1)
+    pool = torch.zeros(B, 64, 576, dtype=torch.bfloat16, device=dev)
+    lys = []
+    for l in range(n_layers):
+        w = I.weights(13 + l, H, D, device=dev)
+        lys.append(quantize_layer(Layer(w.w_dkv, w.w_kr, w.w_q, w.w_uk, w.w_uv, w.w_o, pool,
+                                        table)))
     ws = M.workspace(d, 0, dev)
+    q_cat = torch.empty(B, H, 576, dtype=torch.bfloat16, device=dev)
     o_lat = torch.randn(B, H, 512, dtype=torch.float32, device=dev)
     out = torch.empty(B, D, dtype=torch.bfloat16, device=dev)
-
-    def nbytes(*ts):
-        return sum(t.numel() * t.element_size() for t in ts)
-
+    calls = {
+        "append_absorb": (
+            lambda l: M.mla_append_absorb(d, h, lys[l].w_dkv, lys[l].w_kr, lys[l].w_q,
+                                          lys[l].w_uk, pos, table, pool, q_cat, ws),
+            lambda l: M.mla_append_absorb_fp8(d, h, lys[l].e4m3["w_dkv"], lys[l].e4m3["w_kr"],
+                                              lys[l].e4m3["w_q"], lys[l].w_uk, pos, table, pool,
+                                              q_cat, ws),
+            ("w_dkv", "w_kr", "w_q"), ("w_uk",)),
+        "out_proj": (
+            lambda l: M.mla_out_proj(d, o_lat, lys[l].w_uv, ws, w_o=lys[l].w_o, out=out),
+            lambda l: M.mla_out_proj_fp8(d, o_lat, lys[l].w_uv, lys[l].e4m3["w_o"][0],
+                                         lys[l].e4m3["w_o"][1], out, ws),
+            ("w_o",), ("w_uv",)),
+    }
     res = {}
-    for name, fn, wbytes in (
-            ("bf16", lambda: M.mla_out_proj(d, o_lat, w.w_uv, ws, w_o=w.w_o, out=out),
-             nbytes(w.w_uv, w.w_o)),
-            ("e4m3", lambda: M.mla_out_proj_fp8(d, o_lat, w.w_uv, codes, scale, out, ws),
-             nbytes(w.w_uv, codes, scale))):
-        for _ in range(3):
-            fn()
-        torch.cuda.synchronize()
-        ts = []
-        for _ in range(reps):
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            fn()
-            e1.record()
-            torch.cuda.synchronize()
-            ts.append(e0.elapsed_time(e1) * 1e3)
-        us = sorted(ts)[len(ts) // 2]
-        gbs = wbytes / (us * 1e-6) / 1e9
-        res[name] = {"us_per_layer": us, "weight_bytes_per_layer": wbytes, "gbs": gbs,
-                     "hbm_frac": gbs / peaks.get("hbm_gbs", 6650.0)}
+    ly0 = lys[0]
+    for name, (f_bf16, f_e4m3, quant, kept) in calls.items():
+        kept_b = _nbytes(*[getattr(ly0, k) for k in kept])
+        res[name] = {
+            "bf16": _weight_rate(graph_us_per_call(f_bf16, n_layers),
+                                 kept_b + _nbytes(*[getattr(ly0, k) for k in quant]), peaks),
+            "e4m3": _weight_rate(graph_us_per_call(f_e4m3, n_layers),
+                                 kept_b + sum(_nbytes(*ly0.e4m3[k]) for k in quant), peaks)}
+        res[name]["e4m3_over_bf16_time"] = (res[name]["e4m3"]["us_per_layer"] /
+                                            res[name]["bf16"]["us_per_layer"])
     st = M.mla_get_status()
     if st:
         raise RuntimeError(f"device status {st:#x} in the E4M3 measurement")
-    res["what"] = (f"output projection of one layer (W_UV bf16, then W_O) at B={B}, H={H}, "
-                   f"D={D}, median of {reps}")
-    res["e4m3_over_bf16_time"] = res["e4m3"]["us_per_layer"] / res["bf16"]["us_per_layer"]
-    del w, codes, scale, ws
+    res["what"] = (f"the projection calls of one layer at B={B}, H={H}, D={D}: CUDA-graph replay "
+                   f"of {n_layers} layers with their own weights, median of 10 (W_UK and W_UV "
+                   "stay bf16 in both)")
+    del lys, ws
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_fp8_step(layers, h, pos, lens_dev, lens, cfg, dev, steps):
+    """The headline step with W_DKV, W_KR, W_Q and W_O of every layer stored as E4M3 (the rest
+    unchanged): tokens/s from CUDA-graph replays, and a parity sample against the oracle run
+    with the weights the codes stand for."""
+    import numpy as np
+    import mla_latent_kv_37_b200 as M
+    from oracle import mla_oracle as O
+    from mla_latent_kv_37_b200.step import DecodeStep, quantize_layer
+    B, H, D = cfg["batch"], cfg["heads"], cfg["d_model"]
+    q_layers = [quantize_layer(ly) for ly in layers]
+    step = DecodeStep(q_layers, B, H, D, device=dev, graph=True)
+    for _ in range(3):
+        step.run(h, pos, lens_dev)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        step.run(h, pos, lens_dev)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    st = M.mla_get_status()
+    if st:
+        raise RuntimeError(f"device status {st:#x} in the E4M3 step")
+    # parity: layer 0, sequence 0, 8 heads, oracle with the dequantized weights
+    ly, b = q_layers[0], 0
+    hist = lens[b] - 1
+    w, hb, rows = oracle_sample_inputs(ly, h[0], b, hist)
+    for name in ("w_dkv", "w_kr", "w_q", "w_o"):
+        codes, scale = ly.e4m3[name]
+        n_rows, n_cols = getattr(ly, name).shape
+        setattr(w, name, O.dequantize_rows_e4m3(
+            M.fp8_codes_rows(codes, n_rows, n_cols).cpu().numpy(), scale.cpu().numpy()))
+    heads = list(range(0, H, max(1, H // 8)))[:8]
+    to_bf16 = lambda r: torch.from_numpy(np.asarray(r, dtype=np.float32)).to(torch.bfloat16)
+    ref = O.decode_step(hb, w, rows, hist, H, round_row=to_bf16, heads=heads, with_out=False)
+    got = step.o_heads[0, b][heads].float().cpu().numpy().astype(np.float64)
+    exp = ref["o_heads"]
+    rel = float(np.linalg.norm(got - exp) / np.linalg.norm(exp))
+    mx = float(np.abs(got - exp).max() / np.abs(exp).max())
+    res = {"value": B / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
+           "launch": "CUDA graph of the step",
+           "what": "the headline step with W_DKV, W_KR, W_Q, W_O in E4M3 (W_UK, W_UV bf16; "
+                   "cache bf16)",
+           "parity": {"o_heads_rel_l2": rel, "o_heads_max_abs": mx,
+                      "samples": "layer 0, sequence 0, 8 heads; oracle with the dequantized "
+                                 "weights",
+                      "pass": rel <= 5e-3 and mx <= 2e-2}}
+    del step, q_layers
     torch.cuda.empty_cache()
     return res
 
@@ -843,9 +934,15 @@ def main():
         cpu = cpu_baseline_from(sec, cfg, heads_timed, wall)
 
     # ---------------- the other configurations and the attention sweep (one GPU) ----------
-    configs = sweep = modes = fp8w = None
+    configs = sweep = modes = fp8w = fp8s = None
     if rank == 0 and world == 1 and not args.no_extras:
-        del layers, h, step
+        if B <= 80:
+            del step
+            torch.cuda.empty_cache()
+            fp8s = run_fp8_step(layers, h, pos, lens_dev, lens, cfg, dev, max(3, args.steps // 2))
+        else:
+            del step
+        del layers, h
         torch.cuda.synchronize()
         torch.cuda.empty_cache()
         configs = run_extra_configs(dev, peaks)
@@ -867,7 +964,7 @@ def main():
             "gpu_launches": int(launches), "clocks": clocks, "parity": parity,
             "attention_us_per_layer": roofline["us_per_launch"],
             "configs": configs, "attention_sweep": sweep, "execution_modes": modes,
-            "fp8_weights": fp8w,
+            "fp8_weights": fp8w, "fp8_weights_step": fp8s,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

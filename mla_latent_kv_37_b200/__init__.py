@@ -355,6 +355,14 @@ def fp8_codes_shape(rows, cols):
     return ((rows + 127) // 128 * 128, cols)
 
 
+def fp8_codes_rows(codes, rows, cols):
+    """The codes of a tiled E4M3 buffer rearranged as the [rows, cols] matrix (a layout change
+    on the tensor's device, for inspection and host-side checks)."""
+    rt = codes.shape[0] // 128
+    t = codes.reshape(rt, cols // 128, 128, 128).permute(0, 2, 1, 3).reshape(rt * 128, cols)
+    return t[:rows]
+
+
 def mla_append_absorb_fp8(d: mla_dims, h, w_dkv, w_kr, w_q, w_uk, positions, page_table,
                           cache_pool, q_cat, ws, q_lo=None, stream=None):
     """mla_append_absorb with W_DKV, W_KR, W_Q given as (codes, scale) pairs from

@@ -2,6 +2,8 @@
 
 A step, per layer l (each layer has its own weights, paged cache and hidden state h[l]):
     mla_append_absorb (= mla_cache_append + mla_absorb_q) -> mla_decode_attn -> mla_out_proj
+or, for a layer with E4M3 weights (`Layer.e4m3`, see `quantize_layer`),
+    mla_append_absorb_fp8 -> mla_decode_attn -> mla_out_proj_fp8
 Everything stays on the device; `run_host` adds the host<->device copies of the step's inputs
 and results (pinned buffers), overlapped layer by layer with the kernels, for end-to-end use.
 Marshalling only: no arithmetic.
@@ -12,8 +14,9 @@ import dataclasses
 
 import torch
 
-from . import (dims as make_dims, mla_append_absorb, mla_decode_attn, mla_launch_count,
-               mla_out_proj, workspace)
+from . import (dims as make_dims, fp8_codes_shape, mla_append_absorb, mla_append_absorb_fp8,
+               mla_decode_attn, mla_launch_count, mla_out_proj, mla_out_proj_fp8,
+               mla_quantize_weights_fp8, workspace)
 
 
 @dataclasses.dataclass
@@ -26,6 +29,21 @@ class Layer:
     w_o: torch.Tensor | None
     pool: torch.Tensor        # [num_pages, 64, 576]
     page_table: torch.Tensor  # [B, max_pages] int32
+    # E4M3 copies {"w_dkv", "w_kr", "w_q", "w_o"} -> (codes, scale); None: bf16 weights
+    e4m3: dict | None = None
+
+
+def quantize_layer(layer: Layer) -> Layer:
+    """The layer with E4M3 copies of W_DKV, W_KR, W_Q and W_O (mla_quantize_weights_fp8, on the
+    weights' device and the current stream); W_UK and W_UV stay bf16."""
+    q = {}
+    for name in ("w_dkv", "w_kr", "w_q", "w_o"):
+        w = getattr(layer, name)
+        codes = torch.empty(fp8_codes_shape(*w.shape), dtype=torch.uint8, device=w.device)
+        scale = torch.empty(w.shape[0], dtype=torch.float32, device=w.device)
+        mla_quantize_weights_fp8(w, codes, scale)
+        q[name] = (codes, scale)
+    return dataclasses.replace(layer, e4m3=q)
 
 
 class DecodeStep:
@@ -89,13 +107,23 @@ class DecodeStep:
         return g
 
     def _layer(self, l, h_l, positions, seq_lens, stream=None):
-        d, ly = self.dims, self.layers[l]
-        mla_append_absorb(d, h_l, ly.w_dkv, ly.w_kr, ly.w_q, ly.w_uk, positions, ly.page_table,
-                          ly.pool, self.q_cat, self.ws, q_lo=self.q_lo, stream=stream)
+        d, ly, q = self.dims, self.layers[l], self.layers[l].e4m3
+        if q is not None:
+            mla_append_absorb_fp8(d, h_l, q["w_dkv"], q["w_kr"], q["w_q"], ly.w_uk, positions,
+                                  ly.page_table, ly.pool, self.q_cat, self.ws, q_lo=self.q_lo,
+                                  stream=stream)
+        else:
+            mla_append_absorb(d, h_l, ly.w_dkv, ly.w_kr, ly.w_q, ly.w_uk, positions,
+                              ly.page_table, ly.pool, self.q_cat, self.ws, q_lo=self.q_lo,
+                              stream=stream)
         mla_decode_attn(d, self.q_cat, ly.pool, ly.page_table, seq_lens, self.o_lat, self.ws,
                         lse=self.lse, q_lo=self.q_lo, num_splits=self.num_splits, stream=stream)
-        mla_out_proj(d, self.o_lat, ly.w_uv, self.ws, w_o=ly.w_o, o_heads=self.o_heads[l],
-                     out=self.out[l] if ly.w_o is not None else None, stream=stream)
+        if q is not None:
+            mla_out_proj_fp8(d, self.o_lat, ly.w_uv, q["w_o"][0], q["w_o"][1], self.out[l],
+                             self.ws, o_heads=self.o_heads[l], stream=stream)
+        else:
+            mla_out_proj(d, self.o_lat, ly.w_uv, self.ws, w_o=ly.w_o, o_heads=self.o_heads[l],
+                         out=self.out[l] if ly.w_o is not None else None, stream=stream)
 
     def _run(self, h, positions, seq_lens, stream=None):
         for l in range(len(self.layers)):
@@ -131,6 +159,8 @@ class DecodeStep:
         """End-to-end through the library's native step executor (mla_decode_step_host): the
         host buffers go in and `out` comes back with every copy and launch made in C++."""
         from . import layer_structs, mla_decode_step_host, step_workspace
+        if any(ly.e4m3 is not None for ly in self.layers):
+            raise ValueError("the native step executor takes bf16 weights")
         if getattr(self, "_native", None) is None:
             self._native = (layer_structs(self.dims, self.layers),
                             step_workspace(self.dims, len(self.layers), self.num_splits,
