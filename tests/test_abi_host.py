@@ -231,3 +231,47 @@ def test_step_executor_arguments(M):
                          0x10000, 4)
     assert L.mla_decode_step_host(ctypes.byref(d), 2, lay, f, f, f, f, 0, ws, big, None) == -1
 
+
+
+def test_e4m3_weight_arguments(M):
+    """The E4M3-weight calls check their arguments on the host, before any device work: code
+    widths that are not whole 128-column tiles, missing or misaligned pointers, the fp32
+    path, batches above 80 and d_model not a multiple of 128."""
+    import torch
+    d = _d(M)
+    d32 = M.dims(4, 16, 1024, dtype=torch.float32)
+    L = M.lib()
+    f = ctypes.c_void_p(0x10000)
+    odd = ctypes.c_void_p(0x10008)
+    ws = ctypes.c_void_p(0x100000)
+    big = ctypes.c_size_t(1 << 40)
+    # quantization: cols a positive multiple of 128, pointers present and aligned
+    assert L.mla_quantize_weights_fp8(f, 8, 64, f, f, None) == -5
+    assert L.mla_quantize_weights_fp8(f, 0, 128, f, f, None) == -5
+    assert L.mla_quantize_weights_fp8(None, 8, 128, f, f, None) == -1
+    assert L.mla_quantize_weights_fp8(f, 8, 128, odd, f, None) == -3
+    # append + absorb with E4M3 W_DKV, W_KR, W_Q
+    args = [f, f, f, f, f, f, f, f, f, f, 4, f, 8, f, None, ws, big, None]
+    assert L.mla_append_absorb_fp8(ctypes.byref(d32), *args) == -5
+    assert L.mla_append_absorb_fp8(ctypes.byref(M.dims(81, 16, 1024)), *args) == -2
+    assert L.mla_append_absorb_fp8(ctypes.byref(M.dims(4, 16, 1088)), *args) == -2
+    for i, code in ((1, -1), (6, -1), (7, -1), (13, -1)):  # codes, scale, w_uk, q_cat
+        bad = list(args)
+        bad[i] = None
+        assert L.mla_append_absorb_fp8(ctypes.byref(d), *bad) == code
+    bad = list(args)
+    bad[5] = odd  # W_Q codes
+    assert L.mla_append_absorb_fp8(ctypes.byref(d), *bad) == -3
+    bad = list(args)
+    bad[15] = None  # workspace
+    assert L.mla_append_absorb_fp8(ctypes.byref(d), *bad) == -4
+    # output projection with E4M3 W_O
+    oargs = [f, f, f, f, None, f, ws, big, None]
+    assert L.mla_out_proj_fp8(ctypes.byref(d32), *oargs) == -5
+    assert L.mla_out_proj_fp8(ctypes.byref(M.dims(81, 16, 1024)), *oargs) == -2
+    bad = list(oargs)
+    bad[5] = None  # out
+    assert L.mla_out_proj_fp8(ctypes.byref(d), *bad) == -1
+    bad = list(oargs)
+    bad[2] = odd  # W_O codes
+    assert L.mla_out_proj_fp8(ctypes.byref(d), *bad) == -3
