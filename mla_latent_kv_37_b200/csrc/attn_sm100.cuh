@@ -86,8 +86,6 @@ constexpr uint32_t kOffBar = kOffX + 2 * kXBytes;
 constexpr uint32_t kSmemBytes = kOffBar + 512 + 1024;  // barriers + alignment slack
 // TMEM columns: O half | query latent half | S of two pages (page parity)
 constexpr uint32_t kTmemO = 0, kTmemQ = 256, kTmemS = 384, kTmemCols = 512;
-constexpr int kAhead = 4;  // pages prefetched into L2 ahead of the TMA ring
-constexpr uint32_t kPageBytes = kPage * kRow * 2;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -137,10 +135,18 @@ struct PlanView {
 };
 
 // ------------------------------------------------------------------------------------------
-// Planner: one block.  pages per sequence, prefix sums, equal division of the page list into
-// parts, which parts touch which sequence, and where each sequence's partials go.
+// Planner: one block.  pages per sequence, prefix sums, division of the page list into parts of
+// equal cost, which parts touch which sequence, and where each sequence's partials go.
+//
+// Cost model: a part pays for its pages and, for every sequence that starts inside it, one more
+// segment (a query load, a drained pipeline and an O write-back), which costs about as much as
+// kSegPages pages.  So the division is equal in "virtual pages": every non-empty sequence is
+// kSegPages virtual pages of start-up followed by its real pages, and part c covers the virtual
+// range [c V / C, (c + 1) V / C).  A part whose range begins inside a sequence's start-up begins
+// at that sequence's first page.
 // ------------------------------------------------------------------------------------------
 constexpr int kPlanThreads = 1024;
+constexpr int kSegPages = 3;
 
 __device__ inline int block_exclusive_scan(int v, int* warp_sums, int* total) {
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -179,9 +185,10 @@ __device__ inline int plan_pages(const int32_t* seq_lens, int b, int cap, unsign
   return (len + kPage - 1) / kPage;
 }
 
-// The part that holds global page g of the concatenated list (g = -1 gives -1).
-__device__ inline int part_of_page(int64_t g, int C, int P) {
-  return g < 0 ? -1 : static_cast<int>(((g + 1) * C - 1) / P);
+// The part that holds virtual position v of the list (v = -1 gives -1): part c holds
+// [floor(c V / C), floor((c + 1) V / C)).
+__device__ inline int part_of_page(int64_t v, int C, int64_t V) {
+  return v < 0 ? -1 : static_cast<int>(((v + 1) * C - 1) / V);
 }
 
 // Every value a thread needs comes from its own sequences and two block-wide scans: the parts
@@ -205,11 +212,19 @@ __global__ void __launch_bounds__(kPlanThreads)
   const int chunk = (B + T - 1) / T;
   const int b0 = threadIdx.x * chunk, b1 = min(B, b0 + chunk);
   const int cap = max_pages * kPage;
-  // 1. pages of this thread's sequences, and their exclusive prefix over the whole batch
-  int local = 0;
-  for (int b = b0; b < b1; ++b) local += plan_pages(seq_lens, b, cap, status);
+  // 1. pages of this thread's sequences, and their exclusive prefix over the whole batch; the
+  //    same for the count of non-empty sequences (each adds kSegPages virtual pages)
+  int local = 0, nonempty = 0;
+  for (int b = b0; b < b1; ++b) {
+    const int n = plan_pages(seq_lens, b, cap, status);
+    local += n;
+    nonempty += n > 0;
+  }
   const int run0 = block_exclusive_scan(local, warp_sums, &s_total);
   const int P = s_total;
+  __shared__ int s_seqs;
+  const int rank0 = block_exclusive_scan(nonempty, warp_sums, &s_seqs);
+  const int64_t V = static_cast<int64_t>(P) + static_cast<int64_t>(kSegPages) * s_seqs;
   int C = 0;
   if (P > 0) C = max(1, min(C_req, (P + min_pages_per_part - 1) / min_pages_per_part));
   if (threadIdx.x == 0) {
@@ -217,13 +232,14 @@ __global__ void __launch_bounds__(kPlanThreads)
     plan[1] = C;
     prefix[B] = P;
   }
-  // 2. equal division of the page list; parts beyond C are empty and start no sequence
+  // 2. parts beyond C are empty and start no sequence; every other part start is written by
+  //    the thread of the sequence it starts in (step 3)
   for (int c = threadIdx.x; c <= C_req; c += T) {
-    pstart[c] = (c <= C && C > 0) ? static_cast<int>((static_cast<int64_t>(c) * P) / C) : P;
+    if (c >= C) pstart[c] = P;
     if (c < C_req && c >= C) pseq[c] = B;
   }
   // 3. per sequence: its pages, prefix, the parts that cover it, and the parts starting in it
-  int run = run0, nloc = 0;
+  int run = run0, rank = rank0, nloc = 0;
   for (int b = b0; b < b1; ++b) {
     const int n = plan_pages(seq_lens, b, cap, nullptr);
     pg[b] = n;
@@ -233,22 +249,35 @@ __global__ void __launch_bounds__(kPlanThreads)
       npart[b] = 0;
       continue;
     }
-    const int pf = part_of_page(run, C, P);
-    const int pl = part_of_page(static_cast<int64_t>(run) + n - 1, C, P);
+    // virtual positions: start-up [vs, vs + kSegPages), pages from vp (page k at vp + k)
+    const int64_t vs = static_cast<int64_t>(run) + static_cast<int64_t>(kSegPages) * rank;
+    const int64_t vp = vs + kSegPages;
+    const int pf = part_of_page(vp, C, V);
+    const int pl = part_of_page(vp + n - 1, C, V);
     first[b] = pf;
     npart[b] = pl - pf + 1;
     nloc += pl - pf + 1;
-    for (int c = part_of_page(static_cast<int64_t>(run) - 1, C, P) + 1; c <= pl; ++c) pseq[c] = b;
+    for (int c = part_of_page(vs - 1, C, V) + 1; c <= pl; ++c) {
+      const int64_t u = (static_cast<int64_t>(c) * V) / C;  // the part's first virtual position
+      pstart[c] = run + static_cast<int>(u > vp ? u - vp : 0);
+      pseq[c] = b;
+    }
     run += n;
+    ++rank;
   }
   // 4. where each sequence's partials go
   int srun = block_exclusive_scan(nloc, warp_sums, nullptr);
   run = run0;
+  rank = rank0;
   for (int b = b0; b < b1; ++b) {
     const int n = plan_pages(seq_lens, b, cap, nullptr);
     slot[b] = srun;
-    if (n > 0)
-      srun += part_of_page(static_cast<int64_t>(run) + n - 1, C, P) - part_of_page(run, C, P) + 1;
+    if (n > 0) {
+      const int64_t vp =
+          static_cast<int64_t>(run) + static_cast<int64_t>(kSegPages) * rank + kSegPages;
+      srun += part_of_page(vp + n - 1, C, V) - part_of_page(vp, C, V) + 1;
+      ++rank;
+    }
     run += n;
   }
 }
@@ -489,16 +518,8 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(128)
           atomicOr(p.status, MLA_STATUS_BAD_PAGE);
           my_page = 0;
         }
-        // warm L2 ahead of the ring: each CTA of the pair fetches half of a page's rows
-        if (lane < min(cnt, kAhead))
-          prefetch_l2(p.pool + static_cast<size_t>(my_page) * kPageBytes + rank * (kPageBytes / 2),
-                      kPageBytes / 2);
         for (int j = 0; j < cnt; ++j, ++t) {
           const int page = __shfl_sync(kFull, my_page, j);
-          const int later = __shfl_sync(kFull, my_page, min(j + kAhead, 31));
-          if (lane == 0 && j + kAhead < cnt)
-            prefetch_l2(p.pool + static_cast<size_t>(later) * kPageBytes + rank * (kPageBytes / 2),
-                        kPageBytes / 2);
           if (lane == 0) {
             const int s = t % kSlots;
             if (t >= kSlots) ok = mbar_wait(&bars->empty[s], ((t / kSlots) - 1) & 1, wc);
