@@ -663,6 +663,20 @@ def run_fp8_step(layers, h, pos, lens_dev, lens, cfg, dev, steps):
     e1.record()
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
+    # end to end through the native executor, host buffers in and out (as the headline's e2e)
+    h_host = h.cpu().pin_memory()
+    pos_host, lens_host = pos.cpu().pin_memory(), lens_dev.cpu().pin_memory()
+    out_host = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
+    for _ in range(2):
+        step.run_native(h_host, pos_host, lens_host, out_host)
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record()
+    for _ in range(steps):
+        step.run_native(h_host, pos_host, lens_host, out_host)
+    f1.record()
+    torch.cuda.synchronize()
+    e2e_ms = f0.elapsed_time(f1) / steps
     st = M.mla_get_status()
     if st:
         raise RuntimeError(f"device status {st:#x} in the E4M3 step")
@@ -684,6 +698,10 @@ def run_fp8_step(layers, h, pos, lens_dev, lens, cfg, dev, steps):
     mx = float(np.abs(got - exp).max() / np.abs(exp).max())
     res = {"value": B / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
            "launch": "CUDA graph of the step",
+           "e2e": {"value": B / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
+                   "h2d_bytes_per_step": h_host.numel() * h_host.element_size() + 2 * B * 4,
+                   "d2h_bytes_per_step": out_host.numel() * out_host.element_size(),
+                   "path": "mla_decode_step_host with E4M3 layers"},
            "what": "the headline step with W_DKV, W_KR, W_Q, W_O in E4M3 (W_UK, W_UV bf16; "
                    "cache bf16)",
            "parity": {"o_heads_rel_l2": rel, "o_heads_max_abs": mx,

@@ -297,7 +297,10 @@ int mla_out_proj_fp8(const mla_dims* dims, const float* o_lat, const void* w_uv,
  * Native decode step over a stack of layers, end to end from host memory.
  *
  * mla_layer -- one layer's device-resident weights and paged cache (layouts as in the calls
- * above; w_o must be given: the step's result is `out`).
+ * above; w_o must be given: the step's result is `out`).  With w_q_scale non-NULL the layer's
+ * w_dkv, w_kr, w_q and w_o are E4M3 codes as mla_quantize_weights_fp8 writes them, with the
+ * four row-scale arrays (all required then), and the layer runs mla_append_absorb_fp8 and
+ * mla_out_proj_fp8; with w_q_scale NULL the four scale pointers are ignored.
  *
  * mla_step_workspace_size -- bytes of device workspace mla_decode_step_host needs: device
  *   copies of every layer's h and out, positions, lengths, q_cat, o_lat, lse, o_heads, and the
@@ -327,6 +330,10 @@ typedef struct mla_layer {
   int32_t num_pages;
   const int32_t* page_table;
   int32_t max_pages;
+  const float* w_dkv_scale;
+  const float* w_kr_scale;
+  const float* w_q_scale;
+  const float* w_o_scale;
 } mla_layer;
 
 size_t mla_step_workspace_size(const mla_dims* dims, int32_t n_layers, int32_t num_splits);

@@ -55,7 +55,9 @@ class mla_layer(ctypes.Structure):
     _fields_ = [("w_dkv", ctypes.c_void_p), ("w_kr", ctypes.c_void_p), ("w_q", ctypes.c_void_p),
                 ("w_uk", ctypes.c_void_p), ("w_uv", ctypes.c_void_p), ("w_o", ctypes.c_void_p),
                 ("cache_pool", ctypes.c_void_p), ("num_pages", ctypes.c_int32),
-                ("page_table", ctypes.c_void_p), ("max_pages", ctypes.c_int32)]
+                ("page_table", ctypes.c_void_p), ("max_pages", ctypes.c_int32),
+                ("w_dkv_scale", ctypes.c_void_p), ("w_kr_scale", ctypes.c_void_p),
+                ("w_q_scale", ctypes.c_void_p), ("w_o_scale", ctypes.c_void_p)]
 
 
 _lib = None
@@ -289,24 +291,35 @@ def mla_out_proj(d: mla_dims, o_lat, w_uv, ws, w_o=None, o_heads=None, out=None,
 
 
 def layer_structs(d: mla_dims, layers):
-    """ctypes array of mla_layer for step layers (objects with the Layer fields)."""
+    """ctypes array of mla_layer for step layers (objects with the Layer fields; a layer with
+    `e4m3` copies passes its codes and row scales instead of the bf16 W_DKV, W_KR, W_Q, W_O)."""
     e = _elem(d)
     arr = (mla_layer * len(layers))()
     for i, ly in enumerate(layers):
         H = d.n_heads
-        _need(ly.w_dkv, "w_dkv", e, (d.d_c, d.d_model))
-        _need(ly.w_kr, "w_kr", e, (d.d_rope, d.d_model))
-        _need(ly.w_q, "w_q", e, (H * (d.d_nope + d.d_rope), d.d_model))
-        _need(ly.w_uk, "w_uk", e, (H * d.d_nope, d.d_c))
-        _need(ly.w_uv, "w_uv", e, (H * d.d_v, d.d_c))
+        shapes = {"w_dkv": (d.d_c, d.d_model), "w_kr": (d.d_rope, d.d_model),
+                  "w_q": (H * (d.d_nope + d.d_rope), d.d_model), "w_o": (d.d_model, H * d.d_v)}
         if ly.w_o is None:
             raise ValueError("w_o is required: the step's result is out")
-        _need(ly.w_o, "w_o", e, (d.d_model, H * d.d_v))
+        q = getattr(ly, "e4m3", None)
+        ptrs, scales = {}, {}
+        for n, shp in shapes.items():
+            if q is not None:
+                codes, scale = q[n]
+                _need(codes, n + " codes", torch.uint8, fp8_codes_shape(*shp))
+                _need(scale, n + " scale", torch.float32, (shp[0],))
+                ptrs[n], scales[n] = _ptr(codes), _ptr(scale)
+            else:
+                _need(getattr(ly, n), n, e, shp)
+                ptrs[n], scales[n] = _ptr(getattr(ly, n)), None
+        _need(ly.w_uk, "w_uk", e, (H * d.d_nope, d.d_c))
+        _need(ly.w_uv, "w_uv", e, (H * d.d_v, d.d_c))
         _need(ly.pool, "cache_pool", e)
         _need(ly.page_table, "page_table", torch.int32)
-        arr[i] = mla_layer(_ptr(ly.w_dkv), _ptr(ly.w_kr), _ptr(ly.w_q), _ptr(ly.w_uk),
-                           _ptr(ly.w_uv), _ptr(ly.w_o), _ptr(ly.pool), ly.pool.shape[0],
-                           _ptr(ly.page_table), ly.page_table.shape[1])
+        arr[i] = mla_layer(ptrs["w_dkv"], ptrs["w_kr"], ptrs["w_q"], _ptr(ly.w_uk),
+                           _ptr(ly.w_uv), ptrs["w_o"], _ptr(ly.pool), ly.pool.shape[0],
+                           _ptr(ly.page_table), ly.page_table.shape[1], scales["w_dkv"],
+                           scales["w_kr"], scales["w_q"], scales["w_o"])
     return arr
 
 

@@ -99,8 +99,12 @@ int mla_decode_step_host(const mla_dims* dims, int32_t n_layers, const mla_layer
   if (n_layers < 1 || num_splits < 0) return MLA_ERR_ARG;
   if (!layers || !h_host || !positions_host || !seq_lens_host || !out_host)
     return MLA_ERR_NULL_ARG;
-  for (int l = 0; l < n_layers; ++l)
-    if (!layers[l].w_o) return MLA_ERR_NULL_ARG;  // the step's result is `out`
+  for (int l = 0; l < n_layers; ++l) {
+    const mla_layer& ly = layers[l];
+    if (!ly.w_o) return MLA_ERR_NULL_ARG;  // the step's result is `out`
+    if (ly.w_q_scale && (!ly.w_dkv_scale || !ly.w_kr_scale || !ly.w_o_scale))
+      return MLA_ERR_NULL_ARG;  // an E4M3 layer needs every row scale
+  }
   if (!workspace) return MLA_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(workspace) % 256) return MLA_ERR_ALIGN;
   const StepLayout s = step_layout(dims, n_layers, num_splits);
@@ -148,17 +152,24 @@ int mla_decode_step_host(const mla_dims* dims, int32_t n_layers, const mla_layer
     if ((rc = cuda_rc(cudaStreamWaitEvent(st, ss->ev_in[l], 0)))) return rc;
     void* hl = h_dev + l * layer_bytes;
     void* outl = out_dev + l * layer_bytes;
-    if ((rc = mla_append_absorb(dims, hl, ly.w_dkv, ly.w_kr, ly.w_q, ly.w_uk, pos_dev,
-                                ly.page_table, ly.max_pages, ly.cache_pool, ly.num_pages, q_cat,
-                                nullptr, call_ws, call_bytes, stream)))
-      return rc;
+    const bool e4m3 = ly.w_q_scale != nullptr;
+    rc = e4m3 ? mla_append_absorb_fp8(dims, hl, ly.w_dkv, ly.w_dkv_scale, ly.w_kr, ly.w_kr_scale,
+                                      ly.w_q, ly.w_q_scale, ly.w_uk, pos_dev, ly.page_table,
+                                      ly.max_pages, ly.cache_pool, ly.num_pages, q_cat, nullptr,
+                                      call_ws, call_bytes, stream)
+              : mla_append_absorb(dims, hl, ly.w_dkv, ly.w_kr, ly.w_q, ly.w_uk, pos_dev,
+                                  ly.page_table, ly.max_pages, ly.cache_pool, ly.num_pages,
+                                  q_cat, nullptr, call_ws, call_bytes, stream);
+    if (rc) return rc;
     if ((rc = mla_decode_attn(dims, q_cat, nullptr, ly.cache_pool, ly.num_pages, ly.page_table,
                               ly.max_pages, lens_dev, 0.f, num_splits, call_ws, call_bytes,
                               o_lat, lse, stream)))
       return rc;
-    if ((rc = mla_out_proj(dims, o_lat, ly.w_uv, ly.w_o, o_heads, outl, call_ws, call_bytes,
-                           stream)))
-      return rc;
+    rc = e4m3 ? mla_out_proj_fp8(dims, o_lat, ly.w_uv, ly.w_o, ly.w_o_scale, o_heads, outl,
+                                 call_ws, call_bytes, stream)
+              : mla_out_proj(dims, o_lat, ly.w_uv, ly.w_o, o_heads, outl, call_ws, call_bytes,
+                             stream);
+    if (rc) return rc;
     if ((rc = cuda_rc(cudaEventRecord(ss->ev_out[l], st)))) return rc;
     if ((rc = cuda_rc(cudaStreamWaitEvent(ss->out, ss->ev_out[l], 0)))) return rc;
     if ((rc = cuda_rc(cudaMemcpyAsync(static_cast<char*>(out_host) + l * layer_bytes, outl,

@@ -159,8 +159,6 @@ class DecodeStep:
         """End-to-end through the library's native step executor (mla_decode_step_host): the
         host buffers go in and `out` comes back with every copy and launch made in C++."""
         from . import layer_structs, mla_decode_step_host, step_workspace
-        if any(ly.e4m3 is not None for ly in self.layers):
-            raise ValueError("the native step executor takes bf16 weights")
         if getattr(self, "_native", None) is None:
             self._native = (layer_structs(self.dims, self.layers),
                             step_workspace(self.dims, len(self.layers), self.num_splits,

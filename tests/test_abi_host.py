@@ -230,6 +230,10 @@ def test_step_executor_arguments(M):
     lay[1] = M.mla_layer(0x10000, 0x10000, 0x10000, 0x10000, 0x10000, None, 0x10000, 8,
                          0x10000, 4)
     assert L.mla_decode_step_host(ctypes.byref(d), 2, lay, f, f, f, f, 0, ws, big, None) == -1
+    # an E4M3 layer (w_q_scale given) needs every row scale
+    lay[1] = M.mla_layer(0x10000, 0x10000, 0x10000, 0x10000, 0x10000, 0x10000, 0x10000, 8,
+                         0x10000, 4, 0x10000, None, 0x10000, 0x10000)
+    assert L.mla_decode_step_host(ctypes.byref(d), 2, lay, f, f, f, f, 0, ws, big, None) == -1
 
 
 

@@ -152,3 +152,44 @@ def test_append_absorb_fp8_rejects_large_batch():
                                 torch.empty(B, H, 576, dtype=torch.bfloat16, device="cuda"),
                                 M.workspace(d))
     assert e.value.code == -2
+
+
+def test_e4m3_step_matches_the_oracle():
+    """A two-layer decode step (graph replay) with every layer's W_DKV, W_KR, W_Q and W_O stored as
+    E4M3 (step.quantize_layer): each layer's o_heads and out against the oracle's non-absorbed
+    fp64 step run with the weights the codes stand for."""
+    import mla_latent_kv_37_b200 as M
+    from mla_latent_kv_37_b200.step import DecodeStep, Layer, quantize_layer
+    B, H, D = 4, 128, 1024
+    hist = [100, 0, 700, 64]
+    wls = [Workload(70 + 10 * l, B, H, D, hist) for l in range(2)]
+    layers = [quantize_layer(Layer(dev(wl.w.w_dkv), dev(wl.w.w_kr), dev(wl.w.w_q),
+                                   dev(wl.w.w_uk), dev(wl.w.w_uv), dev(wl.w.w_o),
+                                   dev(wl.cache.pool), dev(wl.cache.page_table)))
+              for wl in wls]
+    step = DecodeStep(layers, B, H, D, graph=True)
+    h = torch.stack([dev(wl.h) for wl in wls])
+    for _ in range(2):
+        step.run(h, dev(wls[0].pos), dev(wls[0].lens))
+    torch.cuda.synchronize()
+    assert M.mla_get_status() == 0
+    for l, (wl, ly) in enumerate(zip(wls, layers)):
+        w = I.Weights(*[O.dequantize_rows_e4m3(
+            M.fp8_codes_rows(ly.e4m3[n][0], *getattr(ly, n).shape).cpu().numpy(),
+            ly.e4m3[n][1].cpu().numpy()) if n in ly.e4m3 else getattr(wl.w, n)
+            for n in ("w_dkv", "w_kr", "w_q", "w_uk", "w_uv", "w_o")])
+        for b in range(B):
+            rows = O.gather_rows(wl.cache.pool, wl.cache.page_table[b].numpy(), hist[b])
+            ref = O.decode_step(wl.h[b], w, rows, hist[b], H,
+                                round_row=lambda r: torch.from_numpy(
+                                    np.asarray(r, dtype=np.float32)).to(torch.bfloat16))
+            assert_close(to_np(step.o_heads[l, b]), ref["o_heads"], torch.bfloat16,
+                         f"o_heads l={l} b={b}")
+            assert_close(to_np(step.out[l, b]), ref["out"], torch.bfloat16, f"out l={l} b={b}")
+    # the native executor (host buffers in and out) gives the device step's bytes
+    out_host = torch.full((2, B, D), float("nan"), dtype=torch.bfloat16).pin_memory()
+    step.run_native(h.cpu().pin_memory(), wls[0].pos.pin_memory(), wls[0].lens.pin_memory(),
+                    out_host)
+    torch.cuda.synchronize()
+    assert M.mla_get_status() == 0
+    assert torch.equal(out_host, step.out.cpu())
