@@ -4,7 +4,8 @@
 //
 // Decode projections multiply large weight matrices by a handful of token vectors, so their
 // cost is the time to stream the weights from HBM once.  The work -- every (128-row tile,
-// 64-wide K block) pair of every group -- is one list of I iterations cut into P equal
+// K block) pair of every group, a K block being one 128-byte piece of a row (64 bf16 or 128
+// E4M3 values) -- is one list of I iterations cut into P equal
 // contiguous ranges, one per CTA (P <= number of SMs), so every SM streams the same number of
 // weight bytes in one wave and its TMA -> shared memory -> tcgen05.mma pipeline never drains
 // between tiles.  A CTA's range splits into segments at tile boundaries; each segment is
@@ -36,7 +37,14 @@
 // Operand layouts in shared memory (128-byte swizzle, filled by TMA):
 //   A K-major : box (64 k, 128 m)   -> [128 rows][128 B], SBO = 1024 B
 //   A MN-major: 2 boxes (64 m, 64 k) -> [64 k rows][128 B] per 64-m half, LBO = 8 KiB
+//   A tiled   : box (128 B, 128 m, kbs) from weights stored as 16 KB tiles -> the K-major layout
 //   X         : box (64 k, 1, n_pad) -> [n_pad rows][128 B], SBO = 1024 B
+//
+// E4M3 instantiation (kFp8): weights and activations are E4M3 bytes, so a K block is 128 values
+// in the same 128-byte rows, and tcgen05.mma.kind::f8f6f4 covers 32 of them per instruction
+// with the bf16 path's descriptors and 32-byte K step.  The activations arrive as n_planes
+// column planes (E4M3 pieces of one activation row) that the epilogue sums, then scales by the
+// weight row's and the activation row's scales.
 #pragma once
 #include "ptx_sm100.cuh"
 #include "rope.cuh"
