@@ -247,3 +247,28 @@ def test_timeout_path_reports_and_recovers(monkeypatch):
     o, l, st = _run(q, cache, lens, 128)
     assert st == 0
     _check(q, cache, lens, o, l)
+
+
+@pytest.mark.parametrize("splits", [1, 5, 0, 200, 1000])
+def test_plan_many_short_and_empty_sequences(splits):
+    """The planner's cost model (each sequence start weighs as a few pages) on a hard mix: 128
+    sequences of 0 to 700 tokens (a quarter empty, many under one page), split into 1 to 1000
+    parts, so that parts begin inside sequences' start-up, some parts stay empty and most
+    sequences are cut several times; every sequence against the oracle."""
+    import random
+    rnd = random.Random(splits + 17)
+    lens = [0 if rnd.random() < 0.25 else rnd.choice([1, 2, 63, 64, 65, rnd.randint(1, 700)])
+            for _ in range(128)]
+    q, cache = _case(300 + splits, lens, 128)
+    o, l, st = _run(q, cache, lens, 128, num_splits=splits)
+    assert st == 0
+    _check(q, cache, lens, o, l)
+
+
+def test_plan_many_parts_fp32():
+    """The fp32 path's planner with more parts than pages in some sequences."""
+    lens = [1, 0, 130, 64, 65, 300, 2, 0]
+    q, cache = _case(23, lens, 16, dtype=torch.float32)
+    o, l, st = _run(q, cache, lens, 16, num_splits=37, dtype=torch.float32)
+    assert st == 0
+    _check(q, cache, lens, o, l, dtype=torch.float32)
