@@ -113,11 +113,12 @@ def test_append_absorb_fp8_matches_oracle(B, H, D, scale):
     pool = dev(wl.cache.pool)
     before = wl.cache.pool.clone()
     q_cat = torch.full((B, H, 576), float("nan"), dtype=torch.bfloat16, device="cuda")
+    q_lo = torch.full((B, H, 576), float("nan"), dtype=torch.bfloat16, device="cuda")
     M.mla_append_absorb_fp8(d, dev(wl.h), dkv, kr, wq, dev(w.w_uk), dev(wl.pos),
-                            dev(wl.cache.page_table), pool, q_cat, M.workspace(d))
+                            dev(wl.cache.page_table), pool, q_cat, M.workspace(d), q_lo=q_lo)
     torch.cuda.synchronize()
     assert M.mla_get_status() == 0
-    pool, q_cat = pool.cpu(), q_cat.cpu()
+    pool, q_cat, q_lo = pool.cpu(), q_cat.cpu(), q_lo.cpu()
     changed = (pool.view(pool.shape[0], 64, -1) != before.view(pool.shape[0], 64, -1)).any(-1)
     w_uk = O.f64(w.w_uk)
     for b, pos in enumerate(wl.history):
@@ -131,6 +132,10 @@ def test_append_absorb_fp8_matches_oracle(B, H, D, scale):
             q_lat = np.stack([w_uk[i * 128:(i + 1) * 128].T @ qn[i] for i in range(H)])
             assert_close(to_np(q_cat[b, :, :512]), q_lat, torch.bfloat16, f"q_lat b={b}")
             assert_close(to_np(q_cat[b, :, 512:]), qr, torch.bfloat16, f"q_rope b={b}")
+            # with the rounding remainder the query carries ~16 significant bits
+            exact = to_np(q_cat[b]) + to_np(q_lo[b])
+            rel = np.linalg.norm(exact[:, :512] - q_lat) / np.linalg.norm(q_lat)
+            assert rel < 1e-4, f"q_lat + q_lo b={b}: {rel:.2e}"
     assert not changed.any(), "append wrote outside the addressed slots"
 
 
