@@ -279,3 +279,58 @@ def test_e4m3_weight_arguments(M):
     bad = list(oargs)
     bad[2] = odd  # W_O codes
     assert L.mla_out_proj_fp8(ctypes.byref(d), *bad) == -3
+
+
+C_PROGRAM = r"""
+#include <stdio.h>
+#include <string.h>
+#include "mla.h"
+
+int main(void) {
+  mla_dims d;
+  memset(&d, 0, sizeof d);
+  d.batch = 4;
+  d.n_heads = 128;
+  d.d_model = 7168;
+  d.d_c = 512;
+  d.d_rope = 64;
+  d.d_nope = 128;
+  d.d_v = 128;
+  d.page_size = 64;
+  d.dtype = MLA_BF16;
+  d.rope_theta = 10000.0f;
+  printf("version %s\n", mla_version());
+  printf("row_bytes %lld\n", (long long)mla_cache_row_bytes(&d));
+  printf("workspace_nonzero %d\n", mla_workspace_size(&d, 0) > 0);
+  printf("null_args %d\n", mla_decode_attn(&d, NULL, NULL, NULL, 1, NULL, 1, NULL, 0.f, 0, NULL,
+                                          0, NULL, NULL, NULL));
+  printf("error_string %s\n", mla_error_string(MLA_ERR_NULL_ARG));
+  return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_links(M, tmp_path):
+    """include/mla.h compiles as strict C99 with every warning an error, and a C program links
+    against the library and calls it: the boundary needs neither C++ nor Python."""
+    import os
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "abi.c"
+    src.write_text(C_PROGRAM)
+    lib_dir = os.path.dirname(M.LIB_PATH)
+    exe = tmp_path / "abi"
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                        "-I", os.path.dirname(HEADER), str(src), "-L", lib_dir, "-lmla_b200",
+                        "-Wl,-rpath," + lib_dir, "-o", str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert out.returncode == 0, out.stderr
+    lines = dict(line.split(" ", 1) for line in out.stdout.strip().splitlines())
+    assert lines["row_bytes"] == "1152"
+    assert lines["workspace_nonzero"] == "1"
+    assert lines["null_args"] == "-1"
+    assert lines["version"]
