@@ -42,7 +42,7 @@ __global__ void append_epilogue_kernel(const float* __restrict__ part, int k_spl
                                        const int32_t* __restrict__ page_table, int max_pages,
                                        T* __restrict__ pool, int num_pages, float theta,
                                        unsigned int* status) {
-  constexpr int kRow = 576, kDc = 512, kDr = 64, kPage = 64;
+  constexpr int kRow = 576, kDc = 512, kPage = 64;
   const int b = blockIdx.y;
   const int q = blockIdx.x * blockDim.x + threadIdx.x;
   if (2 * q >= kRow) return;
@@ -86,7 +86,7 @@ __global__ void wq_epilogue_kernel(const float* __restrict__ part, int k_splits,
                                    int H, const int32_t* __restrict__ positions, float theta,
                                    T* __restrict__ q_cat, __nv_bfloat16* __restrict__ q_lo,
                                    void* __restrict__ qn_out) {
-  constexpr int kDn = 128, kDr = 64, kDq = 192, kRow = 576, kDc = 512;
+  constexpr int kDn = 128, kDq = 192, kRow = 576, kDc = 512;
   const int h = blockIdx.x, b = blockIdx.y;
   const int d = 2 * threadIdx.x;
   if (d >= kDq) return;
