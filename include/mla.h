@@ -261,7 +261,7 @@ int mla_out_proj_folded(const mla_dims* dims, const float* o_lat, const void* w_
  *
  * mla_append_absorb_fp8 -- mla_append_absorb with W_DKV, W_KR and W_Q stored as E4M3 (each
  *   as mla_quantize_weights_fp8 writes it, with its row scales); W_UK stays bf16.  bf16 path
- *   only, batch <= 80 and d_model a multiple of 128 (else MLA_ERR_DIMS).  Each hidden-state
+ *   only, d_model a multiple of 128 (else MLA_ERR_DIMS).  Each hidden-state
  *   row h_b enters the E4M3 x E4M3 product as a power-of-two scale s_b (the smallest power of
  *   two >= max|h_b| / 448) and two E4M3 planes whose sum is h_b / s_b exactly (a bf16 value has
  *   8 significant bits; only parts below E4M3's smallest subnormal, under about 2^-8 of the
@@ -271,11 +271,12 @@ int mla_out_proj_folded(const mla_dims* dims, const float* o_lat, const void* w_
  *
  * mla_out_proj_fp8 -- mla_out_proj with W_O stored as E4M3 codes + row scales (w_o_codes:
  *   W_O [D, H*d_v] as mla_quantize_weights_fp8 writes it, w_o_scale [D]); W_UV stays bf16.
- *   out is required, o_heads optional.  bf16 path only, batch <= 80 (MLA_ERR_DIMS above: the three activation planes below take
- *   3 * round16(batch) of the 256 columns of one MMA).  The codes stream from HBM at one byte
- *   per weight into E4M3 x E4M3 tensor-core products (fp32 sums).  Each o_heads row b enters
- *   as a scale s_b = max|o_b| / 448 and three E4M3 planes whose sum keeps about 12 significant
- *   bits of o_b / s_b; out[b][r] = w_o_scale[r] * s_b * (sum over planes), rounded to bf16.
+ *   out is required, o_heads optional.  bf16 path only.  The codes stream from HBM at one
+ *   byte per weight into E4M3 x E4M3 tensor-core products (fp32 sums).  Each o_heads row b
+ *   enters as a scale s_b = max|o_b| / 448 and E4M3 planes whose sum approximates o_b / s_b:
+ *   three planes (about 12 significant bits) for batches up to 32, two (about 8) above, so that
+ *   planes x round16(batch) fit the 256 columns of one MMA up to batch 128;
+ *   out[b][r] = w_o_scale[r] * s_b * (sum over planes), rounded to bf16.
  *   The workspace of mla_workspace_size serves it (projection part only, as mla_out_proj).
  */
 int mla_quantize_weights_fp8(const void* w, int64_t rows, int64_t cols, void* codes,

@@ -379,7 +379,7 @@ def fp8_codes_rows(codes, rows, cols):
 def mla_append_absorb_fp8(d: mla_dims, h, w_dkv, w_kr, w_q, w_uk, positions, page_table,
                           cache_pool, q_cat, ws, q_lo=None, stream=None):
     """mla_append_absorb with W_DKV, W_KR, W_Q given as (codes, scale) pairs from
-    mla_quantize_weights_fp8 (bf16 path, batch <= 80); W_UK stays bf16."""
+    mla_quantize_weights_fp8 (bf16 path); W_UK stays bf16."""
     H = d.n_heads
     m_q = H * (d.d_nope + d.d_rope)
     pairs = (("w_dkv", w_dkv, d.d_c), ("w_kr", w_kr, d.d_rope), ("w_q", w_q, m_q))
@@ -405,7 +405,7 @@ def mla_append_absorb_fp8(d: mla_dims, h, w_dkv, w_kr, w_q, w_uk, positions, pag
 def mla_out_proj_fp8(d: mla_dims, o_lat, w_uv, w_o_codes, w_o_scale, out, ws, o_heads=None,
                      stream=None):
     """mla_out_proj with W_O stored as E4M3 codes (tiled, as mla_quantize_weights_fp8 writes
-    them) and row scales (bf16 path, batch <= 80)."""
+    them) and row scales (bf16 path)."""
     H = d.n_heads
     _need(o_lat, "o_lat", torch.float32, (d.batch, H, d.d_c))
     _need(w_uv, "w_uv", torch.bfloat16, (H * d.d_v, d.d_c))

@@ -59,17 +59,17 @@ __device__ __forceinline__ float2 e4m3x2_value(uint16_t c) {
   return __half22float2(*reinterpret_cast<const __half2*>(&h));
 }
 
-// fp32 activation rows x_b (K values each) as a scale and three E4M3 planes: s_b = m_b / 448
-// (at least FLT_MIN) with m_b = max_k |x_bk| given as fp32 bits in rowmax[b]; y = x / s_b;
-// p1 = E4M3(y), p2 = E4M3(y - p1), p3 = E4M3(y - p1 - p2), each difference exact in fp32.
-// p1 + p2 + p3 keeps about 12 significant bits of y, so s_b (p1 + p2 + p3) stands in for x_b in a
-// product with E4M3 weights.  planes: [3][rows_pad][K]; rows in [rows, rows_pad) are written as
-// zeros.  Each thread converts 8 consecutive values (grid-stride); K a multiple of 8; x and
-// planes 16- and 8-byte aligned.
+// fp32 activation rows x_b (K values each) as a scale and n_planes (2 or 3) E4M3 planes:
+// s_b = m_b / 448 (at least FLT_MIN) with m_b = max_k |x_bk| given as fp32 bits in rowmax[b];
+// y = x / s_b; p1 = E4M3(y), p2 = E4M3(y - p1), p3 = E4M3(y - p1 - p2), each difference exact
+// in fp32.  The planes' sum keeps about 4 significant bits of y per plane (8 with two, 12 with
+// three), so s_b (p1 + p2 [+ p3]) stands in for x_b in a product with E4M3 weights.  planes:
+// [n_planes][rows_pad][K]; rows in [rows, rows_pad) are written as zeros.  Each thread converts
+// 8 consecutive values (grid-stride); K a multiple of 8; x and planes 16- and 8-byte aligned.
 __global__ void __launch_bounds__(256)
     split_planes_kernel(const float* __restrict__ x, const unsigned int* __restrict__ rowmax,
-                        int rows, long long K, int rows_pad, uint8_t* __restrict__ planes,
-                        float* __restrict__ scale) {
+                        int rows, long long K, int rows_pad, int n_planes,
+                        uint8_t* __restrict__ planes, float* __restrict__ scale) {
   griddep_launch_dependents();
   griddep_wait();
   const long long n8 = K / 8;
@@ -79,7 +79,7 @@ __global__ void __launch_bounds__(256)
        i < static_cast<long long>(plane8); i += static_cast<long long>(gridDim.x) * blockDim.x) {
     const int b = static_cast<int>(i / n8);
     if (b >= rows) {
-      for (int pl = 0; pl < 3; ++pl) out[pl * plane8 + i] = make_uint2(0u, 0u);
+      for (int pl = 0; pl < n_planes; ++pl) out[pl * plane8 + i] = make_uint2(0u, 0u);
       continue;
     }
     const float s = fmaxf(__fdiv_rn(__uint_as_float(rowmax[b]), 448.f), FLT_MIN);
@@ -91,6 +91,7 @@ __global__ void __launch_bounds__(256)
     for (int k = 0; k < 8; ++k) y[k] = __fdiv_rn(y[k], s);
 #pragma unroll
     for (int pl = 0; pl < 3; ++pl) {
+      if (pl == n_planes) break;
       uint32_t c[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {

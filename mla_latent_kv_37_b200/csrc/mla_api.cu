@@ -52,7 +52,7 @@ constexpr int kMaxParts = 1 << 16;  // upper bound on num_splits (host check bef
 constexpr int kSkMinUnits = 2;    // fewest stages' worth of weights a stream-K CTA streams
 constexpr int kSkMaxContrib = 4;  // aim for at most this many CTAs sharing one tile
 constexpr int kSkMaxStages = 12;
-constexpr int kFp8MaxBatch = 80;  // E4M3 W_O product: 3 planes x round16(B) <= 256 MMA columns
+constexpr int kFp8MaxBatch = 128;  // E4M3 products: planes x round16(B) <= 256 MMA columns
 constexpr size_t kSmemPerBlockMax = 232448;  // 227 KiB opt-in limit per CTA
 
 // ------------------------------------------------------------------------------------------
@@ -227,10 +227,12 @@ GemmShape shape_append_wq_e4m3(const mla_dims* d) {
   return {sk::EpiAppendWq::kSplitRow + m, 5 + m / 128, d->d_model, 1, 2 * round16(d->batch),
           round16(d->batch), 1};
 }
-// W_O in E4M3 against o_heads as three E4M3 planes (tcgen05 kind::f8f6f4)
+// W_O in E4M3 against o_heads as E4M3 planes (tcgen05 kind::f8f6f4): three planes (~12
+// significant bits) while they fit the MMA cheaply, two (~8 bits) above 32 rows
+int oh_planes(const mla_dims* d) { return round16(d->batch) <= 32 ? 3 : 2; }
 GemmShape shape_wo_e4m3(const mla_dims* d) {
-  return {d->d_model, (d->d_model + 127) / 128, d->n_heads * kDv, 1, 3 * round16(d->batch),
-          round16(d->batch), 1};
+  return {d->d_model, (d->d_model + 127) / 128, d->n_heads * kDv, 1,
+          oh_planes(d) * round16(d->batch), round16(d->batch), 1};
 }
 
 // Stream-K launch plan: K blocks per stage, CTAs, partial slots per tile, ring depth, smem.
@@ -1213,23 +1215,25 @@ int mla_out_proj_fp8(const mla_dims* dims, const float* o_lat, const void* w_uv,
   sk::EpiWuv e1{H, Bp, static_cast<__nv_bfloat16*>(o_heads), nullptr, oh32, xmax};
   if ((rc = run_streamk(c, s1, q1, B, nullptr, 0.f, a, a, 1 << 30, 0, bm, ws, w, e1, st)))
     return rc;
-  // o_heads row b -> three E4M3 planes and a scale (the W_UV input is consumed by now)
+  // o_heads row b -> E4M3 planes and a scale (the W_UV input is consumed by now)
   const GemmShape s2 = shape_wo_e4m3(dims);
+  const int n_planes = oh_planes(dims);
   const uint64_t K = static_cast<uint64_t>(H) * kDv;
   uint8_t* planes = reinterpret_cast<uint8_t*>(ws + w.o_split);
-  float* x_scale = reinterpret_cast<float*>(ws + w.o_split + align_up(3 * Bp * K, 256));
+  float* x_scale =
+      reinterpret_cast<float*>(ws + w.o_split + align_up(n_planes * Bp * K, 256));
   const size_t groups8 = static_cast<size_t>(Bp) * K / 8;
   launch_pdl(fp8::split_planes_kernel,
              dim3(static_cast<unsigned>(std::min<size_t>((groups8 + 255) / 256, 4 * c->sms))),
              dim3(256), 0, st, static_cast<const float*>(oh32),
-             static_cast<const unsigned int*>(xmax), B, static_cast<long long>(K), Bp, planes,
-             x_scale);
+             static_cast<const unsigned int*>(xmax), B, static_cast<long long>(K), Bp, n_planes,
+             planes, x_scale);
   if ((rc = last_launch())) return rc;
   // out = s_W,r * s_x,b * sum over planes of (W_O codes) x (plane codes), kind::f8f6f4
   const SkPlan q2 = sk_plan(s2, 0, c->sms);
   CUtensorMap a2, b2;
   if ((rc = map_weights_e4m3(&a2, w_o_codes, D, K, q2.kbs))) return rc;
-  if ((rc = map_acts_e4m3(&b2, planes, 3 * Bp, K, s2.n_pad, q2.kbs))) return rc;
+  if ((rc = map_acts_e4m3(&b2, planes, n_planes * Bp, K, s2.n_pad, q2.kbs))) return rc;
   sk::EpiWo e2{D, static_cast<__nv_bfloat16*>(out)};
   E4m3Scales sc;
   sc.a[0] = w_o_scale;

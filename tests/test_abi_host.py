@@ -240,7 +240,7 @@ def test_step_executor_arguments(M):
 def test_e4m3_weight_arguments(M):
     """The E4M3-weight calls check their arguments on the host, before any device work: code
     widths that are not whole 128-column tiles, missing or misaligned pointers, the fp32
-    path, batches above 80 and d_model not a multiple of 128."""
+    path, batches above 128 and d_model not a multiple of 128."""
     import torch
     d = _d(M)
     d32 = M.dims(4, 16, 1024, dtype=torch.float32)
@@ -257,7 +257,7 @@ def test_e4m3_weight_arguments(M):
     # append + absorb with E4M3 W_DKV, W_KR, W_Q
     args = [f, f, f, f, f, f, f, f, f, f, 4, f, 8, f, None, ws, big, None]
     assert L.mla_append_absorb_fp8(ctypes.byref(d32), *args) == -5
-    assert L.mla_append_absorb_fp8(ctypes.byref(M.dims(81, 16, 1024)), *args) == -2
+    assert L.mla_append_absorb_fp8(ctypes.byref(M.dims(129, 16, 1024)), *args) == -2
     assert L.mla_append_absorb_fp8(ctypes.byref(M.dims(4, 16, 1088)), *args) == -2
     for i, code in ((1, -1), (6, -1), (7, -1), (13, -1)):  # codes, scale, w_uk, q_cat
         bad = list(args)
@@ -272,7 +272,7 @@ def test_e4m3_weight_arguments(M):
     # output projection with E4M3 W_O
     oargs = [f, f, f, f, None, f, ws, big, None]
     assert L.mla_out_proj_fp8(ctypes.byref(d32), *oargs) == -5
-    assert L.mla_out_proj_fp8(ctypes.byref(M.dims(81, 16, 1024)), *oargs) == -2
+    assert L.mla_out_proj_fp8(ctypes.byref(M.dims(129, 16, 1024)), *oargs) == -2
     bad = list(oargs)
     bad[5] = None  # out
     assert L.mla_out_proj_fp8(ctypes.byref(d), *bad) == -1

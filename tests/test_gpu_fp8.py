@@ -40,8 +40,8 @@ def test_quantize_matches_oracle_bit_for_bit(rows, cols, std):
     assert np.array_equal(untile(codes.cpu(), rows, cols), exp_codes)
 
 
-@pytest.mark.parametrize("B,H,D", [(3, 16, 1024), (32, 128, 7168), (64, 32, 512),
-                                   (80, 16, 1024)])
+@pytest.mark.parametrize("B,H,D", [(3, 16, 1024), (32, 128, 7168), (33, 16, 1024),
+                                   (64, 32, 512), (128, 16, 1024)])
 def test_out_proj_fp8_matches_oracle(B, H, D):
     import mla_latent_kv_37_b200 as M
     hist = [(41 * i + 3) % 200 for i in range(B)]
@@ -72,15 +72,16 @@ def test_out_proj_fp8_matches_oracle(B, H, D):
 
 
 def test_out_proj_fp8_rejects_large_batch():
-    """Batch 81: three E4M3 planes of round16(81) = 96 columns exceed the MMA's 256."""
+    """Batch 129: above the bf16 path's 128 (two E4M3 planes of round16(129) = 144 columns would
+    exceed the MMA's 256)."""
     import mla_latent_kv_37_b200 as M
-    d = M.dims(81, 16, 1024)
+    d = M.dims(129, 16, 1024)
     with pytest.raises(M.MlaError) as e:
-        M.mla_out_proj_fp8(d, torch.empty(81, 16, 512, device="cuda"),
+        M.mla_out_proj_fp8(d, torch.empty(129, 16, 512, device="cuda"),
                            torch.empty(16 * 128, 512, dtype=torch.bfloat16, device="cuda"),
                            torch.empty(1024, 16 * 128, dtype=torch.uint8, device="cuda"),
                            torch.empty(1024, device="cuda"),
-                           torch.empty(81, 1024, dtype=torch.bfloat16, device="cuda"),
+                           torch.empty(129, 1024, dtype=torch.bfloat16, device="cuda"),
                            M.workspace(d))
     assert e.value.code == -2
 
@@ -97,7 +98,7 @@ def _quantize(M, w):
 
 
 @pytest.mark.parametrize("B,H,D,scale", [(32, 128, 7168, 1.0), (5, 16, 1024, 4.0),
-                                         (33, 32, 512, 1.0), (80, 16, 1024, 1.0)])
+                                         (33, 32, 512, 1.0), (128, 16, 1024, 1.0)])
 def test_append_absorb_fp8_matches_oracle(B, H, D, scale):
     """Cache append + absorbed query with W_DKV, W_KR and W_Q stored as E4M3: the appended cache
     rows and q_cat against the oracle's fp64 projections with the weights the codes stand for
@@ -141,7 +142,7 @@ def test_append_absorb_fp8_matches_oracle(B, H, D, scale):
 
 def test_append_absorb_fp8_rejects_large_batch():
     import mla_latent_kv_37_b200 as M
-    B, H, D = 81, 16, 1024
+    B, H, D = 129, 16, 1024
     d = M.dims(B, H, D)
 
     def pair(rows):
