@@ -954,7 +954,7 @@ def main():
     # ---------------- the other configurations and the attention sweep (one GPU) ----------
     configs = sweep = modes = fp8w = fp8s = None
     if rank == 0 and world == 1 and not args.no_extras:
-        if B <= 80:
+        if B <= 128:
             del step
             torch.cuda.empty_cache()
             fp8s = run_fp8_step(layers, h, pos, lens_dev, lens, cfg, dev, max(3, args.steps // 2))
